@@ -1,0 +1,328 @@
+"""Plain fp64 CPU oracle for SLA (Sparse-Linear Attention).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's
+CPU-baseline leg may import this module.  It shares no code with the CUDA path
+and never calls it.  It is slow on purpose: every step is the definition
+written out, with numpy matrix products as the only library primitive.
+
+Sources.  "SLA" below is the paper page "SLA: Beyond Sparsity in Diffusion
+Transformers via Fine-Tunable Sparse-Linear Attention" (arXiv 2509.24006):
+its English abstract and the Chinese card's technical-framework steps 1-4
+fix that attention weights fall into critical / marginal / negligible groups,
+that critical pairs get exact O(N^2) softmax attention, marginal pairs get
+O(N) linear attention and negligible pairs are skipped, and that a backward
+pass exists.  The pages leave open how the classes are chosen, the feature
+map, the combination and the backward math; this oracle takes these readings
+(each restated where it is used):
+
+* R1  classes come from block mean-pooled Q and K: pooled logits
+      s_ij = mean(Q_i) . mean(K_j) * scale; per row, order j by
+      (s_ij descending, j ascending); the first n_h are critical (+1), the
+      last n_l negligible (-1), the rest marginal (0).  Ranking logits is the
+      same as ranking the row softmax of the pooled scores (softmax is
+      strictly increasing within a row).
+* R3  n_h = ceil(k_h*T - 1e-9), n_l = min(floor(k_l*T + 1e-9), T - n_h).
+* R4  phi(x) = elu(x) + 1 (alpha 1): x + 1 for x > 0, exp(x) otherwise.
+* R5  a query block with no critical key block has O_s = 0 and LSE = -inf.
+* R6  linear branch: O_l,t = phi(Q_t)^T H_i / (phi(Q_t) . Z_i) with
+      H_i = sum_{j marginal} phi(K_j)^T V_j and Z_i = sum_{j marginal}
+      sum_{u in j} phi(K_u); no epsilon; 0 when row i has no marginal block.
+* R7  O = O_s + O_l W_proj, W_proj one d x d matrix for all heads.
+* R8  gradients treat the classification as a constant.
+
+Arrays are [B, H, N, d]; blocks are consecutive runs of ``block`` tokens.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "block_counts",
+    "pool",
+    "pooled_logits",
+    "classify",
+    "classify_rows_bruteforce",
+    "phi",
+    "phi_prime",
+    "key_block_summaries",
+    "forward",
+    "forward_bruteforce",
+    "backward",
+    "sla",
+]
+
+
+def block_counts(T: int, k_h: float, k_l: float) -> tuple[int, int]:
+    """Critical and negligible block counts per row (reading R3)."""
+    if not (0.0 <= k_h and 0.0 <= k_l and k_h + k_l <= 1.0 + 1e-12):
+        raise ValueError("need 0 <= k_h, k_l and k_h + k_l <= 1")
+    n_h = min(T, max(0, math.ceil(k_h * T - 1e-9)))
+    n_l = max(0, min(math.floor(k_l * T + 1e-9), T - n_h))
+    return n_h, n_l
+
+
+def pool(x: np.ndarray, block: int) -> np.ndarray:
+    """Mean of each block of ``block`` consecutive tokens: [B,H,N,d] -> [B,H,T,d]."""
+    B, H, N, d = x.shape
+    if N % block:
+        raise ValueError("N must be a multiple of the block size")
+    return x.astype(np.float64).reshape(B, H, N // block, block, d).mean(axis=3)
+
+
+def pooled_logits(q: np.ndarray, k: np.ndarray, block: int, scale: float) -> np.ndarray:
+    """s_ij = mean(Q_i) . mean(K_j) * scale, [B,H,T,T] (reading R1)."""
+    qb, kb = pool(q, block), pool(k, block)
+    return np.einsum("bhid,bhjd->bhij", qb, kb) * scale
+
+
+def classify(logits: np.ndarray, n_h: int, n_l: int) -> np.ndarray:
+    """Three-way block classes from score rows (reading R1): int8 in {+1,0,-1}.
+
+    Each row is ordered by (score descending, key-block index ascending); the
+    first n_h entries are critical, the last n_l negligible.
+    """
+    logits = np.asarray(logits, dtype=np.float64)
+    if np.isnan(logits).any():
+        raise ValueError("NaN scores have no ordering")
+    *lead, T = logits.shape
+    flat = logits.reshape(-1, T)
+    cls = np.zeros(flat.shape, dtype=np.int8)
+    idx = np.arange(T)
+    for r in range(flat.shape[0]):
+        order = np.lexsort((idx, -flat[r]))  # primary: -score, secondary: index
+        cls[r, order[:n_h]] = 1
+        if n_l:
+            cls[r, order[T - n_l:]] = -1
+    return cls.reshape(*lead, T)
+
+
+def classify_rows_bruteforce(row: list[float], n_h: int, n_l: int) -> list[int]:
+    """Pure-Python per-entry rank count; the independent check of ``classify``.
+
+    rank(j) = #{k : s_k > s_j} + #{k < j : s_k == s_j}; critical iff
+    rank < n_h, negligible iff rank >= T - n_l.
+    """
+    T = len(row)
+    out = []
+    for j in range(T):
+        rank = sum(1 for k in range(T) if row[k] > row[j] or (row[k] == row[j] and k < j))
+        out.append(1 if rank < n_h else (-1 if rank >= T - n_l else 0))
+    return out
+
+
+def phi(x: np.ndarray) -> np.ndarray:
+    """elu(x) + 1 with alpha = 1 (reading R4)."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+
+
+def phi_prime(x: np.ndarray) -> np.ndarray:
+    """Derivative of phi: 1 for x > 0, exp(x) otherwise."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.where(x > 0, 1.0, np.exp(np.minimum(x, 0.0)))
+
+
+def key_block_summaries(k: np.ndarray, v: np.ndarray, block: int):
+    """Per key block j: h_j = phi(K_j)^T V_j [d,d] and z_j = sum_u phi(K_u) [d].
+
+    These are the per-key-block summaries through which marginal pairs get
+    O(N) linear attention (SLA abstract; framework step 3).
+    """
+    B, H, N, d = k.shape
+    T = N // block
+    fk = phi(k).reshape(B, H, T, block, d)
+    vb = v.astype(np.float64).reshape(B, H, T, block, d)
+    h = np.einsum("bhtua,bhtuc->bhtac", fk, vb)
+    z = fk.sum(axis=3)
+    return h, z
+
+
+def _tokens(blocks: np.ndarray, block: int) -> np.ndarray:
+    return (blocks[:, None] * block + np.arange(block)[None, :]).reshape(-1)
+
+
+def forward(q, k, v, w_proj, cls, block: int, scale: float | None = None,
+            query_blocks=None):
+    """SLA forward with a given class map ``cls`` [B,H,T,T].
+
+    Returns a dict with o, o_s, o_l [B,H,N,d], lse and den [B,H,N] (fp64).
+    ``query_blocks``, if given, restricts the work to those query-block
+    indices (other rows stay zero / -inf); used to sample large problems.
+    """
+    B, H, N, d = q.shape
+    T = N // block
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    q64, k64, v64 = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    w64 = np.asarray(w_proj, dtype=np.float64)
+    h, z = key_block_summaries(k64, v64, block)
+    o_s = np.zeros((B, H, N, d))
+    o_l = np.zeros((B, H, N, d))
+    lse = np.full((B, H, N), -np.inf)
+    den = np.zeros((B, H, N))
+    rows = range(T) if query_blocks is None else query_blocks
+    for b in range(B):
+        for hh in range(H):
+            for i in rows:
+                t0, t1 = i * block, (i + 1) * block
+                qi = q64[b, hh, t0:t1]
+                crit = np.nonzero(cls[b, hh, i] == 1)[0]
+                marg = np.nonzero(cls[b, hh, i] == 0)[0]
+                # critical pairs: exact softmax attention over all their key tokens
+                if crit.size:
+                    keys = _tokens(crit, block)
+                    s = (qi @ k64[b, hh, keys].T) * scale
+                    m = s.max(axis=1, keepdims=True)
+                    e = np.exp(s - m)
+                    l = e.sum(axis=1, keepdims=True)
+                    o_s[b, hh, t0:t1] = (e @ v64[b, hh, keys]) / l
+                    lse[b, hh, t0:t1] = (m + np.log(l))[:, 0]
+                # marginal pairs: linear attention through the key-block summaries
+                if marg.size:
+                    Hi = h[b, hh, marg].sum(axis=0)
+                    Zi = z[b, hh, marg].sum(axis=0)
+                    fq = phi(qi)
+                    num = fq @ Hi
+                    dn = fq @ Zi
+                    o_l[b, hh, t0:t1] = num / dn[:, None]
+                    den[b, hh, t0:t1] = dn
+                # negligible pairs contribute nothing
+    o = o_s + np.einsum("bhta,ac->bhtc", o_l, w64)
+    return {"o": o, "o_s": o_s, "o_l": o_l, "lse": lse, "den": den}
+
+
+def forward_bruteforce(q, k, v, w_proj, cls, block: int, scale: float | None = None):
+    """Per-token loops over every key with the class looked up per key.
+
+    The linear branch is written per key token,
+    O_l,t = sum_u (phi(Q_t).phi(K_u)) V_u / sum_u phi(Q_t).phi(K_u),
+    u over marginal tokens, so agreement with ``forward`` pins the summary
+    reassociation.  Meant for N <= 256.
+    """
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    q64, k64, v64 = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    w64 = np.asarray(w_proj, dtype=np.float64)
+    o = np.zeros((B, H, N, d))
+    for b in range(B):
+        for hh in range(H):
+            for t in range(N):
+                i = t // block
+                crit_w, crit_v = [], []
+                lin_num = np.zeros(d)
+                lin_den = 0.0
+                fq = phi(q64[b, hh, t])
+                for u in range(N):
+                    c = cls[b, hh, i, u // block]
+                    if c == 1:
+                        crit_w.append(float(q64[b, hh, t] @ k64[b, hh, u]) * scale)
+                        crit_v.append(v64[b, hh, u])
+                    elif c == 0:
+                        a = float(fq @ phi(k64[b, hh, u]))
+                        lin_num += a * v64[b, hh, u]
+                        lin_den += a
+                os_t = np.zeros(d)
+                if crit_w:
+                    mx = max(crit_w)
+                    ex = [math.exp(x - mx) for x in crit_w]
+                    tot = sum(ex)
+                    for e_u, v_u in zip(ex, crit_v):
+                        os_t += (e_u / tot) * v_u
+                ol_t = lin_num / lin_den if lin_den > 0 else np.zeros(d)
+                for c_out in range(d):
+                    o[b, hh, t, c_out] = os_t[c_out] + sum(
+                        ol_t[a] * w64[a, c_out] for a in range(d))
+    return o
+
+
+def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
+             fwd=None):
+    """Gradients of sum(O * dO) w.r.t. Q, K, V and W_proj, classes held fixed (R8).
+
+    Sparse branch (standard softmax-attention backward over critical pairs):
+      D_t = dO_t . O_s,t;  P = exp(S - LSE);  dV_u += P_tu dO_t;
+      dP_tu = dO_t . V_u;  dS = P (dP - D);  dQ_t += scale dS_tu K_u;
+      dK_u += scale dS_tu Q_t.
+    Linear branch (O_l = num/den, num = phi(Q) H_i, den = phi(Q) . Z_i):
+      dO_l = dO W^T; dnum = dO_l / den; dden = -(dO_l . O_l) / den;
+      dphi(Q_t) = H_i dnum_t + Z_i dden_t;  dQ_t += dphi(Q_t) * phi'(Q_t);
+      dH_i = sum_t phi(Q_t) dnum_t^T;  dZ_i = sum_t phi(Q_t) dden_t;
+      dh_j = sum_{i: j marginal in row i} dH_i (likewise dz_j);
+      dphi(K_u) = dh_j V_u + dz_j;  dK_u += dphi(K_u) * phi'(K_u);
+      dV_u += dh_j^T phi(K_u).
+    Projection: dW = sum over b, h, t of O_l,t dO_t^T.
+    """
+    B, H, N, d = q.shape
+    T = N // block
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if fwd is None:
+        fwd = forward(q, k, v, w_proj, cls, block, scale)
+    q64, k64, v64, do64 = (np.asarray(a, dtype=np.float64) for a in (q, k, v, d_o))
+    w64 = np.asarray(w_proj, dtype=np.float64)
+    h, z = key_block_summaries(k64, v64, block)
+    dq = np.zeros_like(q64)
+    dk = np.zeros_like(k64)
+    dv = np.zeros_like(v64)
+    dw = np.einsum("bhta,bhtc->ac", fwd["o_l"], do64)
+    do_l = np.einsum("bhtc,ac->bhta", do64, w64)
+    for b in range(B):
+        for hh in range(H):
+            dh = np.zeros((T, d, d))
+            dz = np.zeros((T, d))
+            for i in range(T):
+                t0, t1 = i * block, (i + 1) * block
+                qi = q64[b, hh, t0:t1]
+                doi = do64[b, hh, t0:t1]
+                crit = np.nonzero(cls[b, hh, i] == 1)[0]
+                marg = np.nonzero(cls[b, hh, i] == 0)[0]
+                if crit.size:
+                    keys = _tokens(crit, block)
+                    kc, vc = k64[b, hh, keys], v64[b, hh, keys]
+                    s = (qi @ kc.T) * scale
+                    p = np.exp(s - fwd["lse"][b, hh, t0:t1, None])
+                    D = np.sum(doi * fwd["o_s"][b, hh, t0:t1], axis=1, keepdims=True)
+                    dv[b, hh, keys] += p.T @ doi
+                    dp = doi @ vc.T
+                    ds = p * (dp - D)
+                    dq[b, hh, t0:t1] += scale * (ds @ kc)
+                    dk[b, hh, keys] += scale * (ds.T @ qi)
+                if marg.size:
+                    Hi = h[b, hh, marg].sum(axis=0)
+                    Zi = z[b, hh, marg].sum(axis=0)
+                    dn = fwd["den"][b, hh, t0:t1]
+                    dol = do_l[b, hh, t0:t1]
+                    dnum = dol / dn[:, None]
+                    dden = -np.sum(dol * fwd["o_l"][b, hh, t0:t1], axis=1) / dn
+                    fq = phi(qi)
+                    dfq = dnum @ Hi.T + dden[:, None] * Zi[None, :]
+                    dq[b, hh, t0:t1] += dfq * phi_prime(qi)
+                    dHi = fq.T @ dnum
+                    dZi = fq.T @ dden
+                    dh[marg] += dHi
+                    dz[marg] += dZi
+            for j in range(T):
+                u0, u1 = j * block, (j + 1) * block
+                kj, vj = k64[b, hh, u0:u1], v64[b, hh, u0:u1]
+                dfk = vj @ dh[j].T + dz[j][None, :]
+                dk[b, hh, u0:u1] += dfk * phi_prime(kj)
+                dv[b, hh, u0:u1] += phi(kj) @ dh[j]
+    return {"dq": dq, "dk": dk, "dv": dv, "dw": dw}
+
+
+def sla(q, k, v, w_proj, block: int, k_h: float, k_l: float, scale: float | None = None):
+    """Classification from the inputs followed by the forward."""
+    d = q.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    T = q.shape[2] // block
+    n_h, n_l = block_counts(T, k_h, k_l)
+    logits = pooled_logits(q, k, block, scale)
+    cls = classify(logits, n_h, n_l)
+    out = forward(q, k, v, w_proj, cls, block, scale)
+    out.update(cls=cls, logits=logits)
+    return out

@@ -1,0 +1,295 @@
+"""Pins for the fp64 oracle: each test checks it against something other than
+itself (a library routine, a closed form, a brute force, finite differences
+or an invariant), chosen so that a dropped term, a wrong sign or index, or a
+transposed operand fails at least one of them."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sla_inputs
+
+
+def _rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+# ---------------------------------------------------------------- counts (R3)
+
+@pytest.mark.parametrize("T,k_h,k_l,expect", [
+    (16, 0.25, 0.25, (4, 4)),      # tiny
+    (128, 0.05, 0.10, (7, 12)),    # mid
+    (512, 0.05, 0.10, (26, 51)),   # Wan-shaped
+    (1182, 0.025, 0.10, (30, 118)),
+    (1182, 0.05, 0.10, (60, 118)),
+    (1182, 0.10, 0.10, (119, 118)),
+    (10, 0.0, 0.0, (0, 0)),
+    (10, 1.0, 0.0, (10, 0)),
+    (10, 0.0, 1.0, (0, 10)),
+    (10, 0.1, 0.9, (1, 9)),
+    (7, 0.5, 0.5, (4, 3)),         # n_l clipped to T - n_h
+])
+def test_block_counts(T, k_h, k_l, expect):
+    assert oracle.block_counts(T, k_h, k_l) == expect
+
+
+def test_block_counts_rejects_bad_fractions():
+    with pytest.raises(ValueError):
+        oracle.block_counts(10, 0.6, 0.5)
+    with pytest.raises(ValueError):
+        oracle.block_counts(10, -0.1, 0.5)
+
+
+# ---------------------------------------------------------------- classification
+
+@pytest.mark.parametrize("T", [1, 2, 5, 16, 33])
+@pytest.mark.parametrize("frac", [(0.0, 0.0), (0.25, 0.25), (0.5, 0.5), (1.0, 0.0), (0.1, 0.6)])
+def test_classify_matches_rank_count(T, frac):
+    n_h, n_l = oracle.block_counts(T, *frac)
+    rng = np.random.default_rng(T * 100 + int(frac[0] * 10))
+    # small integer scores force many ties; -0.0 and 0.0 must tie as well
+    rows = rng.integers(-3, 4, size=(6, T)).astype(np.float64)
+    rows[0, ::2] = -0.0
+    got = oracle.classify(rows, n_h, n_l)
+    for r in range(rows.shape[0]):
+        assert got[r].tolist() == oracle.classify_rows_bruteforce(rows[r].tolist(), n_h, n_l)
+        assert (got[r] == 1).sum() == n_h and (got[r] == -1).sum() == n_l
+
+
+def test_classify_ranks_softmax_like_logits():
+    # ranking the row softmax (the pooled probabilities) gives the same classes
+    rows = _rand((20, 64), 1, 2.0)
+    p = np.exp(rows - rows.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    assert np.array_equal(oracle.classify(rows, 5, 9), oracle.classify(p, 5, 9))
+
+
+def test_classify_rejects_nan():
+    with pytest.raises(ValueError):
+        oracle.classify(np.array([[0.0, np.nan]]), 1, 0)
+
+
+def test_pool_is_block_mean():
+    x = _rand((1, 1, 8, 3), 2)
+    got = oracle.pool(x, 4)
+    assert np.allclose(got[0, 0, 0], x[0, 0, :4].sum(0) / 4)
+    assert np.allclose(got[0, 0, 1], x[0, 0, 4:].sum(0) / 4)
+
+
+def test_pooled_logits_closed_form():
+    q, k = _rand((1, 1, 4, 2), 3), _rand((1, 1, 4, 2), 4)
+    s = oracle.pooled_logits(q, k, 2, 0.5)
+    qb = [(q[0, 0, 0] + q[0, 0, 1]) / 2, (q[0, 0, 2] + q[0, 0, 3]) / 2]
+    kb = [(k[0, 0, 0] + k[0, 0, 1]) / 2, (k[0, 0, 2] + k[0, 0, 3]) / 2]
+    for i in range(2):
+        for j in range(2):
+            assert math.isclose(s[0, 0, i, j], 0.5 * float(qb[i] @ kb[j]), rel_tol=1e-12)
+
+
+def test_phi_closed_form():
+    x = np.array([-2.0, -0.5, 0.0, 0.5, 3.0])
+    assert np.allclose(oracle.phi(x), [math.exp(-2), math.exp(-0.5), 1.0, 1.5, 4.0])
+    assert np.allclose(oracle.phi_prime(x), [math.exp(-2), math.exp(-0.5), 1.0, 1.0, 1.0])
+    # elu(x) + 1 from torch's own elu
+    xt = torch.tensor(x)
+    assert np.allclose(oracle.phi(x), (torch.nn.functional.elu(xt) + 1).numpy())
+
+
+# ---------------------------------------------------------------- forward special cases
+
+def _small(B=1, H=2, N=256, d=16, seed=0):
+    g = np.random.default_rng(seed)
+    q = g.standard_normal((B, H, N, d))
+    k = g.standard_normal((B, H, N, d))
+    v = g.standard_normal((B, H, N, d))
+    w = g.standard_normal((d, d)) / math.sqrt(d)
+    return q, k, v, w
+
+
+def _cls_from(q, k, block, k_h, k_l):
+    T = q.shape[2] // block
+    n_h, n_l = oracle.block_counts(T, k_h, k_l)
+    return oracle.classify(oracle.pooled_logits(q, k, block, 1 / math.sqrt(q.shape[-1])), n_h, n_l)
+
+
+def test_all_critical_is_dense_softmax_attention():
+    q, k, v, w = _small(N=256, d=16)
+    out = oracle.sla(q, k, v, w, 32, 1.0, 0.0)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q), torch.tensor(k), torch.tensor(v)).numpy()
+    assert np.all(out["cls"] == 1)
+    np.testing.assert_allclose(out["o"], ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(out["o_s"], ref, rtol=1e-10, atol=1e-12)
+    assert np.all(out["o_l"] == 0)
+
+
+def test_all_marginal_is_dense_linear_attention():
+    q, k, v, w = _small(N=256, d=16, seed=5)
+    out = oracle.sla(q, k, v, w, 32, 0.0, 0.0)
+    assert np.all(out["cls"] == 0)
+    # Katharopoulos-style normalised linear attention with an explicit N x N
+    # kernel matrix, computed with torch (elu + 1 feature map)
+    tq, tk, tv, tw = (torch.tensor(a) for a in (q, k, v, w))
+    fq = torch.nn.functional.elu(tq) + 1
+    fk = torch.nn.functional.elu(tk) + 1
+    A = fq @ fk.transpose(-1, -2)
+    lin = (A @ tv) / A.sum(-1, keepdim=True)
+    np.testing.assert_allclose(out["o_l"], lin.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(out["o"], (lin @ tw).numpy(), rtol=1e-10, atol=1e-12)
+    assert np.all(out["o_s"] == 0)
+
+
+def test_all_negligible_gives_zero():
+    q, k, v, w = _small(N=128, d=8, seed=6)
+    out = oracle.sla(q, k, v, w, 16, 0.0, 1.0)
+    assert np.all(out["cls"] == -1)
+    assert np.all(out["o"] == 0)
+    assert np.all(np.isneginf(out["lse"]))
+
+
+def test_zero_projection_leaves_sparse_output():
+    q, k, v, w = _small(N=256, d=16, seed=7)
+    out = oracle.sla(q, k, v, np.zeros_like(w), 32, 0.25, 0.25)
+    assert np.array_equal(out["o"], out["o_s"])
+    assert np.abs(out["o_l"]).max() > 0
+
+
+def test_projection_is_right_multiplied():
+    # W_proj a cyclic column shift: O - O_s must be O_l with its columns rotated
+    q, k, v, _ = _small(N=256, d=16, seed=8)
+    d = 16
+    w = np.zeros((d, d))
+    for a in range(d):
+        w[a, (a + 3) % d] = 1.0
+    out = oracle.sla(q, k, v, w, 32, 0.25, 0.25)
+    np.testing.assert_allclose(out["o"] - out["o_s"], np.roll(out["o_l"], 3, axis=-1),
+                               rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("block,k_h,k_l", [(64, 0.25, 0.25), (16, 0.25, 0.25),
+                                           (16, 0.1, 0.5), (32, 0.0, 0.25)])
+def test_blockwise_equals_bruteforce(block, k_h, k_l):
+    q, k, v, w = _small(B=1, H=1, N=256, d=8, seed=block)
+    cls = _cls_from(q, k, block, k_h, k_l)
+    fast = oracle.forward(q, k, v, w, cls, block)["o"]
+    slow = oracle.forward_bruteforce(q, k, v, w, cls, block)
+    np.testing.assert_allclose(fast, slow, rtol=1e-10, atol=1e-12)
+
+
+def test_query_block_subset_matches_full():
+    q, k, v, w = _small(N=256, d=16, seed=9)
+    cls = _cls_from(q, k, 32, 0.25, 0.25)
+    full = oracle.forward(q, k, v, w, cls, 32)
+    part = oracle.forward(q, k, v, w, cls, 32, query_blocks=[1, 6])
+    for i in (1, 6):
+        sl = slice(i * 32, (i + 1) * 32)
+        np.testing.assert_array_equal(part["o"][:, :, sl], full["o"][:, :, sl])
+
+
+def test_in_block_token_permutation():
+    q, k, v, w = _small(N=256, d=16, seed=10)
+    block = 32
+    rng = np.random.default_rng(11)
+    perm = np.concatenate([i * block + rng.permutation(block) for i in range(256 // block)])
+    base = oracle.sla(q, k, v, w, block, 0.25, 0.25)
+    # permuting keys/values inside their blocks changes nothing
+    kv = oracle.sla(q, k[:, :, perm], v[:, :, perm], w, block, 0.25, 0.25)
+    assert np.array_equal(kv["cls"], base["cls"])
+    np.testing.assert_allclose(kv["o"], base["o"], rtol=1e-10, atol=1e-12)
+    # permuting queries inside their blocks permutes the output rows
+    qp = oracle.sla(q[:, :, perm], k, v, w, block, 0.25, 0.25)
+    assert np.array_equal(qp["cls"], base["cls"])
+    np.testing.assert_allclose(qp["o"], base["o"][:, :, perm], rtol=1e-10, atol=1e-12)
+
+
+def test_key_shift_invariance_of_sparse_branch():
+    q, k, v, w = _small(N=256, d=16, seed=12)
+    c = np.random.default_rng(13).standard_normal(16) * 3
+    a = oracle.sla(q, k, v, w, 32, 0.25, 0.25)
+    b = oracle.sla(q, k + c, v, w, 32, 0.25, 0.25)
+    assert np.array_equal(a["cls"], b["cls"])
+    np.testing.assert_allclose(a["o_s"], b["o_s"], rtol=1e-9, atol=1e-12)
+
+
+def test_output_linear_in_v_with_mask_fixed():
+    q, k, v, w = _small(N=256, d=16, seed=14)
+    v2 = np.random.default_rng(15).standard_normal(v.shape)
+    cls = _cls_from(q, k, 32, 0.25, 0.25)
+    f = lambda vv: oracle.forward(q, k, vv, w, cls, 32)["o"]
+    np.testing.assert_allclose(f(v + 2.5 * v2), f(v) + 2.5 * f(v2), rtol=1e-9, atol=1e-11)
+
+
+def test_summaries_closed_form():
+    k = _rand((1, 1, 4, 3), 16)
+    v = _rand((1, 1, 4, 3), 17)
+    h, z = oracle.key_block_summaries(k, v, 2)
+    for j in range(2):
+        hh = np.zeros((3, 3))
+        zz = np.zeros(3)
+        for u in (2 * j, 2 * j + 1):
+            fk = [kk + 1 if kk > 0 else math.exp(kk) for kk in k[0, 0, u]]
+            zz += fk
+            for a in range(3):
+                for c in range(3):
+                    hh[a, c] += fk[a] * v[0, 0, u, c]
+        np.testing.assert_allclose(h[0, 0, j], hh, rtol=1e-12)
+        np.testing.assert_allclose(z[0, 0, j], zz, rtol=1e-12)
+
+
+# ---------------------------------------------------------------- backward
+
+def _loss(q, k, v, w, cls, do, block):
+    return float(np.sum(oracle.forward(q, k, v, w, cls, block)["o"] * do))
+
+
+@pytest.mark.parametrize("block,k_h,k_l,d", [(64, 0.25, 0.25, 8), (16, 0.25, 0.25, 8),
+                                             (16, 0.1, 0.3, 4)])
+def test_backward_matches_central_differences(block, k_h, k_l, d):
+    q, k, v, w = _small(B=1, H=1, N=256, d=d, seed=20 + block)
+    do = np.random.default_rng(21).standard_normal(q.shape)
+    cls = _cls_from(q, k, block, k_h, k_l)  # frozen at the unperturbed point
+    assert set(np.unique(cls)) == {-1, 0, 1}
+    g = oracle.backward(q, k, v, w, cls, do, block)
+    rng = np.random.default_rng(22)
+    eps = 1e-6
+    for name, arr, grad in (("q", q, g["dq"]), ("k", k, g["dk"]),
+                            ("v", v, g["dv"]), ("w", w, g["dw"])):
+        for _ in range(12):
+            idx = tuple(rng.integers(0, s) for s in arr.shape)
+            xp, xm = arr.copy(), arr.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = {"q": q, "k": k, "v": v, "w": w}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = xp, xm
+            fd = (_loss(args_p["q"], args_p["k"], args_p["v"], args_p["w"], cls, do, block)
+                  - _loss(args_m["q"], args_m["k"], args_m["v"], args_m["w"], cls, do, block)) / (2 * eps)
+            assert math.isclose(fd, grad[idx], rel_tol=2e-6, abs_tol=2e-8), (name, idx, fd, grad[idx])
+
+
+def test_sparse_key_gradient_sums_to_zero():
+    # with no marginal pairs only the softmax branch carries gradient, and its
+    # invariance under K -> K + c makes the key gradients sum to zero
+    q, k, v, w = _small(N=256, d=16, seed=30)
+    do = np.random.default_rng(31).standard_normal(q.shape)
+    cls = _cls_from(q, k, 32, 0.5, 0.5)
+    assert not np.any(cls == 0)
+    g = oracle.backward(q, k, v, w, cls, do, 32)
+    np.testing.assert_allclose(g["dk"].sum(axis=2), 0.0, atol=1e-10)
+    assert np.all(g["dw"] == 0)
+
+
+def test_workload_generators_shapes_and_stats():
+    t = sla_inputs.make("tiny")
+    assert t.q.shape == (1, 2, 1024, 64) and t.w_proj.shape == (64, 64)
+    assert np.array_equal(sla_inputs.bf16_round(t.q), t.q)
+    g = sla_inputs.make_grid((2, 8, 8), H=2, name="g")
+    assert g.N == 128 and g.n_valid == 128
+    f = sla_inputs.grid_feature((2, 3, 4))
+    np.testing.assert_allclose((f ** 2).sum(1), 64.0)
+    # zero padding past the grid
+    p = sla_inputs.make_grid((1, 3, 7), H=1, name="p")
+    assert p.N == 64 and p.n_valid == 21 and np.all(p.q[:, :, 21:] == 0)
