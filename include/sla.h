@@ -1,0 +1,165 @@
+/*
+ * sla.h - C ABI of the SLA (Sparse-Linear Attention) hot path on B200 (sm_100a).
+ *
+ * What is computed.  "SLA: Beyond Sparsity in Diffusion Transformers via
+ * Fine-Tunable Sparse-Linear Attention" (arXiv 2509.24006), abstract and the
+ * technical-framework steps of its paper card: attention weights are sorted
+ * into critical, marginal and negligible groups; critical pairs get exact
+ * O(N^2) softmax attention, marginal pairs get O(N) linear attention, and
+ * negligible pairs are skipped, in a forward and a backward pass.  The pages
+ * leave the classifier, feature map, combination and backward open; this
+ * library takes these readings:
+ *   - classes are per (query block i, key block j) of `block` (64) tokens:
+ *     pooled logits s_ij = mean(Q_i) . mean(K_j) * scale; per row the n_crit
+ *     largest (ties: lower j first) are critical, the n_negl smallest are
+ *     negligible, the rest marginal; n_crit = ceil(k_h*T - 1e-9),
+ *     n_negl = min(floor(k_l*T + 1e-9), T - n_crit), T = N / block;
+ *   - critical pairs: softmax attention with scale 1/sqrt(d) (or
+ *     softmax_scale) over all tokens of the row's critical key blocks;
+ *   - marginal pairs: phi(x) = elu(x) + 1; per key block
+ *     h_j = phi(K_j)^T V_j and z_j = sum phi(K_j); per query block
+ *     H_i = sum_{j marginal} h_j, Z_i likewise;
+ *     O_l = phi(Q) H_i / (phi(Q) . Z_i)  (0 if row i has no marginal block);
+ *   - O = O_s + O_l W_proj, W_proj one d x d matrix shared by all heads;
+ *   - the backward treats the classes as constants.
+ *
+ * Conventions (all entry points).
+ *   - Every data pointer is a DEVICE pointer, allocated and owned by the
+ *     caller; the library never allocates or frees memory and keeps no
+ *     state between calls (except the per-process cached TMA encoder entry
+ *     point).  Sizes of caller buffers come from sla_query_sizes().
+ *   - Q, K, V, O, dO: bf16, contiguous [B, H, N, d], 16-byte aligned.
+ *     W_proj: bf16 row-major [d, d].  dQ, dK, dV, dW_proj: fp32.
+ *   - Supported: block == 64, d in {64, 128}, N % 64 == 0, N >= 64,
+ *     1 <= B*H, T = N/64 <= 4096, 0 <= k_h, 0 <= k_l, k_h + k_l <= 1.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     is asynchronous on it.  Argument errors are returned before anything is
+ *     launched.  A failed launch returns SLA_ERR_CUDA.  Errors found on the
+ *     device (a wait that timed out, an index out of range) are recorded in
+ *     an error word inside the workspace and reported by sla_check().
+ *   - Calls that share a workspace must not overlap on the device.
+ *   - Nothing aborts the process and no C++ exception crosses this ABI.
+ */
+#ifndef SLA_H_
+#define SLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SLA_API __attribute__((visibility("default")))
+#else
+#define SLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SLA_OK = 0,
+  SLA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or fraction */
+  SLA_ERR_UNSUPPORTED = 2, /* valid but not implemented (block != 64, d not 64/128) */
+  SLA_ERR_WORKSPACE = 3,   /* workspace or buffer smaller than sla_query_sizes() */
+  SLA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  SLA_ERR_TIMEOUT = 5,     /* a device-side wait gave up (reported by sla_check) */
+  SLA_ERR_DEVICE = 6       /* a device-side invariant failed (reported by sla_check) */
+} sla_status;
+
+/* Problem shape.  softmax_scale <= 0 selects 1/sqrt(d). */
+typedef struct {
+  int B, H, N, d, block;
+  double k_h, k_l;
+  float softmax_scale;
+} sla_shape;
+
+/* Classification output (written by sla_classify*, read by forward/backward;
+ * a mask may be reused across calls, e.g. across denoising steps).
+ *   cls           int8  [B,H,T,T]   +1 critical, 0 marginal, -1 negligible
+ *   crit_idx      int32 [B,H,T,n_crit]  critical key blocks, ascending
+ *   marg_bits     uint32[B,H,T,ceil(T/32)]  bit j%32 of word j/32: j marginal
+ *   crit_col_ptr  int32 [B,H,T+1]   CSR by key block (offsets per (b,h))
+ *   crit_col_idx  int32 [B,H,T*n_crit]  query blocks with j critical, ascending
+ *   pooled_logits fp32  [B,H,T,T]   optional (NULL: not written / not read) */
+typedef struct {
+  int8_t* cls;
+  int32_t* crit_idx;
+  uint32_t* marg_bits;
+  int32_t* crit_col_ptr;
+  int32_t* crit_col_idx;
+  float* pooled_logits;
+} sla_mask;
+
+/* State saved by sla_forward for sla_backward.
+ *   lse   fp32 [B,H,N]      log-sum-exp of the critical scores (-inf if none)
+ *   o_s   fp32 [B,H,N,d]    sparse-branch output
+ *   den   fp32 [B,H,N]      phi(Q).Z_i (0 if the row has no marginal block)
+ *   h_agg bf16 [B,H,T,d,d]  H_i per query block
+ *   z_agg fp32 [B,H,T,d]    Z_i per query block */
+typedef struct {
+  float* lse;
+  float* o_s;
+  float* den;
+  void* h_agg;
+  float* z_agg;
+} sla_saved;
+
+/* Sizes in bytes of every caller buffer for a shape. */
+typedef struct {
+  int T, n_crit, n_negl, n_marg;
+  size_t cls_bytes, crit_idx_bytes, marg_bits_bytes, crit_col_ptr_bytes, crit_col_idx_bytes,
+      pooled_logits_bytes;
+  size_t lse_bytes, o_s_bytes, den_bytes, h_agg_bytes, z_agg_bytes;
+  size_t workspace_bytes; /* one workspace serves classify, forward and backward */
+} sla_sizes;
+
+/* Fill *out for *shape.  Host only; no CUDA call. */
+SLA_API sla_status sla_query_sizes(const sla_shape* shape, sla_sizes* out);
+
+/* Pool Q and K per block, score the pooled rows and classify every
+ * (query block, key block) pair into *mask.  q, k: bf16 [B,H,N,d]. */
+SLA_API sla_status sla_classify(const sla_shape* shape, const void* q, const void* k,
+                        const sla_mask* mask, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* Classify from caller-given fp32 scores [B,H,T,T] (any values but NaN);
+ * same ranking rule and outputs as sla_classify, pooled_logits untouched.
+ * Lets a test feed identical scores to this library and to a reference. */
+SLA_API sla_status sla_classify_from_scores(const sla_shape* shape, const float* logits,
+                                    const sla_mask* mask, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/* Forward with a given mask: writes o (bf16 [B,H,N,d]) and *saved. */
+SLA_API sla_status sla_forward(const sla_shape* shape, const void* q, const void* k, const void* v,
+                       const void* w_proj, const sla_mask* mask, void* o,
+                       const sla_saved* saved, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/* Backward of sum(O * dO) with the mask held fixed.  Needs the *saved state
+ * of the forward on the same inputs and mask.  Writes dq, dk, dv (fp32
+ * [B,H,N,d]) and dw_proj (fp32 [d,d], summed over B, H, N; overwritten). */
+SLA_API sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, const void* v,
+                        const void* w_proj, const sla_mask* mask, const sla_saved* saved,
+                        const void* d_o, float* dq, float* dk, float* dv, float* dw_proj,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Zero the workspace's device error word (asynchronously on `stream`).  Call
+ * once on a new workspace before its first use; sla_check() clears it
+ * afterwards. */
+SLA_API sla_status sla_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronize `stream`, then return and clear the workspace's device error
+ * word (SLA_OK if no device-side error was recorded). */
+SLA_API sla_status sla_check(void* workspace, void* stream);
+
+/* Static description of a status code. */
+SLA_API const char* sla_strerror(sla_status status);
+
+/* Library version, "major.minor.patch". */
+SLA_API const char* sla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLA_H_ */

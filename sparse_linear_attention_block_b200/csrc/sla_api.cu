@@ -1,0 +1,316 @@
+// C-ABI entry points of the SLA hot-path library (declared in sla.h):
+// argument validation, workspace layout, TMA descriptor encoding and the
+// launch sequence of each call.  No allocation happens here.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "sla.h"
+#include "sla_internal.h"
+
+namespace sla {
+
+WorkspaceLayout workspace_layout(int BH, int N, int d) {
+  const int T = N / kBlock, Tp = pad128(T);
+  WorkspaceLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, kAlign);
+    return at;
+  };
+  const size_t bh = size_t(BH);
+  L.err = take(256);
+  L.qbar = take(bh * T * d * 4);
+  L.kbar = take(bh * T * d * 4);
+  L.summ = take(bh * T * d * d * 2);
+  L.zsum = take(bh * T * d * 4);
+  L.dh = take(bh * T * d * d * 2);
+  L.dz = take(bh * T * d * 4);
+  L.mmat = take(bh * Tp * Tp * 2);
+  L.mmat_t = take(bh * Tp * Tp * 2);
+  L.dvec = take(bh * N * 4);
+  L.dnum = take(bh * N * d * 4);
+  L.dden = take(bh * N * 4);
+  L.total = off;
+  return L;
+}
+
+// ------------------------------------------------------------------ TMA encoding
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                  uint64_t batch, uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_bhnd(CUtensorMap* map, const void* base, int BH, int N, int d, int box_rows) {
+  return make_tmap_3d(map, base, uint64_t(d), uint64_t(N), uint64_t(BH), 64, uint32_t(box_rows));
+}
+
+}  // namespace sla
+
+using namespace sla;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void counts(int T, double k_h, double k_l, int* n_h, int* n_l) {
+  long h = static_cast<long>(std::ceil(k_h * T - 1e-9));
+  if (h < 0) h = 0;
+  if (h > T) h = T;
+  long l = static_cast<long>(std::floor(k_l * T + 1e-9));
+  if (l > T - h) l = T - h;
+  if (l < 0) l = 0;
+  *n_h = int(h);
+  *n_l = int(l);
+}
+
+sla_status check_shape(const sla_shape* s, Problem* p) {
+  if (!s) return SLA_ERR_INVALID_ARG;
+  if (s->B < 1 || s->H < 1 || s->N < 1 || s->d < 1 || s->block < 1) return SLA_ERR_INVALID_ARG;
+  if (!(s->k_h >= 0.0) || !(s->k_l >= 0.0) || s->k_h + s->k_l > 1.0 + 1e-12)
+    return SLA_ERR_INVALID_ARG;
+  if (std::isnan(s->softmax_scale) || std::isinf(s->softmax_scale)) return SLA_ERR_INVALID_ARG;
+  if (s->N % s->block != 0) return SLA_ERR_INVALID_ARG;
+  if (s->block != kBlock) return SLA_ERR_UNSUPPORTED;
+  if (s->d != 64 && s->d != 128) return SLA_ERR_UNSUPPORTED;
+  const long long bh = (long long)s->B * s->H;
+  if (bh > 65535) return SLA_ERR_UNSUPPORTED;
+  const int T = s->N / kBlock;
+  if (T > kMaxT) return SLA_ERR_UNSUPPORTED;
+  if (p) {
+    p->B = s->B;
+    p->H = s->H;
+    p->BH = int(bh);
+    p->N = s->N;
+    p->d = s->d;
+    p->T = T;
+    p->Tp = pad128(T);
+    counts(T, s->k_h, s->k_l, &p->n_crit, &p->n_negl);
+    p->scale = s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / std::sqrt(float(s->d));
+    p->scale_log2 = p->scale * 1.4426950408889634f;
+  }
+  return SLA_OK;
+}
+
+sla_status fill_sizes(const Problem& p, sla_sizes* o) {
+  const size_t bh = size_t(p.BH), T = size_t(p.T), N = size_t(p.N), d = size_t(p.d);
+  std::memset(o, 0, sizeof(*o));
+  o->T = p.T;
+  o->n_crit = p.n_crit;
+  o->n_negl = p.n_negl;
+  o->n_marg = p.T - p.n_crit - p.n_negl;
+  o->cls_bytes = bh * T * T;
+  o->crit_idx_bytes = bh * T * size_t(p.n_crit) * 4;
+  o->marg_bits_bytes = bh * T * ((T + 31) / 32) * 4;
+  o->crit_col_ptr_bytes = bh * (T + 1) * 4;
+  o->crit_col_idx_bytes = bh * T * size_t(p.n_crit) * 4;
+  o->pooled_logits_bytes = bh * T * T * 4;
+  o->lse_bytes = bh * N * 4;
+  o->o_s_bytes = bh * N * d * 4;
+  o->den_bytes = bh * N * 4;
+  o->h_agg_bytes = bh * T * d * d * 2;
+  o->z_agg_bytes = bh * T * d * 4;
+  o->workspace_bytes = workspace_layout(p.BH, p.N, p.d).total;
+  return SLA_OK;
+}
+
+sla_status check_mask(const Problem& p, const sla_mask* m, bool need_csr) {
+  if (!m) return SLA_ERR_INVALID_ARG;
+  if (!m->cls || !m->marg_bits) return SLA_ERR_INVALID_ARG;
+  if (p.n_crit > 0 && !m->crit_idx) return SLA_ERR_INVALID_ARG;
+  if (need_csr && (!m->crit_col_ptr || (p.n_crit > 0 && !m->crit_col_idx)))
+    return SLA_ERR_INVALID_ARG;
+  if (!aligned16(m->marg_bits) || (m->crit_idx && !aligned16(m->crit_idx)))
+    return SLA_ERR_INVALID_ARG;
+  return SLA_OK;
+}
+
+sla_status check_ws(const Problem& p, void* ws, size_t ws_bytes, WorkspaceLayout* L) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return SLA_ERR_INVALID_ARG;
+  *L = workspace_layout(p.BH, p.N, p.d);
+  if (ws_bytes < L->total) return SLA_ERR_WORKSPACE;
+  return SLA_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+#define SLA_LAUNCH(expr)                       \
+  do {                                         \
+    if ((expr) != cudaSuccess) return SLA_ERR_CUDA; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+sla_status sla_query_sizes(const sla_shape* shape, sla_sizes* out) {
+  if (!out) return SLA_ERR_INVALID_ARG;
+  Problem p;
+  sla_status st = check_shape(shape, &p);
+  if (st != SLA_OK) return st;
+  return fill_sizes(p, out);
+}
+
+static sla_status classify_impl(const sla_shape* shape, const void* q, const void* k,
+                                const float* logits_in, const sla_mask* mask, void* ws,
+                                size_t ws_bytes, void* stream) {
+  Problem p;
+  sla_status st = check_shape(shape, &p);
+  if (st != SLA_OK) return st;
+  if ((st = check_mask(p, mask, true)) != SLA_OK) return st;
+  WorkspaceLayout L;
+  if ((st = check_ws(p, ws, ws_bytes, &L)) != SLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float* qbar = at<float>(ws, L.qbar);
+  const float* kbar = at<float>(ws, L.kbar);
+  if (!logits_in) {
+    if (!q || !k || !aligned16(q) || !aligned16(k)) return SLA_ERR_INVALID_ARG;
+    SLA_LAUNCH(launch_pool(p, q, k, at<float>(ws, L.qbar), at<float>(ws, L.kbar), s));
+  }
+  SLA_LAUNCH(launch_classify(p, qbar, kbar, logits_in, logits_in ? nullptr : mask->pooled_logits,
+                             mask->cls, mask->crit_idx, mask->marg_bits, s));
+  SLA_LAUNCH(launch_crit_csr(p, mask->cls, mask->crit_col_ptr, mask->crit_col_idx, s));
+  return SLA_OK;
+}
+
+sla_status sla_classify(const sla_shape* shape, const void* q, const void* k,
+                        const sla_mask* mask, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  if (!q || !k) return SLA_ERR_INVALID_ARG;
+  return classify_impl(shape, q, k, nullptr, mask, workspace, workspace_bytes, stream);
+}
+
+sla_status sla_classify_from_scores(const sla_shape* shape, const float* logits,
+                                    const sla_mask* mask, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (!logits || !aligned16(logits)) return SLA_ERR_INVALID_ARG;
+  return classify_impl(shape, nullptr, nullptr, logits, mask, workspace, workspace_bytes,
+                       stream);
+}
+
+static sla_status check_saved(const Problem& p, const sla_saved* sv) {
+  if (!sv || !sv->lse || !sv->o_s || !sv->den || !sv->h_agg || !sv->z_agg)
+    return SLA_ERR_INVALID_ARG;
+  if (!aligned16(sv->o_s) || !aligned16(sv->h_agg) || !aligned16(sv->z_agg) ||
+      !aligned16(sv->lse) || !aligned16(sv->den))
+    return SLA_ERR_INVALID_ARG;
+  (void)p;
+  return SLA_OK;
+}
+
+sla_status sla_forward(const sla_shape* shape, const void* q, const void* k, const void* v,
+                       const void* w_proj, const sla_mask* mask, void* o,
+                       const sla_saved* saved, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  Problem p;
+  sla_status st = check_shape(shape, &p);
+  if (st != SLA_OK) return st;
+  if (!q || !k || !v || !w_proj || !o) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(w_proj) || !aligned16(o))
+    return SLA_ERR_INVALID_ARG;
+  if ((st = check_mask(p, mask, false)) != SLA_OK) return st;
+  if ((st = check_saved(p, saved)) != SLA_OK) return st;
+  WorkspaceLayout L;
+  if ((st = check_ws(p, workspace, workspace_bytes, &L)) != SLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* err = at<int>(workspace, L.err);
+  auto* summ = at<__nv_bfloat16>(workspace, L.summ);
+  auto* mmat = at<__nv_bfloat16>(workspace, L.mmat);
+  float* zsum = at<float>(workspace, L.zsum);
+  auto* h_agg = static_cast<__nv_bfloat16*>(saved->h_agg);
+  // linear branch: summaries, marginal aggregation
+  SLA_LAUNCH(launch_summaries(p, k, v, summ, zsum, err, s));
+  SLA_LAUNCH(launch_expand_marginal(p, mask->marg_bits, mmat, nullptr, s));
+  SLA_LAUNCH(launch_aggregate(p, mmat, summ, h_agg, err, s));
+  SLA_LAUNCH(launch_aggregate_z(p, mask->marg_bits, zsum, saved->z_agg, false, s));
+  // sparse branch, then the combination
+  SLA_LAUNCH(launch_fwd_sparse(p, q, k, v, mask->crit_idx, saved->o_s, saved->lse, err, s));
+  SLA_LAUNCH(launch_fwd_linear(p, q, h_agg, saved->z_agg, w_proj, saved->o_s, o, saved->den,
+                               err, s));
+  return SLA_OK;
+}
+
+sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, const void* v,
+                        const void* w_proj, const sla_mask* mask, const sla_saved* saved,
+                        const void* d_o, float* dq, float* dk, float* dv, float* dw_proj,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  Problem p;
+  sla_status st = check_shape(shape, &p);
+  if (st != SLA_OK) return st;
+  (void)q; (void)k; (void)v; (void)w_proj; (void)mask; (void)saved; (void)d_o;
+  (void)dq; (void)dk; (void)dv; (void)dw_proj; (void)workspace; (void)workspace_bytes;
+  (void)stream;
+  return SLA_ERR_UNSUPPORTED;
+}
+
+sla_status sla_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace || workspace_bytes < 256) return SLA_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(workspace, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SLA_ERR_CUDA;
+  return SLA_OK;
+}
+
+sla_status sla_check(void* workspace, void* stream) {
+  if (!workspace) return SLA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SLA_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SLA_ERR_CUDA;
+  if (word != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return SLA_ERR_CUDA;
+    return static_cast<sla_status>(word);
+  }
+  return SLA_OK;
+}
+
+const char* sla_strerror(sla_status status) {
+  switch (status) {
+    case SLA_OK: return "ok";
+    case SLA_ERR_INVALID_ARG: return "invalid argument";
+    case SLA_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case SLA_ERR_WORKSPACE: return "workspace or buffer too small";
+    case SLA_ERR_CUDA: return "CUDA runtime error";
+    case SLA_ERR_TIMEOUT: return "device-side wait timed out";
+    case SLA_ERR_DEVICE: return "device-side invariant failed";
+  }
+  return "unknown status";
+}
+
+const char* sla_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,81 @@
+// Internal declarations shared by the C-ABI layer and the kernels: the
+// workspace layout and the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "sla.h"
+
+namespace sla {
+
+constexpr int kBlock = 64;       // tokens per block (the only supported block size)
+constexpr int kMaxT = 4096;      // blocks per sequence
+constexpr size_t kAlign = 1024;  // alignment of every workspace region
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Blocks padded to the aggregation GEMM's 128-row tile.
+inline int pad128(int T) { return (T + 127) / 128 * 128; }
+
+// Byte offsets of the regions inside the caller's workspace.
+struct WorkspaceLayout {
+  size_t err;        // int32 device error word (+ padding)
+  size_t qbar;       // fp32 [BH,T,d]   pooled Q
+  size_t kbar;       // fp32 [BH,T,d]   pooled K
+  size_t summ;       // bf16 [BH,T,d*d] h_j (forward) / dH_i contributions A_i (backward)
+  size_t zsum;       // fp32 [BH,T,d]   z_j (forward) / a_i (backward)
+  size_t dh;         // bf16 [BH,T,d*d] dh_j (backward)
+  size_t dz;         // fp32 [BH,T,d]   dz_j (backward)
+  size_t mmat;       // bf16 [BH,Tp,Tp] marginal 0/1 matrix, rows = query blocks
+  size_t mmat_t;     // bf16 [BH,Tp,Tp] its transpose
+  size_t dvec;       // fp32 [BH,N]     D_t = dO_t . O_s,t
+  size_t dnum;       // fp32 [BH,N,d]   dL/d(numerator)
+  size_t dden;       // fp32 [BH,N]     dL/d(denominator)
+  size_t total;
+};
+
+WorkspaceLayout workspace_layout(int BH, int N, int d);
+
+// Validated problem description handed to the launchers.
+struct Problem {
+  int B, H, BH, N, d, T, Tp, n_crit, n_negl;
+  float scale;        // softmax scale
+  float scale_log2;   // scale * log2(e)
+};
+
+// ---- launchers (return cudaGetLastError() of their launches)
+cudaError_t launch_pool(const Problem& p, const void* q, const void* k, float* qbar,
+                        float* kbar, cudaStream_t s);
+cudaError_t launch_classify(const Problem& p, const float* qbar, const float* kbar,
+                            const float* logits_in, float* logits_out, int8_t* cls,
+                            int32_t* crit_idx, uint32_t* marg_bits, cudaStream_t s);
+cudaError_t launch_crit_csr(const Problem& p, const int8_t* cls, int32_t* col_ptr,
+                            int32_t* col_idx, cudaStream_t s);
+cudaError_t launch_expand_marginal(const Problem& p, const uint32_t* marg_bits,
+                                   __nv_bfloat16* mmat, __nv_bfloat16* mmat_t, cudaStream_t s);
+cudaError_t launch_summaries(const Problem& p, const void* k, const void* v,
+                             __nv_bfloat16* summ, float* zsum, int* err, cudaStream_t s);
+cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
+                             const __nv_bfloat16* summ, __nv_bfloat16* out, int* err,
+                             cudaStream_t s);
+cudaError_t launch_aggregate_z(const Problem& p, const uint32_t* marg_bits, const float* z,
+                               float* zout, bool transpose, cudaStream_t s);
+cudaError_t launch_fwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
+                              const int32_t* crit_idx, float* o_s, float* lse, int* err,
+                              cudaStream_t s);
+cudaError_t launch_fwd_linear(const Problem& p, const void* q, const __nv_bfloat16* h_agg,
+                              const float* z_agg, const void* w_proj, const float* o_s,
+                              void* o, float* den, int* err, cudaStream_t s);
+
+// TMA descriptor for a bf16 [BH, N, d] tensor viewed as 3D {d, N, BH} with a
+// box of {64, rows, 1} and 128-byte swizzle.  Returns false on failure.
+bool make_tmap_bhnd(CUtensorMap* map, const void* base, int BH, int N, int d, int box_rows);
+// TMA descriptor for a bf16 3D tensor {inner, rows, batch} (row pitch = inner).
+bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                  uint64_t batch, uint32_t box_inner, uint32_t box_rows);
+
+}  // namespace sla

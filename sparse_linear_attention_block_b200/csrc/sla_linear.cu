@@ -1,0 +1,480 @@
+// Linear-attention branch of SLA for marginal pairs.
+//
+// SLA (arXiv 2509.24006), abstract / framework step 3: marginal attention
+// weights get O(N) linear attention.  Reading used here: feature map
+// phi = elu + 1, per key block h_j = phi(K_j)^T V_j and z_j = sum phi(K_j),
+// per query block H_i = sum of h_j over its marginal key blocks (Z_i alike),
+// O_l = phi(Q) H_i / (phi(Q) . Z_i), and O = O_s + O_l W_proj.
+//
+// Kernels:
+//   summaries_kernel   h_j (tcgen05, bf16 out) and z_j (fp32)      HBM-bound
+//   agg_gemm_kernel    H = M_marg * h as a dense GEMM per head      tensor/HBM
+//   agg_z_kernel       Z_i = sum of z_j over marginal j            small
+//   fwd_linear_kernel  O = O_s + (phi(Q) H_i / den) W_proj         HBM-bound
+#include <cuda_bf16.h>
+
+#include "sla_internal.h"
+#include "sla_ptx.cuh"
+
+namespace sla {
+namespace {
+
+__device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+
+// ------------------------------------------------------------------ summaries
+// One CTA per (key block j, head); 128 threads.  phi(K_j)^T (M = feature a,
+// K = token) and V_j (N = c, K = token) are written MN-major into swizzled
+// shared memory and multiplied by one thread with tcgen05 (M=128, N=D,
+// K=64); for D = 64 the M dimension is zero-padded to 128.
+template <int D>
+__global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __restrict__ k,
+                                                        const __nv_bfloat16* __restrict__ v,
+                                                        __nv_bfloat16* __restrict__ summ,
+                                                        float* __restrict__ zsum, int N, int T,
+                                                        int* err) {
+  constexpr int kChunks = D / 8;
+  constexpr int kGroups = 128 / kChunks;
+  constexpr int kRowsPer = kBlock / kGroups;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sPhiK = base;             // 2 chunks x 64 rows x 128 B = 16 KB (M padded to 128)
+  uint8_t* sV = base + 16384;        // D/64 chunks x 8 KB
+  float* zred = reinterpret_cast<float*>(sV + (D / 64) * 8192);  // [kGroups][D]
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tmem_base;
+  const int j = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  const int warp = t / 32;
+  if (warp == 0) tmem_alloc(&tmem_base, 128);
+  if (t == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  if (D == 64) {  // zero the padding chunk (features 64..127)
+    uint4 z = make_uint4(0, 0, 0, 0);
+    for (int e = t; e < 8192 / 16; e += 128) reinterpret_cast<uint4*>(sPhiK + 8192)[e] = z;
+  }
+  const int c8 = t % kChunks, g = t / kChunks;
+  const size_t off = (size_t(bh) * N + size_t(j) * kBlock) * D;
+  float zacc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+  for (int i = 0; i < kRowsPer; ++i) {
+    const int row = g + i * kGroups;
+    const uint4 uk = *reinterpret_cast<const uint4*>(k + off + size_t(row) * D + c8 * 8);
+    const uint4 uv = *reinterpret_cast<const uint4*>(v + off + size_t(row) * D + c8 * 8);
+    const uint32_t w[4] = {uk.x, uk.y, uk.z, uk.w};
+    uint32_t pw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a = phi_f(bf16_lo(w[e])), b = phi_f(bf16_hi(w[e]));
+      zacc[2 * e] += a;
+      zacc[2 * e + 1] += b;
+      pw[e] = pack_bf16(a, b);
+    }
+    st_sw128_unit(sPhiK, 64, row, c8 * 8, make_uint4(pw[0], pw[1], pw[2], pw[3]));
+    st_sw128_unit(sV, 64, row, c8 * 8, uv);
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) zred[g * D + c8 * 8 + e] = zacc[e];
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  if (t == 0) {
+    constexpr uint32_t idesc = idesc_bf16(128, D, 1, 1);
+    const uint32_t a0 = smem_u32(sPhiK), b0 = smem_u32(sV);
+#pragma unroll
+    for (int ks = 0; ks < kBlock / 16; ++ks)
+      mma_ss(tmem, desc_mnmajor(a0, 64, ks), desc_mnmajor(b0, 64, ks), idesc, ks > 0);
+    mma_commit(&bar);
+  }
+  // z_j while the MMA runs
+  if (t < D) {
+    float s = 0.f;
+#pragma unroll
+    for (int gg = 0; gg < kGroups; ++gg) s += zred[gg * D + t];
+    zsum[(size_t(bh) * T + j) * D + t] = s;
+  }
+  const bool ok = mbar_wait(&bar, 0, err, nullptr);
+  tc_fence_after();
+  if (ok && warp * 32 < D) {
+    const int a = warp * 32 + lane_id();
+    __nv_bfloat16* dst = summ + ((size_t(bh) * T + j) * D + a) * D;
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      float vals[32];
+      tmem_ld32(tmem_addr(tmem, warp * 32, c0), vals);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint4 o;
+        o.x = pack_bf16(vals[q4 * 8 + 0], vals[q4 * 8 + 1]);
+        o.y = pack_bf16(vals[q4 * 8 + 2], vals[q4 * 8 + 3]);
+        o.z = pack_bf16(vals[q4 * 8 + 4], vals[q4 * 8 + 5]);
+        o.w = pack_bf16(vals[q4 * 8 + 6], vals[q4 * 8 + 7]);
+        *reinterpret_cast<uint4*>(dst + c0 + q4 * 8) = o;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_free(tmem, 128);
+}
+
+// ------------------------------------------------------------------ aggregation GEMM
+// C[bh][i][n] = sum_k A[bh][i][k] * B[bh][k][n] with A the bf16 0/1 marginal
+// matrix [Tp x Tp] (K-major) and B the per-block summaries [T x NN]
+// (MN-major), C bf16 [T x NN].  Tile 128 x 128 x 64, 3-stage TMA ring,
+// warp 0 = TMA producer, warp 1 = MMA issuer, all 4 warps = epilogue.
+constexpr int kAggBN = 128, kAggBK = 64, kAggStages = 3;
+constexpr int kAggStageBytes = 128 * kAggBK * 2 + kAggBK * kAggBN * 2;  // 32 KB
+
+__global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
+                                                       const __grid_constant__ CUtensorMap tm_b,
+                                                       __nv_bfloat16* __restrict__ out, int T,
+                                                       int Tp, int NN, int* err) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ uint64_t full[kAggStages], empty[kAggStages], acc_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  const int mt = blockIdx.x, nt = blockIdx.y, bh = blockIdx.z;
+  const int warp = threadIdx.x / 32;
+  const int nk = Tp / kAggBK;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kAggStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&acc_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(&tmem_base, 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (warp == 0 && lane_id() == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+    for (int kt = 0; kt < nk; ++kt) {
+      const int s = kt % kAggStages;
+      if (kt >= kAggStages &&
+          !mbar_wait(&empty[s], ((kt / kAggStages) + 1) & 1, err, &abort_flag))
+        break;
+      uint8_t* sa = base + s * kAggStageBytes;
+      uint8_t* sb = sa + 128 * kAggBK * 2;
+      mbar_arrive_expect_tx(&full[s], kAggStageBytes);
+      tma_load_3d(sa, &full[s], &tm_a, kt * kAggBK, mt * 128, bh);
+      tma_load_3d(sb, &full[s], &tm_b, nt * kAggBN, kt * kAggBK, bh);
+      tma_load_3d(sb + kAggBK * 128, &full[s], &tm_b, nt * kAggBN + 64, kt * kAggBK, bh);
+    }
+  } else if (warp == 1 && lane_id() == 0) {
+    constexpr uint32_t idesc = idesc_bf16(128, kAggBN, 0, 1);
+    for (int kt = 0; kt < nk; ++kt) {
+      const int s = kt % kAggStages;
+      if (!mbar_wait(&full[s], (kt / kAggStages) & 1, err, &abort_flag)) break;
+      tc_fence_after();
+      const uint32_t sa = smem_u32(base + s * kAggStageBytes);
+      const uint32_t sb = sa + 128 * kAggBK * 2;
+#pragma unroll
+      for (int ks = 0; ks < kAggBK / 16; ++ks)
+        mma_ss(tmem, desc_kmajor(sa, 128, ks), desc_mnmajor(sb, kAggBK, ks), idesc,
+               (kt | ks) != 0);
+      mma_commit(&empty[s]);
+    }
+    mma_commit(&acc_bar);
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(&acc_bar, 0, err, &abort_flag);
+  tc_fence_after();
+  const int i = mt * 128 + warp * 32 + lane_id();
+  if (ok) {
+    __nv_bfloat16* dst = out + (size_t(bh) * T + i) * NN + size_t(nt) * kAggBN;
+#pragma unroll 1
+    for (int c0 = 0; c0 < kAggBN; c0 += 32) {
+      float vals[32];
+      tmem_ld32(tmem_addr(tmem, warp * 32, c0), vals);
+      tmem_ld_wait();
+      if (i < T) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint4 o;
+          o.x = pack_bf16(vals[q4 * 8 + 0], vals[q4 * 8 + 1]);
+          o.y = pack_bf16(vals[q4 * 8 + 2], vals[q4 * 8 + 3]);
+          o.z = pack_bf16(vals[q4 * 8 + 4], vals[q4 * 8 + 5]);
+          o.w = pack_bf16(vals[q4 * 8 + 6], vals[q4 * 8 + 7]);
+          *reinterpret_cast<uint4*>(dst + c0 + q4 * 8) = o;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_free(tmem, 128);
+}
+
+// ------------------------------------------------------------------ Z aggregation
+// Forward: Z_i = sum over j marginal in row i of z_j.
+// Transposed (backward): dz_j = sum over i with j marginal in row i of a_i.
+__global__ void agg_z_kernel(const uint32_t* __restrict__ marg_bits, const float* __restrict__ z,
+                             float* __restrict__ zout, int T, int D, int transpose) {
+  const int r = blockIdx.x, bh = blockIdx.y, a = threadIdx.x;
+  const int words = (T + 31) / 32;
+  const uint32_t* mb = marg_bits + size_t(bh) * T * words;
+  const float* zb = z + size_t(bh) * T * D;
+  float acc = 0.f;
+  if (!transpose) {
+    for (int w = 0; w < words; ++w) {
+      uint32_t bits = mb[size_t(r) * words + w];
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1;
+        acc += zb[size_t(w * 32 + b) * D + a];
+      }
+    }
+  } else {
+    for (int i = 0; i < T; ++i)
+      if ((mb[size_t(i) * words + r / 32] >> (r % 32)) & 1u) acc += zb[size_t(i) * D + a];
+  }
+  zout[(size_t(bh) * T + r) * D + a] = acc;
+}
+
+// ------------------------------------------------------------------ linear forward epilogue
+// One CTA per pair of query blocks (128 tokens); 128 threads, one row each.
+//   NUM_h = phi(Q) H_{2p+h}  (tcgen05, both halves for all rows; each row
+//   keeps its own half), den = phi(Q) . Z (fp32), O_l = NUM / den,
+//   O = O_s + O_l W_proj with O_l split into bf16 hi + lo for the product.
+template <int D>
+__global__ void __launch_bounds__(128, 1) fwd_linear_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ h_agg,
+    const float* __restrict__ z_agg, const __nv_bfloat16* __restrict__ w_proj,
+    const float* __restrict__ o_s, __nv_bfloat16* __restrict__ o, float* __restrict__ den_out,
+    int N, int T, int* err) {
+  constexpr int kTile = 128 * D * 2;  // one 128 x D bf16 operand
+  constexpr int kMat = D * D * 2;     // one D x D bf16 operand
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sA = base;                  // phi(Q), later O_l hi   (K-major, 128 rows)
+  uint8_t* sA2 = sA + kTile;           // O_l lo                 (K-major, 128 rows)
+  uint8_t* sH = sA2 + kTile;           // H_{2p}, H_{2p+1}       (MN-major, D k-rows)
+  uint8_t* sW = sH + 2 * kMat;         // W_proj                 (MN-major, D k-rows)
+  float* sZ = reinterpret_cast<float*>(sW + kMat);  // [2][D]
+  __shared__ uint64_t bar[2];
+  __shared__ uint32_t tmem_base;
+  const int p = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, warp = t / 32;
+  const int half = t >> 6;
+  const int blk = 2 * p + half;
+  const bool row_ok = blk < T;
+  const size_t tok = size_t(p) * 128 + t;
+  if (warp == 0) tmem_alloc(&tmem_base, 2 * D);
+  if (t == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_barrier_init();
+  }
+  // H_{2p}, H_{2p+1} and W_proj into MN-major swizzled tiles (rows = a)
+  for (int e = t; e < 3 * D * (D / 8); e += 128) {
+    const int m = e / (D * (D / 8)), rem = e % (D * (D / 8));
+    const int a = rem / (D / 8), c8 = rem % (D / 8);
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (m < 2) {
+      const int b2 = 2 * p + m;
+      if (b2 < T)
+        u = *reinterpret_cast<const uint4*>(h_agg + ((size_t(bh) * T + b2) * D + a) * D + c8 * 8);
+      st_sw128_unit(sH + m * kMat, D, a, c8 * 8, u);
+    } else {
+      u = *reinterpret_cast<const uint4*>(w_proj + size_t(a) * D + c8 * 8);
+      st_sw128_unit(sW, D, a, c8 * 8, u);
+    }
+  }
+  for (int e = t; e < 2 * D; e += 128) {
+    const int m = e / D, b2 = 2 * p + m;
+    sZ[e] = b2 < T ? z_agg[(size_t(bh) * T + b2) * D + (e % D)] : 0.f;
+  }
+  __syncthreads();
+  // phi(Q) row t -> sA (bf16, K-major) and den = phi(Q) . Z_half (fp32)
+  float den = 0.f;
+  {
+    const __nv_bfloat16* qrow = q + (size_t(bh) * N + tok) * D;
+    const float* z = sZ + half * D;
+#pragma unroll 4
+    for (int c8 = 0; c8 < D / 8; ++c8) {
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (row_ok) u = *reinterpret_cast<const uint4*>(qrow + c8 * 8);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      uint32_t pw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a = phi_f(bf16_lo(w[e])), b = phi_f(bf16_hi(w[e]));
+        den = fmaf(a, z[c8 * 8 + 2 * e], den);
+        den = fmaf(b, z[c8 * 8 + 2 * e + 1], den);
+        pw[e] = pack_bf16(a, b);
+      }
+      st_sw128_unit(sA, 128, t, c8 * 8, make_uint4(pw[0], pw[1], pw[2], pw[3]));
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  if (t == 0) {
+    constexpr uint32_t idesc = idesc_bf16(128, D, 0, 1);
+    const uint32_t a0 = smem_u32(sA);
+    for (int m = 0; m < 2; ++m) {
+      const uint32_t b0 = smem_u32(sH + m * kMat);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        mma_ss(tmem + m * D, desc_kmajor(a0, 128, ks), desc_mnmajor(b0, D, ks), idesc, ks > 0);
+    }
+    mma_commit(&bar[0]);
+  }
+  bool ok = mbar_wait(&bar[0], 0, err, nullptr);
+  tc_fence_after();
+  const float inv = (row_ok && den > 0.f) ? 1.0f / den : 0.0f;
+  if (row_ok && lane_id() < 32) den_out[size_t(bh) * N + tok] = row_ok ? den : 0.f;
+  // O_l = NUM / den, split into hi + lo bf16 (K-major rows)
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    float vals[32];
+    tmem_ld32(tmem_addr(tmem + half * D, warp * 32, c0), vals);
+    tmem_ld_wait();
+#pragma unroll
+    for (int u8 = 0; u8 < 4; ++u8) {
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = ok ? vals[u8 * 8 + 2 * e] * inv : 0.f;
+        const float x1 = ok ? vals[u8 * 8 + 2 * e + 1] * inv : 0.f;
+        hi[e] = pack_bf16(x0, x1);
+        lo[e] = pack_bf16(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
+      }
+      st_sw128_unit(sA, 128, t, c0 + u8 * 8, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+      st_sw128_unit(sA2, 128, t, c0 + u8 * 8, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (t == 0) {
+    constexpr uint32_t idesc = idesc_bf16(128, D, 0, 1);
+    const uint32_t b0 = smem_u32(sW);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks)
+      mma_ss(tmem, desc_kmajor(smem_u32(sA), 128, ks), desc_mnmajor(b0, D, ks), idesc, ks > 0);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks)
+      mma_ss(tmem, desc_kmajor(smem_u32(sA2), 128, ks), desc_mnmajor(b0, D, ks), idesc, 1);
+    mma_commit(&bar[1]);
+  }
+  ok = mbar_wait(&bar[1], 0, err, nullptr) && ok;
+  tc_fence_after();
+  {
+    const float* osrow = o_s + (size_t(bh) * N + tok) * D;
+    __nv_bfloat16* orow = o + (size_t(bh) * N + tok) * D;
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      float vals[32];
+      tmem_ld32(tmem_addr(tmem, warp * 32, c0), vals);
+      tmem_ld_wait();
+      if (row_ok && ok) {
+#pragma unroll
+        for (int u8 = 0; u8 < 4; ++u8) {
+          const float4 s0 = *reinterpret_cast<const float4*>(osrow + c0 + u8 * 8);
+          const float4 s1 = *reinterpret_cast<const float4*>(osrow + c0 + u8 * 8 + 4);
+          uint4 r;
+          r.x = pack_bf16(s0.x + vals[u8 * 8 + 0], s0.y + vals[u8 * 8 + 1]);
+          r.y = pack_bf16(s0.z + vals[u8 * 8 + 2], s0.w + vals[u8 * 8 + 3]);
+          r.z = pack_bf16(s1.x + vals[u8 * 8 + 4], s1.y + vals[u8 * 8 + 5]);
+          r.w = pack_bf16(s1.z + vals[u8 * 8 + 6], s1.w + vals[u8 * 8 + 7]);
+          *reinterpret_cast<uint4*>(orow + c0 + u8 * 8) = r;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_free(tmem, 2 * D);
+}
+
+}  // namespace
+
+cudaError_t launch_summaries(const Problem& p, const void* k, const void* v,
+                             __nv_bfloat16* summ, float* zsum, int* err, cudaStream_t s) {
+  dim3 grid(p.T, p.BH);
+  const int groups = 128 / (p.d / 8);
+  const size_t smem = 1024 + 16384 + (p.d / 64) * 8192 + sizeof(float) * groups * p.d;
+  cudaError_t e;
+  if (p.d == 128) {
+    e = cudaFuncSetAttribute(summaries_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem));
+    if (e != cudaSuccess) return e;
+    summaries_kernel<128><<<grid, 128, smem, s>>>((const __nv_bfloat16*)k,
+                                                  (const __nv_bfloat16*)v, summ, zsum, p.N,
+                                                  p.T, err);
+  } else {
+    e = cudaFuncSetAttribute(summaries_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem));
+    if (e != cudaSuccess) return e;
+    summaries_kernel<64><<<grid, 128, smem, s>>>((const __nv_bfloat16*)k,
+                                                 (const __nv_bfloat16*)v, summ, zsum, p.N, p.T,
+                                                 err);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
+                             const __nv_bfloat16* summ, __nv_bfloat16* out, int* err,
+                             cudaStream_t s) {
+  const int NN = p.d * p.d;
+  CUtensorMap ta, tb;
+  if (!make_tmap_3d(&ta, mmat, p.Tp, p.Tp, p.BH, 64, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_3d(&tb, summ, NN, p.T, p.BH, 64, 64)) return cudaErrorInvalidValue;
+  const size_t smem = 1024 + kAggStages * kAggStageBytes;
+  cudaError_t e = cudaFuncSetAttribute(agg_gemm_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.Tp / 128, NN / kAggBN, p.BH);
+  agg_gemm_kernel<<<grid, 128, smem, s>>>(ta, tb, out, p.T, p.Tp, NN, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_aggregate_z(const Problem& p, const uint32_t* marg_bits, const float* z,
+                               float* zout, bool transpose, cudaStream_t s) {
+  dim3 grid(p.T, p.BH);
+  agg_z_kernel<<<grid, p.d, 0, s>>>(marg_bits, z, zout, p.T, p.d, transpose ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_linear(const Problem& p, const void* q, const __nv_bfloat16* h_agg,
+                              const float* z_agg, const void* w_proj, const float* o_s,
+                              void* o, float* den, int* err, cudaStream_t s) {
+  dim3 grid((p.T + 1) / 2, p.BH);
+  const size_t smem = 1024 + 2 * (128 * p.d * 2) + 3 * (p.d * p.d * 2) + 2 * p.d * sizeof(float);
+  cudaError_t e;
+  if (p.d == 128) {
+    e = cudaFuncSetAttribute(fwd_linear_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    fwd_linear_kernel<128><<<grid, 128, smem, s>>>(
+        (const __nv_bfloat16*)q, h_agg, z_agg, (const __nv_bfloat16*)w_proj, o_s,
+        (__nv_bfloat16*)o, den, p.N, p.T, err);
+  } else {
+    e = cudaFuncSetAttribute(fwd_linear_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem));
+    if (e != cudaSuccess) return e;
+    fwd_linear_kernel<64><<<grid, 128, smem, s>>>(
+        (const __nv_bfloat16*)q, h_agg, z_agg, (const __nv_bfloat16*)w_proj, o_s,
+        (__nv_bfloat16*)o, den, p.N, p.T, err);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace sla

@@ -1,0 +1,321 @@
+// Sparse branch of the SLA forward: exact softmax attention restricted to the
+// critical (query block, key block) pairs.
+//
+// SLA (arXiv 2509.24006), abstract / framework step 2: critical weights get
+// full O(N^2)-class attention; negligible ones are skipped (step 4).  For a
+// query token t of block i with critical key blocks C(i):
+//   O_s,t = sum_{u in C(i)} softmax_u(scale Q_t.K_u) V_u,  LSE_t = log sum exp,
+// and O_s,t = 0, LSE_t = -inf when C(i) is empty.
+//
+// Design (sm_100a).  One CTA owns a 128-row tile = query blocks 2p and 2p+1
+// (tcgen05's natural M = 128), and walks the sorted union of their critical
+// key-block lists; rows whose block does not have a given key block critical
+// get probability 0 for it (that work is executed but not counted as
+// executed-block FLOPs).  Warp roles:
+//   warps 0-3  softmax: one query row per thread, S from TMEM, P back to
+//              TMEM (bf16, aliasing S), lazy rescaling of O in TMEM
+//   warp 4     TMA producer: Q tile once, K_j / V_j tiles into a 2-stage ring
+//   warp 5     MMA issuer (one thread): S_n = Q K_n^T into one of two TMEM
+//              buffers, O += P_n V_n with P read from TMEM
+// TMEM: S buffers at columns [0,64) and [64,128), O at [128, 128+D).
+#include <cuda_bf16.h>
+
+#include "sla_internal.h"
+#include "sla_ptx.cuh"
+
+namespace sla {
+namespace {
+
+constexpr int kStages = 2;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct FwdSmem {
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kKVBytes = 64 * D * 2;  // one K or V tile
+  static constexpr int kStageBytes = 2 * kKVBytes;
+  static constexpr int kTiles = kQBytes + kStages * kStageBytes;
+  // + the union list: 2*n_crit uint16 block indices, then 2*n_crit flag bytes
+  static size_t total(int n_crit) { return 1024 + kTiles + size_t(2 * n_crit) * 3 + 16; }
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ crit_idx, int N, int T,
+    int n_crit, float scale_log2, float* __restrict__ o_s, float* __restrict__ lse, int* err) {
+  using L = FwdSmem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = base;
+  uint8_t* sKV = base + L::kQBytes;
+  uint16_t* ulist = reinterpret_cast<uint16_t*>(base + L::kTiles);
+  uint8_t* uflag = base + L::kTiles + 2 * (2 * n_crit);
+
+  __shared__ uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], p_full[2], o_done,
+      mma_done;
+  __shared__ uint32_t tmem_base;
+  __shared__ int n_union, abort_flag;
+
+  const int p = blockIdx.x, bh = blockIdx.y;
+  const int warp = threadIdx.x / 32, lane = lane_id();
+  const int blk0 = 2 * p, blk1 = 2 * p + 1;
+  const bool has1 = blk1 < T;
+
+  if (warp == 0) tmem_alloc(&tmem_base, 256);
+  if (threadIdx.x == 32) {
+    mbar_init(&q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 128);
+    }
+    mbar_init(&o_done, 1);
+    mbar_init(&mma_done, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (threadIdx.x == 128) {
+    // sorted union of the two rows' critical lists; flag bit h = member of half h
+    const int32_t* l0 = crit_idx + (size_t(bh) * T + blk0) * n_crit;
+    const int32_t* l1 = crit_idx + (size_t(bh) * T + (has1 ? blk1 : blk0)) * n_crit;
+    const int n1 = has1 ? n_crit : 0;
+    int a = 0, b = 0, n = 0;
+    while (a < n_crit || b < n1) {
+      const int x = a < n_crit ? l0[a] : 0x7FFFFFFF;
+      const int y = b < n1 ? l1[b] : 0x7FFFFFFF;
+      int j, f;
+      if (x == y) { j = x; f = 3; ++a; ++b; }
+      else if (x < y) { j = x; f = 1; ++a; }
+      else { j = y; f = 2; ++b; }
+      if (j < 0 || j >= T) { set_error(err, SLA_ERR_DEVICE); continue; }
+      ulist[n] = uint16_t(j);
+      uflag[n] = uint8_t(f);
+      ++n;
+    }
+    n_union = n;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const int nU = n_union;
+  const uint32_t tm_o = tmem + 128;
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0 && nU > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&q_full, L::kQBytes);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * 128 * 128, &q_full, &tm_q, c * 64, p * 128, bh);
+      int issued = 0;
+      for (int n = 0; n < nU; ++n) {
+        const int s = n % kStages;
+        if (n >= kStages && !mbar_wait(&kv_empty[s], ((n / kStages) + 1) & 1, err, &abort_flag))
+          break;
+        uint8_t* sk = sKV + s * L::kStageBytes;
+        uint8_t* sv = sk + L::kKVBytes;
+        const int row = int(ulist[n]) * kBlock;
+        mbar_arrive_expect_tx(&kv_full[s], L::kStageBytes);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(sk + c * 64 * 128, &kv_full[s], &tm_k, c * 64, row, bh);
+          tma_load_3d(sv + c * 64 * 128, &kv_full[s], &tm_v, c * 64, row, bh);
+        }
+        ++issued;
+      }
+      if (abort_flag) {
+        // let copies already in flight land before the CTA exits
+        mbar_wait(&q_full, 0, nullptr, nullptr);
+        for (int n = (issued > kStages ? issued - kStages : 0); n < issued; ++n)
+          mbar_wait(&kv_full[n % kStages], (n / kStages) & 1, nullptr, nullptr);
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0 && nU > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(128, 64, 0, 0);
+      constexpr uint32_t idesc_o = idesc_bf16(128, D, 0, 1);
+      const uint32_t q0 = smem_u32(sQ);
+      bool ok = mbar_wait(&q_full, 0, err, &abort_flag);
+      auto issue_s = [&](int n) -> bool {
+        const int s = n % kStages;
+        if (!mbar_wait(&kv_full[s], (n / kStages) & 1, err, &abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t k0 = smem_u32(sKV + s * L::kStageBytes);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ss(tmem + (n & 1) * 64, desc_kmajor(q0, 128, ks), desc_kmajor(k0, 64, ks),
+                 idesc_s, ks > 0);
+        mma_commit(&s_full[n & 1]);
+        return true;
+      };
+      auto issue_pv = [&](int n) -> bool {
+        if (!mbar_wait(&p_full[n & 1], (n >> 1) & 1, err, &abort_flag)) return false;
+        tc_fence_after();
+        const int s = n % kStages;
+        const uint32_t v0 = smem_u32(sKV + s * L::kStageBytes + L::kKVBytes);
+        const uint32_t pt = tmem + (n & 1) * 64;  // P aliases the first 32 columns of S
+#pragma unroll
+        for (int ks = 0; ks < kBlock / 16; ++ks)
+          mma_ts(tm_o, pt + ks * 8, desc_mnmajor(v0, 64, ks), idesc_o, (n | ks) != 0);
+        mma_commit(&o_done);
+        mma_commit(&kv_empty[s]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      if (ok && nU > 1) ok = issue_s(1);
+      for (int n = 0; ok && n < nU; ++n) {
+        ok = issue_pv(n);
+        if (ok && n + 2 < nU) ok = issue_s(n + 2);
+      }
+      mma_commit(&mma_done);
+      mbar_wait(&mma_done, 0, nullptr, nullptr);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warps 0-3
+    const int r = threadIdx.x;  // tile row == TMEM lane
+    const int half = r >> 6;
+    const int blk = blk0 + half;
+    const bool row_ok = blk < T;
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int n = 0; n < nU; ++n) {
+      const uint32_t sb = tmem + lane_base + (n & 1) * 64;
+      ok = mbar_wait(&s_full[n & 1], (n >> 1) & 1, err, &abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      float sv[64];
+      tmem_ld32(sb, reinterpret_cast<float(&)[32]>(sv[0]));
+      tmem_ld32(sb + 32, reinterpret_cast<float(&)[32]>(sv[32]));
+      tmem_ld_wait();
+      const bool member = row_ok && ((uflag[n] >> half) & 1);
+      float alpha = 1.f;
+      if (member) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          sv[e] *= scale_log2;
+          mx = fmaxf(mx, sv[e]);
+        }
+        if (mx > m_run + kRescaleThreshold || m_run == -INFINITY) {
+          alpha = exp2f(m_run - mx);  // 0 when m_run == -inf
+          l_run *= alpha;
+          m_run = mx;
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          sv[e] = exp2f(sv[e] - m_run);
+          sum += sv[e];
+        }
+        l_run += sum;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) sv[e] = 0.f;
+      }
+      {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(sv[2 * e], sv[2 * e + 1]);
+        tmem_st16(sb, pk);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(sv[32 + 2 * e], sv[32 + 2 * e + 1]);
+        tmem_st16(sb + 16, pk);
+      }
+      // O must not be rescaled before the previous P V has landed
+      if (n > 0) {
+        ok = mbar_wait(&o_done, (n - 1) & 1, err, &abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+      }
+      if (__any_sync(0xFFFFFFFFu, alpha != 1.f) && n > 0) {
+        const uint32_t ob = tm_o + lane_base;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 16) {
+          float ov[16];
+          tmem_ld16(ob + c0, ov);
+          tmem_ld_wait();
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(ov[e] * alpha);
+          tmem_st16(ob + c0, w);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[n & 1]);
+    }
+    // ---------------------------------------------------------------- epilogue
+    if (ok && nU > 0) {
+      ok = mbar_wait(&o_done, (nU - 1) & 1, err, &abort_flag);
+      tc_fence_after();
+    }
+    const size_t tok = size_t(p) * 128 + r;
+    const bool have = ok && nU > 0 && l_run > 0.f;
+    const float inv = have ? 1.0f / l_run : 0.f;
+    float* dst = o_s + (size_t(bh) * N + tok) * D;
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      float ov[32];
+      if (nU > 0) {
+        tmem_ld32(tm_o + lane_base + c0, ov);
+        tmem_ld_wait();
+      }
+      if (row_ok) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          float4 x = have ? make_float4(ov[e] * inv, ov[e + 1] * inv, ov[e + 2] * inv,
+                                        ov[e + 3] * inv)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+          *reinterpret_cast<float4*>(dst + c0 + e) = x;
+        }
+      }
+    }
+    if (row_ok)
+      lse[size_t(bh) * N + tok] =
+          have ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_free(tmem, 256);
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
+                              const int32_t* crit_idx, float* o_s, float* lse, int* err,
+                              cudaStream_t s) {
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_bhnd(&tq, q, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_bhnd(&tk, k, p.BH, p.N, p.d, 64)) return cudaErrorInvalidValue;
+  if (!make_tmap_bhnd(&tv, v, p.BH, p.N, p.d, 64)) return cudaErrorInvalidValue;
+  dim3 grid((p.T + 1) / 2, p.BH);
+  cudaError_t e;
+  if (p.d == 128) {
+    const int smem = int(FwdSmem<128>::total(p.n_crit));
+    e = cudaFuncSetAttribute(fwd_sparse_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
+    if (e != cudaSuccess) return e;
+    fwd_sparse_kernel<128><<<grid, 192, smem, s>>>(tq, tk, tv, crit_idx, p.N, p.T, p.n_crit,
+                                                   p.scale_log2, o_s, lse, err);
+  } else {
+    const int smem = int(FwdSmem<64>::total(p.n_crit));
+    e = cudaFuncSetAttribute(fwd_sparse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
+    if (e != cudaSuccess) return e;
+    fwd_sparse_kernel<64><<<grid, 192, smem, s>>>(tq, tk, tv, crit_idx, p.N, p.T, p.n_crit,
+                                                  p.scale_log2, o_s, lse, err);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace sla
