@@ -166,6 +166,11 @@ def forward(q, k, v, w_proj, cls, block: int, scale: float | None = None,
     rows = range(T) if query_blocks is None else query_blocks
     for b in range(B):
         for hh in range(H):
+            # H_i = sum_{j marginal in row i} h_j for every i, written as the
+            # product with the 0/1 marginal indicator matrix of this head
+            marg_ind = (cls[b, hh] == 0).astype(np.float64)
+            H_all = np.tensordot(marg_ind, h[b, hh], axes=(1, 0))
+            Z_all = marg_ind @ z[b, hh]
             for i in rows:
                 t0, t1 = i * block, (i + 1) * block
                 qi = q64[b, hh, t0:t1]
@@ -182,8 +187,7 @@ def forward(q, k, v, w_proj, cls, block: int, scale: float | None = None,
                     lse[b, hh, t0:t1] = (m + np.log(l))[:, 0]
                 # marginal pairs: linear attention through the key-block summaries
                 if marg.size:
-                    Hi = h[b, hh, marg].sum(axis=0)
-                    Zi = z[b, hh, marg].sum(axis=0)
+                    Hi, Zi = H_all[i], Z_all[i]
                     fq = phi(qi)
                     num = fq @ Hi
                     dn = fq @ Zi
@@ -272,8 +276,11 @@ def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
     do_l = np.einsum("bhtc,ac->bhta", do64, w64)
     for b in range(B):
         for hh in range(H):
-            dh = np.zeros((T, d, d))
-            dz = np.zeros((T, d))
+            marg_ind = (cls[b, hh] == 0).astype(np.float64)
+            H_all = np.tensordot(marg_ind, h[b, hh], axes=(1, 0))
+            Z_all = marg_ind @ z[b, hh]
+            dH_all = np.zeros((T, d, d))  # dL/dH_i per query block
+            dZ_all = np.zeros((T, d))
             for i in range(T):
                 t0, t1 = i * block, (i + 1) * block
                 qi = q64[b, hh, t0:t1]
@@ -292,8 +299,7 @@ def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
                     dq[b, hh, t0:t1] += scale * (ds @ kc)
                     dk[b, hh, keys] += scale * (ds.T @ qi)
                 if marg.size:
-                    Hi = h[b, hh, marg].sum(axis=0)
-                    Zi = z[b, hh, marg].sum(axis=0)
+                    Hi, Zi = H_all[i], Z_all[i]
                     dn = fwd["den"][b, hh, t0:t1]
                     dol = do_l[b, hh, t0:t1]
                     dnum = dol / dn[:, None]
@@ -301,10 +307,11 @@ def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
                     fq = phi(qi)
                     dfq = dnum @ Hi.T + dden[:, None] * Zi[None, :]
                     dq[b, hh, t0:t1] += dfq * phi_prime(qi)
-                    dHi = fq.T @ dnum
-                    dZi = fq.T @ dden
-                    dh[marg] += dHi
-                    dz[marg] += dZi
+                    dH_all[i] = fq.T @ dnum
+                    dZ_all[i] = fq.T @ dden
+            # dh_j = sum over rows i in which j is marginal of dL/dH_i
+            dh = np.tensordot(marg_ind.T, dH_all, axes=(1, 0))
+            dz = marg_ind.T @ dZ_all
             for j in range(T):
                 u0, u1 = j * block, (j + 1) * block
                 kj, vj = k64[b, hh, u0:u1], v64[b, hh, u0:u1]
