@@ -269,10 +269,47 @@ sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, co
   Problem p;
   sla_status st = check_shape(shape, &p);
   if (st != SLA_OK) return st;
-  (void)q; (void)k; (void)v; (void)w_proj; (void)mask; (void)saved; (void)d_o;
-  (void)dq; (void)dk; (void)dv; (void)dw_proj; (void)workspace; (void)workspace_bytes;
-  (void)stream;
-  return SLA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !w_proj || !d_o || !dq || !dk || !dv || !dw_proj)
+    return SLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(w_proj) || !aligned16(d_o) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dw_proj))
+    return SLA_ERR_INVALID_ARG;
+  if ((st = check_mask(p, mask, true)) != SLA_OK) return st;
+  if ((st = check_saved(p, saved)) != SLA_OK) return st;
+  WorkspaceLayout L;
+  if ((st = check_ws(p, workspace, workspace_bytes, &L)) != SLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return SLA_ERR_CUDA;
+  int* err = at<int>(workspace, L.err);
+  auto* summ = at<__nv_bfloat16>(workspace, L.summ);
+  auto* dh = at<__nv_bfloat16>(workspace, L.dh);
+  auto* mmat_t = at<__nv_bfloat16>(workspace, L.mmat_t);
+  float* zsum = at<float>(workspace, L.zsum);
+  float* dz = at<float>(workspace, L.dz);
+  float* dvec = at<float>(workspace, L.dvec);
+  float* dnum = at<float>(workspace, L.dnum);
+  float* dden = at<float>(workspace, L.dden);
+  const size_t grad_bytes = size_t(p.BH) * p.N * p.d * sizeof(float);
+  if (cudaMemsetAsync(dq, 0, grad_bytes, s) != cudaSuccess) return SLA_ERR_CUDA;
+  if (cudaMemsetAsync(dw_proj, 0, size_t(p.d) * p.d * sizeof(float), s) != cudaSuccess)
+    return SLA_ERR_CUDA;
+  auto* h_agg = static_cast<const __nv_bfloat16*>(saved->h_agg);
+  // linear-branch preparation: D, dnum, dden, per-block A_i / a_i, dW
+  SLA_LAUNCH(launch_bwd_prep(p, q, d_o, w_proj, saved->o_s, saved->den, h_agg, saved->z_agg, dvec,
+                             dnum, dden, summ, zsum, dw_proj, sms, err, s));
+  // dh_j = sum over rows i with j marginal of A_i (transposed aggregation)
+  SLA_LAUNCH(launch_expand_marginal(p, mask->marg_bits, nullptr, mmat_t, s));
+  SLA_LAUNCH(launch_aggregate(p, mmat_t, summ, dh, err, s));
+  SLA_LAUNCH(launch_aggregate_z(p, mask->marg_bits, zsum, dz, true, s));
+  // sparse branch writes dK, dV and accumulates dQ; the linear branch adds its share
+  SLA_LAUNCH(launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
+                               mask->crit_col_idx, dq, dk, dv, err, s));
+  SLA_LAUNCH(launch_bwd_linear(p, q, k, v, h_agg, saved->z_agg, dh, dz, dnum, dden, dq, dk, dv,
+                               err, s));
+  return SLA_OK;
 }
 
 sla_status sla_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {

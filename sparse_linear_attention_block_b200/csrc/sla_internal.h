@@ -71,6 +71,21 @@ cudaError_t launch_fwd_linear(const Problem& p, const void* q, const __nv_bfloat
                               const float* z_agg, const void* w_proj, const float* o_s,
                               void* o, float* den, int* err, cudaStream_t s);
 
+cudaError_t launch_bwd_prep(const Problem& p, const void* q, const void* d_o, const void* w_proj,
+                            const float* o_s, const float* den, const __nv_bfloat16* h_agg,
+                            const float* z_agg, float* dvec, float* dnum, float* dden,
+                            __nv_bfloat16* summ, float* zsum, float* dw, int num_sms, int* err,
+                            cudaStream_t s);
+cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
+                              const void* d_o, const float* lse, const float* dvec,
+                              const int32_t* col_ptr, const int32_t* col_idx, float* dq,
+                              float* dk, float* dv, int* err, cudaStream_t s);
+cudaError_t launch_bwd_linear(const Problem& p, const void* q, const void* k, const void* v,
+                              const __nv_bfloat16* h_agg, const float* z_agg,
+                              const __nv_bfloat16* dh, const float* dz, const float* dnum,
+                              const float* dden, float* dq, float* dk, float* dv, int* err,
+                              cudaStream_t s);
+
 // TMA descriptor for a bf16 [BH, N, d] tensor viewed as 3D {d, N, BH} with a
 // box of {64, rows, 1} and 128-byte swizzle.  Returns false on failure.
 bool make_tmap_bhnd(CUtensorMap* map, const void* base, int BH, int N, int d, int box_rows);
