@@ -94,13 +94,13 @@ typedef struct {
  *   lse   fp32 [B,H,N]      log-sum-exp of the critical scores (-inf if none)
  *   o_s   fp32 [B,H,N,d]    sparse-branch output
  *   den   fp32 [B,H,N]      phi(Q).Z_i (0 if the row has no marginal block)
- *   h_agg bf16 [B,H,T,d,d]  H_i per query block
+ *   h_agg fp32 [B,H,T,d,d]  H_i per query block
  *   z_agg fp32 [B,H,T,d]    Z_i per query block */
 typedef struct {
   float* lse;
   float* o_s;
   float* den;
-  void* h_agg;
+  float* h_agg;
   float* z_agg;
 } sla_saved;
 

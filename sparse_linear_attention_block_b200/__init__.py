@@ -231,7 +231,7 @@ class Buffers:
             lse=e(B, H, N, dt=torch.float32),
             o_s=e(B, H, N, d, dt=torch.float32),
             den=e(B, H, N, dt=torch.float32),
-            h_agg=e(B, H, T, d, d, dt=torch.bfloat16),
+            h_agg=e(B, H, T, d, d, dt=torch.float32),
             z_agg=e(B, H, T, d, dt=torch.float32),
             workspace=torch.empty(int(s.workspace_bytes) + 1024, dtype=torch.uint8, device=dev),
             mask=MaskStruct(), saved=SavedStruct())

@@ -27,9 +27,10 @@ WorkspaceLayout workspace_layout(int BH, int N, int d) {
   L.err = take(256);
   L.qbar = take(bh * T * d * 4);
   L.kbar = take(bh * T * d * 4);
-  L.summ = take(bh * T * d * d * 2);
+  L.summ_hi = take(bh * T * d * d * 2);
+  L.summ_lo = take(bh * T * d * d * 2);
   L.zsum = take(bh * T * d * 4);
-  L.dh = take(bh * T * d * d * 2);
+  L.dh = take(bh * T * d * d * 4);
   L.dz = take(bh * T * d * 4);
   L.mmat = take(bh * Tp * Tp * 2);
   L.mmat_t = take(bh * Tp * Tp * 2);
@@ -137,7 +138,7 @@ sla_status fill_sizes(const Problem& p, sla_sizes* o) {
   o->lse_bytes = bh * N * 4;
   o->o_s_bytes = bh * N * d * 4;
   o->den_bytes = bh * N * 4;
-  o->h_agg_bytes = bh * T * d * d * 2;
+  o->h_agg_bytes = bh * T * d * d * 4;
   o->z_agg_bytes = bh * T * d * 4;
   o->workspace_bytes = workspace_layout(p.BH, p.N, p.d).total;
   return SLA_OK;
@@ -246,19 +247,19 @@ sla_status sla_forward(const sla_shape* shape, const void* q, const void* k, con
   if ((st = check_ws(p, workspace, workspace_bytes, &L)) != SLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* err = at<int>(workspace, L.err);
-  auto* summ = at<__nv_bfloat16>(workspace, L.summ);
+  auto* summ_hi = at<__nv_bfloat16>(workspace, L.summ_hi);
+  auto* summ_lo = at<__nv_bfloat16>(workspace, L.summ_lo);
   auto* mmat = at<__nv_bfloat16>(workspace, L.mmat);
   float* zsum = at<float>(workspace, L.zsum);
-  auto* h_agg = static_cast<__nv_bfloat16*>(saved->h_agg);
   // linear branch: summaries, marginal aggregation
-  SLA_LAUNCH(launch_summaries(p, k, v, summ, zsum, err, s));
+  SLA_LAUNCH(launch_summaries(p, k, v, summ_hi, summ_lo, zsum, err, s));
   SLA_LAUNCH(launch_expand_marginal(p, mask->marg_bits, mmat, nullptr, s));
-  SLA_LAUNCH(launch_aggregate(p, mmat, summ, h_agg, err, s));
+  SLA_LAUNCH(launch_aggregate(p, mmat, summ_hi, summ_lo, saved->h_agg, err, s));
   SLA_LAUNCH(launch_aggregate_z(p, mask->marg_bits, zsum, saved->z_agg, false, s));
   // sparse branch, then the combination
   SLA_LAUNCH(launch_fwd_sparse(p, q, k, v, mask->crit_idx, saved->o_s, saved->lse, err, s));
-  SLA_LAUNCH(launch_fwd_linear(p, q, h_agg, saved->z_agg, w_proj, saved->o_s, o, saved->den,
-                               err, s));
+  SLA_LAUNCH(launch_fwd_linear(p, q, saved->h_agg, saved->z_agg, w_proj, saved->o_s, o,
+                               saved->den, err, s));
   return SLA_OK;
 }
 
@@ -284,9 +285,10 @@ sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, co
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return SLA_ERR_CUDA;
   int* err = at<int>(workspace, L.err);
-  auto* summ = at<__nv_bfloat16>(workspace, L.summ);
-  auto* dh = at<__nv_bfloat16>(workspace, L.dh);
+  auto* summ_hi = at<__nv_bfloat16>(workspace, L.summ_hi);
+  auto* summ_lo = at<__nv_bfloat16>(workspace, L.summ_lo);
   auto* mmat_t = at<__nv_bfloat16>(workspace, L.mmat_t);
+  float* dh = at<float>(workspace, L.dh);
   float* zsum = at<float>(workspace, L.zsum);
   float* dz = at<float>(workspace, L.dz);
   float* dvec = at<float>(workspace, L.dvec);
@@ -296,19 +298,19 @@ sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, co
   if (cudaMemsetAsync(dq, 0, grad_bytes, s) != cudaSuccess) return SLA_ERR_CUDA;
   if (cudaMemsetAsync(dw_proj, 0, size_t(p.d) * p.d * sizeof(float), s) != cudaSuccess)
     return SLA_ERR_CUDA;
-  auto* h_agg = static_cast<const __nv_bfloat16*>(saved->h_agg);
-  // linear-branch preparation: D, dnum, dden, per-block A_i / a_i, dW
-  SLA_LAUNCH(launch_bwd_prep(p, q, d_o, w_proj, saved->o_s, saved->den, h_agg, saved->z_agg, dvec,
-                             dnum, dden, summ, zsum, dw_proj, sms, err, s));
+  // linear-branch preparation: D, dnum, dden, dW; then per-block A_i / a_i
+  SLA_LAUNCH(launch_bwd_prep(p, q, d_o, w_proj, saved->o_s, saved->den, saved->h_agg, dvec, dnum,
+                             dden, dw_proj, sms, err, s));
+  SLA_LAUNCH(launch_bwd_summ(p, q, dnum, dden, summ_hi, summ_lo, zsum, err, s));
   // dh_j = sum over rows i with j marginal of A_i (transposed aggregation)
   SLA_LAUNCH(launch_expand_marginal(p, mask->marg_bits, nullptr, mmat_t, s));
-  SLA_LAUNCH(launch_aggregate(p, mmat_t, summ, dh, err, s));
+  SLA_LAUNCH(launch_aggregate(p, mmat_t, summ_hi, summ_lo, dh, err, s));
   SLA_LAUNCH(launch_aggregate_z(p, mask->marg_bits, zsum, dz, true, s));
   // sparse branch writes dK, dV and accumulates dQ; the linear branch adds its share
   SLA_LAUNCH(launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
                                mask->crit_col_idx, dq, dk, dv, err, s));
-  SLA_LAUNCH(launch_bwd_linear(p, q, k, v, h_agg, saved->z_agg, dh, dz, dnum, dden, dq, dk, dv,
-                               err, s));
+  SLA_LAUNCH(launch_bwd_linear(p, q, k, v, saved->h_agg, saved->z_agg, dh, dz, dnum, dden, dq, dk,
+                               dv, err, s));
   return SLA_OK;
 }
 

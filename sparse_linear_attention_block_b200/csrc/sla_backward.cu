@@ -14,8 +14,9 @@
 //   W_proj:  dW = sum_t O_l,t^T dO_t
 //
 // Kernels (all tcgen05 for the contractions):
-//   bwd_prep_kernel    per 128-token tile: D, dnum, dden, A_i, a_i; dW accumulated
-//                      in TMEM across the tiles of a persistent CTA
+//   bwd_prep_kernel    per 128-token tile: D, dnum, dden; dW accumulated in TMEM
+//                      across the tiles of a persistent CTA
+//   bwd_summ_kernel    per 128-token tile: A_i (bf16 hi/lo planes) and a_i
 //   bwd_sparse_kernel  per 128-key tile (key blocks 2q, 2q+1): walks the union of
 //                      their critical query blocks (column CSR); dK, dV in TMEM,
 //                      dQ^T per query block reduced into fp32 dQ with atomics
@@ -53,42 +54,63 @@ __device__ __forceinline__ void load_rows_sw(uint8_t* dst, int rows, const __nv_
   }
 }
 
-// ============================================================================ bwd_prep
+// Load an fp32 [rows x D] global matrix into bf16 hi/lo 128B-swizzled tiles
+// (64-column chunks of `rows` rows); rows >= valid_rows are zero.
 template <int D>
-struct PrepSmem {
-  static constexpr int kTile = 128 * 128 * 2;  // 128 rows x 2 chunks (D = 64 is padded)
-  static constexpr int kTotal = 1024 + 7 * kTile;
-};
+__device__ __forceinline__ void load_split_sw(uint8_t* hi_t, uint8_t* lo_t, int rows,
+                                              const float* src, int valid_rows, int tid,
+                                              int nthreads) {
+  for (int e = tid; e < rows * (D / 8); e += nthreads) {
+    const int r = e / (D / 8), c8 = e % (D / 8);
+    float x[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (r < valid_rows) {
+      const float4 u0 = *reinterpret_cast<const float4*>(src + size_t(r) * D + c8 * 8);
+      const float4 u1 = *reinterpret_cast<const float4*>(src + size_t(r) * D + c8 * 8 + 4);
+      x[0] = u0.x; x[1] = u0.y; x[2] = u0.z; x[3] = u0.w;
+      x[4] = u1.x; x[5] = u1.y; x[6] = u1.z; x[7] = u1.w;
+    }
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      h[i] = pack_bf16(x[2 * i], x[2 * i + 1]);
+      l[i] = pack_bf16(x[2 * i] - bf16_lo(h[i]), x[2 * i + 1] - bf16_hi(h[i]));
+    }
+    st_sw128_unit(hi_t, rows, r, c8 * 8, make_uint4(h[0], h[1], h[2], h[3]));
+    st_sw128_unit(lo_t, rows, r, c8 * 8, make_uint4(l[0], l[1], l[2], l[3]));
+  }
+}
+
+// ============================================================================ bwd_prep
+// Persistent over 128-token tiles (query blocks 2p, 2p+1); 128 threads, one
+// row each; thread 0 issues the MMAs.  Per tile:
+//   G = dO W^T, NUM_h = phi(Q) (H_h,hi + H_h,lo)           (tcgen05)
+//   O_l = NUM / den, D = dO . O_s, dnum = G / den, dden = -(G . O_l) / den
+//   dW += (O_l,hi + O_l,lo)^T dO  accumulated in TMEM over the CTA's tiles
+constexpr int kTile32 = 128 * 128 * 2;  // 128 rows x 2 chunks (D = 64 padded)
 
 template <int D>
 __global__ void __launch_bounds__(128, 1) bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ d_o,
     const __nv_bfloat16* __restrict__ w_proj, const float* __restrict__ o_s,
-    const float* __restrict__ den, const __nv_bfloat16* __restrict__ h_agg,
-    const float* __restrict__ z_agg, float* __restrict__ dvec, float* __restrict__ dnum,
-    float* __restrict__ dden, __nv_bfloat16* __restrict__ summ, float* __restrict__ zsum,
-    float* __restrict__ dw, int N, int T, int BH, int* err) {
-  using L = PrepSmem<D>;
+    const float* __restrict__ den, const float* __restrict__ h_agg, float* __restrict__ dvec,
+    float* __restrict__ dnum, float* __restrict__ dden, float* __restrict__ dw, int N, int T,
+    int BH, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sA = base;                  // phi(Q)            [t][a]
-  uint8_t* sDO = sA + L::kTile;        // dO                [t][c]
-  uint8_t* sW = sDO + L::kTile;        // W_proj            [a][c]
-  uint8_t* sH0 = sW + L::kTile;        // H_{2p}  [a][c], later O_l hi [t][a]
-  uint8_t* sH1 = sH0 + L::kTile;       // H_{2p+1}[a][c], later O_l lo [t][a]
-  uint8_t* sDN = sH1 + L::kTile;       // dnum (bf16)       [t][c]
-  float* sZ = reinterpret_cast<float*>(sDN + L::kTile);  // [2][D]
-  float* sDd = sZ + 2 * D;                               // dden [128]
-  __shared__ uint64_t bar[2];
+  uint8_t* sA = base;                  // phi(Q)                      [t][a]
+  uint8_t* sDO = sA + kTile32;         // dO                          [t][c]
+  uint8_t* sW = sDO + kTile32;         // W_proj                      [a][c]
+  uint8_t* sHh = sW + kTile32;         // H hi [a][c], later O_l hi   [t][a]
+  uint8_t* sHl = sHh + kTile32;        // H lo [a][c], later O_l lo   [t][a]
+  __shared__ uint64_t bar[3];
   __shared__ uint32_t tmem_base;
   const int t = threadIdx.x, warp = t / 32, half = t >> 6;
   const int P = (T + 1) / 2, ntiles = P * BH;
-  constexpr uint32_t kCols = 4 * D;  // G | NUM0/A_0 | NUM1/A_1 | dW
+  constexpr uint32_t kCols = 4 * D;  // G | NUM0 | NUM1 | dW
   if (warp == 0) tmem_alloc(&tmem_base, kCols);
   if (t == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+    for (int b = 0; b < 3; ++b) mbar_init(&bar[b], 1);
     fence_barrier_init();
   }
   load_rows_sw<D>(sW, D, w_proj, D, t, 128);
@@ -98,23 +120,13 @@ __global__ void __launch_bounds__(128, 1) bwd_prep_kernel(
   const uint32_t tmem = tmem_base;
   const uint32_t lane_base = uint32_t(warp * 32) << 16;
   int it = 0;
-  bool ok = true;
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     const int bh = tile / P, p = tile % P;
     const int blk = 2 * p + half;
     const bool row_ok = blk < T;
     const size_t tok = size_t(p) * 128 + t;
     const size_t rowoff = (size_t(bh) * N + tok) * D;
-    // H_{2p}, H_{2p+1} ([a][c]), Z, dO tile, phi(Q) tile
-    for (int m = 0; m < 2; ++m) {
-      const int b2 = 2 * p + m;
-      load_rows_sw<D>(m ? sH1 : sH0, D, h_agg + (size_t(bh) * T + (b2 < T ? b2 : 0)) * D * D,
-                      b2 < T ? D : 0, t, 128);
-    }
-    for (int e = t; e < 2 * D; e += 128) {
-      const int b2 = 2 * p + e / D;
-      sZ[e] = b2 < T ? z_agg[(size_t(bh) * T + b2) * D + e % D] : 0.f;
-    }
+    bool ok = true;
     load_rows_sw<D>(sDO, 128, d_o + (size_t(bh) * N + size_t(p) * 128) * D,
                     min(128, N - p * 128), t, 128);
     for (int c8 = 0; c8 < D / 8; ++c8) {
@@ -126,27 +138,35 @@ __global__ void __launch_bounds__(128, 1) bwd_prep_kernel(
       for (int e = 0; e < 4; ++e) pw[e] = pack_bf16(phi_f(bf16_lo(w[e])), phi_f(bf16_hi(w[e])));
       st_sw128_unit(sA, 128, t, c8 * 8, make_uint4(pw[0], pw[1], pw[2], pw[3]));
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (t == 0) {
-      // G = dO W^T ; NUM_h = phi(Q) H_h
-      constexpr uint32_t id_g = idesc_bf16(128, D, 0, 0);
-      constexpr uint32_t id_n = idesc_bf16(128, D, 0, 1);
+    for (int m = 0; m < 2; ++m) {
+      const int b2 = 2 * p + m;
+      load_split_sw<D>(sHh, sHl, D, h_agg + (size_t(bh) * T + (b2 < T ? b2 : 0)) * D * D,
+                       b2 < T ? D : 0, t, 128);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (t == 0) {
+        constexpr uint32_t id_g = idesc_bf16(128, D, 0, 0);
+        constexpr uint32_t id_n = idesc_bf16(128, D, 0, 1);
+        if (m == 0) {
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks)
-        mma_ss(tmem, desc_kmajor(smem_u32(sDO), 128, ks), desc_kmajor(smem_u32(sW), D, ks), id_g,
-               ks > 0);
-      for (int m = 0; m < 2; ++m)
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_ss(tmem, desc_kmajor(smem_u32(sDO), 128, ks), desc_kmajor(smem_u32(sW), D, ks),
+                   id_g, ks > 0);
+        }
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
+        for (int ks = 0; ks < D / 16; ++ks) {
           mma_ss(tmem + (1 + m) * D, desc_kmajor(smem_u32(sA), 128, ks),
-                 desc_mnmajor(smem_u32(m ? sH1 : sH0), D, ks), id_n, ks > 0);
-      mma_commit(&bar[0]);
+                 desc_mnmajor(smem_u32(sHh), D, ks), id_n, ks > 0);
+          mma_ss(tmem + (1 + m) * D, desc_kmajor(smem_u32(sA), 128, ks),
+                 desc_mnmajor(smem_u32(sHl), D, ks), id_n, 1);
+        }
+        mma_commit(&bar[m]);
+      }
+      ok = mbar_wait(&bar[m], it & 1, err, nullptr) && ok;
+      tc_fence_after();
     }
-    ok = mbar_wait(&bar[0], it & 1, err, nullptr);
-    tc_fence_after();
     // per row: O_l, D, dnum, dden
     const float dn = row_ok ? den[size_t(bh) * N + tok] : 0.f;
     const float inv = dn > 0.f ? 1.0f / dn : 0.f;
@@ -157,14 +177,13 @@ __global__ void __launch_bounds__(128, 1) bwd_prep_kernel(
       tmem_ld16(tmem + lane_base + c0, g);
       tmem_ld16(tmem + lane_base + (1 + half) * D + c0, nm);
       tmem_ld_wait();
-      uint32_t ol_hi[8], ol_lo[8], dnb[8];
+      uint32_t ol_hi[8], ol_lo[8];
 #pragma unroll
       for (int e = 0; e < 16; e += 2) {
         const float o0 = nm[e] * inv, o1 = nm[e + 1] * inv;
         gdot = fmaf(g[e], o0, fmaf(g[e + 1], o1, gdot));
         ol_hi[e / 2] = pack_bf16(o0, o1);
         ol_lo[e / 2] = pack_bf16(o0 - bf16_lo(ol_hi[e / 2]), o1 - bf16_hi(ol_hi[e / 2]));
-        dnb[e / 2] = pack_bf16(g[e] * inv, g[e + 1] * inv);
       }
       if (row_ok) {
         const float* osr = o_s + rowoff + c0;
@@ -185,79 +204,32 @@ __global__ void __launch_bounds__(128, 1) bwd_prep_kernel(
               make_float4(g[e + 4] * inv, g[e + 5] * inv, g[e + 6] * inv, g[e + 7] * inv);
         }
       }
-      st_sw128_unit(sH0, 128, t, c0, make_uint4(ol_hi[0], ol_hi[1], ol_hi[2], ol_hi[3]));
-      st_sw128_unit(sH0, 128, t, c0 + 8, make_uint4(ol_hi[4], ol_hi[5], ol_hi[6], ol_hi[7]));
-      st_sw128_unit(sH1, 128, t, c0, make_uint4(ol_lo[0], ol_lo[1], ol_lo[2], ol_lo[3]));
-      st_sw128_unit(sH1, 128, t, c0 + 8, make_uint4(ol_lo[4], ol_lo[5], ol_lo[6], ol_lo[7]));
-      st_sw128_unit(sDN, 128, t, c0, make_uint4(dnb[0], dnb[1], dnb[2], dnb[3]));
-      st_sw128_unit(sDN, 128, t, c0 + 8, make_uint4(dnb[4], dnb[5], dnb[6], dnb[7]));
+      st_sw128_unit(sHh, 128, t, c0, make_uint4(ol_hi[0], ol_hi[1], ol_hi[2], ol_hi[3]));
+      st_sw128_unit(sHh, 128, t, c0 + 8, make_uint4(ol_hi[4], ol_hi[5], ol_hi[6], ol_hi[7]));
+      st_sw128_unit(sHl, 128, t, c0, make_uint4(ol_lo[0], ol_lo[1], ol_lo[2], ol_lo[3]));
+      st_sw128_unit(sHl, 128, t, c0 + 8, make_uint4(ol_lo[4], ol_lo[5], ol_lo[6], ol_lo[7]));
     }
-    const float ddn = (row_ok && dn > 0.f) ? -gdot * inv : 0.f;
-    sDd[t] = ddn;
     if (row_ok) {
       dvec[size_t(bh) * N + tok] = dsum;
-      dden[size_t(bh) * N + tok] = ddn;
+      dden[size_t(bh) * N + tok] = dn > 0.f ? -gdot * inv : 0.f;
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (t == 0) {
-      // A_h = phi(Q_h)^T dnum_h (K = the 64 tokens of block 2p+h); dW += O_l^T dO
-      constexpr uint32_t id_a = idesc_bf16(128, D, 1, 1);
-      for (int m = 0; m < 2; ++m)
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_ss(tmem + (1 + m) * D, desc_mnmajor(smem_u32(sA) + m * 8192, 128, ks),
-                 desc_mnmajor(smem_u32(sDN) + m * 8192, 128, ks), id_a, ks > 0);
+      constexpr uint32_t id_w = idesc_bf16(128, D, 1, 1);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        mma_ss(tmem + 3 * D, desc_mnmajor(smem_u32(sH0), 128, ks),
-               desc_mnmajor(smem_u32(sDO), 128, ks), id_a, (it | ks) != 0);
-        mma_ss(tmem + 3 * D, desc_mnmajor(smem_u32(sH1), 128, ks),
-               desc_mnmajor(smem_u32(sDO), 128, ks), id_a, 1);
+        mma_ss(tmem + 3 * D, desc_mnmajor(smem_u32(sHh), 128, ks),
+               desc_mnmajor(smem_u32(sDO), 128, ks), id_w, (it | ks) != 0);
+        mma_ss(tmem + 3 * D, desc_mnmajor(smem_u32(sHl), 128, ks),
+               desc_mnmajor(smem_u32(sDO), 128, ks), id_w, 1);
       }
-      mma_commit(&bar[1]);
+      mma_commit(&bar[2]);
     }
-    ok = mbar_wait(&bar[1], it & 1, err, nullptr) && ok;
+    ok = mbar_wait(&bar[2], it & 1, err, nullptr) && ok;
     tc_fence_after();
-    // A_h rows (lane = feature a) -> summaries; a_h = sum_t phi(Q_t)[a] dden_t
-    if (warp * 32 < D) {
-      const int a = t;
-#pragma unroll 1
-      for (int m = 0; m < 2; ++m) {
-        const int b2 = 2 * p + m;
-        __nv_bfloat16* dst = summ + ((size_t(bh) * T + (b2 < T ? b2 : 0)) * D + a) * D;
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float v[32];
-          tmem_ld32(tmem + lane_base + (1 + m) * D + c0, v);
-          tmem_ld_wait();
-          if (b2 < T) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              uint4 o;
-              o.x = pack_bf16(v[e], v[e + 1]);
-              o.y = pack_bf16(v[e + 2], v[e + 3]);
-              o.z = pack_bf16(v[e + 4], v[e + 5]);
-              o.w = pack_bf16(v[e + 6], v[e + 7]);
-              *reinterpret_cast<uint4*>(dst + c0 + e) = o;
-            }
-          }
-        }
-        if (b2 < T) {
-          float acc = 0.f;
-          for (int r = 0; r < 64; ++r) {
-            const int row = m * 64 + r;
-            const uint8_t* pa = sA + (a >> 6) * 128 * 128 + sw128_offset(row, a & 63);
-            acc = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(pa)), sDd[row],
-                       acc);
-          }
-          zsum[(size_t(bh) * T + b2) * D + a] = acc;
-        }
-      }
-    }
-    tc_fence_before();
     const int failed = __syncthreads_or(!ok);  // CTA-uniform exit on a timed-out wait
     tc_fence_after();
     if (failed) break;
@@ -276,6 +248,119 @@ __global__ void __launch_bounds__(128, 1) bwd_prep_kernel(
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_free(tmem, kCols);
+}
+
+// ============================================================================ bwd_summ
+// Per 128-token tile: A_h = phi(Q_h)^T dnum_h for the two query blocks
+// (M = feature a, N = c, K = the block's 64 tokens; hi*hi + hi*lo + lo*hi),
+// written as bf16 hi/lo planes, and a_h = sum_t phi(Q_t) dden_t (fp32).
+template <int D>
+__global__ void __launch_bounds__(128, 1) bwd_summ_kernel(
+    const __nv_bfloat16* __restrict__ q, const float* __restrict__ dnum,
+    const float* __restrict__ dden, __nv_bfloat16* __restrict__ summ_hi,
+    __nv_bfloat16* __restrict__ summ_lo, float* __restrict__ zsum, int N, int T, int* err) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQh = base;                 // phi(Q) hi [t][a]
+  uint8_t* sQl = sQh + kTile32;        // phi(Q) lo
+  uint8_t* sNh = sQl + kTile32;        // dnum hi   [t][c]
+  uint8_t* sNl = sNh + kTile32;        // dnum lo
+  __shared__ float sDd[128];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tmem_base;
+  const int p = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, warp = t / 32, half = t >> 6;
+  const bool row_ok = 2 * p + half < T;
+  const size_t tok = size_t(p) * 128 + t;
+  const size_t rowoff = (size_t(bh) * N + tok) * D;
+  if (warp == 0) tmem_alloc(&tmem_base, 2 * D);
+  if (t == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  for (int c8 = 0; c8 < D / 8; ++c8) {
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (row_ok) u = *reinterpret_cast<const uint4*>(q + rowoff + c8 * 8);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a = row_ok ? phi_f(bf16_lo(w[e])) : 0.f, b = row_ok ? phi_f(bf16_hi(w[e])) : 0.f;
+      h[e] = pack_bf16(a, b);
+      l[e] = pack_bf16(a - bf16_lo(h[e]), b - bf16_hi(h[e]));
+    }
+    st_sw128_unit(sQh, 128, t, c8 * 8, make_uint4(h[0], h[1], h[2], h[3]));
+    st_sw128_unit(sQl, 128, t, c8 * 8, make_uint4(l[0], l[1], l[2], l[3]));
+  }
+  load_split_sw<D>(sNh, sNl, 128, dnum + (size_t(bh) * N + size_t(p) * 128) * D,
+                   min(128, N - p * 128), t, 128);
+  sDd[t] = row_ok ? dden[size_t(bh) * N + tok] : 0.f;
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  if (t == 0) {
+    constexpr uint32_t id = idesc_bf16(128, D, 1, 1);
+    for (int m = 0; m < 2; ++m) {
+      const uint32_t o = m * 8192;  // the block's 64 token rows inside each chunk
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t qh = desc_mnmajor(smem_u32(sQh) + o, 128, ks);
+        const uint64_t ql = desc_mnmajor(smem_u32(sQl) + o, 128, ks);
+        const uint64_t nh = desc_mnmajor(smem_u32(sNh) + o, 128, ks);
+        const uint64_t nl = desc_mnmajor(smem_u32(sNl) + o, 128, ks);
+        mma_ss(tmem + m * D, qh, nh, id, ks > 0);
+        mma_ss(tmem + m * D, qh, nl, id, 1);
+        mma_ss(tmem + m * D, ql, nh, id, 1);
+      }
+    }
+    mma_commit(&bar);
+  }
+  const bool ok = mbar_wait(&bar, 0, err, nullptr);
+  tc_fence_after();
+  if (warp * 32 < D) {
+    const int a = t;
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+#pragma unroll 1
+    for (int m = 0; m < 2; ++m) {
+      const int b2 = 2 * p + m;
+      const size_t o = ((size_t(bh) * T + (b2 < T ? b2 : 0)) * D + a) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + m * D + c0, v);
+        tmem_ld_wait();
+        if (b2 < T && ok) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint32_t h[4], l[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              h[i] = pack_bf16(v[e + 2 * i], v[e + 2 * i + 1]);
+              l[i] = pack_bf16(v[e + 2 * i] - bf16_lo(h[i]), v[e + 2 * i + 1] - bf16_hi(h[i]));
+            }
+            *reinterpret_cast<uint4*>(summ_hi + o + c0 + e) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4*>(summ_lo + o + c0 + e) = make_uint4(l[0], l[1], l[2], l[3]);
+          }
+        }
+      }
+      if (b2 < T) {
+        float acc = 0.f;
+        for (int r = 0; r < 64; ++r) {
+          const int row = m * 64 + r;
+          const uint32_t so = (a >> 6) * 128 * 128 + sw128_offset(row, a & 63);
+          const float ph = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sQh + so));
+          const float pl = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sQl + so));
+          acc = fmaf(ph + pl, sDd[row], acc);
+        }
+        zsum[(size_t(bh) * T + b2) * D + a] = acc;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_free(tmem, 2 * D);
 }
 
 // ============================================================================ bwd_sparse
@@ -526,90 +611,76 @@ __global__ void __launch_bounds__(192, 1) bwd_sparse_kernel(
 }
 
 // ============================================================================ bwd_linear
-template <int D>
-struct LinSmem {
-  static constexpr int kTile = 128 * 128 * 2;
-  static constexpr int kTotal = 1024 + 4 * kTile;
-};
-
+// Per 128-token tile (blocks 2p, 2p+1 as query blocks and as key blocks);
+// 128 threads, one row each; thread 0 issues the MMAs; the two halves' H
+// (resp. dh) pass through one shared-memory slot in turn.
+//   phase 1: dQ += ((dnum_hi + dnum_lo) (H_hi + H_lo)^T + dden Z) * phi'(Q)
+//   phase 2: dK += (V (dh_hi + dh_lo)^T + dz) * phi'(K)
+//            dV += (phi(K)_hi + phi(K)_lo) (dh_hi + dh_lo)
+// (products drop the lo*lo term).
 template <int D>
 __global__ void __launch_bounds__(128, 1) bwd_linear_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-    const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ h_agg,
-    const float* __restrict__ z_agg, const __nv_bfloat16* __restrict__ dh,
+    const __nv_bfloat16* __restrict__ v, const float* __restrict__ h_agg,
+    const float* __restrict__ z_agg, const float* __restrict__ dh,
     const float* __restrict__ dz, const float* __restrict__ dnum, const float* __restrict__ dden,
     float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dv, int N, int T,
     int* err) {
-  using L = LinSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* s0 = base;             // phase 1: dnum hi  | phase 2: V       [t][c]
-  uint8_t* s1 = s0 + L::kTile;    // phase 1: dnum lo  | phase 2: phi(K)  [t][a]
-  uint8_t* s2 = s1 + L::kTile;    // phase 1: H_{2p}   | phase 2: dh_{2p}   [a][c]
-  uint8_t* s3 = s2 + L::kTile;    // phase 1: H_{2p+1} | phase 2: dh_{2p+1} [a][c]
+  uint8_t* s0 = base;             // phase 1: dnum hi | phase 2: V        [t][c]
+  uint8_t* s1 = s0 + kTile32;     // phase 1: dnum lo | phase 2: phi(K) hi [t][a]
+  uint8_t* s2 = s1 + kTile32;     //                    phase 2: phi(K) lo [t][a]
+  uint8_t* sMh = s2 + kTile32;    // H / dh hi [a][c]
+  uint8_t* sMl = sMh + kTile32;   // H / dh lo [a][c]
   __shared__ float sZ[2][D];
-  __shared__ uint64_t bar[2];
+  __shared__ uint64_t bar[4];
   __shared__ uint32_t tmem_base;
   const int p = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, warp = t / 32, half = t >> 6;
-  const int blk = 2 * p + half;
-  const bool row_ok = blk < T;
+  const bool row_ok = 2 * p + half < T;
   const size_t tok = size_t(p) * 128 + t;
   const size_t rowoff = (size_t(bh) * N + tok) * D;
   const uint32_t lane_base = uint32_t(warp * 32) << 16;
   constexpr uint32_t kCols = 4 * D;
   if (warp == 0) tmem_alloc(&tmem_base, kCols);
   if (t == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+    for (int b = 0; b < 4; ++b) mbar_init(&bar[b], 1);
     fence_barrier_init();
   }
-  // ---------------- phase 1: dQ_l = (dnum H^T + dden Z) * phi'(Q)
-  for (int m = 0; m < 2; ++m) {
-    const int b2 = 2 * p + m;
-    load_rows_sw<D>(m ? s3 : s2, D, h_agg + (size_t(bh) * T + (b2 < T ? b2 : 0)) * D * D,
-                    b2 < T ? D : 0, t, 128);
-  }
+  // ---------------- phase 1: dQ
+  load_split_sw<D>(s0, s1, 128, dnum + (size_t(bh) * N + size_t(p) * 128) * D,
+                   min(128, N - p * 128), t, 128);
   for (int e = t; e < 2 * D; e += 128) {
     const int b2 = 2 * p + e / D;
     sZ[e / D][e % D] = b2 < T ? z_agg[(size_t(bh) * T + b2) * D + e % D] : 0.f;
   }
-  for (int c8 = 0; c8 < D / 8; ++c8) {
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-    if (row_ok) {
-      a = *reinterpret_cast<const float4*>(dnum + rowoff + c8 * 8);
-      b = *reinterpret_cast<const float4*>(dnum + rowoff + c8 * 8 + 4);
-    }
-    const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    uint32_t hi[4], lo[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      hi[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
-      lo[e] = pack_bf16(x[2 * e] - bf16_lo(hi[e]), x[2 * e + 1] - bf16_hi(hi[e]));
-    }
-    st_sw128_unit(s0, 128, t, c8 * 8, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-    st_sw128_unit(s1, 128, t, c8 * 8, make_uint4(lo[0], lo[1], lo[2], lo[3]));
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base;
-  if (t == 0) {
-    constexpr uint32_t id = idesc_bf16(128, D, 0, 0);
-    for (int m = 0; m < 2; ++m) {
-      const uint32_t hb = smem_u32(m ? s3 : s2);
+  bool ok = true;
+  for (int m = 0; m < 2; ++m) {
+    const int b2 = 2 * p + m;
+    load_split_sw<D>(sMh, sMl, D, h_agg + (size_t(bh) * T + (b2 < T ? b2 : 0)) * D * D,
+                     b2 < T ? D : 0, t, 128);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (t == 0) {
+      constexpr uint32_t id = idesc_bf16(128, D, 0, 0);
+      const uint32_t hh = smem_u32(sMh), hl = smem_u32(sMl);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
-        mma_ss(tmem + m * D, desc_kmajor(smem_u32(s0), 128, ks), desc_kmajor(hb, D, ks), id,
-               ks > 0);
-        mma_ss(tmem + m * D, desc_kmajor(smem_u32(s1), 128, ks), desc_kmajor(hb, D, ks), id, 1);
+        const uint64_t ah = desc_kmajor(smem_u32(s0), 128, ks);
+        const uint64_t al = desc_kmajor(smem_u32(s1), 128, ks);
+        mma_ss(tmem_base + m * D, ah, desc_kmajor(hh, D, ks), id, ks > 0);
+        mma_ss(tmem_base + m * D, ah, desc_kmajor(hl, D, ks), id, 1);
+        mma_ss(tmem_base + m * D, al, desc_kmajor(hh, D, ks), id, 1);
       }
+      mma_commit(&bar[m]);
     }
-    mma_commit(&bar[0]);
+    ok = mbar_wait(&bar[m], 0, err, nullptr) && ok;
+    tc_fence_after();
   }
-  bool ok = mbar_wait(&bar[0], 0, err, nullptr);
-  tc_fence_after();
+  const uint32_t tmem = tmem_base;
   {
     const float ddn = row_ok ? dden[size_t(bh) * N + tok] : 0.f;
 #pragma unroll 1
@@ -625,12 +696,10 @@ __global__ void __launch_bounds__(128, 1) bwd_linear_kernel(
 #pragma unroll
         for (int e = 0; e < 16; e += 4) {
           float4 cur = *reinterpret_cast<float4*>(dst + e);
-          const float qa = bf16_lo(w[e / 2]), qb = bf16_hi(w[e / 2]);
-          const float qc = bf16_lo(w[e / 2 + 1]), qd = bf16_hi(w[e / 2 + 1]);
-          cur.x += (g[e] + ddn * sZ[half][c0 + e]) * dphi_f(qa);
-          cur.y += (g[e + 1] + ddn * sZ[half][c0 + e + 1]) * dphi_f(qb);
-          cur.z += (g[e + 2] + ddn * sZ[half][c0 + e + 2]) * dphi_f(qc);
-          cur.w += (g[e + 3] + ddn * sZ[half][c0 + e + 3]) * dphi_f(qd);
+          cur.x += (g[e] + ddn * sZ[half][c0 + e]) * dphi_f(bf16_lo(w[e / 2]));
+          cur.y += (g[e + 1] + ddn * sZ[half][c0 + e + 1]) * dphi_f(bf16_hi(w[e / 2]));
+          cur.z += (g[e + 2] + ddn * sZ[half][c0 + e + 2]) * dphi_f(bf16_lo(w[e / 2 + 1]));
+          cur.w += (g[e + 3] + ddn * sZ[half][c0 + e + 3]) * dphi_f(bf16_hi(w[e / 2 + 1]));
           *reinterpret_cast<float4*>(dst + e) = cur;
         }
       }
@@ -639,12 +708,7 @@ __global__ void __launch_bounds__(128, 1) bwd_linear_kernel(
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // ---------------- phase 2: dK_l = (V dh^T + dz) * phi'(K),  dV_l = phi(K) dh
-  for (int m = 0; m < 2; ++m) {
-    const int b2 = 2 * p + m;
-    load_rows_sw<D>(m ? s3 : s2, D, dh + (size_t(bh) * T + (b2 < T ? b2 : 0)) * D * D,
-                    b2 < T ? D : 0, t, 128);
-  }
+  // ---------------- phase 2: dK, dV
   for (int e = t; e < 2 * D; e += 128) {
     const int b2 = 2 * p + e / D;
     sZ[e / D][e % D] = b2 < T ? dz[(size_t(bh) * T + b2) * D + e % D] : 0.f;
@@ -657,32 +721,44 @@ __global__ void __launch_bounds__(128, 1) bwd_linear_kernel(
     }
     st_sw128_unit(s0, 128, t, c8 * 8, uv);
     const uint32_t w[4] = {uk.x, uk.y, uk.z, uk.w};
-    uint32_t pw[4];
+    uint32_t h[4], l[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) pw[e] = pack_bf16(phi_f(bf16_lo(w[e])), phi_f(bf16_hi(w[e])));
-    st_sw128_unit(s1, 128, t, c8 * 8, make_uint4(pw[0], pw[1], pw[2], pw[3]));
+    for (int e = 0; e < 4; ++e) {
+      const float a = phi_f(bf16_lo(w[e])), b = phi_f(bf16_hi(w[e]));
+      h[e] = pack_bf16(a, b);
+      l[e] = pack_bf16(a - bf16_lo(h[e]), b - bf16_hi(h[e]));
+    }
+    st_sw128_unit(s1, 128, t, c8 * 8, make_uint4(h[0], h[1], h[2], h[3]));
+    st_sw128_unit(s2, 128, t, c8 * 8, make_uint4(l[0], l[1], l[2], l[3]));
   }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (t == 0) {
-    constexpr uint32_t id_k = idesc_bf16(128, D, 0, 0);
-    constexpr uint32_t id_v = idesc_bf16(128, D, 0, 1);
-    for (int m = 0; m < 2; ++m) {
-      const uint32_t hb = smem_u32(m ? s3 : s2);
+  for (int m = 0; m < 2; ++m) {
+    const int b2 = 2 * p + m;
+    load_split_sw<D>(sMh, sMl, D, dh + (size_t(bh) * T + (b2 < T ? b2 : 0)) * D * D,
+                     b2 < T ? D : 0, t, 128);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (t == 0) {
+      constexpr uint32_t id_k = idesc_bf16(128, D, 0, 0);
+      constexpr uint32_t id_v = idesc_bf16(128, D, 0, 1);
+      const uint32_t hh = smem_u32(sMh), hl = smem_u32(sMl);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
-        mma_ss(tmem + m * D, desc_kmajor(smem_u32(s0), 128, ks), desc_kmajor(hb, D, ks), id_k,
-               ks > 0);
-        mma_ss(tmem + (2 + m) * D, desc_kmajor(smem_u32(s1), 128, ks), desc_mnmajor(hb, D, ks),
-               id_v, ks > 0);
+        const uint64_t av = desc_kmajor(smem_u32(s0), 128, ks);
+        const uint64_t kh = desc_kmajor(smem_u32(s1), 128, ks);
+        const uint64_t kl = desc_kmajor(smem_u32(s2), 128, ks);
+        mma_ss(tmem + m * D, av, desc_kmajor(hh, D, ks), id_k, ks > 0);
+        mma_ss(tmem + m * D, av, desc_kmajor(hl, D, ks), id_k, 1);
+        mma_ss(tmem + (2 + m) * D, kh, desc_mnmajor(hh, D, ks), id_v, ks > 0);
+        mma_ss(tmem + (2 + m) * D, kh, desc_mnmajor(hl, D, ks), id_v, 1);
+        mma_ss(tmem + (2 + m) * D, kl, desc_mnmajor(hh, D, ks), id_v, 1);
       }
+      mma_commit(&bar[2 + m]);
     }
-    mma_commit(&bar[1]);
+    ok = mbar_wait(&bar[2 + m], 0, err, nullptr) && ok;
+    tc_fence_after();
   }
-  ok = mbar_wait(&bar[1], 0, err, nullptr) && ok;
-  tc_fence_after();
 #pragma unroll 1
   for (int c0 = 0; c0 < D; c0 += 16) {
     float gk[16], gv[16];
@@ -725,25 +801,42 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }  // namespace
 
 cudaError_t launch_bwd_prep(const Problem& p, const void* q, const void* d_o, const void* w_proj,
-                            const float* o_s, const float* den, const __nv_bfloat16* h_agg,
-                            const float* z_agg, float* dvec, float* dnum, float* dden,
-                            __nv_bfloat16* summ, float* zsum, float* dw, int num_sms, int* err,
+                            const float* o_s, const float* den, const float* h_agg, float* dvec,
+                            float* dnum, float* dden, float* dw, int num_sms, int* err,
                             cudaStream_t s) {
   const int tiles = ((p.T + 1) / 2) * p.BH;
   const int grid = tiles < num_sms ? tiles : num_sms;
+  const size_t smem = 1024 + 5 * kTile32;
   cudaError_t e;
-#define SLA_PREP(DD)                                                                         \
-  e = set_smem(bwd_prep_kernel<DD>, PrepSmem<DD>::kTotal);                                  \
-  if (e != cudaSuccess) return e;                                                            \
-  bwd_prep_kernel<DD><<<grid, 128, PrepSmem<DD>::kTotal, s>>>(                               \
-      (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o, (const __nv_bfloat16*)w_proj, o_s, \
-      den, h_agg, z_agg, dvec, dnum, dden, summ, zsum, dw, p.N, p.T, p.BH, err);
   if (p.d == 128) {
-    SLA_PREP(128)
+    if ((e = set_smem(bwd_prep_kernel<128>, smem)) != cudaSuccess) return e;
+    bwd_prep_kernel<128><<<grid, 128, smem, s>>>(
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o, (const __nv_bfloat16*)w_proj, o_s,
+        den, h_agg, dvec, dnum, dden, dw, p.N, p.T, p.BH, err);
   } else {
-    SLA_PREP(64)
+    if ((e = set_smem(bwd_prep_kernel<64>, smem)) != cudaSuccess) return e;
+    bwd_prep_kernel<64><<<grid, 128, smem, s>>>(
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o, (const __nv_bfloat16*)w_proj, o_s,
+        den, h_agg, dvec, dnum, dden, dw, p.N, p.T, p.BH, err);
   }
-#undef SLA_PREP
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_summ(const Problem& p, const void* q, const float* dnum,
+                            const float* dden, __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo,
+                            float* zsum, int* err, cudaStream_t s) {
+  dim3 grid((p.T + 1) / 2, p.BH);
+  const size_t smem = 1024 + 4 * kTile32;
+  cudaError_t e;
+  if (p.d == 128) {
+    if ((e = set_smem(bwd_summ_kernel<128>, smem)) != cudaSuccess) return e;
+    bwd_summ_kernel<128><<<grid, 128, smem, s>>>((const __nv_bfloat16*)q, dnum, dden, summ_hi,
+                                                 summ_lo, zsum, p.N, p.T, err);
+  } else {
+    if ((e = set_smem(bwd_summ_kernel<64>, smem)) != cudaSuccess) return e;
+    bwd_summ_kernel<64><<<grid, 128, smem, s>>>((const __nv_bfloat16*)q, dnum, dden, summ_hi,
+                                                summ_lo, zsum, p.N, p.T, err);
+  }
   return cudaGetLastError();
 }
 
@@ -777,24 +870,23 @@ cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, co
 }
 
 cudaError_t launch_bwd_linear(const Problem& p, const void* q, const void* k, const void* v,
-                              const __nv_bfloat16* h_agg, const float* z_agg,
-                              const __nv_bfloat16* dh, const float* dz, const float* dnum,
-                              const float* dden, float* dq, float* dk, float* dv, int* err,
-                              cudaStream_t s) {
+                              const float* h_agg, const float* z_agg, const float* dh,
+                              const float* dz, const float* dnum, const float* dden, float* dq,
+                              float* dk, float* dv, int* err, cudaStream_t s) {
   dim3 grid((p.T + 1) / 2, p.BH);
+  const size_t smem = 1024 + 5 * kTile32;
   cudaError_t e;
-#define SLA_LIN(DD)                                                                          \
-  e = set_smem(bwd_linear_kernel<DD>, LinSmem<DD>::kTotal);                                 \
-  if (e != cudaSuccess) return e;                                                            \
-  bwd_linear_kernel<DD><<<grid, 128, LinSmem<DD>::kTotal, s>>>(                              \
-      (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, h_agg, z_agg, \
-      dh, dz, dnum, dden, dq, dk, dv, p.N, p.T, err);
   if (p.d == 128) {
-    SLA_LIN(128)
+    if ((e = set_smem(bwd_linear_kernel<128>, smem)) != cudaSuccess) return e;
+    bwd_linear_kernel<128><<<grid, 128, smem, s>>>(
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, h_agg, z_agg,
+        dh, dz, dnum, dden, dq, dk, dv, p.N, p.T, err);
   } else {
-    SLA_LIN(64)
+    if ((e = set_smem(bwd_linear_kernel<64>, smem)) != cudaSuccess) return e;
+    bwd_linear_kernel<64><<<grid, 128, smem, s>>>(
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, h_agg, z_agg,
+        dh, dz, dnum, dden, dq, dk, dv, p.N, p.T, err);
   }
-#undef SLA_LIN
   return cudaGetLastError();
 }
 

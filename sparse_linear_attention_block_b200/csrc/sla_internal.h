@@ -26,9 +26,10 @@ struct WorkspaceLayout {
   size_t err;        // int32 device error word (+ padding)
   size_t qbar;       // fp32 [BH,T,d]   pooled Q
   size_t kbar;       // fp32 [BH,T,d]   pooled K
-  size_t summ;       // bf16 [BH,T,d*d] h_j (forward) / dH_i contributions A_i (backward)
+  size_t summ_hi;    // bf16 [BH,T,d*d] h_j (forward) / A_i (backward), high part
+  size_t summ_lo;    // bf16 [BH,T,d*d] the low part (value = hi + lo)
   size_t zsum;       // fp32 [BH,T,d]   z_j (forward) / a_i (backward)
-  size_t dh;         // bf16 [BH,T,d*d] dh_j (backward)
+  size_t dh;         // fp32 [BH,T,d*d] dh_j (backward)
   size_t dz;         // fp32 [BH,T,d]   dz_j (backward)
   size_t mmat;       // bf16 [BH,Tp,Tp] marginal 0/1 matrix, rows = query blocks
   size_t mmat_t;     // bf16 [BH,Tp,Tp] its transpose
@@ -58,33 +59,34 @@ cudaError_t launch_crit_csr(const Problem& p, const int8_t* cls, int32_t* col_pt
 cudaError_t launch_expand_marginal(const Problem& p, const uint32_t* marg_bits,
                                    __nv_bfloat16* mmat, __nv_bfloat16* mmat_t, cudaStream_t s);
 cudaError_t launch_summaries(const Problem& p, const void* k, const void* v,
-                             __nv_bfloat16* summ, float* zsum, int* err, cudaStream_t s);
+                             __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* zsum,
+                             int* err, cudaStream_t s);
 cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
-                             const __nv_bfloat16* summ, __nv_bfloat16* out, int* err,
-                             cudaStream_t s);
+                             const __nv_bfloat16* summ_hi, const __nv_bfloat16* summ_lo,
+                             float* out, int* err, cudaStream_t s);
 cudaError_t launch_aggregate_z(const Problem& p, const uint32_t* marg_bits, const float* z,
                                float* zout, bool transpose, cudaStream_t s);
 cudaError_t launch_fwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
                               const int32_t* crit_idx, float* o_s, float* lse, int* err,
                               cudaStream_t s);
-cudaError_t launch_fwd_linear(const Problem& p, const void* q, const __nv_bfloat16* h_agg,
+cudaError_t launch_fwd_linear(const Problem& p, const void* q, const float* h_agg,
                               const float* z_agg, const void* w_proj, const float* o_s,
                               void* o, float* den, int* err, cudaStream_t s);
-
 cudaError_t launch_bwd_prep(const Problem& p, const void* q, const void* d_o, const void* w_proj,
-                            const float* o_s, const float* den, const __nv_bfloat16* h_agg,
-                            const float* z_agg, float* dvec, float* dnum, float* dden,
-                            __nv_bfloat16* summ, float* zsum, float* dw, int num_sms, int* err,
+                            const float* o_s, const float* den, const float* h_agg, float* dvec,
+                            float* dnum, float* dden, float* dw, int num_sms, int* err,
                             cudaStream_t s);
+cudaError_t launch_bwd_summ(const Problem& p, const void* q, const float* dnum,
+                            const float* dden, __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo,
+                            float* zsum, int* err, cudaStream_t s);
 cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
                               const void* d_o, const float* lse, const float* dvec,
                               const int32_t* col_ptr, const int32_t* col_idx, float* dq,
                               float* dk, float* dv, int* err, cudaStream_t s);
 cudaError_t launch_bwd_linear(const Problem& p, const void* q, const void* k, const void* v,
-                              const __nv_bfloat16* h_agg, const float* z_agg,
-                              const __nv_bfloat16* dh, const float* dz, const float* dnum,
-                              const float* dden, float* dq, float* dk, float* dv, int* err,
-                              cudaStream_t s);
+                              const float* h_agg, const float* z_agg, const float* dh,
+                              const float* dz, const float* dnum, const float* dden, float* dq,
+                              float* dk, float* dv, int* err, cudaStream_t s);
 
 // TMA descriptor for a bf16 [BH, N, d] tensor viewed as 3D {d, N, BH} with a
 // box of {64, rows, 1} and 128-byte swizzle.  Returns false on failure.

@@ -6,11 +6,17 @@
 // per query block H_i = sum of h_j over its marginal key blocks (Z_i alike),
 // O_l = phi(Q) H_i / (phi(Q) . Z_i), and O = O_s + O_l W_proj.
 //
+// Precision.  The gradient through phi(Q) involves H_i - O_l Z_i, a
+// difference of nearly equal terms, so the linear branch keeps ~16 mantissa
+// bits: fp32 values x are carried as a bf16 pair x = hi + lo and products use
+// hi*hi + hi*lo + lo*hi (the 0/1 marginal matrix is exact in bf16, so the
+// aggregation needs only M*h_hi + M*h_lo).  Accumulation is fp32 in TMEM.
+//
 // Kernels:
-//   summaries_kernel   h_j (tcgen05, bf16 out) and z_j (fp32)      HBM-bound
-//   agg_gemm_kernel    H = M_marg * h as a dense GEMM per head      tensor/HBM
-//   agg_z_kernel       Z_i = sum of z_j over marginal j            small
-//   fwd_linear_kernel  O = O_s + (phi(Q) H_i / den) W_proj         HBM-bound
+//   summaries_kernel   h_j as bf16 hi/lo planes (tcgen05), z_j fp32     HBM-bound
+//   agg_gemm_kernel    fp32 C = M * (B_hi + B_lo), M the 0/1 matrix      tensor/HBM
+//   agg_z_kernel       Z_i = sum of z_j over marginal j                 small
+//   fwd_linear_kernel  O = O_s + (phi(Q) H_i / den) W_proj              HBM-bound
 #include <cuda_bf16.h>
 
 #include "sla_internal.h"
@@ -23,13 +29,14 @@ __device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : __e
 
 // ------------------------------------------------------------------ summaries
 // One CTA per (key block j, head); 128 threads.  phi(K_j)^T (M = feature a,
-// K = token) and V_j (N = c, K = token) are written MN-major into swizzled
-// shared memory and multiplied by one thread with tcgen05 (M=128, N=D,
-// K=64); for D = 64 the M dimension is zero-padded to 128.
+// K = token; as hi and lo bf16 tiles) and V_j (N = c) are written MN-major
+// into swizzled shared memory; h_j = phi_hi^T V + phi_lo^T V by tcgen05
+// (M=128, N=D, K=64; for D = 64 the M dimension is zero-padded to 128).
 template <int D>
 __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __restrict__ k,
                                                         const __nv_bfloat16* __restrict__ v,
-                                                        __nv_bfloat16* __restrict__ summ,
+                                                        __nv_bfloat16* __restrict__ summ_hi,
+                                                        __nv_bfloat16* __restrict__ summ_lo,
                                                         float* __restrict__ zsum, int N, int T,
                                                         int* err) {
   constexpr int kChunks = D / 8;
@@ -38,8 +45,9 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sPhiK = base;             // 2 chunks x 64 rows x 128 B = 16 KB (M padded to 128)
-  uint8_t* sV = base + 16384;        // D/64 chunks x 8 KB
+  uint8_t* sPhiH = base;           // 2 chunks x 64 rows x 128 B = 16 KB (M padded to 128)
+  uint8_t* sPhiL = base + 16384;   // same for the lo part
+  uint8_t* sV = base + 32768;      // D/64 chunks x 8 KB
   float* zred = reinterpret_cast<float*>(sV + (D / 64) * 8192);  // [kGroups][D]
   __shared__ uint64_t bar;
   __shared__ uint32_t tmem_base;
@@ -50,9 +58,12 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
     mbar_init(&bar, 1);
     fence_barrier_init();
   }
-  if (D == 64) {  // zero the padding chunk (features 64..127)
-    uint4 z = make_uint4(0, 0, 0, 0);
-    for (int e = t; e < 8192 / 16; e += 128) reinterpret_cast<uint4*>(sPhiK + 8192)[e] = z;
+  if (D == 64) {  // zero the padding chunks (features 64..127)
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int e = t; e < 8192 / 16; e += 128) {
+      reinterpret_cast<uint4*>(sPhiH + 8192)[e] = z;
+      reinterpret_cast<uint4*>(sPhiL + 8192)[e] = z;
+    }
   }
   const int c8 = t % kChunks, g = t / kChunks;
   const size_t off = (size_t(bh) * N + size_t(j) * kBlock) * D;
@@ -63,15 +74,17 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
     const uint4 uk = *reinterpret_cast<const uint4*>(k + off + size_t(row) * D + c8 * 8);
     const uint4 uv = *reinterpret_cast<const uint4*>(v + off + size_t(row) * D + c8 * 8);
     const uint32_t w[4] = {uk.x, uk.y, uk.z, uk.w};
-    uint32_t pw[4];
+    uint32_t ph[4], pl[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float a = phi_f(bf16_lo(w[e])), b = phi_f(bf16_hi(w[e]));
       zacc[2 * e] += a;
       zacc[2 * e + 1] += b;
-      pw[e] = pack_bf16(a, b);
+      ph[e] = pack_bf16(a, b);
+      pl[e] = pack_bf16(a - bf16_lo(ph[e]), b - bf16_hi(ph[e]));
     }
-    st_sw128_unit(sPhiK, 64, row, c8 * 8, make_uint4(pw[0], pw[1], pw[2], pw[3]));
+    st_sw128_unit(sPhiH, 64, row, c8 * 8, make_uint4(ph[0], ph[1], ph[2], ph[3]));
+    st_sw128_unit(sPhiL, 64, row, c8 * 8, make_uint4(pl[0], pl[1], pl[2], pl[3]));
     st_sw128_unit(sV, 64, row, c8 * 8, uv);
   }
 #pragma unroll
@@ -83,13 +96,14 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
   const uint32_t tmem = tmem_base;
   if (t == 0) {
     constexpr uint32_t idesc = idesc_bf16(128, D, 1, 1);
-    const uint32_t a0 = smem_u32(sPhiK), b0 = smem_u32(sV);
+    const uint32_t ah = smem_u32(sPhiH), al = smem_u32(sPhiL), b0 = smem_u32(sV);
 #pragma unroll
-    for (int ks = 0; ks < kBlock / 16; ++ks)
-      mma_ss(tmem, desc_mnmajor(a0, 64, ks), desc_mnmajor(b0, 64, ks), idesc, ks > 0);
+    for (int ks = 0; ks < kBlock / 16; ++ks) {
+      mma_ss(tmem, desc_mnmajor(ah, 64, ks), desc_mnmajor(b0, 64, ks), idesc, ks > 0);
+      mma_ss(tmem, desc_mnmajor(al, 64, ks), desc_mnmajor(b0, 64, ks), idesc, 1);
+    }
     mma_commit(&bar);
   }
-  // z_j while the MMA runs
   if (t < D) {
     float s = 0.f;
 #pragma unroll
@@ -100,20 +114,23 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
   tc_fence_after();
   if (ok && warp * 32 < D) {
     const int a = warp * 32 + lane_id();
-    __nv_bfloat16* dst = summ + ((size_t(bh) * T + j) * D + a) * D;
-#pragma unroll
+    const size_t o = ((size_t(bh) * T + j) * D + a) * D;
+#pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       float vals[32];
       tmem_ld32(tmem_addr(tmem, warp * 32, c0), vals);
       tmem_ld_wait();
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        uint4 o;
-        o.x = pack_bf16(vals[q4 * 8 + 0], vals[q4 * 8 + 1]);
-        o.y = pack_bf16(vals[q4 * 8 + 2], vals[q4 * 8 + 3]);
-        o.z = pack_bf16(vals[q4 * 8 + 4], vals[q4 * 8 + 5]);
-        o.w = pack_bf16(vals[q4 * 8 + 6], vals[q4 * 8 + 7]);
-        *reinterpret_cast<uint4*>(dst + c0 + q4 * 8) = o;
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = vals[q4 * 8 + 2 * e], x1 = vals[q4 * 8 + 2 * e + 1];
+          hi[e] = pack_bf16(x0, x1);
+          lo[e] = pack_bf16(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
+        }
+        *reinterpret_cast<uint4*>(summ_hi + o + c0 + q4 * 8) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(summ_lo + o + c0 + q4 * 8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
     }
   }
@@ -123,17 +140,21 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
 }
 
 // ------------------------------------------------------------------ aggregation GEMM
-// C[bh][i][n] = sum_k A[bh][i][k] * B[bh][k][n] with A the bf16 0/1 marginal
-// matrix [Tp x Tp] (K-major) and B the per-block summaries [T x NN]
-// (MN-major), C bf16 [T x NN].  Tile 128 x 128 x 64, 3-stage TMA ring,
-// warp 0 = TMA producer, warp 1 = MMA issuer, all 4 warps = epilogue.
-constexpr int kAggBN = 128, kAggBK = 64, kAggStages = 3;
-constexpr int kAggStageBytes = 128 * kAggBK * 2 + kAggBK * kAggBN * 2;  // 32 KB
+// C[bh][i][n] = sum_k A[bh][i][k] * (Bhi + Blo)[bh][k][n] with A the bf16 0/1
+// marginal matrix [Tp x Tp] (K-major), B the per-block summaries [T x NN]
+// as bf16 hi/lo planes (MN-major), C fp32 [T x NN].  Tile 128 x 128 x 64,
+// 2-stage TMA ring, warp 0 = TMA producer, warp 1 = MMA issuer, all 4 warps
+// = epilogue.  Two CTAs per SM overlap one's epilogue with the other's MMAs.
+constexpr int kAggBN = 128, kAggBK = 64, kAggStages = 2;
+constexpr int kAggA = 128 * kAggBK * 2;        // 16 KB
+constexpr int kAggB = kAggBK * kAggBN * 2;     // 16 KB per plane
+constexpr int kAggStageBytes = kAggA + 2 * kAggB;
 
 __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
-                                                       const __grid_constant__ CUtensorMap tm_b,
-                                                       __nv_bfloat16* __restrict__ out, int T,
-                                                       int Tp, int NN, int* err) {
+                                                       const __grid_constant__ CUtensorMap tm_bh,
+                                                       const __grid_constant__ CUtensorMap tm_bl,
+                                                       float* __restrict__ out, int T, int Tp,
+                                                       int NN, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -160,19 +181,27 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
 
   if (warp == 0 && lane_id() == 0) {
     tma_prefetch_desc(&tm_a);
-    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_bh);
+    tma_prefetch_desc(&tm_bl);
+    int issued = 0;
     for (int kt = 0; kt < nk; ++kt) {
       const int s = kt % kAggStages;
       if (kt >= kAggStages &&
           !mbar_wait(&empty[s], ((kt / kAggStages) + 1) & 1, err, &abort_flag))
         break;
       uint8_t* sa = base + s * kAggStageBytes;
-      uint8_t* sb = sa + 128 * kAggBK * 2;
+      uint8_t* sb = sa + kAggA;
       mbar_arrive_expect_tx(&full[s], kAggStageBytes);
       tma_load_3d(sa, &full[s], &tm_a, kt * kAggBK, mt * 128, bh);
-      tma_load_3d(sb, &full[s], &tm_b, nt * kAggBN, kt * kAggBK, bh);
-      tma_load_3d(sb + kAggBK * 128, &full[s], &tm_b, nt * kAggBN + 64, kt * kAggBK, bh);
+      for (int c = 0; c < 2; ++c) {
+        tma_load_3d(sb + c * 8192, &full[s], &tm_bh, nt * kAggBN + c * 64, kt * kAggBK, bh);
+        tma_load_3d(sb + kAggB + c * 8192, &full[s], &tm_bl, nt * kAggBN + c * 64, kt * kAggBK, bh);
+      }
+      ++issued;
     }
+    if (abort_flag)
+      for (int kt = (issued > kAggStages ? issued - kAggStages : 0); kt < issued; ++kt)
+        mbar_wait(&full[kt % kAggStages], (kt / kAggStages) & 1, nullptr, nullptr);
   } else if (warp == 1 && lane_id() == 0) {
     constexpr uint32_t idesc = idesc_bf16(128, kAggBN, 0, 1);
     for (int kt = 0; kt < nk; ++kt) {
@@ -180,11 +209,13 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
       if (!mbar_wait(&full[s], (kt / kAggStages) & 1, err, &abort_flag)) break;
       tc_fence_after();
       const uint32_t sa = smem_u32(base + s * kAggStageBytes);
-      const uint32_t sb = sa + 128 * kAggBK * 2;
+      const uint32_t sb = sa + kAggA;
 #pragma unroll
-      for (int ks = 0; ks < kAggBK / 16; ++ks)
+      for (int ks = 0; ks < kAggBK / 16; ++ks) {
         mma_ss(tmem, desc_kmajor(sa, 128, ks), desc_mnmajor(sb, kAggBK, ks), idesc,
                (kt | ks) != 0);
+        mma_ss(tmem, desc_kmajor(sa, 128, ks), desc_mnmajor(sb + kAggB, kAggBK, ks), idesc, 1);
+      }
       mma_commit(&empty[s]);
     }
     mma_commit(&acc_bar);
@@ -194,7 +225,7 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
   tc_fence_after();
   const int i = mt * 128 + warp * 32 + lane_id();
   if (ok) {
-    __nv_bfloat16* dst = out + (size_t(bh) * T + i) * NN + size_t(nt) * kAggBN;
+    float* dst = out + (size_t(bh) * T + i) * NN + size_t(nt) * kAggBN;
 #pragma unroll 1
     for (int c0 = 0; c0 < kAggBN; c0 += 32) {
       float vals[32];
@@ -202,14 +233,9 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
       tmem_ld_wait();
       if (i < T) {
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint4 o;
-          o.x = pack_bf16(vals[q4 * 8 + 0], vals[q4 * 8 + 1]);
-          o.y = pack_bf16(vals[q4 * 8 + 2], vals[q4 * 8 + 3]);
-          o.z = pack_bf16(vals[q4 * 8 + 4], vals[q4 * 8 + 5]);
-          o.w = pack_bf16(vals[q4 * 8 + 6], vals[q4 * 8 + 7]);
-          *reinterpret_cast<uint4*>(dst + c0 + q4 * 8) = o;
-        }
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst + c0 + e) =
+              make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
       }
     }
   }
@@ -246,26 +272,26 @@ __global__ void agg_z_kernel(const uint32_t* __restrict__ marg_bits, const float
 
 // ------------------------------------------------------------------ linear forward epilogue
 // One CTA per pair of query blocks (128 tokens); 128 threads, one row each.
-//   NUM_h = phi(Q) H_{2p+h}  (tcgen05, both halves for all rows; each row
-//   keeps its own half), den = phi(Q) . Z (fp32), O_l = NUM / den,
-//   O = O_s + O_l W_proj with O_l split into bf16 hi + lo for the product.
+//   NUM_h = phi(Q) (H_{2p+h,hi} + H_{2p+h,lo})   (tcgen05; the two halves in
+//   turn, each row keeps its own), den = phi(Q) . Z (fp32), O_l = NUM / den,
+//   O = O_s + (O_l,hi + O_l,lo) W_proj.
 template <int D>
 __global__ void __launch_bounds__(128, 1) fwd_linear_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ h_agg,
+    const __nv_bfloat16* __restrict__ q, const float* __restrict__ h_agg,
     const float* __restrict__ z_agg, const __nv_bfloat16* __restrict__ w_proj,
     const float* __restrict__ o_s, __nv_bfloat16* __restrict__ o, float* __restrict__ den_out,
     int N, int T, int* err) {
-  constexpr int kTile = 128 * D * 2;  // one 128 x D bf16 operand
-  constexpr int kMat = D * D * 2;     // one D x D bf16 operand
+  constexpr int kTile = 128 * 128 * 2;  // 128 rows x 2 chunks (D = 64 padded)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sA = base;                  // phi(Q), later O_l hi   (K-major, 128 rows)
-  uint8_t* sA2 = sA + kTile;           // O_l lo                 (K-major, 128 rows)
-  uint8_t* sH = sA2 + kTile;           // H_{2p}, H_{2p+1}       (MN-major, D k-rows)
-  uint8_t* sW = sH + 2 * kMat;         // W_proj                 (MN-major, D k-rows)
-  float* sZ = reinterpret_cast<float*>(sW + kMat);  // [2][D]
-  __shared__ uint64_t bar[2];
+  uint8_t* sA = base;                  // phi(Q), later O_l hi    (K-major, 128 rows)
+  uint8_t* sA2 = sA + kTile;           // O_l lo                  (K-major, 128 rows)
+  uint8_t* sHh = sA2 + kTile;          // H hi                    (MN-major, D k-rows)
+  uint8_t* sHl = sHh + kTile;          // H lo
+  uint8_t* sW = sHl + kTile;           // W_proj                  (MN-major, D k-rows)
+  __shared__ float sZ[2][D];
+  __shared__ uint64_t bar[3];
   __shared__ uint32_t tmem_base;
   const int p = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, warp = t / 32;
   const int half = t >> 6;
@@ -274,35 +300,22 @@ __global__ void __launch_bounds__(128, 1) fwd_linear_kernel(
   const size_t tok = size_t(p) * 128 + t;
   if (warp == 0) tmem_alloc(&tmem_base, 2 * D);
   if (t == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+    for (int b = 0; b < 3; ++b) mbar_init(&bar[b], 1);
     fence_barrier_init();
   }
-  // H_{2p}, H_{2p+1} and W_proj into MN-major swizzled tiles (rows = a)
-  for (int e = t; e < 3 * D * (D / 8); e += 128) {
-    const int m = e / (D * (D / 8)), rem = e % (D * (D / 8));
-    const int a = rem / (D / 8), c8 = rem % (D / 8);
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (m < 2) {
-      const int b2 = 2 * p + m;
-      if (b2 < T)
-        u = *reinterpret_cast<const uint4*>(h_agg + ((size_t(bh) * T + b2) * D + a) * D + c8 * 8);
-      st_sw128_unit(sH + m * kMat, D, a, c8 * 8, u);
-    } else {
-      u = *reinterpret_cast<const uint4*>(w_proj + size_t(a) * D + c8 * 8);
-      st_sw128_unit(sW, D, a, c8 * 8, u);
-    }
+  for (int e = t; e < D * (D / 8); e += 128) {
+    const int a = e / (D / 8), c8 = e % (D / 8);
+    st_sw128_unit(sW, D, a, c8 * 8, *reinterpret_cast<const uint4*>(w_proj + size_t(a) * D + c8 * 8));
   }
   for (int e = t; e < 2 * D; e += 128) {
     const int m = e / D, b2 = 2 * p + m;
-    sZ[e] = b2 < T ? z_agg[(size_t(bh) * T + b2) * D + (e % D)] : 0.f;
+    sZ[m][e % D] = b2 < T ? z_agg[(size_t(bh) * T + b2) * D + (e % D)] : 0.f;
   }
   __syncthreads();
   // phi(Q) row t -> sA (bf16, K-major) and den = phi(Q) . Z_half (fp32)
   float den = 0.f;
   {
     const __nv_bfloat16* qrow = q + (size_t(bh) * N + tok) * D;
-    const float* z = sZ + half * D;
 #pragma unroll 4
     for (int c8 = 0; c8 < D / 8; ++c8) {
       uint4 u = make_uint4(0, 0, 0, 0);
@@ -312,33 +325,60 @@ __global__ void __launch_bounds__(128, 1) fwd_linear_kernel(
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float a = phi_f(bf16_lo(w[e])), b = phi_f(bf16_hi(w[e]));
-        den = fmaf(a, z[c8 * 8 + 2 * e], den);
-        den = fmaf(b, z[c8 * 8 + 2 * e + 1], den);
+        den = fmaf(a, sZ[half][c8 * 8 + 2 * e], den);
+        den = fmaf(b, sZ[half][c8 * 8 + 2 * e + 1], den);
         pw[e] = pack_bf16(a, b);
       }
       st_sw128_unit(sA, 128, t, c8 * 8, make_uint4(pw[0], pw[1], pw[2], pw[3]));
     }
   }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base;
-  if (t == 0) {
-    constexpr uint32_t idesc = idesc_bf16(128, D, 0, 1);
-    const uint32_t a0 = smem_u32(sA);
-    for (int m = 0; m < 2; ++m) {
-      const uint32_t b0 = smem_u32(sH + m * kMat);
+  const uint32_t tmem_hold = 0;
+  (void)tmem_hold;
+  bool ok = true;
+  for (int m = 0; m < 2; ++m) {
+    // H_{2p+m} (fp32) -> hi / lo tiles
+    const int b2 = 2 * p + m;
+    const float* hsrc = h_agg + (size_t(bh) * T + (b2 < T ? b2 : 0)) * D * D;
+    for (int e = t; e < D * (D / 8); e += 128) {
+      const int a = e / (D / 8), c8 = e % (D / 8);
+      float x[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (b2 < T) {
+        const float4 u0 = *reinterpret_cast<const float4*>(hsrc + size_t(a) * D + c8 * 8);
+        const float4 u1 = *reinterpret_cast<const float4*>(hsrc + size_t(a) * D + c8 * 8 + 4);
+        x[0] = u0.x; x[1] = u0.y; x[2] = u0.z; x[3] = u0.w;
+        x[4] = u1.x; x[5] = u1.y; x[6] = u1.z; x[7] = u1.w;
+      }
+      uint32_t hi[4], lo[4];
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks)
-        mma_ss(tmem + m * D, desc_kmajor(a0, 128, ks), desc_mnmajor(b0, D, ks), idesc, ks > 0);
+      for (int i = 0; i < 4; ++i) {
+        hi[i] = pack_bf16(x[2 * i], x[2 * i + 1]);
+        lo[i] = pack_bf16(x[2 * i] - bf16_lo(hi[i]), x[2 * i + 1] - bf16_hi(hi[i]));
+      }
+      st_sw128_unit(sHh, D, a, c8 * 8, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+      st_sw128_unit(sHl, D, a, c8 * 8, make_uint4(lo[0], lo[1], lo[2], lo[3]));
     }
-    mma_commit(&bar[0]);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (t == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, D, 0, 1);
+      const uint32_t a0 = smem_u32(sA);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        mma_ss(tmem_base + m * D, desc_kmajor(a0, 128, ks), desc_mnmajor(smem_u32(sHh), D, ks),
+               idesc, ks > 0);
+        mma_ss(tmem_base + m * D, desc_kmajor(a0, 128, ks), desc_mnmajor(smem_u32(sHl), D, ks),
+               idesc, 1);
+      }
+      mma_commit(&bar[m]);
+    }
+    ok = mbar_wait(&bar[m], 0, err, nullptr) && ok;
+    tc_fence_after();
   }
-  bool ok = mbar_wait(&bar[0], 0, err, nullptr);
-  tc_fence_after();
+  const uint32_t tmem = tmem_base;
   const float inv = (row_ok && den > 0.f) ? 1.0f / den : 0.0f;
-  if (row_ok && lane_id() < 32) den_out[size_t(bh) * N + tok] = row_ok ? den : 0.f;
+  if (row_ok) den_out[size_t(bh) * N + tok] = den;
   // O_l = NUM / den, split into hi + lo bf16 (K-major rows)
 #pragma unroll 1
   for (int c0 = 0; c0 < D; c0 += 32) {
@@ -367,14 +407,13 @@ __global__ void __launch_bounds__(128, 1) fwd_linear_kernel(
     constexpr uint32_t idesc = idesc_bf16(128, D, 0, 1);
     const uint32_t b0 = smem_u32(sW);
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks)
+    for (int ks = 0; ks < D / 16; ++ks) {
       mma_ss(tmem, desc_kmajor(smem_u32(sA), 128, ks), desc_mnmajor(b0, D, ks), idesc, ks > 0);
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks)
       mma_ss(tmem, desc_kmajor(smem_u32(sA2), 128, ks), desc_mnmajor(b0, D, ks), idesc, 1);
-    mma_commit(&bar[1]);
+    }
+    mma_commit(&bar[2]);
   }
-  ok = mbar_wait(&bar[1], 0, err, nullptr) && ok;
+  ok = mbar_wait(&bar[2], 0, err, nullptr) && ok;
   tc_fence_after();
   {
     const float* osrow = o_s + (size_t(bh) * N + tok) * D;
@@ -404,45 +443,47 @@ __global__ void __launch_bounds__(128, 1) fwd_linear_kernel(
   if (warp == 0) tmem_free(tmem, 2 * D);
 }
 
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+}
+
 }  // namespace
 
 cudaError_t launch_summaries(const Problem& p, const void* k, const void* v,
-                             __nv_bfloat16* summ, float* zsum, int* err, cudaStream_t s) {
+                             __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* zsum,
+                             int* err, cudaStream_t s) {
   dim3 grid(p.T, p.BH);
   const int groups = 128 / (p.d / 8);
-  const size_t smem = 1024 + 16384 + (p.d / 64) * 8192 + sizeof(float) * groups * p.d;
+  const size_t smem = 1024 + 32768 + (p.d / 64) * 8192 + sizeof(float) * groups * p.d;
   cudaError_t e;
   if (p.d == 128) {
-    e = cudaFuncSetAttribute(summaries_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem));
-    if (e != cudaSuccess) return e;
+    if ((e = set_smem(summaries_kernel<128>, smem)) != cudaSuccess) return e;
     summaries_kernel<128><<<grid, 128, smem, s>>>((const __nv_bfloat16*)k,
-                                                  (const __nv_bfloat16*)v, summ, zsum, p.N,
-                                                  p.T, err);
+                                                  (const __nv_bfloat16*)v, summ_hi, summ_lo,
+                                                  zsum, p.N, p.T, err);
   } else {
-    e = cudaFuncSetAttribute(summaries_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem));
-    if (e != cudaSuccess) return e;
+    if ((e = set_smem(summaries_kernel<64>, smem)) != cudaSuccess) return e;
     summaries_kernel<64><<<grid, 128, smem, s>>>((const __nv_bfloat16*)k,
-                                                 (const __nv_bfloat16*)v, summ, zsum, p.N, p.T,
-                                                 err);
+                                                 (const __nv_bfloat16*)v, summ_hi, summ_lo, zsum,
+                                                 p.N, p.T, err);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
-                             const __nv_bfloat16* summ, __nv_bfloat16* out, int* err,
-                             cudaStream_t s) {
+                             const __nv_bfloat16* summ_hi, const __nv_bfloat16* summ_lo,
+                             float* out, int* err, cudaStream_t s) {
   const int NN = p.d * p.d;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tbh, tbl;
   if (!make_tmap_3d(&ta, mmat, p.Tp, p.Tp, p.BH, 64, 128)) return cudaErrorInvalidValue;
-  if (!make_tmap_3d(&tb, summ, NN, p.T, p.BH, 64, 64)) return cudaErrorInvalidValue;
+  if (!make_tmap_3d(&tbh, summ_hi, NN, p.T, p.BH, 64, 64)) return cudaErrorInvalidValue;
+  if (!make_tmap_3d(&tbl, summ_lo, NN, p.T, p.BH, 64, 64)) return cudaErrorInvalidValue;
   const size_t smem = 1024 + kAggStages * kAggStageBytes;
-  cudaError_t e = cudaFuncSetAttribute(agg_gemm_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e = set_smem(agg_gemm_kernel, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.Tp / 128, NN / kAggBN, p.BH);
-  agg_gemm_kernel<<<grid, 128, smem, s>>>(ta, tb, out, p.T, p.Tp, NN, err);
+  agg_gemm_kernel<<<grid, 128, smem, s>>>(ta, tbh, tbl, out, p.T, p.Tp, NN, err);
   return cudaGetLastError();
 }
 
@@ -453,23 +494,19 @@ cudaError_t launch_aggregate_z(const Problem& p, const uint32_t* marg_bits, cons
   return cudaGetLastError();
 }
 
-cudaError_t launch_fwd_linear(const Problem& p, const void* q, const __nv_bfloat16* h_agg,
+cudaError_t launch_fwd_linear(const Problem& p, const void* q, const float* h_agg,
                               const float* z_agg, const void* w_proj, const float* o_s,
                               void* o, float* den, int* err, cudaStream_t s) {
   dim3 grid((p.T + 1) / 2, p.BH);
-  const size_t smem = 1024 + 2 * (128 * p.d * 2) + 3 * (p.d * p.d * 2) + 2 * p.d * sizeof(float);
+  const size_t smem = 1024 + 5 * (128 * 128 * 2);
   cudaError_t e;
   if (p.d == 128) {
-    e = cudaFuncSetAttribute(fwd_linear_kernel<128>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
+    if ((e = set_smem(fwd_linear_kernel<128>, smem)) != cudaSuccess) return e;
     fwd_linear_kernel<128><<<grid, 128, smem, s>>>(
         (const __nv_bfloat16*)q, h_agg, z_agg, (const __nv_bfloat16*)w_proj, o_s,
         (__nv_bfloat16*)o, den, p.N, p.T, err);
   } else {
-    e = cudaFuncSetAttribute(fwd_linear_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem));
-    if (e != cudaSuccess) return e;
+    if ((e = set_smem(fwd_linear_kernel<64>, smem)) != cudaSuccess) return e;
     fwd_linear_kernel<64><<<grid, 128, smem, s>>>(
         (const __nv_bfloat16*)q, h_agg, z_agg, (const __nv_bfloat16*)w_proj, o_s,
         (__nv_bfloat16*)o, den, p.N, p.T, err);

@@ -91,8 +91,11 @@ def test_backward_sparse_key_gradient_sums_to_zero():
     run.forward()
     run.backward(wl.d_o)
     dk = run.np(run.dk)
-    scale = np.abs(dk).sum(axis=2)
-    assert np.all(np.abs(dk.sum(axis=2)) <= 1e-4 * scale + 1e-6)
+    # exact only in exact arithmetic: bf16 P in the forward's P V product makes
+    # D = dO . O_s differ slightly from sum_u P dP, a per-row common mode
+    resid = np.abs(dk.sum(axis=2)).sum(axis=-1)
+    total = np.abs(dk).sum(axis=(2, 3))
+    assert np.all(resid <= 3e-3 * total), (resid / total)
 
 
 def test_backward_wan_full_size_sampled():
