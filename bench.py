@@ -1,0 +1,386 @@
+"""Benchmark of the SLA hot path on B200: one step = classification + forward +
+backward of sparse-linear attention on a Wan2.1-1.3B-shaped training
+workload (B=1, H=12, N=32768 tokens from a 21x30x52 latent grid padded to
+64-token blocks, d=128, k_h=5%, k_l=10%, synthetic inputs, seed = rank).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sla|reference]
+
+Prints one JSON line (rank 0).  ``value`` is executed-block TFLOP/s of the
+whole step: (forward 4*b^2*d + backward 10*b^2*d) per critical
+(query block, key block) pair, summed over ranks, divided by the max over
+ranks of the device time per step.  With N > 1 every rank runs an
+independent replica of the step (weak scaling, no collective on the data
+path).  ``--impl reference`` times the fp64 CPU oracle on a bounded sample
+of the same workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SLA fwd/bwd ms and executed-block TFLOP/s (% bf16 peak) at N=32768,H=12,d=128"
+WORKLOAD = dict(name="train", B=1, H=12, d=128, grid=(21, 30, 52), block=64, k_h=0.05, k_l=0.10)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(wl, n_crit):
+    return {
+        "workload": "Wan2.1-1.3B-shaped SLA training step (classify+forward+backward): "
+                    "B=1 H=12 N=32768 (21x30x52 grid padded) d=128 block=64 k_h=0.05 k_l=0.10",
+        "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "block": wl.block, "k_h": wl.k_h,
+        "k_l": wl.k_l, "n_crit": n_crit, "global_batch": wl.B, "seq_len": wl.N,
+        "l2": "inputs larger than L2 (Q/K/V/dO bf16 = 403 MB per step)",
+        "parallelism": "independent replica per GPU",
+    }
+
+
+def executed_block_flops(wl, n_crit):
+    pairs = wl.B * wl.H * wl.T * n_crit
+    fwd = pairs * 4 * wl.block * wl.block * wl.d
+    bwd = pairs * 10 * wl.block * wl.block * wl.d
+    return fwd, bwd
+
+
+def kernel_work(wl, n_crit):
+    """Algorithmic work per launch of each kernel: ('tensor', FLOP) or ('hbm', bytes)."""
+    B, H, N, d, T = wl.B, wl.H, wl.N, wl.d, wl.T
+    BH = B * H
+    Tp = (T + 127) // 128 * 128
+    tok = BH * N
+    pairs = BH * T * n_crit
+    b = wl.block
+    return {
+        "pool": ("hbm", 2 * tok * d * 2 + 2 * BH * T * d * 4),
+        "summaries": ("hbm", 2 * tok * d * 2 + BH * T * d * d * 4 + BH * T * d * 4),
+        "aggregate": ("tensor", 2 * BH * T * T * d * d),
+        "aggregate_t": ("tensor", 2 * BH * T * T * d * d),
+        "fwd_sparse": ("tensor", pairs * 4 * b * b * d),
+        "fwd_linear": ("hbm", tok * d * (2 + 4 + 2) + BH * T * d * d * 4 + tok * 4),
+        "bwd_prep": ("hbm", tok * d * (2 + 2 + 4 + 4) + BH * T * d * d * 4 + tok * 4 * 3),
+        "bwd_summ": ("hbm", tok * d * (2 + 4) + BH * T * d * d * 4 + tok * 4),
+        "bwd_sparse": ("tensor", pairs * 10 * b * b * d),
+        "bwd_linear": ("hbm", tok * d * (3 * 2 + 4 + 3 * 8) + 2 * BH * T * d * d * 4),
+        "expand_marginal": ("hbm", BH * Tp * Tp * 2),
+        "expand_marginal_t": ("hbm", BH * Tp * Tp * 2),
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [x.strip() for x in ln.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = [x for x in threadpool_info() if x.get("user_api") == "blas"]
+        if info:
+            return int(info[0]["num_threads"])
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample_step(wl, heads):
+    """classification + forward + backward of the fp64 oracle on `heads`."""
+    import oracle
+    sub = lambda a: a[:, heads]
+    T = wl.T
+    n_h, n_l = oracle.block_counts(T, wl.k_h, wl.k_l)
+    logits = oracle.pooled_logits(sub(wl.q), sub(wl.k), wl.block, wl.scale)
+    cls = oracle.classify(logits, n_h, n_l)
+    fwd = oracle.forward(sub(wl.q), sub(wl.k), sub(wl.v), wl.w_proj, cls, wl.block, wl.scale)
+    oracle.backward(sub(wl.q), sub(wl.k), sub(wl.v), wl.w_proj, cls, sub(wl.d_o), wl.block,
+                    wl.scale, fwd=fwd)
+    return n_h
+
+
+def time_oracle(wl, heads, steps, warmup):
+    t_all = []
+    n_h = 0
+    for i in range(warmup + steps):
+        t0 = time.perf_counter()
+        n_h = oracle_sample_step(wl, heads)
+        if i >= warmup:
+            t_all.append(time.perf_counter() - t0)
+    sample = wl.B * len(heads) * wl.T * n_h * 14 * wl.block * wl.block * wl.d
+    sec = statistics.mean(t_all)
+    return sample / sec / 1e12, sec
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import sla_inputs
+    wl = sla_inputs.make("train", seed=0)
+    heads = [0]
+    tflops, sec = time_oracle(wl, heads, args.steps, args.warmup)
+    n_crit = oracle_n_crit(wl)
+    cfg = workload_config(wl, n_crit)
+    sample = (f"head 0 of 12 of the same workload per step (classify+forward+backward, fp64 "
+              f"numpy on {blas_threads()} BLAS threads), {sec:.2f} s per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def oracle_n_crit(wl):
+    import oracle
+    return oracle.block_counts(wl.T, wl.k_h, wl.k_l)[0]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["sla", "reference"], default="sla")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import sla_inputs
+    import sparse_linear_attention_block_b200 as slab
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    wl = sla_inputs.make("train", seed=rank)
+    shape = slab.make_shape(wl.B, wl.H, wl.N, wl.d, wl.block, wl.k_h, wl.k_l)
+    buf = slab.Buffers.allocate(shape, device=dev, with_logits=False)
+    n_crit = buf.sizes.n_crit
+    to_dev = lambda a: torch.from_numpy(a).to(torch.bfloat16).to(dev)
+    q, k, v, w, do = (to_dev(x) for x in (wl.q, wl.k, wl.v, wl.w_proj, wl.d_o))
+    o = torch.empty_like(q)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk, dv = torch.empty_like(dq), torch.empty_like(dq)
+    dw = torch.empty(w.shape, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(qq=q, kk=k, vv=v, ww=w, dd=do):
+        slab.sla_classify(shape, qq, kk, buf.mask, buf.workspace, stream)
+        slab.sla_forward(shape, qq, kk, vv, ww, buf.mask, o, buf.saved, buf.workspace, stream)
+        slab.sla_backward(shape, qq, kk, vv, ww, buf.mask, buf.saved, dd, dq, dk, dv, dw,
+                          buf.workspace, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    slab.sla_check(buf.workspace, stream)
+    torch.cuda.synchronize()
+    barrier()
+
+    # ------------------------------------------------------------ timed region
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    slab.sla_check(buf.workspace, stream)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    clocks = clk.summary()
+
+    fwd_flops, bwd_flops = executed_block_flops(wl, n_crit)
+    value = world * (fwd_flops + bwd_flops) / (ms * 1e-3) / 1e12
+
+    # ------------------------------------------------------------ per-kernel times
+    slab.sla_profile_begin()
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    prof = slab.sla_profile_end()
+    launches_per_step = sum(n for n, _ in prof.values()) / args.steps
+    pk, src = peaks()
+    work = kernel_work(wl, n_crit)
+    per_kernel = {name: {"launches": n, "ms_per_launch": tot / n,
+                         "share": tot / sum(t for _, t in prof.values())}
+                  for name, (n, tot) in prof.items()}
+    dominant = max(prof, key=lambda n: prof[n][1])
+    kind, amount = work.get(dominant, ("tensor", 0))
+    avg_s = prof[dominant][1] / prof[dominant][0] * 1e-3
+    if kind == "tensor":
+        achieved = amount / avg_s / 1e12
+        peak = pk["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "kernel": dominant,
+                "peak_source": f"{src} sustained bf16"}
+    else:
+        achieved = amount / avg_s / 1e9
+        peak = pk["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None, "kernel": dominant,
+                "peak_source": f"{src} HBM copy"}
+    fwd_ms = sum(prof[n][1] for n in ("summaries", "expand_marginal", "aggregate",
+                                      "aggregate_z", "fwd_sparse", "fwd_linear")
+                 if n in prof) / args.steps
+    cls_ms = sum(prof[n][1] for n in ("pool", "classify", "crit_csr") if n in prof) / args.steps
+    bwd_ms = sum(t for n, (_, t) in prof.items()) / args.steps - fwd_ms - cls_ms
+
+    # ------------------------------------------------------------ end to end
+    e2e = None
+    if not args.no_e2e:
+        hosts = [torch.from_numpy(x).to(torch.bfloat16).pin_memory()
+                 for x in (wl.q, wl.k, wl.v, wl.w_proj, wl.d_o)]
+        devs = [torch.empty_like(h, device=dev) for h in hosts]
+        dw_host = torch.empty(dw.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(h.numel() * h.element_size() for h in hosts)
+        d2h = dw_host.numel() * dw_host.element_size()
+
+        def e2e_step():
+            for hsrc, ddst in zip(hosts, devs):
+                ddst.copy_(hsrc, non_blocking=True)
+            step(*devs)
+            dw_host.copy_(dw, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps)
+        e2e = {"value": world * (fwd_flops + bwd_flops) / (e_ms * 1e-3) / 1e12,
+               "unit": "TFLOP/s", "ms_per_step": e_ms, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+
+    # ------------------------------------------------------------ CPU oracle baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tfl, sec = time_oracle(wl, [0], 1, 0)
+        cpu = {"value": tfl, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"head 0 of 12 of this workload, one classify+forward+backward step "
+                         f"of the fp64 oracle ({sec:.1f} s), same executed-block FLOP count"}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peak_t = pk["bf16_tflops_sustained"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(wl, n_crit),
+        "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "classify_ms": cls_ms,
+        "fwd_tflops": fwd_flops / (fwd_ms * 1e-3) / 1e12,
+        "bwd_tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12,
+        "frac_of_bf16_peak": value / world / peak_t,
+        "kernels": per_kernel, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "clocks": clocks, "gpu_launches": int(round(launches_per_step * args.steps)),
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

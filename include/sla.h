@@ -155,6 +155,22 @@ SLA_API sla_status sla_check(void* workspace, void* stream);
 /* Static description of a status code. */
 SLA_API const char* sla_strerror(sla_status status);
 
+/* Per-kernel device time collected by the opt-in profiler. */
+typedef struct {
+  const char* name; /* static string, e.g. "fwd_sparse" */
+  int launches;
+  double total_ms;
+} sla_kernel_stat;
+
+/* Start recording: until sla_profile_end(), every kernel the library
+ * launches is bracketed by two CUDA events on its stream (diagnostic only;
+ * adds a few microseconds per launch).  Process-wide. */
+SLA_API sla_status sla_profile_begin(void);
+
+/* Stop recording, wait for the recorded launches, and write up to max_out
+ * per-kernel totals (in first-launch order) to out; *n_out = entries written. */
+SLA_API sla_status sla_profile_end(sla_kernel_stat* out, int max_out, int* n_out);
+
 /* Library version, "major.minor.patch". */
 SLA_API const char* sla_version(void);
 

@@ -22,7 +22,8 @@ __all__ = [
     "SlaError", "Shape", "Sizes", "MaskStruct", "SavedStruct", "Buffers", "lib", "lib_path",
     "sla_query_sizes", "sla_classify", "sla_classify_from_scores", "sla_forward",
     "sla_backward", "sla_workspace_init", "sla_check", "sla_strerror", "sla_version",
-    "EXPORTED_SYMBOLS", "STATUS",
+    "sla_profile_begin", "sla_profile_end", "KernelStat", "make_shape", "EXPORTED_SYMBOLS",
+    "STATUS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -33,7 +34,7 @@ STATUS = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED", 3: "S
 
 EXPORTED_SYMBOLS = ["sla_query_sizes", "sla_classify", "sla_classify_from_scores",
                     "sla_forward", "sla_backward", "sla_workspace_init", "sla_check",
-                    "sla_strerror", "sla_version"]
+                    "sla_strerror", "sla_version", "sla_profile_begin", "sla_profile_end"]
 
 
 class SlaError(RuntimeError):
@@ -57,6 +58,11 @@ class MaskStruct(ctypes.Structure):
 class SavedStruct(ctypes.Structure):
     _fields_ = [("lse", ctypes.c_void_p), ("o_s", ctypes.c_void_p), ("den", ctypes.c_void_p),
                 ("h_agg", ctypes.c_void_p), ("z_agg", ctypes.c_void_p)]
+
+
+class KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int),
+                ("total_ms", ctypes.c_double)]
 
 
 class Sizes(ctypes.Structure):
@@ -94,8 +100,11 @@ def lib() -> ctypes.CDLL:
         L.sla_strerror.restype = ctypes.c_char_p
         L.sla_version.argtypes = []
         L.sla_version.restype = ctypes.c_char_p
+        L.sla_profile_begin.argtypes = []
+        L.sla_profile_end.argtypes = [P(KernelStat), st, P(st)]
         for n in ("sla_query_sizes", "sla_classify", "sla_classify_from_scores", "sla_forward",
-                  "sla_backward", "sla_workspace_init", "sla_check"):
+                  "sla_backward", "sla_workspace_init", "sla_check", "sla_profile_begin",
+                  "sla_profile_end"):
             getattr(L, n).restype = st
         _lib = L
     return _lib
@@ -146,6 +155,18 @@ def sla_strerror(status: int) -> str:
 
 def sla_version() -> str:
     return lib().sla_version().decode()
+
+
+def sla_profile_begin():
+    _check(lib().sla_profile_begin(), "sla_profile_begin")
+
+
+def sla_profile_end(max_out: int = 64) -> dict:
+    """Per-kernel {name: (launches, total_ms)} since sla_profile_begin()."""
+    arr = (KernelStat * max_out)()
+    n = ctypes.c_int(0)
+    _check(lib().sla_profile_end(arr, max_out, ctypes.byref(n)), "sla_profile_end")
+    return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n.value)}
 
 
 def sla_workspace_init(workspace, stream=None):

@@ -8,6 +8,8 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include "sla.h"
 #include "sla_internal.h"
@@ -167,9 +169,44 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
-#define SLA_LAUNCH(expr)                       \
-  do {                                         \
-    if ((expr) != cudaSuccess) return SLA_ERR_CUDA; \
+// ------------------------------------------------------------------ opt-in profiler
+// When enabled by sla_profile_begin(), every kernel launch of the library is
+// bracketed by a pair of CUDA events on its stream; sla_profile_end() folds
+// them into per-kernel launch counts and total device time.
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+
+bool prof_mark(cudaStream_t s, cudaEvent_t* ev) {
+  if (cudaEventCreate(ev) != cudaSuccess) return false;
+  return cudaEventRecord(*ev, s) == cudaSuccess;
+}
+
+template <typename F>
+cudaError_t launch_named(const char* name, cudaStream_t s, F&& launch) {
+  bool on;
+  {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    on = g_prof_on;
+  }
+  if (!on) return launch();
+  ProfRec r{name, nullptr, nullptr};
+  if (!prof_mark(s, &r.a)) return cudaErrorUnknown;
+  const cudaError_t e = launch();
+  if (!prof_mark(s, &r.b)) return cudaErrorUnknown;
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  g_prof.push_back(r);
+  return e;
+}
+
+#define SLA_LAUNCH(name, stream, expr)                                            \
+  do {                                                                            \
+    if (launch_named(name, stream, [&] { return (expr); }) != cudaSuccess)        \
+      return SLA_ERR_CUDA;                                                        \
   } while (0)
 
 }  // namespace
@@ -198,11 +235,11 @@ static sla_status classify_impl(const sla_shape* shape, const void* q, const voi
   const float* kbar = at<float>(ws, L.kbar);
   if (!logits_in) {
     if (!q || !k || !aligned16(q) || !aligned16(k)) return SLA_ERR_INVALID_ARG;
-    SLA_LAUNCH(launch_pool(p, q, k, at<float>(ws, L.qbar), at<float>(ws, L.kbar), s));
+    SLA_LAUNCH("pool", s, launch_pool(p, q, k, at<float>(ws, L.qbar), at<float>(ws, L.kbar), s));
   }
-  SLA_LAUNCH(launch_classify(p, qbar, kbar, logits_in, logits_in ? nullptr : mask->pooled_logits,
+  SLA_LAUNCH("classify", s, launch_classify(p, qbar, kbar, logits_in, logits_in ? nullptr : mask->pooled_logits,
                              mask->cls, mask->crit_idx, mask->marg_bits, s));
-  SLA_LAUNCH(launch_crit_csr(p, mask->cls, mask->crit_col_ptr, mask->crit_col_idx, s));
+  SLA_LAUNCH("crit_csr", s, launch_crit_csr(p, mask->cls, mask->crit_col_ptr, mask->crit_col_idx, s));
   return SLA_OK;
 }
 
@@ -252,13 +289,13 @@ sla_status sla_forward(const sla_shape* shape, const void* q, const void* k, con
   auto* mmat = at<__nv_bfloat16>(workspace, L.mmat);
   float* zsum = at<float>(workspace, L.zsum);
   // linear branch: summaries, marginal aggregation
-  SLA_LAUNCH(launch_summaries(p, k, v, summ_hi, summ_lo, zsum, err, s));
-  SLA_LAUNCH(launch_expand_marginal(p, mask->marg_bits, mmat, nullptr, s));
-  SLA_LAUNCH(launch_aggregate(p, mmat, summ_hi, summ_lo, saved->h_agg, err, s));
-  SLA_LAUNCH(launch_aggregate_z(p, mask->marg_bits, zsum, saved->z_agg, false, s));
+  SLA_LAUNCH("summaries", s, launch_summaries(p, k, v, summ_hi, summ_lo, zsum, err, s));
+  SLA_LAUNCH("expand_marginal", s, launch_expand_marginal(p, mask->marg_bits, mmat, nullptr, s));
+  SLA_LAUNCH("aggregate", s, launch_aggregate(p, mmat, summ_hi, summ_lo, saved->h_agg, err, s));
+  SLA_LAUNCH("aggregate_z", s, launch_aggregate_z(p, mask->marg_bits, zsum, saved->z_agg, false, s));
   // sparse branch, then the combination
-  SLA_LAUNCH(launch_fwd_sparse(p, q, k, v, mask->crit_idx, saved->o_s, saved->lse, err, s));
-  SLA_LAUNCH(launch_fwd_linear(p, q, saved->h_agg, saved->z_agg, w_proj, saved->o_s, o,
+  SLA_LAUNCH("fwd_sparse", s, launch_fwd_sparse(p, q, k, v, mask->crit_idx, saved->o_s, saved->lse, err, s));
+  SLA_LAUNCH("fwd_linear", s, launch_fwd_linear(p, q, saved->h_agg, saved->z_agg, w_proj, saved->o_s, o,
                                saved->den, err, s));
   return SLA_OK;
 }
@@ -299,17 +336,17 @@ sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, co
   if (cudaMemsetAsync(dw_proj, 0, size_t(p.d) * p.d * sizeof(float), s) != cudaSuccess)
     return SLA_ERR_CUDA;
   // linear-branch preparation: D, dnum, dden, dW; then per-block A_i / a_i
-  SLA_LAUNCH(launch_bwd_prep(p, q, d_o, w_proj, saved->o_s, saved->den, saved->h_agg, dvec, dnum,
+  SLA_LAUNCH("bwd_prep", s, launch_bwd_prep(p, q, d_o, w_proj, saved->o_s, saved->den, saved->h_agg, dvec, dnum,
                              dden, dw_proj, sms, err, s));
-  SLA_LAUNCH(launch_bwd_summ(p, q, dnum, dden, summ_hi, summ_lo, zsum, err, s));
+  SLA_LAUNCH("bwd_summ", s, launch_bwd_summ(p, q, dnum, dden, summ_hi, summ_lo, zsum, err, s));
   // dh_j = sum over rows i with j marginal of A_i (transposed aggregation)
-  SLA_LAUNCH(launch_expand_marginal(p, mask->marg_bits, nullptr, mmat_t, s));
-  SLA_LAUNCH(launch_aggregate(p, mmat_t, summ_hi, summ_lo, dh, err, s));
-  SLA_LAUNCH(launch_aggregate_z(p, mask->marg_bits, zsum, dz, true, s));
+  SLA_LAUNCH("expand_marginal_t", s, launch_expand_marginal(p, mask->marg_bits, nullptr, mmat_t, s));
+  SLA_LAUNCH("aggregate_t", s, launch_aggregate(p, mmat_t, summ_hi, summ_lo, dh, err, s));
+  SLA_LAUNCH("aggregate_z_t", s, launch_aggregate_z(p, mask->marg_bits, zsum, dz, true, s));
   // sparse branch writes dK, dV and accumulates dQ; the linear branch adds its share
-  SLA_LAUNCH(launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
+  SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
                                mask->crit_col_idx, dq, dk, dv, err, s));
-  SLA_LAUNCH(launch_bwd_linear(p, q, k, v, saved->h_agg, saved->z_agg, dh, dz, dnum, dden, dq, dk,
+  SLA_LAUNCH("bwd_linear", s, launch_bwd_linear(p, q, k, v, saved->h_agg, saved->z_agg, dh, dz, dnum, dden, dq, dk,
                                dv, err, s));
   return SLA_OK;
 }
@@ -351,5 +388,50 @@ const char* sla_strerror(sla_status status) {
 }
 
 const char* sla_version(void) { return "0.1.0"; }
+
+sla_status sla_profile_begin(void) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  for (auto& r : g_prof) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  g_prof.clear();
+  g_prof_on = true;
+  return SLA_OK;
+}
+
+sla_status sla_profile_end(sla_kernel_stat* out, int max_out, int* n_out) {
+  if (!n_out || (max_out > 0 && !out)) return SLA_ERR_INVALID_ARG;
+  std::vector<ProfRec> recs;
+  {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    g_prof_on = false;
+    recs.swap(g_prof);
+  }
+  sla_status st = SLA_OK;
+  int n = 0;
+  for (auto& r : recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+      st = SLA_ERR_CUDA;
+    int slot = -1;
+    for (int i = 0; i < n && i < max_out; ++i)
+      if (std::string(out[i].name) == r.name) slot = i;
+    if (slot < 0 && n < max_out) {
+      slot = n++;
+      out[slot].name = r.name;
+      out[slot].launches = 0;
+      out[slot].total_ms = 0.0;
+    }
+    if (slot >= 0) {
+      out[slot].launches += 1;
+      out[slot].total_ms += ms;
+    }
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  *n_out = n;
+  return st;
+}
 
 }  // extern "C"
