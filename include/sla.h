@@ -129,6 +129,23 @@ SLA_API sla_status sla_classify_from_scores(const sla_shape* shape, const float*
                                     const sla_mask* mask, void* workspace,
                                     size_t workspace_bytes, void* stream);
 
+/* Same classification as sla_classify, for callers that cannot allocate
+ * device memory when they classify (for example code running inside CUDA
+ * graph capture, allocator-less embedded or real-time runtimes, or hosts
+ * whose device memory comes from a pool they may not grow).  It takes no
+ * workspace: its only scratch (pooled Q and K) is a fixed 16 MiB array built
+ * into the library, present on every GPU that loads it until the process
+ * exits, and it calls no allocating routine.  The paper has no counterpart;
+ * this is a packaging variant.
+ *   - Limit: 2 * B*H*T*d*4 bytes <= 16 MiB (B*H*T*d <= 2M); larger shapes get
+ *     SLA_ERR_WORKSPACE.  Other arguments and outputs as sla_classify.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call shares the one array: calls that overlap on the GPU (other
+ *     streams, other threads) race on it and must be serialized by the caller. */
+SLA_API sla_status sla_classify_noalloc(const sla_shape* shape, const void* q, const void* k,
+                                        const sla_mask* mask, void* stream);
+
 /* Forward with a given mask: writes o (bf16 [B,H,N,d]) and *saved. */
 SLA_API sla_status sla_forward(const sla_shape* shape, const void* q, const void* k, const void* v,
                        const void* w_proj, const sla_mask* mask, void* o,

@@ -34,7 +34,8 @@ STATUS = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED", 3: "S
 
 EXPORTED_SYMBOLS = ["sla_query_sizes", "sla_classify", "sla_classify_from_scores",
                     "sla_forward", "sla_backward", "sla_workspace_init", "sla_check",
-                    "sla_strerror", "sla_version", "sla_profile_begin", "sla_profile_end"]
+                    "sla_strerror", "sla_version", "sla_profile_begin", "sla_profile_end",
+                    "sla_classify_noalloc"]
 
 
 class SlaError(RuntimeError):
@@ -100,6 +101,8 @@ def lib() -> ctypes.CDLL:
         L.sla_strerror.restype = ctypes.c_char_p
         L.sla_version.argtypes = []
         L.sla_version.restype = ctypes.c_char_p
+        L.sla_classify_noalloc.argtypes = [P(Shape), vp, vp, P(MaskStruct), vp]
+        L.sla_classify_noalloc.restype = st
         L.sla_profile_begin.argtypes = []
         L.sla_profile_end.argtypes = [P(KernelStat), st, P(st)]
         for n in ("sla_query_sizes", "sla_classify", "sla_classify_from_scores", "sla_forward",
@@ -182,6 +185,14 @@ def sla_classify(shape: Shape, q, k, mask: MaskStruct, workspace, stream=None):
     _check(lib().sla_classify(ctypes.byref(shape), _ptr(q), _ptr(k), ctypes.byref(mask),
                               _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _stream(stream)), "sla_classify")
+
+
+def sla_classify_noalloc(shape: Shape, q, k, mask: MaskStruct, stream=None):
+    """Classification without a workspace, for callers that cannot allocate
+    device memory (scratch is a fixed 16 MiB array inside the library; see
+    sla.h for the size limit and the one-time per-device set-up)."""
+    _check(lib().sla_classify_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), ctypes.byref(mask),
+                                      _stream(stream)), "sla_classify_noalloc")
 
 
 def sla_classify_from_scores(shape: Shape, logits, mask: MaskStruct, workspace, stream=None):
