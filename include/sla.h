@@ -94,14 +94,12 @@ typedef struct {
  *   lse   fp32 [B,H,N]      log-sum-exp of the critical scores (-inf if none)
  *   o_s   fp32 [B,H,N,d]    sparse-branch output
  *   den   fp32 [B,H,N]      phi(Q).Z_i (0 if the row has no marginal block)
- *   h_agg fp32 [B,H,T,d,d]  H_i per query block
- *   z_agg fp32 [B,H,T,d]    Z_i per query block */
+ *   hz_agg fp32 [B,H,T,d*d+d]  per query block: H_i (d x d, row-major) then Z_i (d) */
 typedef struct {
   float* lse;
   float* o_s;
   float* den;
-  float* h_agg;
-  float* z_agg;
+  float* hz_agg;
 } sla_saved;
 
 /* Sizes in bytes of every caller buffer for a shape. */
@@ -109,7 +107,7 @@ typedef struct {
   int T, n_crit, n_negl, n_marg;
   size_t cls_bytes, crit_idx_bytes, marg_bits_bytes, crit_col_ptr_bytes, crit_col_idx_bytes,
       pooled_logits_bytes;
-  size_t lse_bytes, o_s_bytes, den_bytes, h_agg_bytes, z_agg_bytes;
+  size_t lse_bytes, o_s_bytes, den_bytes, hz_agg_bytes;
   size_t workspace_bytes; /* one workspace serves classify, forward and backward */
 } sla_sizes;
 

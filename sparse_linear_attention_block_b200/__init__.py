@@ -58,7 +58,7 @@ class MaskStruct(ctypes.Structure):
 
 class SavedStruct(ctypes.Structure):
     _fields_ = [("lse", ctypes.c_void_p), ("o_s", ctypes.c_void_p), ("den", ctypes.c_void_p),
-                ("h_agg", ctypes.c_void_p), ("z_agg", ctypes.c_void_p)]
+                ("hz_agg", ctypes.c_void_p)]
 
 
 class KernelStat(ctypes.Structure):
@@ -72,7 +72,7 @@ class Sizes(ctypes.Structure):
         (n, ctypes.c_size_t) for n in (
             "cls_bytes", "crit_idx_bytes", "marg_bits_bytes", "crit_col_ptr_bytes",
             "crit_col_idx_bytes", "pooled_logits_bytes", "lse_bytes", "o_s_bytes", "den_bytes",
-            "h_agg_bytes", "z_agg_bytes", "workspace_bytes")]
+            "hz_agg_bytes", "workspace_bytes")]
 
 
 _lib = None
@@ -237,8 +237,7 @@ class Buffers:
     lse: object
     o_s: object
     den: object
-    h_agg: object
-    z_agg: object
+    hz_agg: object
     workspace: object
     mask: MaskStruct
     saved: SavedStruct
@@ -263,8 +262,7 @@ class Buffers:
             lse=e(B, H, N, dt=torch.float32),
             o_s=e(B, H, N, d, dt=torch.float32),
             den=e(B, H, N, dt=torch.float32),
-            h_agg=e(B, H, T, d, d, dt=torch.float32),
-            z_agg=e(B, H, T, d, dt=torch.float32),
+            hz_agg=e(B, H, T, d * d + d, dt=torch.float32),
             workspace=torch.empty(int(s.workspace_bytes) + 1024, dtype=torch.uint8, device=dev),
             mask=MaskStruct(), saved=SavedStruct())
         # the C ABI wants a 1024-byte aligned workspace
@@ -272,7 +270,6 @@ class Buffers:
         b.workspace = b.workspace[off:off + int(s.workspace_bytes)]
         b.mask = MaskStruct(_ptr(b.cls), _ptr(b.crit_idx), _ptr(b.marg_bits),
                             _ptr(b.crit_col_ptr), _ptr(b.crit_col_idx), _ptr(b.pooled_logits))
-        b.saved = SavedStruct(_ptr(b.lse), _ptr(b.o_s), _ptr(b.den), _ptr(b.h_agg),
-                              _ptr(b.z_agg))
+        b.saved = SavedStruct(_ptr(b.lse), _ptr(b.o_s), _ptr(b.den), _ptr(b.hz_agg))
         sla_workspace_init(b.workspace, stream)
         return b

@@ -29,11 +29,10 @@ WorkspaceLayout workspace_layout(int BH, int N, int d) {
   L.err = take(256);
   L.qbar = take(bh * T * d * 4);
   L.kbar = take(bh * T * d * 4);
-  L.summ_hi = take(bh * T * d * d * 2);
-  L.summ_lo = take(bh * T * d * d * 2);
-  L.zsum = take(bh * T * d * 4);
-  L.dh = take(bh * T * d * d * 4);
-  L.dz = take(bh * T * d * 4);
+  const size_t W = size_t(summary_width(d));
+  L.summ_hi = take(bh * T * W * 2);
+  L.summ_lo = take(bh * T * W * 2);
+  L.dh = take(bh * T * W * 4);
   L.mmat = take(bh * Tp * Tp * 2);
   L.mmat_t = take(bh * Tp * Tp * 2);
   L.dvec = take(bh * N * 4);
@@ -140,8 +139,7 @@ sla_status fill_sizes(const Problem& p, sla_sizes* o) {
   o->lse_bytes = bh * N * 4;
   o->o_s_bytes = bh * N * d * 4;
   o->den_bytes = bh * N * 4;
-  o->h_agg_bytes = bh * T * d * d * 4;
-  o->z_agg_bytes = bh * T * d * 4;
+  o->hz_agg_bytes = bh * T * size_t(summary_width(p.d)) * 4;
   o->workspace_bytes = workspace_layout(p.BH, p.N, p.d).total;
   return SLA_OK;
 }
@@ -259,10 +257,9 @@ sla_status sla_classify_from_scores(const sla_shape* shape, const float* logits,
 }
 
 static sla_status check_saved(const Problem& p, const sla_saved* sv) {
-  if (!sv || !sv->lse || !sv->o_s || !sv->den || !sv->h_agg || !sv->z_agg)
-    return SLA_ERR_INVALID_ARG;
-  if (!aligned16(sv->o_s) || !aligned16(sv->h_agg) || !aligned16(sv->z_agg) ||
-      !aligned16(sv->lse) || !aligned16(sv->den))
+  if (!sv || !sv->lse || !sv->o_s || !sv->den || !sv->hz_agg) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(sv->o_s) || !aligned16(sv->hz_agg) || !aligned16(sv->lse) ||
+      !aligned16(sv->den))
     return SLA_ERR_INVALID_ARG;
   (void)p;
   return SLA_OK;
@@ -287,16 +284,14 @@ sla_status sla_forward(const sla_shape* shape, const void* q, const void* k, con
   auto* summ_hi = at<__nv_bfloat16>(workspace, L.summ_hi);
   auto* summ_lo = at<__nv_bfloat16>(workspace, L.summ_lo);
   auto* mmat = at<__nv_bfloat16>(workspace, L.mmat);
-  float* zsum = at<float>(workspace, L.zsum);
-  // linear branch: summaries, marginal aggregation
-  SLA_LAUNCH("summaries", s, launch_summaries(p, k, v, summ_hi, summ_lo, zsum, err, s));
+  // linear branch: (h_j | z_j) summaries, then (H_i | Z_i) by one aggregation GEMM
+  SLA_LAUNCH("summaries", s, launch_summaries(p, k, v, summ_hi, summ_lo, err, s));
   SLA_LAUNCH("expand_marginal", s, launch_expand_marginal(p, mask->marg_bits, mmat, nullptr, s));
-  SLA_LAUNCH("aggregate", s, launch_aggregate(p, mmat, summ_hi, summ_lo, saved->h_agg, err, s));
-  SLA_LAUNCH("aggregate_z", s, launch_aggregate_z(p, mask->marg_bits, zsum, saved->z_agg, false, s));
+  SLA_LAUNCH("aggregate", s, launch_aggregate(p, mmat, summ_hi, summ_lo, saved->hz_agg, err, s));
   // sparse branch, then the combination
   SLA_LAUNCH("fwd_sparse", s, launch_fwd_sparse(p, q, k, v, mask->crit_idx, saved->o_s, saved->lse, err, s));
-  SLA_LAUNCH("fwd_linear", s, launch_fwd_linear(p, q, saved->h_agg, saved->z_agg, w_proj, saved->o_s, o,
-                               saved->den, err, s));
+  SLA_LAUNCH("fwd_linear", s, launch_fwd_linear(p, q, saved->hz_agg, w_proj, saved->o_s, o,
+                                                saved->den, err, s));
   return SLA_OK;
 }
 
@@ -326,8 +321,6 @@ sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, co
   auto* summ_lo = at<__nv_bfloat16>(workspace, L.summ_lo);
   auto* mmat_t = at<__nv_bfloat16>(workspace, L.mmat_t);
   float* dh = at<float>(workspace, L.dh);
-  float* zsum = at<float>(workspace, L.zsum);
-  float* dz = at<float>(workspace, L.dz);
   float* dvec = at<float>(workspace, L.dvec);
   float* dnum = at<float>(workspace, L.dnum);
   float* dden = at<float>(workspace, L.dden);
@@ -336,18 +329,17 @@ sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, co
   if (cudaMemsetAsync(dw_proj, 0, size_t(p.d) * p.d * sizeof(float), s) != cudaSuccess)
     return SLA_ERR_CUDA;
   // linear-branch preparation: D, dnum, dden, dW; then per-block A_i / a_i
-  SLA_LAUNCH("bwd_prep", s, launch_bwd_prep(p, q, d_o, w_proj, saved->o_s, saved->den, saved->h_agg, dvec, dnum,
-                             dden, dw_proj, sms, err, s));
-  SLA_LAUNCH("bwd_summ", s, launch_bwd_summ(p, q, dnum, dden, summ_hi, summ_lo, zsum, err, s));
-  // dh_j = sum over rows i with j marginal of A_i (transposed aggregation)
+  SLA_LAUNCH("bwd_prep", s, launch_bwd_prep(p, q, d_o, w_proj, saved->o_s, saved->den,
+                                            saved->hz_agg, dvec, dnum, dden, dw_proj, sms, err, s));
+  SLA_LAUNCH("bwd_summ", s, launch_bwd_summ(p, q, dnum, dden, summ_hi, summ_lo, err, s));
+  // (dh_j | dz_j) = sum over rows i with j marginal of (A_i | a_i): transposed aggregation
   SLA_LAUNCH("expand_marginal_t", s, launch_expand_marginal(p, mask->marg_bits, nullptr, mmat_t, s));
   SLA_LAUNCH("aggregate_t", s, launch_aggregate(p, mmat_t, summ_hi, summ_lo, dh, err, s));
-  SLA_LAUNCH("aggregate_z_t", s, launch_aggregate_z(p, mask->marg_bits, zsum, dz, true, s));
   // sparse branch writes dK, dV and accumulates dQ; the linear branch adds its share
   SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
                                mask->crit_col_idx, dq, dk, dv, err, s));
-  SLA_LAUNCH("bwd_linear", s, launch_bwd_linear(p, q, k, v, saved->h_agg, saved->z_agg, dh, dz, dnum, dden, dq, dk,
-                               dv, err, s));
+  SLA_LAUNCH("bwd_linear", s, launch_bwd_linear(p, q, k, v, saved->hz_agg, dh, dnum, dden, dq, dk,
+                                                dv, err, s));
   return SLA_OK;
 }
 

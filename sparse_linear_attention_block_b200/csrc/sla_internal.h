@@ -3,10 +3,10 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
-#include <cuda_bf16.h>
 
 #include "sla.h"
 
@@ -21,16 +21,18 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Blocks padded to the aggregation GEMM's 128-row tile.
 inline int pad128(int T) { return (T + 127) / 128 * 128; }
 
+// Width of one per-block summary row: the d x d matrix followed by the d-vector
+// (h_j | z_j, H_i | Z_i, and their backward counterparts).
+inline int summary_width(int d) { return d * d + d; }
+
 // Byte offsets of the regions inside the caller's workspace.
 struct WorkspaceLayout {
   size_t err;        // int32 device error word (+ padding)
   size_t qbar;       // fp32 [BH,T,d]   pooled Q
   size_t kbar;       // fp32 [BH,T,d]   pooled K
-  size_t summ_hi;    // bf16 [BH,T,d*d] h_j (forward) / A_i (backward), high part
-  size_t summ_lo;    // bf16 [BH,T,d*d] the low part (value = hi + lo)
-  size_t zsum;       // fp32 [BH,T,d]   z_j (forward) / a_i (backward)
-  size_t dh;         // fp32 [BH,T,d*d] dh_j (backward)
-  size_t dz;         // fp32 [BH,T,d]   dz_j (backward)
+  size_t summ_hi;    // bf16 [BH,T,d*d+d] (h_j|z_j) forward, (A_i|a_i) backward: high part
+  size_t summ_lo;    // bf16 [BH,T,d*d+d] the low part (value = hi + lo)
+  size_t dh;         // fp32 [BH,T,d*d+d] (dh_j|dz_j) backward
   size_t mmat;       // bf16 [BH,Tp,Tp] marginal 0/1 matrix, rows = query blocks
   size_t mmat_t;     // bf16 [BH,Tp,Tp] its transpose
   size_t dvec;       // fp32 [BH,N]     D_t = dO_t . O_s,t
@@ -59,34 +61,32 @@ cudaError_t launch_crit_csr(const Problem& p, const int8_t* cls, int32_t* col_pt
 cudaError_t launch_expand_marginal(const Problem& p, const uint32_t* marg_bits,
                                    __nv_bfloat16* mmat, __nv_bfloat16* mmat_t, cudaStream_t s);
 cudaError_t launch_summaries(const Problem& p, const void* k, const void* v,
-                             __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* zsum,
-                             int* err, cudaStream_t s);
+                             __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, int* err,
+                             cudaStream_t s);
 cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
                              const __nv_bfloat16* summ_hi, const __nv_bfloat16* summ_lo,
                              float* out, int* err, cudaStream_t s);
-cudaError_t launch_aggregate_z(const Problem& p, const uint32_t* marg_bits, const float* z,
-                               float* zout, bool transpose, cudaStream_t s);
 cudaError_t launch_fwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
                               const int32_t* crit_idx, float* o_s, float* lse, int* err,
                               cudaStream_t s);
-cudaError_t launch_fwd_linear(const Problem& p, const void* q, const float* h_agg,
-                              const float* z_agg, const void* w_proj, const float* o_s,
-                              void* o, float* den, int* err, cudaStream_t s);
+cudaError_t launch_fwd_linear(const Problem& p, const void* q, const float* hz_agg,
+                              const void* w_proj, const float* o_s, void* o, float* den,
+                              int* err, cudaStream_t s);
 cudaError_t launch_bwd_prep(const Problem& p, const void* q, const void* d_o, const void* w_proj,
-                            const float* o_s, const float* den, const float* h_agg, float* dvec,
+                            const float* o_s, const float* den, const float* hz_agg, float* dvec,
                             float* dnum, float* dden, float* dw, int num_sms, int* err,
                             cudaStream_t s);
 cudaError_t launch_bwd_summ(const Problem& p, const void* q, const float* dnum,
                             const float* dden, __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo,
-                            float* zsum, int* err, cudaStream_t s);
+                            int* err, cudaStream_t s);
 cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
                               const void* d_o, const float* lse, const float* dvec,
                               const int32_t* col_ptr, const int32_t* col_idx, float* dq,
                               float* dk, float* dv, int* err, cudaStream_t s);
 cudaError_t launch_bwd_linear(const Problem& p, const void* q, const void* k, const void* v,
-                              const float* h_agg, const float* z_agg, const float* dh,
-                              const float* dz, const float* dnum, const float* dden, float* dq,
-                              float* dk, float* dv, int* err, cudaStream_t s);
+                              const float* hz_agg, const float* dhz, const float* dnum,
+                              const float* dden, float* dq, float* dk, float* dv, int* err,
+                              cudaStream_t s);
 
 // TMA descriptor for a bf16 [BH, N, d] tensor viewed as 3D {d, N, BH} with a
 // box of {64, rows, 1} and 128-byte swizzle.  Returns false on failure.

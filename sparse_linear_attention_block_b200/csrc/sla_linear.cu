@@ -12,20 +12,21 @@
 // hi*hi + hi*lo + lo*hi (the 0/1 marginal matrix is exact in bf16, so the
 // aggregation needs only M*h_hi + M*h_lo).  Accumulation is fp32 in TMEM.
 //
+// Layout.  A per-block summary row is the d x d matrix followed by the
+// d-vector: (h_j | z_j), (H_i | Z_i); one GEMM aggregates both.
+//
 // Kernels:
-//   summaries_kernel   h_j as bf16 hi/lo planes (tcgen05), z_j fp32     HBM-bound
+//   summaries_kernel   (h_j | z_j) as bf16 hi/lo planes (tcgen05)      HBM-bound
 //   agg_gemm_kernel    fp32 C = M * (B_hi + B_lo), M the 0/1 matrix      tensor/HBM
-//   agg_z_kernel       Z_i = sum of z_j over marginal j                 small
 //   fwd_linear_kernel  O = O_s + (phi(Q) H_i / den) W_proj              HBM-bound
 #include <cuda_bf16.h>
 
 #include "sla_internal.h"
 #include "sla_ptx.cuh"
+#include "sla_tile.cuh"
 
 namespace sla {
 namespace {
-
-__device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 
 // ------------------------------------------------------------------ summaries
 // One CTA per (key block j, head); 128 threads.  phi(K_j)^T (M = feature a,
@@ -37,11 +38,11 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
                                                         const __nv_bfloat16* __restrict__ v,
                                                         __nv_bfloat16* __restrict__ summ_hi,
                                                         __nv_bfloat16* __restrict__ summ_lo,
-                                                        float* __restrict__ zsum, int N, int T,
-                                                        int* err) {
+                                                        int N, int T, int* err) {
   constexpr int kChunks = D / 8;
   constexpr int kGroups = 128 / kChunks;
   constexpr int kRowsPer = kBlock / kGroups;
+  constexpr int W = D * D + D;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -67,25 +68,29 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
   }
   const int c8 = t % kChunks, g = t / kChunks;
   const size_t off = (size_t(bh) * N + size_t(j) * kBlock) * D;
+  uint4 uk[kRowsPer], uv[kRowsPer];
+#pragma unroll
+  for (int i = 0; i < kRowsPer; ++i) {
+    const int row = g + i * kGroups;
+    uk[i] = __ldg(reinterpret_cast<const uint4*>(k + off + size_t(row) * D + c8 * 8));
+    uv[i] = __ldg(reinterpret_cast<const uint4*>(v + off + size_t(row) * D + c8 * 8));
+  }
   float zacc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
   for (int i = 0; i < kRowsPer; ++i) {
     const int row = g + i * kGroups;
-    const uint4 uk = *reinterpret_cast<const uint4*>(k + off + size_t(row) * D + c8 * 8);
-    const uint4 uv = *reinterpret_cast<const uint4*>(v + off + size_t(row) * D + c8 * 8);
-    const uint32_t w[4] = {uk.x, uk.y, uk.z, uk.w};
+    const uint32_t w[4] = {uk[i].x, uk[i].y, uk[i].z, uk[i].w};
     uint32_t ph[4], pl[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float a = phi_f(bf16_lo(w[e])), b = phi_f(bf16_hi(w[e]));
       zacc[2 * e] += a;
       zacc[2 * e + 1] += b;
-      ph[e] = pack_bf16(a, b);
-      pl[e] = pack_bf16(a - bf16_lo(ph[e]), b - bf16_hi(ph[e]));
+      split2(a, b, ph[e], pl[e]);
     }
     st_sw128_unit(sPhiH, 64, row, c8 * 8, make_uint4(ph[0], ph[1], ph[2], ph[3]));
     st_sw128_unit(sPhiL, 64, row, c8 * 8, make_uint4(pl[0], pl[1], pl[2], pl[3]));
-    st_sw128_unit(sV, 64, row, c8 * 8, uv);
+    st_sw128_unit(sV, 64, row, c8 * 8, uv[i]);
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) zred[g * D + c8 * 8 + e] = zacc[e];
@@ -104,17 +109,24 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
     }
     mma_commit(&bar);
   }
-  if (t < D) {
-    float s = 0.f;
+  const size_t rowbase = (size_t(bh) * T + j) * W;
+  if (t < D / 2) {  // z_j (fp32 sum) -> hi/lo at column d*d
+    float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-    for (int gg = 0; gg < kGroups; ++gg) s += zred[gg * D + t];
-    zsum[(size_t(bh) * T + j) * D + t] = s;
+    for (int gg = 0; gg < kGroups; ++gg) {
+      s0 += zred[gg * D + 2 * t];
+      s1 += zred[gg * D + 2 * t + 1];
+    }
+    uint32_t h, l;
+    split2(s0, s1, h, l);
+    reinterpret_cast<uint32_t*>(summ_hi + rowbase + D * D)[t] = h;
+    reinterpret_cast<uint32_t*>(summ_lo + rowbase + D * D)[t] = l;
   }
   const bool ok = mbar_wait(&bar, 0, err, nullptr);
   tc_fence_after();
   if (ok && warp * 32 < D) {
     const int a = warp * 32 + lane_id();
-    const size_t o = ((size_t(bh) * T + j) * D + a) * D;
+    const size_t o = rowbase + size_t(a) * D;
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       float vals[32];
@@ -124,11 +136,7 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x0 = vals[q4 * 8 + 2 * e], x1 = vals[q4 * 8 + 2 * e + 1];
-          hi[e] = pack_bf16(x0, x1);
-          lo[e] = pack_bf16(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
-        }
+        for (int e = 0; e < 4; ++e) split2(vals[q4 * 8 + 2 * e], vals[q4 * 8 + 2 * e + 1], hi[e], lo[e]);
         *reinterpret_cast<uint4*>(summ_hi + o + c0 + q4 * 8) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4*>(summ_lo + o + c0 + q4 * 8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
@@ -141,8 +149,8 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
 
 // ------------------------------------------------------------------ aggregation GEMM
 // C[bh][i][n] = sum_k A[bh][i][k] * (Bhi + Blo)[bh][k][n] with A the bf16 0/1
-// marginal matrix [Tp x Tp] (K-major), B the per-block summaries [T x NN]
-// as bf16 hi/lo planes (MN-major), C fp32 [T x NN].  Tile 128 x 128 x 64,
+// marginal matrix [Tp x Tp] (K-major), B the per-block summary rows [T x W]
+// as bf16 hi/lo planes (MN-major), C fp32 [T x W].  Tile 128 x 128 x 64,
 // 2-stage TMA ring, warp 0 = TMA producer, warp 1 = MMA issuer, all 4 warps
 // = epilogue.  Two CTAs per SM overlap one's epilogue with the other's MMAs.
 constexpr int kAggBN = 128, kAggBK = 64, kAggStages = 2;
@@ -231,7 +239,7 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
       float vals[32];
       tmem_ld32(tmem_addr(tmem, warp * 32, c0), vals);
       tmem_ld_wait();
-      if (i < T) {
+      if (i < T && nt * kAggBN + c0 < NN) {  // NN is a multiple of 32
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
           *reinterpret_cast<float4*>(dst + c0 + e) =
@@ -244,131 +252,81 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
   if (warp == 0) tmem_free(tmem, 128);
 }
 
-// ------------------------------------------------------------------ Z aggregation
-// Forward: Z_i = sum over j marginal in row i of z_j.
-// Transposed (backward): dz_j = sum over i with j marginal in row i of a_i.
-__global__ void agg_z_kernel(const uint32_t* __restrict__ marg_bits, const float* __restrict__ z,
-                             float* __restrict__ zout, int T, int D, int transpose) {
-  const int r = blockIdx.x, bh = blockIdx.y, a = threadIdx.x;
-  const int words = (T + 31) / 32;
-  const uint32_t* mb = marg_bits + size_t(bh) * T * words;
-  const float* zb = z + size_t(bh) * T * D;
-  float acc = 0.f;
-  if (!transpose) {
-    for (int w = 0; w < words; ++w) {
-      uint32_t bits = mb[size_t(r) * words + w];
-      while (bits) {
-        const int b = __ffs(bits) - 1;
-        bits &= bits - 1;
-        acc += zb[size_t(w * 32 + b) * D + a];
-      }
-    }
-  } else {
-    for (int i = 0; i < T; ++i)
-      if ((mb[size_t(i) * words + r / 32] >> (r % 32)) & 1u) acc += zb[size_t(i) * D + a];
-  }
-  zout[(size_t(bh) * T + r) * D + a] = acc;
-}
-
 // ------------------------------------------------------------------ linear forward epilogue
-// One CTA per pair of query blocks (128 tokens); 128 threads, one row each.
+// One CTA per pair of query blocks (128 tokens); 256 threads: thread t owns
+// row r = t % 128 (its TMEM lane) and column half t / 128.
 //   NUM_h = phi(Q) (H_{2p+h,hi} + H_{2p+h,lo})   (tcgen05; the two halves in
-//   turn, each row keeps its own), den = phi(Q) . Z (fp32), O_l = NUM / den,
-//   O = O_s + (O_l,hi + O_l,lo) W_proj.
+//   turn, each row keeps its own), den = phi(Q) . Z (fp32 from phi hi+lo),
+//   O_l = NUM / den, O = O_s + (O_l,hi + O_l,lo) W_proj.
 template <int D>
-__global__ void __launch_bounds__(128, 1) fwd_linear_kernel(
-    const __nv_bfloat16* __restrict__ q, const float* __restrict__ h_agg,
-    const float* __restrict__ z_agg, const __nv_bfloat16* __restrict__ w_proj,
-    const float* __restrict__ o_s, __nv_bfloat16* __restrict__ o, float* __restrict__ den_out,
-    int N, int T, int* err) {
+__global__ void __launch_bounds__(256, 1) fwd_linear_kernel(
+    const __nv_bfloat16* __restrict__ q, const float* __restrict__ hz_agg,
+    const __nv_bfloat16* __restrict__ w_proj, const float* __restrict__ o_s,
+    __nv_bfloat16* __restrict__ o, float* __restrict__ den_out, int N, int T, int* err) {
   constexpr int kTile = 128 * 128 * 2;  // 128 rows x 2 chunks (D = 64 padded)
+  constexpr int W = D * D + D;
+  constexpr int DH = D / 2;             // columns per thread
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sA = base;                  // phi(Q), later O_l hi    (K-major, 128 rows)
-  uint8_t* sA2 = sA + kTile;           // O_l lo                  (K-major, 128 rows)
-  uint8_t* sHh = sA2 + kTile;          // H hi                    (MN-major, D k-rows)
+  uint8_t* sA = base;                  // phi(Q) hi, later O_l hi  (K-major, 128 rows)
+  uint8_t* sA2 = sA + kTile;           // phi(Q) lo, later O_l lo
+  uint8_t* sHh = sA2 + kTile;          // H hi                      (MN-major, D k-rows)
   uint8_t* sHl = sHh + kTile;          // H lo
-  uint8_t* sW = sHl + kTile;           // W_proj                  (MN-major, D k-rows)
+  uint8_t* sW = sHl + kTile;           // W_proj                    (MN-major, D k-rows)
   __shared__ float sZ[2][D];
+  __shared__ float sDen[2][128];
   __shared__ uint64_t bar[3];
   __shared__ uint32_t tmem_base;
   const int p = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, warp = t / 32;
-  const int half = t >> 6;
-  const int blk = 2 * p + half;
-  const bool row_ok = blk < T;
-  const size_t tok = size_t(p) * 128 + t;
+  const int r = t & 127, ch = t >> 7, half = r >> 6;
+  const bool row_ok = 2 * p + half < T;
+  const int valid_rows = (2 * p + 1 < T) ? 128 : 64;
+  const size_t tok = size_t(p) * 128 + r;
+  const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
   if (warp == 0) tmem_alloc(&tmem_base, 2 * D);
   if (t == 0) {
     for (int b = 0; b < 3; ++b) mbar_init(&bar[b], 1);
     fence_barrier_init();
   }
-  for (int e = t; e < D * (D / 8); e += 128) {
-    const int a = e / (D / 8), c8 = e % (D / 8);
-    st_sw128_unit(sW, D, a, c8 * 8, *reinterpret_cast<const uint4*>(w_proj + size_t(a) * D + c8 * 8));
-  }
-  for (int e = t; e < 2 * D; e += 128) {
+  for (int e = t; e < 2 * D; e += 256) {
     const int m = e / D, b2 = 2 * p + m;
-    sZ[m][e % D] = b2 < T ? z_agg[(size_t(bh) * T + b2) * D + (e % D)] : 0.f;
+    sZ[m][e % D] = b2 < T ? hz_agg[(size_t(bh) * T + b2) * W + D * D + (e % D)] : 0.f;
   }
+  load_rows_sw<D>(sW, D, w_proj, D, t, 256);
+  load_phi_sw<D>(sA, sA2, 128, q + (size_t(bh) * N + size_t(p) * 128) * D, valid_rows, t, 256);
+  load_split_sw<D>(sHh, sHl, D, hz_agg + (size_t(bh) * T + 2 * p) * W, D, t, 256);
+  fence_proxy_async_smem();
+  tc_fence_before();
   __syncthreads();
-  // phi(Q) row t -> sA (bf16, K-major) and den = phi(Q) . Z_half (fp32)
-  float den = 0.f;
+  tc_fence_after();
+  // den = phi(Q) . Z_half, fp32 from the hi + lo parts
   {
-    const __nv_bfloat16* qrow = q + (size_t(bh) * N + tok) * D;
-#pragma unroll 4
-    for (int c8 = 0; c8 < D / 8; ++c8) {
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (row_ok) u = *reinterpret_cast<const uint4*>(qrow + c8 * 8);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-      uint32_t pw[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float a = phi_f(bf16_lo(w[e])), b = phi_f(bf16_hi(w[e]));
-        den = fmaf(a, sZ[half][c8 * 8 + 2 * e], den);
-        den = fmaf(b, sZ[half][c8 * 8 + 2 * e + 1], den);
-        pw[e] = pack_bf16(a, b);
-      }
-      st_sw128_unit(sA, 128, t, c8 * 8, make_uint4(pw[0], pw[1], pw[2], pw[3]));
-    }
+    float acc = 0.f;
+    for (int c = ch * DH; c < (ch + 1) * DH; ++c)
+      acc = fmaf(ld_sw_bf16(sA, 128, r, c) + ld_sw_bf16(sA2, 128, r, c), sZ[half][c], acc);
+    sDen[ch][r] = acc;
   }
-  const uint32_t tmem_hold = 0;
-  (void)tmem_hold;
+  const uint32_t tmem = tmem_base;
   bool ok = true;
+  constexpr uint32_t idesc = idesc_bf16(128, D, 0, 1);
   for (int m = 0; m < 2; ++m) {
-    // H_{2p+m} (fp32) -> hi / lo tiles
-    const int b2 = 2 * p + m;
-    const float* hsrc = h_agg + (size_t(bh) * T + (b2 < T ? b2 : 0)) * D * D;
-    for (int e = t; e < D * (D / 8); e += 128) {
-      const int a = e / (D / 8), c8 = e % (D / 8);
-      float x[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      if (b2 < T) {
-        const float4 u0 = *reinterpret_cast<const float4*>(hsrc + size_t(a) * D + c8 * 8);
-        const float4 u1 = *reinterpret_cast<const float4*>(hsrc + size_t(a) * D + c8 * 8 + 4);
-        x[0] = u0.x; x[1] = u0.y; x[2] = u0.z; x[3] = u0.w;
-        x[4] = u1.x; x[5] = u1.y; x[6] = u1.z; x[7] = u1.w;
-      }
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        hi[i] = pack_bf16(x[2 * i], x[2 * i + 1]);
-        lo[i] = pack_bf16(x[2 * i] - bf16_lo(hi[i]), x[2 * i + 1] - bf16_hi(hi[i]));
-      }
-      st_sw128_unit(sHh, D, a, c8 * 8, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-      st_sw128_unit(sHl, D, a, c8 * 8, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+    if (m == 1) {
+      const int b2 = 2 * p + 1;
+      load_split_sw<D>(sHh, sHl, D, hz_agg + (size_t(bh) * T + (b2 < T ? b2 : 0)) * W,
+                       b2 < T ? D : 0, t, 256);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
     if (t == 0) {
-      constexpr uint32_t idesc = idesc_bf16(128, D, 0, 1);
       const uint32_t a0 = smem_u32(sA);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
-        mma_ss(tmem_base + m * D, desc_kmajor(a0, 128, ks), desc_mnmajor(smem_u32(sHh), D, ks),
+        mma_ss(tmem + m * D, desc_kmajor(a0, 128, ks), desc_mnmajor(smem_u32(sHh), D, ks),
                idesc, ks > 0);
-        mma_ss(tmem_base + m * D, desc_kmajor(a0, 128, ks), desc_mnmajor(smem_u32(sHl), D, ks),
+        mma_ss(tmem + m * D, desc_kmajor(a0, 128, ks), desc_mnmajor(smem_u32(sHl), D, ks),
                idesc, 1);
       }
       mma_commit(&bar[m]);
@@ -376,27 +334,25 @@ __global__ void __launch_bounds__(128, 1) fwd_linear_kernel(
     ok = mbar_wait(&bar[m], 0, err, nullptr) && ok;
     tc_fence_after();
   }
-  const uint32_t tmem = tmem_base;
+  __syncthreads();  // sDen complete; phi(Q) tiles no longer read by any MMA
+  const float den = sDen[0][r] + sDen[1][r];
   const float inv = (row_ok && den > 0.f) ? 1.0f / den : 0.0f;
-  if (row_ok) den_out[size_t(bh) * N + tok] = den;
+  if (row_ok && ch == 0) den_out[size_t(bh) * N + tok] = den;
   // O_l = NUM / den, split into hi + lo bf16 (K-major rows)
 #pragma unroll 1
-  for (int c0 = 0; c0 < D; c0 += 32) {
+  for (int c0 = ch * DH; c0 < (ch + 1) * DH; c0 += 32) {
     float vals[32];
-    tmem_ld32(tmem_addr(tmem + half * D, warp * 32, c0), vals);
+    tmem_ld32(tmem + lane_base + half * D + c0, vals);
     tmem_ld_wait();
 #pragma unroll
     for (int u8 = 0; u8 < 4; ++u8) {
       uint32_t hi[4], lo[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float x0 = ok ? vals[u8 * 8 + 2 * e] * inv : 0.f;
-        const float x1 = ok ? vals[u8 * 8 + 2 * e + 1] * inv : 0.f;
-        hi[e] = pack_bf16(x0, x1);
-        lo[e] = pack_bf16(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
-      }
-      st_sw128_unit(sA, 128, t, c0 + u8 * 8, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-      st_sw128_unit(sA2, 128, t, c0 + u8 * 8, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+      for (int e = 0; e < 4; ++e)
+        split2(ok ? vals[u8 * 8 + 2 * e] * inv : 0.f, ok ? vals[u8 * 8 + 2 * e + 1] * inv : 0.f,
+               hi[e], lo[e]);
+      st_sw128_unit(sA, 128, r, c0 + u8 * 8, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+      st_sw128_unit(sA2, 128, r, c0 + u8 * 8, make_uint4(lo[0], lo[1], lo[2], lo[3]));
     }
   }
   fence_proxy_async_smem();
@@ -404,7 +360,6 @@ __global__ void __launch_bounds__(128, 1) fwd_linear_kernel(
   __syncthreads();
   tc_fence_after();
   if (t == 0) {
-    constexpr uint32_t idesc = idesc_bf16(128, D, 0, 1);
     const uint32_t b0 = smem_u32(sW);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
@@ -419,21 +374,23 @@ __global__ void __launch_bounds__(128, 1) fwd_linear_kernel(
     const float* osrow = o_s + (size_t(bh) * N + tok) * D;
     __nv_bfloat16* orow = o + (size_t(bh) * N + tok) * D;
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
+    for (int c0 = ch * DH; c0 < (ch + 1) * DH; c0 += 32) {
       float vals[32];
-      tmem_ld32(tmem_addr(tmem, warp * 32, c0), vals);
+      tmem_ld32(tmem + lane_base + c0, vals);
       tmem_ld_wait();
       if (row_ok && ok) {
+        float4 s[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s[u] = __ldg(reinterpret_cast<const float4*>(osrow + c0) + u);
 #pragma unroll
         for (int u8 = 0; u8 < 4; ++u8) {
-          const float4 s0 = *reinterpret_cast<const float4*>(osrow + c0 + u8 * 8);
-          const float4 s1 = *reinterpret_cast<const float4*>(osrow + c0 + u8 * 8 + 4);
-          uint4 r;
-          r.x = pack_bf16(s0.x + vals[u8 * 8 + 0], s0.y + vals[u8 * 8 + 1]);
-          r.y = pack_bf16(s0.z + vals[u8 * 8 + 2], s0.w + vals[u8 * 8 + 3]);
-          r.z = pack_bf16(s1.x + vals[u8 * 8 + 4], s1.y + vals[u8 * 8 + 5]);
-          r.w = pack_bf16(s1.z + vals[u8 * 8 + 6], s1.w + vals[u8 * 8 + 7]);
-          *reinterpret_cast<uint4*>(orow + c0 + u8 * 8) = r;
+          const float4 s0 = s[2 * u8], s1 = s[2 * u8 + 1];
+          uint4 rr;
+          rr.x = pack_bf16(s0.x + vals[u8 * 8 + 0], s0.y + vals[u8 * 8 + 1]);
+          rr.y = pack_bf16(s0.z + vals[u8 * 8 + 2], s0.w + vals[u8 * 8 + 3]);
+          rr.z = pack_bf16(s1.x + vals[u8 * 8 + 4], s1.y + vals[u8 * 8 + 5]);
+          rr.w = pack_bf16(s1.z + vals[u8 * 8 + 6], s1.w + vals[u8 * 8 + 7]);
+          *reinterpret_cast<uint4*>(orow + c0 + u8 * 8) = rr;
         }
       }
     }
@@ -451,8 +408,8 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }  // namespace
 
 cudaError_t launch_summaries(const Problem& p, const void* k, const void* v,
-                             __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* zsum,
-                             int* err, cudaStream_t s) {
+                             __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, int* err,
+                             cudaStream_t s) {
   dim3 grid(p.T, p.BH);
   const int groups = 128 / (p.d / 8);
   const size_t smem = 1024 + 32768 + (p.d / 64) * 8192 + sizeof(float) * groups * p.d;
@@ -461,12 +418,12 @@ cudaError_t launch_summaries(const Problem& p, const void* k, const void* v,
     if ((e = set_smem(summaries_kernel<128>, smem)) != cudaSuccess) return e;
     summaries_kernel<128><<<grid, 128, smem, s>>>((const __nv_bfloat16*)k,
                                                   (const __nv_bfloat16*)v, summ_hi, summ_lo,
-                                                  zsum, p.N, p.T, err);
+                                                  p.N, p.T, err);
   } else {
     if ((e = set_smem(summaries_kernel<64>, smem)) != cudaSuccess) return e;
     summaries_kernel<64><<<grid, 128, smem, s>>>((const __nv_bfloat16*)k,
-                                                 (const __nv_bfloat16*)v, summ_hi, summ_lo, zsum,
-                                                 p.N, p.T, err);
+                                                 (const __nv_bfloat16*)v, summ_hi, summ_lo, p.N,
+                                                 p.T, err);
   }
   return cudaGetLastError();
 }
@@ -474,7 +431,7 @@ cudaError_t launch_summaries(const Problem& p, const void* k, const void* v,
 cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
                              const __nv_bfloat16* summ_hi, const __nv_bfloat16* summ_lo,
                              float* out, int* err, cudaStream_t s) {
-  const int NN = p.d * p.d;
+  const int NN = summary_width(p.d);
   CUtensorMap ta, tbh, tbl;
   if (!make_tmap_3d(&ta, mmat, p.Tp, p.Tp, p.BH, 64, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_3d(&tbh, summ_hi, NN, p.T, p.BH, 64, 64)) return cudaErrorInvalidValue;
@@ -482,34 +439,27 @@ cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
   const size_t smem = 1024 + kAggStages * kAggStageBytes;
   cudaError_t e = set_smem(agg_gemm_kernel, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.Tp / 128, NN / kAggBN, p.BH);
+  dim3 grid(p.Tp / 128, (NN + kAggBN - 1) / kAggBN, p.BH);
   agg_gemm_kernel<<<grid, 128, smem, s>>>(ta, tbh, tbl, out, p.T, p.Tp, NN, err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_aggregate_z(const Problem& p, const uint32_t* marg_bits, const float* z,
-                               float* zout, bool transpose, cudaStream_t s) {
-  dim3 grid(p.T, p.BH);
-  agg_z_kernel<<<grid, p.d, 0, s>>>(marg_bits, z, zout, p.T, p.d, transpose ? 1 : 0);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_fwd_linear(const Problem& p, const void* q, const float* h_agg,
-                              const float* z_agg, const void* w_proj, const float* o_s,
-                              void* o, float* den, int* err, cudaStream_t s) {
+cudaError_t launch_fwd_linear(const Problem& p, const void* q, const float* hz_agg,
+                              const void* w_proj, const float* o_s, void* o, float* den,
+                              int* err, cudaStream_t s) {
   dim3 grid((p.T + 1) / 2, p.BH);
   const size_t smem = 1024 + 5 * (128 * 128 * 2);
   cudaError_t e;
   if (p.d == 128) {
     if ((e = set_smem(fwd_linear_kernel<128>, smem)) != cudaSuccess) return e;
-    fwd_linear_kernel<128><<<grid, 128, smem, s>>>(
-        (const __nv_bfloat16*)q, h_agg, z_agg, (const __nv_bfloat16*)w_proj, o_s,
-        (__nv_bfloat16*)o, den, p.N, p.T, err);
+    fwd_linear_kernel<128><<<grid, 256, smem, s>>>((const __nv_bfloat16*)q, hz_agg,
+                                                   (const __nv_bfloat16*)w_proj, o_s,
+                                                   (__nv_bfloat16*)o, den, p.N, p.T, err);
   } else {
     if ((e = set_smem(fwd_linear_kernel<64>, smem)) != cudaSuccess) return e;
-    fwd_linear_kernel<64><<<grid, 128, smem, s>>>(
-        (const __nv_bfloat16*)q, h_agg, z_agg, (const __nv_bfloat16*)w_proj, o_s,
-        (__nv_bfloat16*)o, den, p.N, p.T, err);
+    fwd_linear_kernel<64><<<grid, 256, smem, s>>>((const __nv_bfloat16*)q, hz_agg,
+                                                  (const __nv_bfloat16*)w_proj, o_s,
+                                                  (__nv_bfloat16*)o, den, p.N, p.T, err);
   }
   return cudaGetLastError();
 }

@@ -54,7 +54,7 @@ def test_query_sizes_wan_shape(L):
     assert s.crit_idx_bytes == 12 * 512 * 26 * 4
     assert s.marg_bits_bytes == 12 * 512 * 16 * 4
     assert s.o_s_bytes == 12 * 32768 * 128 * 4
-    assert s.h_agg_bytes == 12 * 512 * 128 * 128 * 4
+    assert s.hz_agg_bytes == 12 * 512 * (128 * 128 + 128) * 4
     assert s.workspace_bytes > 0
 
 
