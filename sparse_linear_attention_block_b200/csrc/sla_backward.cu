@@ -41,8 +41,7 @@ __global__ void __launch_bounds__(256, 1) bwd_prep_kernel(
     int BH, int* err) {
   constexpr int W = D * D + D, DH = D / 2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* base = align_smem_1024(smem_raw);
   uint8_t* sA = base;                  // phi(Q)                      [t][a]
   uint8_t* sDO = sA + kTile32;         // dO                          [t][c]
   uint8_t* sW = sDO + kTile32;         // W_proj                      [a][c]
@@ -201,8 +200,7 @@ __global__ void __launch_bounds__(256, 1) bwd_summ_kernel(
     __nv_bfloat16* __restrict__ summ_lo, int N, int T, int* err) {
   constexpr int W = D * D + D, DH = D / 2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* base = align_smem_1024(smem_raw);
   uint8_t* sQh = base;                 // phi(Q) hi [t][a]
   uint8_t* sQl = sQh + kTile32;        // phi(Q) lo
   uint8_t* sNh = sQl + kTile32;        // dnum hi   [t][c]
@@ -305,8 +303,7 @@ __global__ void __launch_bounds__(256, 1) bwd_linear_kernel(
     float* __restrict__ dv, int N, int T, int* err) {
   constexpr int W = D * D + D, DH = D / 2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* base = align_smem_1024(smem_raw);
   uint8_t* s0 = base;             // phase 1: dnum hi | phase 2: V         [t][c]
   uint8_t* s1 = s0 + kTile32;     // phase 1: dnum lo | phase 2: phi(K) hi [t][a]
   uint8_t* s2 = s1 + kTile32;     //                    phase 2: phi(K) lo [t][a]

@@ -68,29 +68,96 @@ __device__ __forceinline__ uint32_t ordered_bits(float x) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Distinct 64-bit rank key: larger = earlier in (score desc, index asc).
-__device__ __forceinline__ uint64_t rank_key(float s, int j) {
-  return (uint64_t(ordered_bits(s)) << 32) | uint64_t(0xFFFFFFFFu - uint32_t(j));
+// The n-th element (n >= 1) of one row in the order (score desc, index asc),
+// or with `flip` in the reverse order (score asc, index desc), found by one
+// warp: an exact radix select on the order-preserving 32-bit score (four
+// 8-bit digits, most significant first, histogram in shared memory) followed
+// by one pass that breaks ties by index.  Returns the element's (possibly
+// complemented) ordered score v and its index jt; an element is at or before
+// it in the order iff its value is > v, or == v with index <= jt (>= jt when
+// flipped).
+struct Threshold {
+  uint32_t v;
+  int jt;
+};
+
+__device__ Threshold warp_select(const float* row, int T, int n, bool flip, uint32_t* hist) {
+  constexpr uint32_t kAll = 0xFFFFFFFFu;
+  const int lane = lane_id();
+  uint32_t prefix = 0, mask = 0;
+  int need = n;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int j = lane; j < T; j += 32) {
+      uint32_t o = ordered_bits(row[j]);
+      if (flip) o = ~o;
+      if ((o & mask) == prefix) atomicAdd(&hist[(o >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    // lane l owns digits 255-8l down to 248-8l; scan from the top digit
+    uint32_t c[8];
+    int s = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      c[e] = hist[255 - 8 * lane - e];
+      s += int(c[e]);
+    }
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kAll, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int excl = incl - s;
+    const bool mine = excl < need && need <= incl;
+    const int src = __ffs(__ballot_sync(kAll, mine)) - 1;
+    int digit = 0, above = 0;
+    if (mine) {
+      int acc = excl;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (acc + int(c[e]) >= need) {
+          digit = 255 - 8 * lane - e;
+          above = acc;
+          break;
+        }
+        acc += int(c[e]);
+      }
+    }
+    digit = __shfl_sync(kAll, digit, src);
+    above = __shfl_sync(kAll, above, src);
+    prefix |= uint32_t(digit) << shift;
+    mask |= 255u << shift;
+    need -= above;
+    __syncwarp();
+  }
+  // ties on the score: the need-th equal element in index order
+  int jt = -1, seen = 0;
+  const int last = ((T - 1) / 32) * 32;
+  for (int step = 0; step <= last / 32 && jt < 0; ++step) {
+    const int j0 = flip ? last - 32 * step : 32 * step;
+    const int j = j0 + lane;
+    bool eq = false;
+    if (j < T) {
+      uint32_t o = ordered_bits(row[j]);
+      if (flip) o = ~o;
+      eq = o == prefix;
+    }
+    uint32_t m = __ballot_sync(kAll, eq);
+    const int cnt = __popc(m);
+    if (seen + cnt >= need) {
+      for (int k = need - seen; k > 1; --k) m &= flip ? ~(1u << (31 - __clz(m))) : (m - 1);
+      jt = j0 + (flip ? 31 - __clz(m) : __ffs(m) - 1);
+    }
+    seen += cnt;
+  }
+  return {prefix, jt};
 }
 
-// The n-th largest of the keys of one row (n >= 1), computed by one warp with
-// a bitwise greedy search: the result is the largest K with
-// #{key >= K} >= n, which is the n-th largest because keys are distinct.
-// `flip` ranks the complemented keys instead (n-th smallest original key).
-__device__ uint64_t warp_kth_largest(const float* row, int T, int n, bool flip) {
-  uint64_t K = 0;
-  for (int bit = 63; bit >= 0; --bit) {
-    const uint64_t cand = K | (1ull << bit);
-    int cnt = 0;
-    for (int j = lane_id(); j < T; j += 32) {
-      uint64_t key = rank_key(row[j], j);
-      if (flip) key = ~key;
-      cnt += key >= cand;
-    }
-    cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-    if (cnt >= n) K = cand;
-  }
-  return K;
+__device__ __forceinline__ bool before_or_at(uint32_t o, int j, Threshold t, bool flip) {
+  if (flip) o = ~o;
+  return o > t.v || (o == t.v && (flip ? j >= t.jt : j <= t.jt));
 }
 
 constexpr int kRowsPerCta = 8;  // one warp per query-block row
@@ -151,8 +218,9 @@ __global__ void __launch_bounds__(256) classify_kernel(
   }
   if (!row_ok) return;
 
-  const uint64_t kh = n_crit > 0 ? warp_kth_largest(row, T, n_crit, false) : ~0ull;
-  const uint64_t kl = n_negl > 0 ? warp_kth_largest(row, T, n_negl, true) : ~0ull;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sk + kKTile * kStride) + warp * 256;
+  const Threshold th = n_crit > 0 ? warp_select(row, T, n_crit, false, hist) : Threshold{0, -1};
+  const Threshold tl = n_negl > 0 ? warp_select(row, T, n_negl, true, hist) : Threshold{0, -1};
   const size_t rbase = size_t(bh) * T + i;
   int8_t* crow = cls + rbase * T;
   int32_t* idx = crit_idx + rbase * n_crit;
@@ -164,16 +232,16 @@ __global__ void __launch_bounds__(256) classify_kernel(
     int c = 0;
     bool in = j < T;
     if (in) {
-      const uint64_t key = rank_key(row[j], j);
-      if (n_crit > 0 && key >= kh) c = 1;
-      else if (n_negl > 0 && ~key >= kl) c = -1;
+      const uint32_t o = ordered_bits(row[j]);
+      if (n_crit > 0 && before_or_at(o, j, th, false)) c = 1;
+      else if (n_negl > 0 && before_or_at(o, j, tl, true)) c = -1;
       crow[j] = int8_t(c);
     }
     const uint32_t crit_mask = __ballot_sync(0xFFFFFFFFu, in && c == 1);
     const uint32_t marg_mask = __ballot_sync(0xFFFFFFFFu, in && c == 0);
     if (in && c == 1) {
       const int pos = written + __popc(crit_mask & ((1u << lane) - 1u));
-      idx[pos] = j;
+      if (pos < n_crit) idx[pos] = j;
     }
     written += __popc(crit_mask);
     if (lane == 0) mrow[j0 / 32] = marg_mask;
@@ -181,27 +249,38 @@ __global__ void __launch_bounds__(256) classify_kernel(
 }
 
 // ------------------------------------------------------------------ column CSR
-// One CTA per head: for every key block j the ascending list of query blocks
-// i with cls[i][j] == +1.  Offsets are relative to the head.
-__global__ void __launch_bounds__(1024) crit_csr_kernel(const int8_t* __restrict__ cls,
-                                                        int32_t* __restrict__ col_ptr,
-                                                        int32_t* __restrict__ col_idx, int T,
-                                                        int n_crit) {
+// For every key block j the ascending list of query blocks i with
+// cls[i][j] == +1 (offsets relative to the head), in three launches:
+//   csr_count_kernel  one warp per column: count -> col_ptr[j+1]
+//   csr_scan_kernel   one CTA per head: inclusive scan of col_ptr[1..T] in place
+//   csr_fill_kernel   one warp per column: rows in ascending order by ballots
+constexpr int kCsrWarps = 8;
+
+__global__ void __launch_bounds__(256) csr_count_kernel(const int8_t* __restrict__ cls,
+                                                        int32_t* __restrict__ col_ptr, int T) {
+  const int bh = blockIdx.y, j = blockIdx.x * kCsrWarps + threadIdx.x / 32, lane = lane_id();
+  if (j >= T) return;
+  const int8_t* c = cls + size_t(bh) * T * T + j;
+  int cnt = 0;
+#pragma unroll 4
+  for (int i = lane; i < T; i += 32) cnt += c[size_t(i) * T] == 1;
+  cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+  if (lane == 0) col_ptr[size_t(bh) * (T + 1) + j + 1] = cnt;
+}
+
+__global__ void __launch_bounds__(1024) csr_scan_kernel(int32_t* __restrict__ col_ptr, int T) {
   __shared__ int wsum[32];
   __shared__ int carry;
-  const int bh = blockIdx.x;
-  const int8_t* c = cls + size_t(bh) * T * T;
-  int32_t* ptr = col_ptr + size_t(bh) * (T + 1);
-  int32_t* out = col_idx + size_t(bh) * T * n_crit;
-  if (threadIdx.x == 0) carry = 0;
+  int32_t* ptr = col_ptr + size_t(blockIdx.x) * (T + 1);
+  if (threadIdx.x == 0) {
+    carry = 0;
+    ptr[0] = 0;
+  }
   __syncthreads();
-  for (int j0 = 0; j0 < T; j0 += blockDim.x) {
+  for (int j0 = 1; j0 <= T; j0 += blockDim.x) {
     const int j = j0 + threadIdx.x;
-    int cnt = 0;
-    if (j < T)
-      for (int i = 0; i < T; ++i) cnt += c[size_t(i) * T + j] == 1;
-    // block-wide exclusive scan of cnt
-    int x = cnt;
+    const int v = j <= T ? ptr[j] : 0;
+    int x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
@@ -210,28 +289,41 @@ __global__ void __launch_bounds__(1024) crit_csr_kernel(const int8_t* __restrict
     if (lane_id() == 31) wsum[threadIdx.x / 32] = x;
     __syncthreads();
     if (threadIdx.x < 32) {
-      int s = threadIdx.x < (blockDim.x + 31) / 32 ? wsum[threadIdx.x] : 0;
+      int s = wsum[threadIdx.x];
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xFFFFFFFFu, s, o);
         if (lane_id() >= o) s += y;
       }
-      wsum[threadIdx.x] = s;  // inclusive
+      wsum[threadIdx.x] = s;  // inclusive over warps
     }
     __syncthreads();
     const int warp_off = threadIdx.x >= 32 ? wsum[threadIdx.x / 32 - 1] : 0;
-    const int start = carry + warp_off + x - cnt;
-    if (j < T) {
-      ptr[j] = start;
-      int pos = start;
-      for (int i = 0; i < T; ++i)
-        if (c[size_t(i) * T + j] == 1) out[pos++] = i;
-    }
+    if (j <= T) ptr[j] = carry + warp_off + x;
     __syncthreads();
     if (threadIdx.x == 0) carry += wsum[31];
     __syncthreads();
   }
-  if (threadIdx.x == 0) ptr[T] = carry;
+}
+
+__global__ void __launch_bounds__(256) csr_fill_kernel(const int8_t* __restrict__ cls,
+                                                       const int32_t* __restrict__ col_ptr,
+                                                       int32_t* __restrict__ col_idx, int T,
+                                                       int n_crit) {
+  const int bh = blockIdx.y, j = blockIdx.x * kCsrWarps + threadIdx.x / 32, lane = lane_id();
+  if (j >= T) return;
+  const int8_t* c = cls + size_t(bh) * T * T + j;
+  int32_t* out = col_idx + size_t(bh) * T * n_crit;
+  const int cap = T * n_crit;
+  int pos = col_ptr[size_t(bh) * (T + 1) + j];
+  for (int i0 = 0; i0 < T; i0 += 32) {
+    const int i = i0 + lane;
+    const bool hit = i < T && c[size_t(i) * T] == 1;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, hit);
+    const int at = pos + __popc(m & ((1u << lane) - 1u));
+    if (hit && at < cap) out[at] = i;
+    pos += __popc(m);
+  }
 }
 
 // ------------------------------------------------------------------ marginal matrix
@@ -277,7 +369,8 @@ cudaError_t launch_classify(const Problem& p, const float* qbar, const float* kb
                             int32_t* crit_idx, uint32_t* marg_bits, cudaStream_t s) {
   dim3 grid((p.T + kRowsPerCta - 1) / kRowsPerCta, p.BH);
   const size_t smem =
-      sizeof(float) * (size_t(kRowsPerCta) * p.T + kRowsPerCta * p.d + kKTile * (p.d + 4));
+      sizeof(float) * (size_t(kRowsPerCta) * p.T + kRowsPerCta * p.d + kKTile * (p.d + 4)) +
+      sizeof(uint32_t) * kRowsPerCta * 256;  // per-warp radix histograms
   cudaError_t e;
   if (p.d == 128) {
     e = cudaFuncSetAttribute(classify_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -299,8 +392,10 @@ cudaError_t launch_classify(const Problem& p, const float* qbar, const float* kb
 
 cudaError_t launch_crit_csr(const Problem& p, const int8_t* cls, int32_t* col_ptr,
                             int32_t* col_idx, cudaStream_t s) {
-  const int threads = p.T >= 1024 ? 1024 : ((p.T + 31) / 32) * 32;
-  crit_csr_kernel<<<p.BH, threads, 0, s>>>(cls, col_ptr, col_idx, p.T, p.n_crit);
+  dim3 grid((p.T + kCsrWarps - 1) / kCsrWarps, p.BH);
+  csr_count_kernel<<<grid, 32 * kCsrWarps, 0, s>>>(cls, col_ptr, p.T);
+  csr_scan_kernel<<<p.BH, 1024, 0, s>>>(col_ptr, p.T);
+  if (p.n_crit > 0) csr_fill_kernel<<<grid, 32 * kCsrWarps, 0, s>>>(cls, col_ptr, col_idx, p.T, p.n_crit);
   return cudaGetLastError();
 }
 

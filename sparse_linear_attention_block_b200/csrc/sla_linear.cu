@@ -44,8 +44,7 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
   constexpr int kRowsPer = kBlock / kGroups;
   constexpr int W = D * D + D;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* base = align_smem_1024(smem_raw);
   uint8_t* sPhiH = base;           // 2 chunks x 64 rows x 128 B = 16 KB (M padded to 128)
   uint8_t* sPhiL = base + 16384;   // same for the lo part
   uint8_t* sV = base + 32768;      // D/64 chunks x 8 KB
@@ -164,8 +163,7 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
                                                        float* __restrict__ out, int T, int Tp,
                                                        int NN, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* base = align_smem_1024(smem_raw);
   __shared__ uint64_t full[kAggStages], empty[kAggStages], acc_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
@@ -267,8 +265,7 @@ __global__ void __launch_bounds__(256, 1) fwd_linear_kernel(
   constexpr int W = D * D + D;
   constexpr int DH = D / 2;             // columns per thread
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* base = align_smem_1024(smem_raw);
   uint8_t* sA = base;                  // phi(Q) hi, later O_l hi  (K-major, 128 rows)
   uint8_t* sA2 = sA + kTile;           // phi(Q) lo, later O_l lo
   uint8_t* sHh = sA2 + kTile;          // H hi                      (MN-major, D k-rows)

@@ -27,6 +27,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 
+// First 1024-byte aligned address at or after the dynamic shared buffer `p`,
+// derived by pointer arithmetic so that the compiler keeps treating it as
+// shared memory (a round trip through an integer would make every access a
+// generic one).
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* p) {
+  return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ bool elect_one() { return lane_id() == 0; }
 
 // Device error word: first error wins.

@@ -17,8 +17,10 @@
 //                    one computes P, dS while the other drains its dQ;
 //   warp 8           TMA producer: K, V once; Q_i, dO_i, LSE_i, D_i per stage;
 //   warp 9           single-thread tcgen05 issuer.
-// dQ_i^T leaves TMEM into the query block's (now free) stage buffer as fp32
-// [64 q][d] and is added to dQ in global memory by one TMA bulk reduce-add.
+// The warpgroup returns the stage to the producer as soon as the MMAs of its
+// query block are done, reads dQ_i^T from TMEM into registers (freeing the
+// buffer for the next S^T) and adds it into fp32 dQ with coalesced
+// fire-and-forget reductions.
 // TMEM (512 columns): per buffer b in {0,1}: S^T at 128b (later dQ^T), dP^T at
 // 128b + 64; dV at 256, dK at 256 + d.
 #include <cuda_bf16.h>
@@ -50,24 +52,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// global[dst .. dst+bytes) += shared[src ..) as fp32, one bulk operation
-__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes) {
-  asm volatile(
-      "cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-          reinterpret_cast<uint64_t>(dst)),
-      "r"(smem_u32(src)), "r"(bytes)
-      : "memory");
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-__device__ __forceinline__ void bulk_wait_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
 template <int D>
 __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -78,8 +62,7 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
     float* __restrict__ dv, int* err) {
   using L = SbSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* base = align_smem_1024(smem_raw);
   uint8_t* sK = base;
   uint8_t* sV = sK + L::kKV;
   uint8_t* sSt = sV + L::kKV;
@@ -88,7 +71,7 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
   uint8_t* uflag = reinterpret_cast<uint8_t*>(ulist + 2 * T);
 
   __shared__ uint64_t kv_full, st_full[kNSt], st_empty[kNSt], s_full[2], p_full[2], m_done[2],
-      tfree[2], stg_ready[2], fin;
+      tfree[2], fin;
   __shared__ uint32_t tmem_base;
   __shared__ int n_union, abort_flag;
   const int qp = blockIdx.x, bh = blockIdx.y;
@@ -109,38 +92,47 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
       mbar_init(&p_full[b], 128);
       mbar_init(&m_done[b], 1);
       mbar_init(&tfree[b], 128);
-      mbar_init(&stg_ready[b], 128);
     }
     mbar_init(&fin, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
-  if (threadIdx.x == 256) {
+  if (warp == 8) {
     // union of the critical query blocks of key blocks 2q and 2q+1; flag bit h
-    // = query block critical for key block 2q+h
+    // = query block critical for key block 2q+h.  The two column lists are
+    // staged in the (still idle) stage buffers with coalesced loads, then
+    // merged from shared memory by one lane.
     const int32_t* cp = col_ptr + size_t(bh) * (T + 1);
     const int32_t* ci = col_idx + size_t(bh) * T * n_crit;
     int a = cp[kb0], ae = cp[kb0 + 1];
     int b = has1 ? cp[kb1] : 0, be = has1 ? cp[kb1 + 1] : 0;
     const int cap = T * n_crit;
-    if (a < 0 || ae > cap || a > ae || b < 0 || be > cap || b > be) {
-      set_error(err, SLA_ERR_DEVICE);
+    if (a < 0 || ae > cap || a > ae || b < 0 || be > cap || b > be || ae - a > T || be - b > T) {
+      if (lane == 0) set_error(err, SLA_ERR_DEVICE);
       a = ae = b = be = 0;
     }
-    int n = 0;
-    while (a < ae || b < be) {
-      const int x = a < ae ? ci[a] : 0x7FFFFFFF;
-      const int y = b < be ? ci[b] : 0x7FFFFFFF;
-      int i, f;
-      if (x == y) { i = x; f = 3; ++a; ++b; }
-      else if (x < y) { i = x; f = 1; ++a; }
-      else { i = y; f = 2; ++b; }
-      if (i < 0 || i >= T || n >= 2 * T) { set_error(err, SLA_ERR_DEVICE); continue; }
-      ulist[n] = uint16_t(i);
-      uflag[n] = uint8_t(f);
-      ++n;
+    const int la = ae - a, lb = be - b;
+    int32_t* la_s = reinterpret_cast<int32_t*>(sSt);  // up to T + T entries
+    int32_t* lb_s = la_s + la;
+    for (int x = lane; x < la; x += 32) la_s[x] = ci[a + x];
+    for (int x = lane; x < lb; x += 32) lb_s[x] = ci[b + x];
+    __syncwarp();
+    if (lane == 0) {
+      int ia = 0, ib = 0, n = 0;
+      while (ia < la || ib < lb) {
+        const int x = ia < la ? la_s[ia] : 0x7FFFFFFF;
+        const int y = ib < lb ? lb_s[ib] : 0x7FFFFFFF;
+        int i, f;
+        if (x == y) { i = x; f = 3; ++ia; ++ib; }
+        else if (x < y) { i = x; f = 1; ++ia; }
+        else { i = y; f = 2; ++ib; }
+        if (i < 0 || i >= T || n >= 2 * T) { set_error(err, SLA_ERR_DEVICE); continue; }
+        ulist[n] = uint16_t(i);
+        uflag[n] = uint8_t(f);
+        ++n;
+      }
+      n_union = n;
     }
-    n_union = n;
   }
   tc_fence_before();
   __syncthreads();
@@ -151,6 +143,7 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && nU > 0) {
+      fence_proxy_async_smem();  // list staging used these buffers generically
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(&kv_full, 2 * L::kKV);
@@ -252,7 +245,6 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
     uint8_t* ds_tile = sDS + wg * L::kDS;
     bool ok = true;
-    bool issued_bulk = false;
     for (int n = wg; n < nU; n += 2) {
       const int s = n % kNSt;
       uint8_t* st = sSt + s * L::kStage;
@@ -293,32 +285,26 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
       mbar_arrive(&p_full[wg]);
       if (!(ok = mbar_wait(&m_done[wg], (n >> 1) & 1, err, &abort_flag))) break;
       tc_fence_after();
-      // dQ_i^T (lane = feature a, 64 query columns) -> this stage's buffer as
-      // fp32 [q][a]; Q_i and dO_i there are no longer read by any MMA
-      float* stg = reinterpret_cast<float*>(st);
+      // The MMAs are done with Q_i, dO_i and this warpgroup read LSE_i, D_i:
+      // hand the stage back to the producer before draining dQ.
+      if (wq == 0 && lane == 0) mbar_arrive(&st_empty[s]);
+      // dQ_i^T (lane = feature a, 64 query columns) added into dQ with
+      // fire-and-forget fp32 reductions; for each query the 32 lanes of a
+      // warp cover 32 consecutive features (one coalesced 128-byte request).
+      float v[64];
       if (wq * 32 < D) {
-#pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          float v[32];
-          tmem_ld32(st_t + c0, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) stg[(c0 + e) * D + r] = v[e] * scale;
-        }
+        tmem_ld32(st_t, reinterpret_cast<float(&)[32]>(v[0]));
+        tmem_ld32(st_t + 32, reinterpret_cast<float(&)[32]>(v[32]));
+        tmem_ld_wait();
       }
       tc_fence_before();
-      mbar_arrive(&tfree[wg]);
-      fence_proxy_async_smem();
-      mbar_arrive(&stg_ready[wg]);  // a bounded wait below, so a missing thread cannot hang it
-      if (wq == 0 && lane == 0) {
-        if (!(ok = mbar_wait(&stg_ready[wg], (n >> 1) & 1, err, &abort_flag))) break;
-        bulk_reduce_add_f32(dq + (size_t(bh) * N + size_t(i) * 64) * D, stg, 64 * D * 4);
-        bulk_wait_read_all();
-        issued_bulk = true;
-        mbar_arrive(&st_empty[s]);
+      mbar_arrive(&tfree[wg]);  // the buffer is free once dQ^T is in registers
+      if (wq * 32 < D) {
+        float* dst = dq + (size_t(bh) * N + size_t(i) * 64) * D + r;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) atomicAdd(dst + size_t(e) * D, v[e] * scale);
       }
     }
-    if (issued_bulk) bulk_wait_all();
     // dK (warpgroup 0) and dV (warpgroup 1) of this tile's keys
     if (nU > 0) {
       ok = mbar_wait(&fin, 0, err, &abort_flag) && ok;

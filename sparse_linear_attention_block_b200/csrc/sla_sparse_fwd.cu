@@ -46,8 +46,7 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
     int n_crit, float scale_log2, float* __restrict__ o_s, float* __restrict__ lse, int* err) {
   using L = FwdSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* base = align_smem_1024(smem_raw);
   uint8_t* sQ = base;
   uint8_t* sKV = base + L::kQBytes;
   uint16_t* ulist = reinterpret_cast<uint16_t*>(base + L::kTiles);
@@ -79,25 +78,31 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
     abort_flag = 0;
     fence_barrier_init();
   }
-  if (threadIdx.x == 128) {
-    // sorted union of the two rows' critical lists; flag bit h = member of half h
-    const int32_t* l0 = crit_idx + (size_t(bh) * T + blk0) * n_crit;
-    const int32_t* l1 = crit_idx + (size_t(bh) * T + (has1 ? blk1 : blk0)) * n_crit;
+  if (warp == 4) {
+    // sorted union of the two rows' critical lists; flag bit h = member of
+    // half h.  Both rows are staged in the (still idle) K/V stage buffers
+    // with coalesced loads and merged from shared memory by one lane.
     const int n1 = has1 ? n_crit : 0;
-    int a = 0, b = 0, n = 0;
-    while (a < n_crit || b < n1) {
-      const int x = a < n_crit ? l0[a] : 0x7FFFFFFF;
-      const int y = b < n1 ? l1[b] : 0x7FFFFFFF;
-      int j, f;
-      if (x == y) { j = x; f = 3; ++a; ++b; }
-      else if (x < y) { j = x; f = 1; ++a; }
-      else { j = y; f = 2; ++b; }
-      if (j < 0 || j >= T) { set_error(err, SLA_ERR_DEVICE); continue; }
-      ulist[n] = uint16_t(j);
-      uflag[n] = uint8_t(f);
-      ++n;
+    const int32_t* l0 = crit_idx + (size_t(bh) * T + blk0) * n_crit;  // row 2p+1 follows
+    int32_t* ls = reinterpret_cast<int32_t*>(sKV);
+    for (int x = lane; x < n_crit + n1; x += 32) ls[x] = l0[x];
+    __syncwarp();
+    if (lane == 0) {
+      int a = 0, b = 0, n = 0;
+      while (a < n_crit || b < n1) {
+        const int x = a < n_crit ? ls[a] : 0x7FFFFFFF;
+        const int y = b < n1 ? ls[n_crit + b] : 0x7FFFFFFF;
+        int j, f;
+        if (x == y) { j = x; f = 3; ++a; ++b; }
+        else if (x < y) { j = x; f = 1; ++a; }
+        else { j = y; f = 2; ++b; }
+        if (j < 0 || j >= T) { set_error(err, SLA_ERR_DEVICE); continue; }
+        ulist[n] = uint16_t(j);
+        uflag[n] = uint8_t(f);
+        ++n;
+      }
+      n_union = n;
     }
-    n_union = n;
   }
   tc_fence_before();
   __syncthreads();
@@ -109,6 +114,7 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
   if (warp == 4) {
     // ---------------------------------------------------------------- producer
     if (lane == 0 && nU > 0) {
+      fence_proxy_async_smem();  // list staging used these buffers generically
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
