@@ -215,12 +215,14 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
       if (!mbar_wait(&full[s], (kt / kAggStages) & 1, err, &abort_flag)) break;
       tc_fence_after();
       const uint32_t sa = smem_u32(base + s * kAggStageBytes);
-      const uint32_t sb = sa + kAggA;
+      const uint64_t ad = desc_kmajor_base(sa);
+      const uint64_t bhd = desc_mnmajor_base(sa + kAggA, kAggBK);
+      const uint64_t bld = desc_mnmajor_base(sa + kAggA + kAggB, kAggBK);
 #pragma unroll
       for (int ks = 0; ks < kAggBK / 16; ++ks) {
-        mma_ss(tmem, desc_kmajor(sa, 128, ks), desc_mnmajor(sb, kAggBK, ks), idesc,
-               (kt | ks) != 0);
-        mma_ss(tmem, desc_kmajor(sa, 128, ks), desc_mnmajor(sb + kAggB, kAggBK, ks), idesc, 1);
+        const uint64_t a = desc_advance(ad, kmajor_step_bytes(128, ks));
+        mma_ss(tmem, a, desc_advance(bhd, mnmajor_step_bytes(ks)), idesc, (kt | ks) != 0);
+        mma_ss(tmem, a, desc_advance(bld, mnmajor_step_bytes(ks)), idesc, 1);
       }
       mma_commit(&empty[s]);
     }

@@ -266,6 +266,27 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile_saddr, int krows,
   return sdesc_sw128(tile_saddr + ks * 16 * 128, krows * 128, 1024);
 }
 
+// Byte offset of MMA K-step `ks` inside a K-major tile of `rows` rows, and
+// inside an MN-major tile; compile-time constants for unrolled loops.
+__host__ __device__ constexpr uint32_t kmajor_step_bytes(int rows, int ks) {
+  return uint32_t(((ks * 16) >> 6) * rows * 128 + ((ks * 16) & 63) * 2);
+}
+__host__ __device__ constexpr uint32_t mnmajor_step_bytes(int ks) { return uint32_t(ks * 16 * 128); }
+
+// Advance a descriptor's start address by `bytes` (16-byte units in the low
+// field; callers stay inside one shared-memory window so nothing carries).
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + uint64_t(bytes >> 4);
+}
+
+// Base descriptors of a tile (K-step 0), to be advanced per K-step.
+__device__ __forceinline__ uint64_t desc_kmajor_base(uint32_t tile_saddr) {
+  return sdesc_sw128(tile_saddr, 16, 1024);
+}
+__device__ __forceinline__ uint64_t desc_mnmajor_base(uint32_t tile_saddr, int krows) {
+  return sdesc_sw128(tile_saddr, krows * 128, 1024);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate) {

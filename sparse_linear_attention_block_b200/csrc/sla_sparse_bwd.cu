@@ -52,6 +52,13 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// 16-byte fire-and-forget fp32 reduction into global memory
+__device__ __forceinline__ void red_add_v4(float* dst, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
 template <int D>
 __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -71,7 +78,7 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
   uint8_t* uflag = reinterpret_cast<uint8_t*>(ulist + 2 * T);
 
   __shared__ uint64_t kv_full, st_full[kNSt], st_empty[kNSt], s_full[2], p_full[2], m_done[2],
-      tfree[2], fin;
+      tfree[2], wsync[2], fin;
   __shared__ uint32_t tmem_base;
   __shared__ int n_union, abort_flag;
   const int qp = blockIdx.x, bh = blockIdx.y;
@@ -92,6 +99,7 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
       mbar_init(&p_full[b], 128);
       mbar_init(&m_done[b], 1);
       mbar_init(&tfree[b], 128);
+      mbar_init(&wsync[b], 128);
     }
     mbar_init(&fin, 1);
     abort_flag = 0;
@@ -181,7 +189,8 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
       constexpr uint32_t id_g = idesc_bf16(128, D, 0, 1);   // dV, dK (A from TMEM)
       constexpr uint32_t id_q = idesc_bf16(128, 64, 1, 1);  // dQ^T = K^T dS^T
       bool ok = mbar_wait(&kv_full, 0, err, &abort_flag);
-      const uint32_t k0 = smem_u32(sK), v0 = smem_u32(sV);
+      const uint64_t kd_k = desc_kmajor_base(smem_u32(sK)), vd_k = desc_kmajor_base(smem_u32(sV));
+      const uint64_t kd_mn = desc_mnmajor_base(smem_u32(sK), 128);
       // Two in-order streams, issued whichever is ready first:
       //   S(n):  S^T_n, dP^T_n into buffer n&1 (needs stage n loaded and, for
       //          n >= 2, dQ^T_{n-2} drained from that buffer; at most one
@@ -196,10 +205,13 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
           tc_fence_after();
           const uint32_t q0 = smem_u32(sSt + (ns % kNSt) * L::kStage), do0 = q0 + L::kQ;
           const uint32_t st_t = tmem + (ns & 1) * 128, dp_t = st_t + 64;
+          const uint64_t qd = desc_kmajor_base(q0), dod = desc_kmajor_base(do0);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
-            mma_ss(st_t, desc_kmajor(k0, 128, ks), desc_kmajor(q0, 64, ks), id_s, ks > 0);
-            mma_ss(dp_t, desc_kmajor(v0, 128, ks), desc_kmajor(do0, 64, ks), id_s, ks > 0);
+            mma_ss(st_t, desc_advance(kd_k, kmajor_step_bytes(128, ks)),
+                   desc_advance(qd, kmajor_step_bytes(64, ks)), id_s, ks > 0);
+            mma_ss(dp_t, desc_advance(vd_k, kmajor_step_bytes(128, ks)),
+                   desc_advance(dod, kmajor_step_bytes(64, ks)), id_s, ks > 0);
           }
           mma_commit(&s_full[ns & 1]);
           ++ns;
@@ -210,15 +222,19 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
           const int b = ng & 1;
           const uint32_t q0 = smem_u32(sSt + (ng % kNSt) * L::kStage), do0 = q0 + L::kQ;
           const uint32_t st_t = tmem + b * 128, dp_t = st_t + 64;
+          const uint64_t qd = desc_mnmajor_base(q0, 64), dod = desc_mnmajor_base(do0, 64);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
-            mma_ts(tmem + kDV, st_t + ks * 8, desc_mnmajor(do0, 64, ks), id_g, (ng | ks) != 0);
-            mma_ts(tmem + kDK, dp_t + ks * 8, desc_mnmajor(q0, 64, ks), id_g, (ng | ks) != 0);
+            mma_ts(tmem + kDV, st_t + ks * 8, desc_advance(dod, mnmajor_step_bytes(ks)), id_g,
+                   (ng | ks) != 0);
+            mma_ts(tmem + kDK, dp_t + ks * 8, desc_advance(qd, mnmajor_step_bytes(ks)), id_g,
+                   (ng | ks) != 0);
           }
-          const uint32_t ds0 = smem_u32(sDS + b * L::kDS);
+          const uint64_t dsd = desc_mnmajor_base(smem_u32(sDS + b * L::kDS), 128);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)  // dQ^T overwrites S^T (its P was consumed by dV above)
-            mma_ss(st_t, desc_mnmajor(k0, 128, ks), desc_mnmajor(ds0, 128, ks), id_q, ks > 0);
+            mma_ss(st_t, desc_advance(kd_mn, mnmajor_step_bytes(ks)),
+                   desc_advance(dsd, mnmajor_step_bytes(ks)), id_q, ks > 0);
           mma_commit(&m_done[b]);
           ++ng;
           progressed = true;
@@ -245,6 +261,15 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
     uint8_t* ds_tile = sDS + wg * L::kDS;
     bool ok = true;
+    uint32_t wphase = 0;
+    // warpgroup barrier with a bounded wait (a thread that gave up cannot
+    // leave the other 127 stuck, as a named barrier would)
+    auto wg_sync = [&]() -> bool {
+      mbar_arrive(&wsync[wg]);
+      const bool r = mbar_wait(&wsync[wg], wphase & 1, err, &abort_flag);
+      ++wphase;
+      return r;
+    };
     for (int n = wg; n < nU; n += 2) {
       const int s = n % kNSt;
       uint8_t* st = sSt + s * L::kStage;
@@ -289,8 +314,7 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
       // hand the stage back to the producer before draining dQ.
       if (wq == 0 && lane == 0) mbar_arrive(&st_empty[s]);
       // dQ_i^T (lane = feature a, 64 query columns) added into dQ with
-      // fire-and-forget fp32 reductions; for each query the 32 lanes of a
-      // warp cover 32 consecutive features (one coalesced 128-byte request).
+      // fire-and-forget fp32 reductions.
       float v[64];
       if (wq * 32 < D) {
         tmem_ld32(st_t, reinterpret_cast<float(&)[32]>(v[0]));
@@ -299,11 +323,31 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
       }
       tc_fence_before();
       mbar_arrive(&tfree[wg]);  // the buffer is free once dQ^T is in registers
-      if (wq * 32 < D) {
-        float* dst = dq + (size_t(bh) * N + size_t(i) * 64) * D + r;
+      // Transpose through this warpgroup's dS^T tile (its MMA is done and the
+      // tile is not written again before this warpgroup's next query block),
+      // 32 queries at a time, then add 16-byte vectors into dQ.
+      float* stg = reinterpret_cast<float*>(ds_tile);
+      float* gdq = dq + (size_t(bh) * N + size_t(i) * 64) * D;
 #pragma unroll
-        for (int e = 0; e < 64; ++e) atomicAdd(dst + size_t(e) * D, v[e] * scale);
+      for (int h = 0; h < 2; ++h) {
+        if (ok) {
+          if (wq * 32 < D) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) stg[e * D + r] = v[32 * h + e] * scale;
+          }
+          ok = wg_sync();
+        }
+        if (ok) {
+          const float4* s4 = reinterpret_cast<const float4*>(stg);
+#pragma unroll
+          for (int idx = r; idx < 32 * D / 4; idx += 128) {
+            const int qq = idx / (D / 4), a4 = idx % (D / 4);
+            red_add_v4(gdq + size_t(32 * h + qq) * D + a4 * 4, s4[idx]);
+          }
+          ok = wg_sync();
+        }
       }
+      if (!ok) break;
     }
     // dK (warpgroup 0) and dV (warpgroup 1) of this tile's keys
     if (nU > 0) {

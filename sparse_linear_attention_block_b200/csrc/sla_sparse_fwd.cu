@@ -149,17 +149,17 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
     if (lane == 0 && nU > 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, 64, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16(128, D, 0, 1);
-      const uint32_t q0 = smem_u32(sQ);
+      const uint64_t qd = desc_kmajor_base(smem_u32(sQ));
       bool ok = mbar_wait(&q_full, 0, err, &abort_flag);
       auto issue_s = [&](int n) -> bool {
         const int s = n % kStages;
         if (!mbar_wait(&kv_full[s], (n / kStages) & 1, err, &abort_flag)) return false;
         tc_fence_after();
-        const uint32_t k0 = smem_u32(sKV + s * L::kStageBytes);
+        const uint64_t kd = desc_kmajor_base(smem_u32(sKV + s * L::kStageBytes));
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          mma_ss(tmem + (n & 1) * 64, desc_kmajor(q0, 128, ks), desc_kmajor(k0, 64, ks),
-                 idesc_s, ks > 0);
+          mma_ss(tmem + (n & 1) * 64, desc_advance(qd, kmajor_step_bytes(128, ks)),
+                 desc_advance(kd, kmajor_step_bytes(64, ks)), idesc_s, ks > 0);
         mma_commit(&s_full[n & 1]);
         return true;
       };
@@ -167,11 +167,11 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
         if (!mbar_wait(&p_full[n & 1], (n >> 1) & 1, err, &abort_flag)) return false;
         tc_fence_after();
         const int s = n % kStages;
-        const uint32_t v0 = smem_u32(sKV + s * L::kStageBytes + L::kKVBytes);
+        const uint64_t vd = desc_mnmajor_base(smem_u32(sKV + s * L::kStageBytes + L::kKVBytes), 64);
         const uint32_t pt = tmem + (n & 1) * 64;  // P aliases the first 32 columns of S
 #pragma unroll
         for (int ks = 0; ks < kBlock / 16; ++ks)
-          mma_ts(tm_o, pt + ks * 8, desc_mnmajor(v0, 64, ks), idesc_o, (n | ks) != 0);
+          mma_ts(tm_o, pt + ks * 8, desc_advance(vd, mnmajor_step_bytes(ks)), idesc_o, (n | ks) != 0);
         mma_commit(&o_done);
         mma_commit(&kv_empty[s]);
         return true;
