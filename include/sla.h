@@ -94,12 +94,14 @@ typedef struct {
  *   lse   fp32 [B,H,N]      log-sum-exp of the critical scores (-inf if none)
  *   o_s   fp32 [B,H,N,d]    sparse-branch output
  *   den   fp32 [B,H,N]      phi(Q).Z_i (0 if the row has no marginal block)
- *   hz_agg fp32 [B,H,T,d*d+d]  per query block: H_i (d x d, row-major) then Z_i (d) */
+ *   hz_agg bf16 [2][B,H,T,d*d+d]  per query block: H_i (d x d, row-major) then
+ *          Z_i (d), stored as a high plane followed by a low plane (value =
+ *          hi + lo, about 16 significant bits); 4 bytes per element in all */
 typedef struct {
   float* lse;
   float* o_s;
   float* den;
-  float* hz_agg;
+  void* hz_agg;
 } sla_saved;
 
 /* Sizes in bytes of every caller buffer for a shape. */

@@ -262,7 +262,7 @@ class Buffers:
             lse=e(B, H, N, dt=torch.float32),
             o_s=e(B, H, N, d, dt=torch.float32),
             den=e(B, H, N, dt=torch.float32),
-            hz_agg=e(B, H, T, d * d + d, dt=torch.float32),
+            hz_agg=e(2, B, H, T, d * d + d, dt=torch.bfloat16),  # hi plane, lo plane
             workspace=torch.empty(int(s.workspace_bytes) + 1024, dtype=torch.uint8, device=dev),
             mask=MaskStruct(), saved=SavedStruct())
         # the C ABI wants a 1024-byte aligned workspace

@@ -32,7 +32,7 @@ WorkspaceLayout workspace_layout(int BH, int N, int d) {
   const size_t W = size_t(summary_width(d));
   L.summ_hi = take(bh * T * W * 2);
   L.summ_lo = take(bh * T * W * 2);
-  L.dh = take(bh * T * W * 4);
+  L.dh = take(bh * T * W * 4);  // two bf16 planes
   L.mmat = take(bh * Tp * Tp * 2);
   L.mmat_t = take(bh * Tp * Tp * 2);
   L.dvec = take(bh * N * 4);
@@ -70,6 +70,25 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t r
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_strided(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint64_t stride1, uint64_t stride2, uint32_t box0, uint32_t box1) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1 * 2, stride2 * 2};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_summary(CUtensorMap* map, const void* plane, int rows, int d) {
+  return make_tmap_strided(map, plane, uint64_t(d), uint64_t(d), uint64_t(rows), uint64_t(d),
+                           uint64_t(summary_width(d)), 64, uint32_t(d));
 }
 
 bool make_tmap_bhnd(CUtensorMap* map, const void* base, int BH, int N, int d, int box_rows) {
@@ -287,10 +306,12 @@ sla_status sla_forward(const sla_shape* shape, const void* q, const void* k, con
   // linear branch: (h_j | z_j) summaries, then (H_i | Z_i) by one aggregation GEMM
   SLA_LAUNCH("summaries", s, launch_summaries(p, k, v, summ_hi, summ_lo, err, s));
   SLA_LAUNCH("expand_marginal", s, launch_expand_marginal(p, mask->marg_bits, mmat, nullptr, s));
-  SLA_LAUNCH("aggregate", s, launch_aggregate(p, mmat, summ_hi, summ_lo, saved->hz_agg, err, s));
+  auto* hz_hi = static_cast<__nv_bfloat16*>(saved->hz_agg);
+  auto* hz_lo = hz_hi + size_t(p.BH) * p.T * summary_width(p.d);
+  SLA_LAUNCH("aggregate", s, launch_aggregate(p, mmat, summ_hi, summ_lo, hz_hi, hz_lo, err, s));
   // sparse branch, then the combination
   SLA_LAUNCH("fwd_sparse", s, launch_fwd_sparse(p, q, k, v, mask->crit_idx, saved->o_s, saved->lse, err, s));
-  SLA_LAUNCH("fwd_linear", s, launch_fwd_linear(p, q, saved->hz_agg, w_proj, saved->o_s, o,
+  SLA_LAUNCH("fwd_linear", s, launch_fwd_linear(p, q, hz_hi, hz_lo, w_proj, saved->o_s, o,
                                                 saved->den, err, s));
   return SLA_OK;
 }
@@ -320,7 +341,10 @@ sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, co
   auto* summ_hi = at<__nv_bfloat16>(workspace, L.summ_hi);
   auto* summ_lo = at<__nv_bfloat16>(workspace, L.summ_lo);
   auto* mmat_t = at<__nv_bfloat16>(workspace, L.mmat_t);
-  float* dh = at<float>(workspace, L.dh);
+  auto* dh_hi = at<__nv_bfloat16>(workspace, L.dh);
+  auto* dh_lo = dh_hi + size_t(p.BH) * p.T * summary_width(p.d);
+  const auto* hz_hi = static_cast<const __nv_bfloat16*>(saved->hz_agg);
+  const auto* hz_lo = hz_hi + size_t(p.BH) * p.T * summary_width(p.d);
   float* dvec = at<float>(workspace, L.dvec);
   float* dnum = at<float>(workspace, L.dnum);
   float* dden = at<float>(workspace, L.dden);
@@ -330,16 +354,16 @@ sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, co
     return SLA_ERR_CUDA;
   // linear-branch preparation: D, dnum, dden, dW; then per-block A_i / a_i
   SLA_LAUNCH("bwd_prep", s, launch_bwd_prep(p, q, d_o, w_proj, saved->o_s, saved->den,
-                                            saved->hz_agg, dvec, dnum, dden, dw_proj, sms, err, s));
+                                            hz_hi, hz_lo, dvec, dnum, dden, dw_proj, sms, err, s));
   SLA_LAUNCH("bwd_summ", s, launch_bwd_summ(p, q, dnum, dden, summ_hi, summ_lo, err, s));
   // (dh_j | dz_j) = sum over rows i with j marginal of (A_i | a_i): transposed aggregation
   SLA_LAUNCH("expand_marginal_t", s, launch_expand_marginal(p, mask->marg_bits, nullptr, mmat_t, s));
-  SLA_LAUNCH("aggregate_t", s, launch_aggregate(p, mmat_t, summ_hi, summ_lo, dh, err, s));
+  SLA_LAUNCH("aggregate_t", s, launch_aggregate(p, mmat_t, summ_hi, summ_lo, dh_hi, dh_lo, err, s));
   // sparse branch writes dK, dV and accumulates dQ; the linear branch adds its share
   SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
                                mask->crit_col_idx, dq, dk, dv, err, s));
-  SLA_LAUNCH("bwd_linear", s, launch_bwd_linear(p, q, k, v, saved->hz_agg, dh, dnum, dden, dq, dk,
-                                                dv, err, s));
+  SLA_LAUNCH("bwd_linear", s, launch_bwd_linear(p, q, k, v, hz_hi, hz_lo, dh_hi, dh_lo, dnum, dden,
+                                                dq, dk, dv, err, s));
   return SLA_OK;
 }
 

@@ -36,7 +36,8 @@ template <int D>
 __global__ void __launch_bounds__(256, 1) bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ d_o,
     const __nv_bfloat16* __restrict__ w_proj, const float* __restrict__ o_s,
-    const float* __restrict__ den, const float* __restrict__ hz_agg, float* __restrict__ dvec,
+    const float* __restrict__ den, const __nv_bfloat16* __restrict__ hz_hi,
+    const __nv_bfloat16* __restrict__ hz_lo, float* __restrict__ dvec,
     float* __restrict__ dnum, float* __restrict__ dden, float* __restrict__ dw, int N, int T,
     int BH, int* err) {
   constexpr int W = D * D + D, DH = D / 2;
@@ -77,8 +78,9 @@ __global__ void __launch_bounds__(256, 1) bwd_prep_kernel(
     load_phi_sw<D>(sA, nullptr, 128, q + tile_off, valid_rows, t, 256);
     for (int m = 0; m < 2; ++m) {
       const int b2 = 2 * p + m;
-      load_split_sw<D>(sHh, sHl, D, hz_agg + (size_t(bh) * T + (b2 < T ? b2 : 0)) * W,
-                       b2 < T ? D : 0, t, 256);
+      const size_t hrow = (size_t(bh) * T + (b2 < T ? b2 : 0)) * W;
+      load_rows_sw<D>(sHh, D, hz_hi + hrow, b2 < T ? D : 0, t, 256);
+      load_rows_sw<D>(sHl, D, hz_lo + hrow, b2 < T ? D : 0, t, 256);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
@@ -297,8 +299,9 @@ __global__ void __launch_bounds__(256, 1) bwd_summ_kernel(
 template <int D>
 __global__ void __launch_bounds__(256, 1) bwd_linear_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-    const __nv_bfloat16* __restrict__ v, const float* __restrict__ hz_agg,
-    const float* __restrict__ dhz, const float* __restrict__ dnum,
+    const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ hz_hi,
+    const __nv_bfloat16* __restrict__ hz_lo, const __nv_bfloat16* __restrict__ dh_hi,
+    const __nv_bfloat16* __restrict__ dh_lo, const float* __restrict__ dnum,
     const float* __restrict__ dden, float* __restrict__ dq, float* __restrict__ dk,
     float* __restrict__ dv, int N, int T, int* err) {
   constexpr int W = D * D + D, DH = D / 2;
@@ -330,13 +333,16 @@ __global__ void __launch_bounds__(256, 1) bwd_linear_kernel(
   load_split_sw<D>(s0, s1, 128, dnum + tile_off, valid_rows, t, 256);
   for (int e = t; e < 2 * D; e += 256) {
     const int b2 = 2 * p + e / D;
-    sZ[e / D][e % D] = b2 < T ? hz_agg[(size_t(bh) * T + b2) * W + D * D + e % D] : 0.f;
+    const size_t zo = (size_t(bh) * T + b2) * W + D * D + e % D;
+    sZ[e / D][e % D] =
+        b2 < T ? __bfloat162float(hz_hi[zo]) + __bfloat162float(hz_lo[zo]) : 0.f;
   }
   bool ok = true;
   for (int m = 0; m < 2; ++m) {
     const int b2 = 2 * p + m;
-    load_split_sw<D>(sMh, sMl, D, hz_agg + (size_t(bh) * T + (b2 < T ? b2 : 0)) * W,
-                     b2 < T ? D : 0, t, 256);
+    const size_t hrow = (size_t(bh) * T + (b2 < T ? b2 : 0)) * W;
+    load_rows_sw<D>(sMh, D, hz_hi + hrow, b2 < T ? D : 0, t, 256);
+    load_rows_sw<D>(sMl, D, hz_lo + hrow, b2 < T ? D : 0, t, 256);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -392,14 +398,17 @@ __global__ void __launch_bounds__(256, 1) bwd_linear_kernel(
   // ---------------- phase 2: dK, dV
   for (int e = t; e < 2 * D; e += 256) {
     const int b2 = 2 * p + e / D;
-    sZ[e / D][e % D] = b2 < T ? dhz[(size_t(bh) * T + b2) * W + D * D + e % D] : 0.f;
+    const size_t zo = (size_t(bh) * T + b2) * W + D * D + e % D;
+    sZ[e / D][e % D] =
+        b2 < T ? __bfloat162float(dh_hi[zo]) + __bfloat162float(dh_lo[zo]) : 0.f;
   }
   load_rows_sw<D>(s0, 128, v + tile_off, valid_rows, t, 256);
   load_phi_sw<D>(s1, s2, 128, k + tile_off, valid_rows, t, 256);
   for (int m = 0; m < 2; ++m) {
     const int b2 = 2 * p + m;
-    load_split_sw<D>(sMh, sMl, D, dhz + (size_t(bh) * T + (b2 < T ? b2 : 0)) * W,
-                     b2 < T ? D : 0, t, 256);
+    const size_t hrow = (size_t(bh) * T + (b2 < T ? b2 : 0)) * W;
+    load_rows_sw<D>(sMh, D, dh_hi + hrow, b2 < T ? D : 0, t, 256);
+    load_rows_sw<D>(sMl, D, dh_lo + hrow, b2 < T ? D : 0, t, 256);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -472,7 +481,8 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }  // namespace
 
 cudaError_t launch_bwd_prep(const Problem& p, const void* q, const void* d_o, const void* w_proj,
-                            const float* o_s, const float* den, const float* hz_agg, float* dvec,
+                            const float* o_s, const float* den, const __nv_bfloat16* hz_hi,
+                            const __nv_bfloat16* hz_lo, float* dvec,
                             float* dnum, float* dden, float* dw, int num_sms, int* err,
                             cudaStream_t s) {
   const int tiles = ((p.T + 1) / 2) * p.BH;
@@ -483,12 +493,12 @@ cudaError_t launch_bwd_prep(const Problem& p, const void* q, const void* d_o, co
     if ((e = set_smem(bwd_prep_kernel<128>, smem)) != cudaSuccess) return e;
     bwd_prep_kernel<128><<<grid, 256, smem, s>>>(
         (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o, (const __nv_bfloat16*)w_proj, o_s,
-        den, hz_agg, dvec, dnum, dden, dw, p.N, p.T, p.BH, err);
+        den, hz_hi, hz_lo, dvec, dnum, dden, dw, p.N, p.T, p.BH, err);
   } else {
     if ((e = set_smem(bwd_prep_kernel<64>, smem)) != cudaSuccess) return e;
     bwd_prep_kernel<64><<<grid, 256, smem, s>>>(
         (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o, (const __nv_bfloat16*)w_proj, o_s,
-        den, hz_agg, dvec, dnum, dden, dw, p.N, p.T, p.BH, err);
+        den, hz_hi, hz_lo, dvec, dnum, dden, dw, p.N, p.T, p.BH, err);
   }
   return cudaGetLastError();
 }
@@ -512,7 +522,9 @@ cudaError_t launch_bwd_summ(const Problem& p, const void* q, const float* dnum,
 }
 
 cudaError_t launch_bwd_linear(const Problem& p, const void* q, const void* k, const void* v,
-                              const float* hz_agg, const float* dhz, const float* dnum,
+                              const __nv_bfloat16* hz_hi, const __nv_bfloat16* hz_lo,
+                              const __nv_bfloat16* dh_hi, const __nv_bfloat16* dh_lo,
+                              const float* dnum,
                               const float* dden, float* dq, float* dk, float* dv, int* err,
                               cudaStream_t s) {
   dim3 grid((p.T + 1) / 2, p.BH);
@@ -521,12 +533,14 @@ cudaError_t launch_bwd_linear(const Problem& p, const void* q, const void* k, co
   if (p.d == 128) {
     if ((e = set_smem(bwd_linear_kernel<128>, smem)) != cudaSuccess) return e;
     bwd_linear_kernel<128><<<grid, 256, smem, s>>>(
-        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, hz_agg, dhz,
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, hz_hi, hz_lo,
+        dh_hi, dh_lo,
         dnum, dden, dq, dk, dv, p.N, p.T, err);
   } else {
     if ((e = set_smem(bwd_linear_kernel<64>, smem)) != cudaSuccess) return e;
     bwd_linear_kernel<64><<<grid, 256, smem, s>>>(
-        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, hz_agg, dhz,
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, hz_hi, hz_lo,
+        dh_hi, dh_lo,
         dnum, dden, dq, dk, dv, p.N, p.T, err);
   }
   return cudaGetLastError();

@@ -32,7 +32,7 @@ struct WorkspaceLayout {
   size_t kbar;       // fp32 [BH,T,d]   pooled K
   size_t summ_hi;    // bf16 [BH,T,d*d+d] (h_j|z_j) forward, (A_i|a_i) backward: high part
   size_t summ_lo;    // bf16 [BH,T,d*d+d] the low part (value = hi + lo)
-  size_t dh;         // fp32 [BH,T,d*d+d] (dh_j|dz_j) backward
+  size_t dh;         // bf16 [2][BH,T,d*d+d] (dh_j|dz_j) backward: hi plane, lo plane
   size_t mmat;       // bf16 [BH,Tp,Tp] marginal 0/1 matrix, rows = query blocks
   size_t mmat_t;     // bf16 [BH,Tp,Tp] its transpose
   size_t dvec;       // fp32 [BH,N]     D_t = dO_t . O_s,t
@@ -65,15 +65,17 @@ cudaError_t launch_summaries(const Problem& p, const void* k, const void* v,
                              cudaStream_t s);
 cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
                              const __nv_bfloat16* summ_hi, const __nv_bfloat16* summ_lo,
-                             float* out, int* err, cudaStream_t s);
+                             __nv_bfloat16* out_hi, __nv_bfloat16* out_lo, int* err,
+                             cudaStream_t s);
 cudaError_t launch_fwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
                               const int32_t* crit_idx, float* o_s, float* lse, int* err,
                               cudaStream_t s);
-cudaError_t launch_fwd_linear(const Problem& p, const void* q, const float* hz_agg,
-                              const void* w_proj, const float* o_s, void* o, float* den,
-                              int* err, cudaStream_t s);
+cudaError_t launch_fwd_linear(const Problem& p, const void* q, const __nv_bfloat16* hz_hi,
+                              const __nv_bfloat16* hz_lo, const void* w_proj, const float* o_s,
+                              void* o, float* den, int* err, cudaStream_t s);
 cudaError_t launch_bwd_prep(const Problem& p, const void* q, const void* d_o, const void* w_proj,
-                            const float* o_s, const float* den, const float* hz_agg, float* dvec,
+                            const float* o_s, const float* den, const __nv_bfloat16* hz_hi,
+                            const __nv_bfloat16* hz_lo, float* dvec,
                             float* dnum, float* dden, float* dw, int num_sms, int* err,
                             cudaStream_t s);
 cudaError_t launch_bwd_summ(const Problem& p, const void* q, const float* dnum,
@@ -84,7 +86,9 @@ cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, co
                               const int32_t* col_ptr, const int32_t* col_idx, float* dq,
                               float* dk, float* dv, int* err, cudaStream_t s);
 cudaError_t launch_bwd_linear(const Problem& p, const void* q, const void* k, const void* v,
-                              const float* hz_agg, const float* dhz, const float* dnum,
+                              const __nv_bfloat16* hz_hi, const __nv_bfloat16* hz_lo,
+                              const __nv_bfloat16* dh_hi, const __nv_bfloat16* dh_lo,
+                              const float* dnum,
                               const float* dden, float* dq, float* dk, float* dv, int* err,
                               cudaStream_t s);
 
@@ -94,5 +98,13 @@ bool make_tmap_bhnd(CUtensorMap* map, const void* base, int BH, int N, int d, in
 // TMA descriptor for a bf16 3D tensor {inner, rows, batch} (row pitch = inner).
 bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
                   uint64_t batch, uint32_t box_inner, uint32_t box_rows);
+// TMA descriptor for a bf16 3D tensor {d0, d1, d2} with explicit element
+// strides of dimensions 1 and 2 (multiples of 8), box {box0, box1, 1}.
+bool make_tmap_strided(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint64_t stride1, uint64_t stride2, uint32_t box0, uint32_t box1);
+// The d x d block of every per-block summary row of a bf16 plane [rows, d*d+d],
+// viewed as {c, a, row} so that a box {64, d, 1} lands as a 128-byte-swizzled
+// tile of d rows (a) per 64-column chunk (c).
+bool make_tmap_summary(CUtensorMap* map, const void* plane, int rows, int d);
 
 }  // namespace sla

@@ -17,8 +17,8 @@
 //
 // Kernels:
 //   summaries_kernel   (h_j | z_j) as bf16 hi/lo planes (tcgen05)      HBM-bound
-//   agg_gemm_kernel    fp32 C = M * (B_hi + B_lo), M the 0/1 matrix      tensor/HBM
-//   fwd_linear_kernel  O = O_s + (phi(Q) H_i / den) W_proj              HBM-bound
+//   agg_gemm_kernel    C = M * (B_hi + B_lo), M the 0/1 matrix, C as hi/lo  tensor/HBM
+// (the combination O = O_s + (phi(Q) H_i / den) W_proj is in sla_fwd_linear.cu)
 #include <cuda_bf16.h>
 
 #include "sla_internal.h"
@@ -149,7 +149,9 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
 // ------------------------------------------------------------------ aggregation GEMM
 // C[bh][i][n] = sum_k A[bh][i][k] * (Bhi + Blo)[bh][k][n] with A the bf16 0/1
 // marginal matrix [Tp x Tp] (K-major), B the per-block summary rows [T x W]
-// as bf16 hi/lo planes (MN-major), C fp32 [T x W].  Tile 128 x 128 x 64,
+// as bf16 hi/lo planes (MN-major); C (fp32 in TMEM) is written back as bf16
+// hi/lo planes [T x W] (C = hi + lo), the operand format of its consumers.
+// Tile 128 x 128 x 64,
 // 2-stage TMA ring, warp 0 = TMA producer, warp 1 = MMA issuer, all 4 warps
 // = epilogue.  Two CTAs per SM overlap one's epilogue with the other's MMAs.
 constexpr int kAggBN = 128, kAggBK = 64, kAggStages = 2;
@@ -160,8 +162,9 @@ constexpr int kAggStageBytes = kAggA + 2 * kAggB;
 __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                                                        const __grid_constant__ CUtensorMap tm_bh,
                                                        const __grid_constant__ CUtensorMap tm_bl,
-                                                       float* __restrict__ out, int T, int Tp,
-                                                       int NN, int* err) {
+                                                       __nv_bfloat16* __restrict__ out_hi,
+                                                       __nv_bfloat16* __restrict__ out_lo, int T,
+                                                       int Tp, int NN, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = align_smem_1024(smem_raw);
   __shared__ uint64_t full[kAggStages], empty[kAggStages], acc_bar;
@@ -233,7 +236,7 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
   tc_fence_after();
   const int i = mt * 128 + warp * 32 + lane_id();
   if (ok) {
-    float* dst = out + (size_t(bh) * T + i) * NN + size_t(nt) * kAggBN;
+    const size_t o = (size_t(bh) * T + i) * NN + size_t(nt) * kAggBN;
 #pragma unroll 1
     for (int c0 = 0; c0 < kAggBN; c0 += 32) {
       float vals[32];
@@ -241,162 +244,19 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
       tmem_ld_wait();
       if (i < T && nt * kAggBN + c0 < NN) {  // NN is a multiple of 32
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst + c0 + e) =
-              make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_free(tmem, 128);
-}
-
-// ------------------------------------------------------------------ linear forward epilogue
-// One CTA per pair of query blocks (128 tokens); 256 threads: thread t owns
-// row r = t % 128 (its TMEM lane) and column half t / 128.
-//   NUM_h = phi(Q) (H_{2p+h,hi} + H_{2p+h,lo})   (tcgen05; the two halves in
-//   turn, each row keeps its own), den = phi(Q) . Z (fp32 from phi hi+lo),
-//   O_l = NUM / den, O = O_s + (O_l,hi + O_l,lo) W_proj.
-template <int D>
-__global__ void __launch_bounds__(256, 1) fwd_linear_kernel(
-    const __nv_bfloat16* __restrict__ q, const float* __restrict__ hz_agg,
-    const __nv_bfloat16* __restrict__ w_proj, const float* __restrict__ o_s,
-    __nv_bfloat16* __restrict__ o, float* __restrict__ den_out, int N, int T, int* err) {
-  constexpr int kTile = 128 * 128 * 2;  // 128 rows x 2 chunks (D = 64 padded)
-  constexpr int W = D * D + D;
-  constexpr int DH = D / 2;             // columns per thread
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = align_smem_1024(smem_raw);
-  uint8_t* sA = base;                  // phi(Q) hi, later O_l hi  (K-major, 128 rows)
-  uint8_t* sA2 = sA + kTile;           // phi(Q) lo, later O_l lo
-  uint8_t* sHh = sA2 + kTile;          // H hi                      (MN-major, D k-rows)
-  uint8_t* sHl = sHh + kTile;          // H lo
-  uint8_t* sW = sHl + kTile;           // W_proj                    (MN-major, D k-rows)
-  __shared__ float sZ[2][D];
-  __shared__ float sDen[2][128];
-  __shared__ uint64_t bar[3];
-  __shared__ uint32_t tmem_base;
-  const int p = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, warp = t / 32;
-  const int r = t & 127, ch = t >> 7, half = r >> 6;
-  const bool row_ok = 2 * p + half < T;
-  const int valid_rows = (2 * p + 1 < T) ? 128 : 64;
-  const size_t tok = size_t(p) * 128 + r;
-  const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
-  if (warp == 0) tmem_alloc(&tmem_base, 2 * D);
-  if (t == 0) {
-    for (int b = 0; b < 3; ++b) mbar_init(&bar[b], 1);
-    fence_barrier_init();
-  }
-  for (int e = t; e < 2 * D; e += 256) {
-    const int m = e / D, b2 = 2 * p + m;
-    sZ[m][e % D] = b2 < T ? hz_agg[(size_t(bh) * T + b2) * W + D * D + (e % D)] : 0.f;
-  }
-  load_rows_sw<D>(sW, D, w_proj, D, t, 256);
-  load_phi_sw<D>(sA, sA2, 128, q + (size_t(bh) * N + size_t(p) * 128) * D, valid_rows, t, 256);
-  load_split_sw<D>(sHh, sHl, D, hz_agg + (size_t(bh) * T + 2 * p) * W, D, t, 256);
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  // den = phi(Q) . Z_half, fp32 from the hi + lo parts
-  {
-    float acc = 0.f;
-    for (int c = ch * DH; c < (ch + 1) * DH; ++c)
-      acc = fmaf(ld_sw_bf16(sA, 128, r, c) + ld_sw_bf16(sA2, 128, r, c), sZ[half][c], acc);
-    sDen[ch][r] = acc;
-  }
-  const uint32_t tmem = tmem_base;
-  bool ok = true;
-  constexpr uint32_t idesc = idesc_bf16(128, D, 0, 1);
-  for (int m = 0; m < 2; ++m) {
-    if (m == 1) {
-      const int b2 = 2 * p + 1;
-      load_split_sw<D>(sHh, sHl, D, hz_agg + (size_t(bh) * T + (b2 < T ? b2 : 0)) * W,
-                       b2 < T ? D : 0, t, 256);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      tc_fence_after();
-    }
-    if (t == 0) {
-      const uint32_t a0 = smem_u32(sA);
+        for (int e = 0; e < 32; e += 8) {
+          uint32_t h[4], l[4];
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        mma_ss(tmem + m * D, desc_kmajor(a0, 128, ks), desc_mnmajor(smem_u32(sHh), D, ks),
-               idesc, ks > 0);
-        mma_ss(tmem + m * D, desc_kmajor(a0, 128, ks), desc_mnmajor(smem_u32(sHl), D, ks),
-               idesc, 1);
-      }
-      mma_commit(&bar[m]);
-    }
-    ok = mbar_wait(&bar[m], 0, err, nullptr) && ok;
-    tc_fence_after();
-  }
-  __syncthreads();  // sDen complete; phi(Q) tiles no longer read by any MMA
-  const float den = sDen[0][r] + sDen[1][r];
-  const float inv = (row_ok && den > 0.f) ? 1.0f / den : 0.0f;
-  if (row_ok && ch == 0) den_out[size_t(bh) * N + tok] = den;
-  // O_l = NUM / den, split into hi + lo bf16 (K-major rows)
-#pragma unroll 1
-  for (int c0 = ch * DH; c0 < (ch + 1) * DH; c0 += 32) {
-    float vals[32];
-    tmem_ld32(tmem + lane_base + half * D + c0, vals);
-    tmem_ld_wait();
-#pragma unroll
-    for (int u8 = 0; u8 < 4; ++u8) {
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        split2(ok ? vals[u8 * 8 + 2 * e] * inv : 0.f, ok ? vals[u8 * 8 + 2 * e + 1] * inv : 0.f,
-               hi[e], lo[e]);
-      st_sw128_unit(sA, 128, r, c0 + u8 * 8, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-      st_sw128_unit(sA2, 128, r, c0 + u8 * 8, make_uint4(lo[0], lo[1], lo[2], lo[3]));
-    }
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (t == 0) {
-    const uint32_t b0 = smem_u32(sW);
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      mma_ss(tmem, desc_kmajor(smem_u32(sA), 128, ks), desc_mnmajor(b0, D, ks), idesc, ks > 0);
-      mma_ss(tmem, desc_kmajor(smem_u32(sA2), 128, ks), desc_mnmajor(b0, D, ks), idesc, 1);
-    }
-    mma_commit(&bar[2]);
-  }
-  ok = mbar_wait(&bar[2], 0, err, nullptr) && ok;
-  tc_fence_after();
-  {
-    const float* osrow = o_s + (size_t(bh) * N + tok) * D;
-    __nv_bfloat16* orow = o + (size_t(bh) * N + tok) * D;
-#pragma unroll 1
-    for (int c0 = ch * DH; c0 < (ch + 1) * DH; c0 += 32) {
-      float vals[32];
-      tmem_ld32(tmem + lane_base + c0, vals);
-      tmem_ld_wait();
-      if (row_ok && ok) {
-        float4 s[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) s[u] = __ldg(reinterpret_cast<const float4*>(osrow + c0) + u);
-#pragma unroll
-        for (int u8 = 0; u8 < 4; ++u8) {
-          const float4 s0 = s[2 * u8], s1 = s[2 * u8 + 1];
-          uint4 rr;
-          rr.x = pack_bf16(s0.x + vals[u8 * 8 + 0], s0.y + vals[u8 * 8 + 1]);
-          rr.y = pack_bf16(s0.z + vals[u8 * 8 + 2], s0.w + vals[u8 * 8 + 3]);
-          rr.z = pack_bf16(s1.x + vals[u8 * 8 + 4], s1.y + vals[u8 * 8 + 5]);
-          rr.w = pack_bf16(s1.z + vals[u8 * 8 + 6], s1.w + vals[u8 * 8 + 7]);
-          *reinterpret_cast<uint4*>(orow + c0 + u8 * 8) = rr;
+          for (int u = 0; u < 4; ++u) split2(vals[e + 2 * u], vals[e + 2 * u + 1], h[u], l[u]);
+          *reinterpret_cast<uint4*>(out_hi + o + c0 + e) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(out_lo + o + c0 + e) = make_uint4(l[0], l[1], l[2], l[3]);
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_free(tmem, 2 * D);
+  if (warp == 0) tmem_free(tmem, 128);
 }
 
 template <typename K>
@@ -429,7 +289,8 @@ cudaError_t launch_summaries(const Problem& p, const void* k, const void* v,
 
 cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
                              const __nv_bfloat16* summ_hi, const __nv_bfloat16* summ_lo,
-                             float* out, int* err, cudaStream_t s) {
+                             __nv_bfloat16* out_hi, __nv_bfloat16* out_lo, int* err,
+                             cudaStream_t s) {
   const int NN = summary_width(p.d);
   CUtensorMap ta, tbh, tbl;
   if (!make_tmap_3d(&ta, mmat, p.Tp, p.Tp, p.BH, 64, 128)) return cudaErrorInvalidValue;
@@ -439,27 +300,7 @@ cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
   cudaError_t e = set_smem(agg_gemm_kernel, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.Tp / 128, (NN + kAggBN - 1) / kAggBN, p.BH);
-  agg_gemm_kernel<<<grid, 128, smem, s>>>(ta, tbh, tbl, out, p.T, p.Tp, NN, err);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_fwd_linear(const Problem& p, const void* q, const float* hz_agg,
-                              const void* w_proj, const float* o_s, void* o, float* den,
-                              int* err, cudaStream_t s) {
-  dim3 grid((p.T + 1) / 2, p.BH);
-  const size_t smem = 1024 + 5 * (128 * 128 * 2);
-  cudaError_t e;
-  if (p.d == 128) {
-    if ((e = set_smem(fwd_linear_kernel<128>, smem)) != cudaSuccess) return e;
-    fwd_linear_kernel<128><<<grid, 256, smem, s>>>((const __nv_bfloat16*)q, hz_agg,
-                                                   (const __nv_bfloat16*)w_proj, o_s,
-                                                   (__nv_bfloat16*)o, den, p.N, p.T, err);
-  } else {
-    if ((e = set_smem(fwd_linear_kernel<64>, smem)) != cudaSuccess) return e;
-    fwd_linear_kernel<64><<<grid, 256, smem, s>>>((const __nv_bfloat16*)q, hz_agg,
-                                                  (const __nv_bfloat16*)w_proj, o_s,
-                                                  (__nv_bfloat16*)o, den, p.N, p.T, err);
-  }
+  agg_gemm_kernel<<<grid, 128, smem, s>>>(ta, tbh, tbl, out_hi, out_lo, p.T, p.Tp, NN, err);
   return cudaGetLastError();
 }
 
