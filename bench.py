@@ -75,11 +75,10 @@ def kernel_work(wl, n_crit):
         "aggregate": ("tensor", 2 * BH * T * T * d * d),
         "aggregate_t": ("tensor", 2 * BH * T * T * d * d),
         "fwd_sparse": ("tensor", pairs * 4 * b * b * d),
-        "fwd_linear": ("hbm", tok * d * (2 + 4 + 2) + BH * T * d * d * 4 + tok * 4),
-        "bwd_prep": ("hbm", tok * d * (2 + 2 + 4 + 4) + BH * T * d * d * 4 + tok * 4 * 3),
-        "bwd_summ": ("hbm", tok * d * (2 + 4) + BH * T * d * d * 4 + tok * 4),
+        "fwd_linear": ("hbm", tok * d * (2 + 4 + 2) + BH * T * (d * d + d) * 4 + tok * 4),
+        "bwd_q": ("hbm", tok * d * (2 + 2 + 4 + 4) + 2 * BH * T * (d * d + d) * 4 + tok * 4 * 2),
         "bwd_sparse": ("tensor", pairs * 10 * b * b * d),
-        "bwd_linear": ("hbm", tok * d * (3 * 2 + 4 + 3 * 8) + 2 * BH * T * d * d * 4),
+        "bwd_k": ("hbm", tok * d * (2 + 2 + 8 + 8) + BH * T * (d * d + d) * 4),
         "expand_marginal": ("hbm", BH * Tp * Tp * 2),
         "expand_marginal_t": ("hbm", BH * Tp * Tp * 2),
     }

@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG_DIR, "libsla.so")
 
 SOURCES = ["sla_api.cu", "sla_classify.cu", "sla_linear.cu", "sla_fwd_linear.cu",
-           "sla_sparse_fwd.cu", "sla_backward.cu", "sla_sparse_bwd.cu", "sla_noalloc.cu"]
+           "sla_sparse_fwd.cu", "sla_bwd_linear.cu", "sla_sparse_bwd.cu", "sla_noalloc.cu"]
 HEADERS = ["sla_internal.h", "sla_ptx.cuh", "sla_tile.cuh"]
 
 NVCC_FLAGS = [

@@ -36,8 +36,6 @@ WorkspaceLayout workspace_layout(int BH, int N, int d) {
   L.mmat = take(bh * Tp * Tp * 2);
   L.mmat_t = take(bh * Tp * Tp * 2);
   L.dvec = take(bh * N * 4);
-  L.dnum = take(bh * N * d * 4);
-  L.dden = take(bh * N * 4);
   L.total = off;
   return L;
 }
@@ -346,24 +344,19 @@ sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, co
   const auto* hz_hi = static_cast<const __nv_bfloat16*>(saved->hz_agg);
   const auto* hz_lo = hz_hi + size_t(p.BH) * p.T * summary_width(p.d);
   float* dvec = at<float>(workspace, L.dvec);
-  float* dnum = at<float>(workspace, L.dnum);
-  float* dden = at<float>(workspace, L.dden);
-  const size_t grad_bytes = size_t(p.BH) * p.N * p.d * sizeof(float);
-  if (cudaMemsetAsync(dq, 0, grad_bytes, s) != cudaSuccess) return SLA_ERR_CUDA;
   if (cudaMemsetAsync(dw_proj, 0, size_t(p.d) * p.d * sizeof(float), s) != cudaSuccess)
     return SLA_ERR_CUDA;
-  // linear-branch preparation: D, dnum, dden, dW; then per-block A_i / a_i
-  SLA_LAUNCH("bwd_prep", s, launch_bwd_prep(p, q, d_o, w_proj, saved->o_s, saved->den,
-                                            hz_hi, hz_lo, dvec, dnum, dden, dw_proj, sms, err, s));
-  SLA_LAUNCH("bwd_summ", s, launch_bwd_summ(p, q, dnum, dden, summ_hi, summ_lo, err, s));
+  // linear branch, query side: D, dQ's linear share (written), dW, and the
+  // per-block (A_i | a_i) rows
+  SLA_LAUNCH("bwd_q", s, launch_bwd_q(p, q, d_o, w_proj, saved->o_s, saved->den, hz_hi, hz_lo,
+                                      dvec, dq, summ_hi, summ_lo, dw_proj, sms, err, s));
   // (dh_j | dz_j) = sum over rows i with j marginal of (A_i | a_i): transposed aggregation
   SLA_LAUNCH("expand_marginal_t", s, launch_expand_marginal(p, mask->marg_bits, nullptr, mmat_t, s));
   SLA_LAUNCH("aggregate_t", s, launch_aggregate(p, mmat_t, summ_hi, summ_lo, dh_hi, dh_lo, err, s));
-  // sparse branch writes dK, dV and accumulates dQ; the linear branch adds its share
+  // sparse branch adds to dQ and writes dK, dV; the linear branch's key side adds its share
   SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
                                mask->crit_col_idx, dq, dk, dv, err, s));
-  SLA_LAUNCH("bwd_linear", s, launch_bwd_linear(p, q, k, v, hz_hi, hz_lo, dh_hi, dh_lo, dnum, dden,
-                                                dq, dk, dv, err, s));
+  SLA_LAUNCH("bwd_k", s, launch_bwd_k(p, k, v, dh_hi, dh_lo, dk, dv, sms, err, s));
   return SLA_OK;
 }
 

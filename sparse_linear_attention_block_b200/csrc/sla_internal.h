@@ -36,8 +36,6 @@ struct WorkspaceLayout {
   size_t mmat;       // bf16 [BH,Tp,Tp] marginal 0/1 matrix, rows = query blocks
   size_t mmat_t;     // bf16 [BH,Tp,Tp] its transpose
   size_t dvec;       // fp32 [BH,N]     D_t = dO_t . O_s,t
-  size_t dnum;       // fp32 [BH,N,d]   dL/d(numerator)
-  size_t dden;       // fp32 [BH,N]     dL/d(denominator)
   size_t total;
 };
 
@@ -73,24 +71,18 @@ cudaError_t launch_fwd_sparse(const Problem& p, const void* q, const void* k, co
 cudaError_t launch_fwd_linear(const Problem& p, const void* q, const __nv_bfloat16* hz_hi,
                               const __nv_bfloat16* hz_lo, const void* w_proj, const float* o_s,
                               void* o, float* den, int* err, cudaStream_t s);
-cudaError_t launch_bwd_prep(const Problem& p, const void* q, const void* d_o, const void* w_proj,
-                            const float* o_s, const float* den, const __nv_bfloat16* hz_hi,
-                            const __nv_bfloat16* hz_lo, float* dvec,
-                            float* dnum, float* dden, float* dw, int num_sms, int* err,
-                            cudaStream_t s);
-cudaError_t launch_bwd_summ(const Problem& p, const void* q, const float* dnum,
-                            const float* dden, __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo,
-                            int* err, cudaStream_t s);
+cudaError_t launch_bwd_q(const Problem& p, const void* q, const void* d_o, const void* w_proj,
+                         const float* o_s, const float* den, const __nv_bfloat16* hz_hi,
+                         const __nv_bfloat16* hz_lo, float* dvec, float* dq,
+                         __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* dw, int num_sms,
+                         int* err, cudaStream_t s);
 cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
                               const void* d_o, const float* lse, const float* dvec,
                               const int32_t* col_ptr, const int32_t* col_idx, float* dq,
                               float* dk, float* dv, int* err, cudaStream_t s);
-cudaError_t launch_bwd_linear(const Problem& p, const void* q, const void* k, const void* v,
-                              const __nv_bfloat16* hz_hi, const __nv_bfloat16* hz_lo,
-                              const __nv_bfloat16* dh_hi, const __nv_bfloat16* dh_lo,
-                              const float* dnum,
-                              const float* dden, float* dq, float* dk, float* dv, int* err,
-                              cudaStream_t s);
+cudaError_t launch_bwd_k(const Problem& p, const void* k, const void* v,
+                         const __nv_bfloat16* dh_hi, const __nv_bfloat16* dh_lo, float* dk,
+                         float* dv, int num_sms, int* err, cudaStream_t s);
 
 // TMA descriptor for a bf16 [BH, N, d] tensor viewed as 3D {d, N, BH} with a
 // box of {64, rows, 1} and 128-byte swizzle.  Returns false on failure.
