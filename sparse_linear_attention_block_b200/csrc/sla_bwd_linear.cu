@@ -16,7 +16,8 @@
 // columns (every product has M = 128; d = 64 pads with zeros), take H_i and
 // dh_j as bf16 hi/lo planes by TMA, and keep the forward's split-bf16
 // precision (hi*hi + hi*lo + lo*hi where a value is fp32).
-//   bwd_q_kernel  persistent, one CTA per SM, per query block: D_t, dden,
+//   bwd_q_kernel  persistent, one CTA (two warpgroups, one per half of the
+//                 block's tokens) per SM, per query block: D_t, dden,
 //                 A_i | a_i (summary rows for the transposed aggregation),
 //                 dQ's linear share (written; the sparse branch adds to it),
 //                 dW accumulated in TMEM across the CTA's blocks
@@ -59,7 +60,7 @@ constexpr int kQT = 16384;  // a [64 t][128] or [128][64 t] bf16 tile
 constexpr int kBqSmem = 1024 + 2 * kQH + kQT + 2 * kQT + 2 * kQT;
 
 template <int D>
-__global__ void __launch_bounds__(128, 1) bwd_q_kernel(
+__global__ void __launch_bounds__(256, 1) bwd_q_kernel(
     const __grid_constant__ CUtensorMap tm_hh, const __grid_constant__ CUtensorMap tm_hl,
     const __grid_constant__ CUtensorMap tm_do, const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* __restrict__ d_o, const __nv_bfloat16* __restrict__ w_proj,
@@ -70,8 +71,9 @@ __global__ void __launch_bounds__(128, 1) bwd_q_kernel(
     int* err) {
   constexpr int W = D * D + D;
   constexpr int kU = D / 8;
-  constexpr int kRowsPerPass = 128 / kU;
+  constexpr int kRowsPerPass = 256 / kU;
   constexpr int kPass = 64 / kRowsPerPass;
+  constexpr int DH = D / 2;  // A_i columns per warpgroup
   // TMEM columns: W (packed A), dW, G^T, NUM^T -> O_l^T (packed), dQ^T, A_i
   constexpr uint32_t kW = 0, kDW = 64, kG = 192, kNum = 256, kDq = 320, kA = 384;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -88,9 +90,13 @@ __global__ void __launch_bounds__(128, 1) bwd_q_kernel(
   __shared__ float sRed[2][4][64];  // per-warp partial sums: G . O_l and dO . O_s
   __shared__ uint64_t bar_in, bar_c1, bar_c2;
   __shared__ uint32_t tmem_base;
+  // warpgroup g owns tokens [32g, 32g+32) of each block (TMEM columns), and
+  // its thread f = t % 128 owns feature f (TMEM lane)
   const int t = threadIdx.x, warp = t / 32, lane = int(lane_id());
-  const bool lane_ok = warp * 32 < D;
-  const uint32_t lane_base = uint32_t(warp * 32) << 16;
+  const int g = t >> 7, f = t & 127, wq = warp & 3;
+  const bool lane_ok = wq * 32 < D;
+  const uint32_t lane_base = uint32_t(wq * 32) << 16;
+  const int t0 = 32 * g;  // first token of this warpgroup
   auto tok_of = [&](int blk) { return size_t(blk / T) * N + size_t(blk % T) * 64; };
 
   if (warp == 0) tmem_alloc(&tmem_base, 512);
@@ -101,11 +107,11 @@ __global__ void __launch_bounds__(128, 1) bwd_q_kernel(
     fence_barrier_init();
   }
   if (D == 64) {  // zero the feature padding of the H and phi tiles
-    for (int e = t; e < (kQH - 8192) / 16; e += 128) {
+    for (int e = t; e < (kQH - 8192) / 16; e += 256) {
       reinterpret_cast<uint4*>(sHh + 8192)[e] = make_uint4(0, 0, 0, 0);
       reinterpret_cast<uint4*>(sHl + 8192)[e] = make_uint4(0, 0, 0, 0);
     }
-    for (int e = t; e < 8192 / 16; e += 128) {
+    for (int e = t; e < 8192 / 16; e += 256) {
       reinterpret_cast<uint4*>(sPh + 8192)[e] = make_uint4(0, 0, 0, 0);
       reinterpret_cast<uint4*>(sPl + 8192)[e] = make_uint4(0, 0, 0, 0);
     }
@@ -130,11 +136,12 @@ __global__ void __launch_bounds__(128, 1) bwd_q_kernel(
     tma_prefetch_desc(&tm_do);
     request_in(blockIdx.x);
   }
-  // W into TMEM as the A operand of G^T = W dO^T: lane c holds row c of W
+  // W into TMEM as the A operand of G^T = W dO^T: lane c holds row c of W;
+  // warpgroup g writes the columns of W's half g
   if (lane_ok) {
-    const uint4* wr = reinterpret_cast<const uint4*>(w_proj + size_t(t) * D);
+    const uint4* wr = reinterpret_cast<const uint4*>(w_proj + size_t(f) * D);
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
+    for (int c0 = g * DH; c0 < (g + 1) * DH; c0 += 32) {
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -150,22 +157,27 @@ __global__ void __launch_bounds__(128, 1) bwd_q_kernel(
   tmem_st_wait();
   const int u = t % kU, r0 = t / kU;
   uint4 qv[kPass];
-  auto load_q = [&](int blk) {
+  float os[32];  // O_s[t0 + j][f] of the block about to be processed
+  auto load_in = [&](int blk) {  // Q (phi input) and this thread's O_s column
     const size_t tk = tok_of(blk);
 #pragma unroll
     for (int b = 0; b < kPass; ++b)
       qv[b] = __ldg(reinterpret_cast<const uint4*>(q + (tk + r0 + b * kRowsPerPass) * D) + u);
+    if (lane_ok) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) os[j] = __ldg(o_s + (tk + t0 + j) * D + f);
+    }
   };
   auto load_zd = [&](int blk) {  // Z_i (hi + lo) and 1 / den of block blk
     if (t < D)
       sZ[t] = __bfloat162float(hz_hi[size_t(blk) * W + D * D + t]) +
               __bfloat162float(hz_lo[size_t(blk) * W + D * D + t]);
-    if (t < 64) {
-      const float dn = den[tok_of(blk) + t];
-      sInv[t] = dn > 0.f ? 1.0f / dn : 0.f;
+    if (t >= 128 && t < 192) {
+      const float dn = den[tok_of(blk) + (t - 128)];
+      sInv[t - 128] = dn > 0.f ? 1.0f / dn : 0.f;
     }
   };
-  load_q(blockIdx.x);
+  load_in(blockIdx.x);
   load_zd(blockIdx.x);
   bool ok = true;
   int k = 0;
@@ -213,62 +225,48 @@ __global__ void __launch_bounds__(128, 1) bwd_q_kernel(
       }
       mma_commit(&bar_c1);
     }
-    // ---- D_t = dO_t . O_s,t while the products run (lane = feature c)
+    // ---- D_t = dO_t . O_s,t while the products run (this warpgroup's 32 tokens)
     if (lane_ok) {
       const bool in_ok = mbar_wait(&bar_in, k & 1, err, nullptr);
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        float pd[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) pd[j] = __ldg(o_s + (tok0 + 32 * h + j) * D + t);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) pd[j] *= in_ok ? tile_at(sDO, 64, 32 * h + j, t) : 0.f;
-        sRed[1][warp][32 * h + lane] = warp_reduce_scatter32(pd);
-      }
+      for (int j = 0; j < 32; ++j) os[j] *= in_ok ? tile_at(sDO, 64, t0 + j, f) : 0.f;
+      sRed[1][wq][t0 + lane] = warp_reduce_scatter32(os);
     }
     ok = mbar_wait(&bar_c1, k & 1, err, nullptr) && ok;
     tc_fence_after();
     if (__syncthreads_or(!ok)) break;  // CTA-uniform exit; no copy is in flight
     // ---- O_l = NUM / den (back into TMEM, packed, as dW's A operand), dnum^T tiles,
     //      per-token partial sums of G . O_l
+    float nm[32], gv[32];
     if (lane_ok) {
-      float nm[64];
-      tmem_ld32(tmem + lane_base + kNum, reinterpret_cast<float(&)[32]>(nm[0]));
-      tmem_ld32(tmem + lane_base + kNum + 32, reinterpret_cast<float(&)[32]>(nm[32]));
+      tmem_ld32(tmem + lane_base + kNum + t0, nm);
+      tmem_ld32(tmem + lane_base + kG + t0, gv);
       tmem_ld_wait();
+    }
+    tc_fence_before();
+    __syncthreads();  // every NUM^T column read before the packed O_l overwrites them
+    tc_fence_after();
+    if (lane_ok) {
+      uint32_t dnh[16], dnl[16], ph[16], pl[16];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float g[32];
-        tmem_ld32(tmem + lane_base + kG + 32 * h, g);
-        tmem_ld_wait();
-        uint32_t dnh[16], dnl[16];
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float i0 = sInv[32 * h + j], i1 = sInv[32 * h + j + 1];
-          const float o0 = nm[32 * h + j] * i0, o1 = nm[32 * h + j + 1] * i1;
-          nm[32 * h + j] = o0;
-          nm[32 * h + j + 1] = o1;
-          split2(g[j] * i0, g[j + 1] * i1, dnh[j / 2], dnl[j / 2]);
-          g[j] *= o0;
-          g[j + 1] *= o1;
-        }
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          st_sw128_unit(sNh, 128, t, 32 * h + 8 * q4,
-                        make_uint4(dnh[4 * q4], dnh[4 * q4 + 1], dnh[4 * q4 + 2], dnh[4 * q4 + 3]));
-          st_sw128_unit(sNl, 128, t, 32 * h + 8 * q4,
-                        make_uint4(dnl[4 * q4], dnl[4 * q4 + 1], dnl[4 * q4 + 2], dnl[4 * q4 + 3]));
-        }
-        sRed[0][warp][32 * h + lane] = warp_reduce_scatter32(g);
+      for (int j = 0; j < 32; j += 2) {
+        const float i0 = sInv[t0 + j], i1 = sInv[t0 + j + 1];
+        const float o0 = nm[j] * i0, o1 = nm[j + 1] * i1;
+        split2(o0, o1, ph[j / 2], pl[j / 2]);
+        split2(gv[j] * i0, gv[j + 1] * i1, dnh[j / 2], dnl[j / 2]);
+        gv[j] *= o0;
+        gv[j + 1] *= o1;
       }
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t ph[16], pl[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) split2(nm[32 * h + 2 * e], nm[32 * h + 2 * e + 1], ph[e], pl[e]);
-        tmem_st16(tmem + lane_base + kNum + 16 * h, ph);
-        tmem_st16(tmem + lane_base + kNum + 32 + 16 * h, pl);
+      for (int q4 = 0; q4 < 4; ++q4) {
+        st_sw128_unit(sNh, 128, f, t0 + 8 * q4,
+                      make_uint4(dnh[4 * q4], dnh[4 * q4 + 1], dnh[4 * q4 + 2], dnh[4 * q4 + 3]));
+        st_sw128_unit(sNl, 128, f, t0 + 8 * q4,
+                      make_uint4(dnl[4 * q4], dnl[4 * q4 + 1], dnl[4 * q4 + 2], dnl[4 * q4 + 3]));
       }
+      tmem_st16(tmem + lane_base + kNum + 16 * g, ph);
+      tmem_st16(tmem + lane_base + kNum + 32 + 16 * g, pl);
+      sRed[0][wq][t0 + lane] = warp_reduce_scatter32(gv);
       tmem_st_wait();
     }
     fence_proxy_async_smem();
@@ -286,8 +284,7 @@ __global__ void __launch_bounds__(128, 1) bwd_q_kernel(
     }
     __syncthreads();
     tc_fence_after();
-    // ---- dW += O_l^T dO;  dQ^T = H (dnum_hi + dnum_lo)^T (+ H_lo dnum_hi^T);
-    //      A_i = phi^T dnum (split products)
+    // ---- dW += O_l^T dO;  dQ^T = H dnum^T (split products);  A_i = phi^T dnum
     if (t == 0) {
       constexpr uint32_t id_w = idesc_bf16(128, D, 0, 1);
       constexpr uint32_t id_q = idesc_bf16(128, 64, 0, 1);
@@ -323,41 +320,42 @@ __global__ void __launch_bounds__(128, 1) bwd_q_kernel(
       }
       mma_commit(&bar_c2);
     }
-    // ---- a_i = phi(Q_i)^T dden (fp32 from phi hi + lo), the Z part of the summary row
-    if (t < D) {
-      float acc = 0.f;
+    // ---- a_i = phi(Q_i)^T dden (fp32 from phi hi + lo): each warpgroup sums
+    //      its 32 tokens, warpgroup 0 adds the halves and writes the Z part
+    float ai = 0.f;
+    if (f < D) {
 #pragma unroll 8
-      for (int tt = 0; tt < 64; ++tt)
-        acc = fmaf(tile_at(sPh, 64, tt, t) + tile_at(sPl, 64, tt, t), sDd[tt], acc);
-      const __nv_bfloat16 h = __float2bfloat16_rn(acc);
-      summ_hi[size_t(blk) * W + D * D + t] = h;
-      summ_lo[size_t(blk) * W + D * D + t] = __float2bfloat16_rn(acc - __bfloat162float(h));
+      for (int j = 0; j < 32; ++j)
+        ai = fmaf(tile_at(sPh, 64, t0 + j, f) + tile_at(sPl, 64, t0 + j, f), sDd[t0 + j], ai);
+      if (g == 1) (&sRed[0][0][0])[f] = ai;  // sRed[0] (256 floats) is free again
+    }
+    __syncthreads();
+    if (g == 0 && f < D) {
+      ai += (&sRed[0][0][0])[f];
+      const __nv_bfloat16 h = __float2bfloat16_rn(ai);
+      summ_hi[size_t(blk) * W + D * D + f] = h;
+      summ_lo[size_t(blk) * W + D * D + f] = __float2bfloat16_rn(ai - __bfloat162float(h));
     }
     ok = mbar_wait(&bar_c2, k & 1, err, nullptr);
     tc_fence_after();
     if (__syncthreads_or(!ok)) break;
     if (t == 0 && nxt < nblk) request_in(nxt);  // H, dO tiles are free again
-    if (nxt < nblk) load_q(nxt);
-    // ---- dQ's linear share (lane = feature a): (dQ^T + dden Z_a) * phi'(q), written
+    if (nxt < nblk) load_in(nxt);
     if (lane_ok) {
-      const float za = sZ[t];
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        float v[32];
-        tmem_ld32(tmem + lane_base + kDq + 32 * h, v);
-        tmem_ld_wait();
+      // ---- dQ's linear share (lane = feature a, this warpgroup's tokens), written
+      const float za = sZ[f];
+      float v[32];
+      tmem_ld32(tmem + lane_base + kDq + t0, v);
+      tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int tt = 32 * h + j;
-          const float dph = fminf(tile_at(sPh, 64, tt, t) + tile_at(sPl, 64, tt, t), 1.0f);
-          dq[(tok0 + tt) * D + t] = fmaf(sDd[tt], za, v[j]) * dph;
-        }
+      for (int j = 0; j < 32; ++j) {
+        const float dph = fminf(tile_at(sPh, 64, t0 + j, f) + tile_at(sPl, 64, t0 + j, f), 1.0f);
+        dq[(tok0 + t0 + j) * D + f] = fmaf(sDd[t0 + j], za, v[j]) * dph;
       }
-      // A_i, row a of the summary (hi/lo planes)
-      const size_t srow = size_t(blk) * W + size_t(t) * D;
+      // A_i, row a of the summary (hi/lo planes), this warpgroup's column half
+      const size_t srow = size_t(blk) * W + size_t(f) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        float v[32];
+      for (int c0 = g * DH; c0 < (g + 1) * DH; c0 += 32) {
         tmem_ld32(tmem + lane_base + kA + c0, v);
         tmem_ld_wait();
 #pragma unroll
@@ -375,15 +373,15 @@ __global__ void __launch_bounds__(128, 1) bwd_q_kernel(
     tc_fence_after();
     if (nxt < nblk) load_zd(nxt);
   }
-  // this CTA's share of dW (lane = row c of dW)
+  // this CTA's share of dW (lane = row c of dW, this warpgroup's column half)
   if (ok && k > 0 && lane_ok) {
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
+    for (int c0 = g * DH; c0 < (g + 1) * DH; c0 += 32) {
       float v[32];
       tmem_ld32(tmem + lane_base + kDW + c0, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) atomicAdd(dw + size_t(t) * D + c0 + e, v[e]);
+      for (int e = 0; e < 32; ++e) atomicAdd(dw + size_t(f) * D + c0 + e, v[e]);
     }
   }
   tc_fence_before();
@@ -605,14 +603,14 @@ cudaError_t launch_bwd_q(const Problem& p, const void* q, const void* d_o, const
   if (p.d == 128) {
     e = cudaFuncSetAttribute(bwd_q_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBqSmem);
     if (e != cudaSuccess) return e;
-    bwd_q_kernel<128><<<grid, 128, kBqSmem, s>>>(
+    bwd_q_kernel<128><<<grid, 256, kBqSmem, s>>>(
         th, tl, tdo, (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o,
         (const __nv_bfloat16*)w_proj, o_s, den, hz_hi, hz_lo, dvec, dq, summ_hi, summ_lo, dw, p.N,
         p.T, nblk, err);
   } else {
     e = cudaFuncSetAttribute(bwd_q_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBqSmem);
     if (e != cudaSuccess) return e;
-    bwd_q_kernel<64><<<grid, 128, kBqSmem, s>>>(
+    bwd_q_kernel<64><<<grid, 256, kBqSmem, s>>>(
         th, tl, tdo, (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o,
         (const __nv_bfloat16*)w_proj, o_s, den, hz_hi, hz_lo, dvec, dq, summ_hi, summ_lo, dw, p.N,
         p.T, nblk, err);
