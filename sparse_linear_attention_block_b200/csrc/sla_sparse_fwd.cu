@@ -14,9 +14,12 @@
 // executed-block FLOPs).  Warp roles:
 //   warps 0-3  softmax: one query row per thread, S from TMEM, P back to
 //              TMEM (bf16, aliasing S), lazy rescaling of O in TMEM
-//   warp 4     TMA producer: Q tile once, K_j / V_j tiles into a 2-stage ring
-//   warp 5     MMA issuer (one thread): S_n = Q K_n^T into one of two TMEM
-//              buffers, O += P_n V_n with P read from TMEM
+//   warp 4     TMA producer: Q tile once; K_j tiles into a 2-slot ring whose
+//              slot is freed as soon as S_n = Q K_n^T has been computed, V_j
+//              into a 2-slot ring freed by P_n V_n (separate rings keep the K
+//              copies off the softmax -> P V -> S chain)
+//   warp 5     MMA issuer (one thread): S_n into one of two TMEM buffers,
+//              O += P_n V_n with P read from TMEM
 // TMEM: S buffers at columns [0,64) and [64,128), O at [128, 128+D).
 #include <cuda_bf16.h>
 
@@ -33,8 +36,7 @@ template <int D>
 struct FwdSmem {
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVBytes = 64 * D * 2;  // one K or V tile
-  static constexpr int kStageBytes = 2 * kKVBytes;
-  static constexpr int kTiles = kQBytes + kStages * kStageBytes;
+  static constexpr int kTiles = kQBytes + 2 * kStages * kKVBytes;  // K slots, then V slots
   // + the union list: 2*n_crit uint16 block indices, then 2*n_crit flag bytes
   static size_t total(int n_crit) { return 1024 + kTiles + size_t(2 * n_crit) * 3 + 16; }
 };
@@ -52,8 +54,8 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
   uint16_t* ulist = reinterpret_cast<uint16_t*>(base + L::kTiles);
   uint8_t* uflag = base + L::kTiles + 2 * (2 * n_crit);
 
-  __shared__ uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], p_full[2], o_done,
-      mma_done;
+  __shared__ uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages],
+      v_empty[kStages], s_full[2], p_full[2], o_done, mma_done;
   __shared__ uint32_t tmem_base;
   __shared__ int n_union, abort_flag;
 
@@ -66,8 +68,10 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
   if (threadIdx.x == 32) {
     mbar_init(&q_full, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -121,27 +125,48 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
       mbar_arrive_expect_tx(&q_full, L::kQBytes);
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * 128 * 128, &q_full, &tm_q, c * 64, p * 128, bh);
-      int issued = 0;
-      for (int n = 0; n < nU; ++n) {
+      // K_n needs S_{n-2} done, V_n needs P_{n-2} V_{n-2} done; the pipe
+      // completes S_0, S_1, PV_0, S_2, PV_1, S_3, ... so requests go out in
+      // that order: K_0 V_0 K_1 V_1 K_2 K_3, then V_m K_{m+2} for m >= 2.
+      int nk = 0, nv = 0;  // K and V copies issued
+      auto load_k = [&](int n) -> bool {
         const int s = n % kStages;
-        if (n >= kStages && !mbar_wait(&kv_empty[s], ((n / kStages) + 1) & 1, err, &abort_flag))
-          break;
-        uint8_t* sk = sKV + s * L::kStageBytes;
-        uint8_t* sv = sk + L::kKVBytes;
-        const int row = int(ulist[n]) * kBlock;
-        mbar_arrive_expect_tx(&kv_full[s], L::kStageBytes);
+        if (n >= kStages && !mbar_wait(&k_empty[s], ((n / kStages) + 1) & 1, err, &abort_flag))
+          return false;
+        uint8_t* sk = sKV + s * L::kKVBytes;
+        mbar_arrive_expect_tx(&k_full[s], L::kKVBytes);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(sk + c * 64 * 128, &kv_full[s], &tm_k, c * 64, row, bh);
-          tma_load_3d(sv + c * 64 * 128, &kv_full[s], &tm_v, c * 64, row, bh);
-        }
-        ++issued;
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sk + c * 64 * 128, &k_full[s], &tm_k, c * 64, int(ulist[n]) * kBlock, bh);
+        ++nk;
+        return true;
+      };
+      auto load_v = [&](int n) -> bool {
+        const int s = n % kStages;
+        if (n >= kStages && !mbar_wait(&v_empty[s], ((n / kStages) + 1) & 1, err, &abort_flag))
+          return false;
+        uint8_t* sv = sKV + (kStages + s) * L::kKVBytes;
+        mbar_arrive_expect_tx(&v_full[s], L::kKVBytes);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sv + c * 64 * 128, &v_full[s], &tm_v, c * 64, int(ulist[n]) * kBlock, bh);
+        ++nv;
+        return true;
+      };
+      bool go = true;
+      for (int n = 0; go && n < kStages && n < nU; ++n) go = load_k(n) && load_v(n);
+      for (int n = kStages; go && n < 2 * kStages && n < nU; ++n) go = load_k(n);
+      for (int m = kStages; go && m < nU; ++m) {
+        go = load_v(m);
+        if (go && m + kStages < nU) go = load_k(m + kStages);
       }
       if (abort_flag) {
         // let copies already in flight land before the CTA exits
         mbar_wait(&q_full, 0, nullptr, nullptr);
-        for (int n = (issued > kStages ? issued - kStages : 0); n < issued; ++n)
-          mbar_wait(&kv_full[n % kStages], (n / kStages) & 1, nullptr, nullptr);
+        for (int n = (nk > kStages ? nk - kStages : 0); n < nk; ++n)
+          mbar_wait(&k_full[n % kStages], (n / kStages) & 1, nullptr, nullptr);
+        for (int n = (nv > kStages ? nv - kStages : 0); n < nv; ++n)
+          mbar_wait(&v_full[n % kStages], (n / kStages) & 1, nullptr, nullptr);
       }
     }
   } else if (warp == 5) {
@@ -153,27 +178,30 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
       bool ok = mbar_wait(&q_full, 0, err, &abort_flag);
       auto issue_s = [&](int n) -> bool {
         const int s = n % kStages;
-        if (!mbar_wait(&kv_full[s], (n / kStages) & 1, err, &abort_flag)) return false;
+        if (!mbar_wait(&k_full[s], (n / kStages) & 1, err, &abort_flag)) return false;
         tc_fence_after();
-        const uint64_t kd = desc_kmajor_base(smem_u32(sKV + s * L::kStageBytes));
+        const uint64_t kd = desc_kmajor_base(smem_u32(sKV + s * L::kKVBytes));
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
           mma_ss(tmem + (n & 1) * 64, desc_advance(qd, kmajor_step_bytes(128, ks)),
                  desc_advance(kd, kmajor_step_bytes(64, ks)), idesc_s, ks > 0);
         mma_commit(&s_full[n & 1]);
+        mma_commit(&k_empty[s]);
         return true;
       };
       auto issue_pv = [&](int n) -> bool {
-        if (!mbar_wait(&p_full[n & 1], (n >> 1) & 1, err, &abort_flag)) return false;
-        tc_fence_after();
         const int s = n % kStages;
-        const uint64_t vd = desc_mnmajor_base(smem_u32(sKV + s * L::kStageBytes + L::kKVBytes), 64);
+        if (!mbar_wait(&p_full[n & 1], (n >> 1) & 1, err, &abort_flag) ||
+            !mbar_wait(&v_full[s], (n / kStages) & 1, err, &abort_flag))
+          return false;
+        tc_fence_after();
+        const uint64_t vd = desc_mnmajor_base(smem_u32(sKV + (kStages + s) * L::kKVBytes), 64);
         const uint32_t pt = tmem + (n & 1) * 64;  // P aliases the first 32 columns of S
 #pragma unroll
         for (int ks = 0; ks < kBlock / 16; ++ks)
           mma_ts(tm_o, pt + ks * 8, desc_advance(vd, mnmajor_step_bytes(ks)), idesc_o, (n | ks) != 0);
         mma_commit(&o_done);
-        mma_commit(&kv_empty[s]);
+        mma_commit(&v_empty[s]);
         return true;
       };
       if (ok) ok = issue_s(0);
@@ -206,12 +234,10 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
       const bool member = row_ok && ((uflag[n] >> half) & 1);
       float alpha = 1.f;
       if (member) {
-        float mx = -INFINITY;
+        float mx = -INFINITY;  // the scale is positive: max of the raw scores, then scaled
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          sv[e] *= scale_log2;
-          mx = fmaxf(mx, sv[e]);
-        }
+        for (int e = 0; e < 64; ++e) mx = fmaxf(mx, sv[e]);
+        mx *= scale_log2;
         if (mx > m_run + kRescaleThreshold || m_run == -INFINITY) {
           alpha = exp2f(m_run - mx);  // 0 when m_run == -inf
           l_run *= alpha;
@@ -220,7 +246,7 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
         float sum = 0.f;
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
-          sv[e] = exp2f(sv[e] - m_run);
+          sv[e] = exp2f(fmaf(sv[e], scale_log2, -m_run));
           sum += sv[e];
         }
         l_run += sum;
