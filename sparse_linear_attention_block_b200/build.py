@@ -20,7 +20,7 @@ LIB = os.path.join(PKG_DIR, "libsla.so")
 
 SOURCES = ["sla_api.cu", "sla_classify.cu", "sla_linear.cu", "sla_fwd_linear.cu",
            "sla_sparse_fwd.cu", "sla_bwd_linear.cu", "sla_sparse_bwd.cu", "sla_noalloc.cu"]
-HEADERS = ["sla_internal.h", "sla_ptx.cuh", "sla_tile.cuh"]
+HEADERS = ["sla_internal.h", "sla_ptx.cuh", "sla_tile.cuh", "sla_union.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -27,6 +27,7 @@
 
 #include "sla_internal.h"
 #include "sla_ptx.cuh"
+#include "sla_union.cuh"
 
 namespace sla {
 namespace {
@@ -107,9 +108,8 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
   }
   if (warp == 8) {
     // union of the critical query blocks of key blocks 2q and 2q+1; flag bit h
-    // = query block critical for key block 2q+h.  The two column lists are
-    // staged in the (still idle) stage buffers with coalesced loads, then
-    // merged from shared memory by one lane.
+    // = query block critical for key block 2q+h (bitmap scratch in the still
+    // idle stage buffers)
     const int32_t* cp = col_ptr + size_t(bh) * (T + 1);
     const int32_t* ci = col_idx + size_t(bh) * T * n_crit;
     int a = cp[kb0], ae = cp[kb0 + 1];
@@ -119,28 +119,9 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
       if (lane == 0) set_error(err, SLA_ERR_DEVICE);
       a = ae = b = be = 0;
     }
-    const int la = ae - a, lb = be - b;
-    int32_t* la_s = reinterpret_cast<int32_t*>(sSt);  // up to T + T entries
-    int32_t* lb_s = la_s + la;
-    for (int x = lane; x < la; x += 32) la_s[x] = ci[a + x];
-    for (int x = lane; x < lb; x += 32) lb_s[x] = ci[b + x];
-    __syncwarp();
-    if (lane == 0) {
-      int ia = 0, ib = 0, n = 0;
-      while (ia < la || ib < lb) {
-        const int x = ia < la ? la_s[ia] : 0x7FFFFFFF;
-        const int y = ib < lb ? lb_s[ib] : 0x7FFFFFFF;
-        int i, f;
-        if (x == y) { i = x; f = 3; ++ia; ++ib; }
-        else if (x < y) { i = x; f = 1; ++ia; }
-        else { i = y; f = 2; ++ib; }
-        if (i < 0 || i >= T || n >= 2 * T) { set_error(err, SLA_ERR_DEVICE); continue; }
-        ulist[n] = uint16_t(i);
-        uflag[n] = uint8_t(f);
-        ++n;
-      }
-      n_union = n;
-    }
+    const int n = warp_union(ci + a, ae - a, ci + b, be - b, T, reinterpret_cast<uint32_t*>(sSt),
+                             ulist, uflag, err);
+    if (lane == 0) n_union = n;
   }
   tc_fence_before();
   __syncthreads();
@@ -151,7 +132,7 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && nU > 0) {
-      fence_proxy_async_smem();  // list staging used these buffers generically
+      fence_proxy_async_smem();  // the union's scratch used these buffers generically
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(&kv_full, 2 * L::kKV);

@@ -25,6 +25,7 @@
 
 #include "sla_internal.h"
 #include "sla_ptx.cuh"
+#include "sla_union.cuh"
 
 namespace sla {
 namespace {
@@ -83,30 +84,12 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
     fence_barrier_init();
   }
   if (warp == 4) {
-    // sorted union of the two rows' critical lists; flag bit h = member of
-    // half h.  Both rows are staged in the (still idle) K/V stage buffers
-    // with coalesced loads and merged from shared memory by one lane.
-    const int n1 = has1 ? n_crit : 0;
+    // sorted union of the two rows' critical lists (bitmap scratch in the
+    // still idle K/V slots); flag bit h = member of row 2p+h
     const int32_t* l0 = crit_idx + (size_t(bh) * T + blk0) * n_crit;  // row 2p+1 follows
-    int32_t* ls = reinterpret_cast<int32_t*>(sKV);
-    for (int x = lane; x < n_crit + n1; x += 32) ls[x] = l0[x];
-    __syncwarp();
-    if (lane == 0) {
-      int a = 0, b = 0, n = 0;
-      while (a < n_crit || b < n1) {
-        const int x = a < n_crit ? ls[a] : 0x7FFFFFFF;
-        const int y = b < n1 ? ls[n_crit + b] : 0x7FFFFFFF;
-        int j, f;
-        if (x == y) { j = x; f = 3; ++a; ++b; }
-        else if (x < y) { j = x; f = 1; ++a; }
-        else { j = y; f = 2; ++b; }
-        if (j < 0 || j >= T) { set_error(err, SLA_ERR_DEVICE); continue; }
-        ulist[n] = uint16_t(j);
-        uflag[n] = uint8_t(f);
-        ++n;
-      }
-      n_union = n;
-    }
+    const int n = warp_union(l0, n_crit, l0 + n_crit, has1 ? n_crit : 0, T,
+                             reinterpret_cast<uint32_t*>(sKV), ulist, uflag, err);
+    if (lane == 0) n_union = n;
   }
   tc_fence_before();
   __syncthreads();
@@ -118,7 +101,7 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
   if (warp == 4) {
     // ---------------------------------------------------------------- producer
     if (lane == 0 && nU > 0) {
-      fence_proxy_async_smem();  // list staging used these buffers generically
+      fence_proxy_async_smem();  // the union's scratch used these buffers generically
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
