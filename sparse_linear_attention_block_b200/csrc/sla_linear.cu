@@ -151,28 +151,30 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
 // marginal matrix [Tp x Tp] (K-major), B the per-block summary rows [T x W]
 // as bf16 hi/lo planes (MN-major); C (fp32 in TMEM) is written back as bf16
 // hi/lo planes [T x W] (C = hi + lo), the operand format of its consumers.
-// Tile 128 x 128 x 64,
-// 2-stage TMA ring, warp 0 = TMA producer, warp 1 = MMA issuer, all 4 warps
-// = epilogue.  Two CTAs per SM overlap one's epilogue with the other's MMAs.
-constexpr int kAggBN = 128, kAggBK = 64, kAggStages = 2;
-constexpr int kAggA = 128 * kAggBK * 2;        // 16 KB
+// One CTA covers up to 512 rows (four 128 x 128 accumulators, all of TMEM)
+// of one 128-column slice, so each B slice is read once and A once per
+// slice; K in steps of 64 through a 2-stage TMA ring.  Warp 0 = TMA
+// producer, warp 1 = MMA issuer, all 4 warps = epilogue.
+constexpr int kAggBN = 128, kAggBK = 64, kAggStages = 2, kAggMT = 4;
+constexpr int kAggA = 128 * kAggBK * 2;        // 16 KB per 128-row tile
 constexpr int kAggB = kAggBK * kAggBN * 2;     // 16 KB per plane
-constexpr int kAggStageBytes = kAggA + 2 * kAggB;
+constexpr int kAggStageBytes = kAggMT * kAggA + 2 * kAggB;
 
-__global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
-                                                       const __grid_constant__ CUtensorMap tm_bh,
-                                                       const __grid_constant__ CUtensorMap tm_bl,
-                                                       __nv_bfloat16* __restrict__ out_hi,
-                                                       __nv_bfloat16* __restrict__ out_lo, int T,
-                                                       int Tp, int NN, int* err) {
+__global__ void __launch_bounds__(128, 1) agg_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
+                                                          const __grid_constant__ CUtensorMap tm_bh,
+                                                          const __grid_constant__ CUtensorMap tm_bl,
+                                                          __nv_bfloat16* __restrict__ out_hi,
+                                                          __nv_bfloat16* __restrict__ out_lo,
+                                                          int T, int Tp, int NN, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = align_smem_1024(smem_raw);
   __shared__ uint64_t full[kAggStages], empty[kAggStages], acc_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
-  const int mt = blockIdx.x, nt = blockIdx.y, bh = blockIdx.z;
+  const int mg = blockIdx.x, nt = blockIdx.y, bh = blockIdx.z;
   const int warp = threadIdx.x / 32;
   const int nk = Tp / kAggBK;
+  const int nmt = min(kAggMT, Tp / 128 - mg * kAggMT);  // 128-row tiles of this CTA
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAggStages; ++s) {
       mbar_init(&full[s], 1);
@@ -182,7 +184,7 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
     abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0) tmem_alloc(&tmem_base, 128);
+  if (warp == 0) tmem_alloc(&tmem_base, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -199,9 +201,10 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
           !mbar_wait(&empty[s], ((kt / kAggStages) + 1) & 1, err, &abort_flag))
         break;
       uint8_t* sa = base + s * kAggStageBytes;
-      uint8_t* sb = sa + kAggA;
-      mbar_arrive_expect_tx(&full[s], kAggStageBytes);
-      tma_load_3d(sa, &full[s], &tm_a, kt * kAggBK, mt * 128, bh);
+      uint8_t* sb = sa + kAggMT * kAggA;
+      mbar_arrive_expect_tx(&full[s], nmt * kAggA + 2 * kAggB);
+      for (int m = 0; m < nmt; ++m)
+        tma_load_3d(sa + m * kAggA, &full[s], &tm_a, kt * kAggBK, (mg * kAggMT + m) * 128, bh);
       for (int c = 0; c < 2; ++c) {
         tma_load_3d(sb + c * 8192, &full[s], &tm_bh, nt * kAggBN + c * 64, kt * kAggBK, bh);
         tma_load_3d(sb + kAggB + c * 8192, &full[s], &tm_bl, nt * kAggBN + c * 64, kt * kAggBK, bh);
@@ -218,14 +221,17 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
       if (!mbar_wait(&full[s], (kt / kAggStages) & 1, err, &abort_flag)) break;
       tc_fence_after();
       const uint32_t sa = smem_u32(base + s * kAggStageBytes);
-      const uint64_t ad = desc_kmajor_base(sa);
-      const uint64_t bhd = desc_mnmajor_base(sa + kAggA, kAggBK);
-      const uint64_t bld = desc_mnmajor_base(sa + kAggA + kAggB, kAggBK);
+      const uint64_t bhd = desc_mnmajor_base(sa + kAggMT * kAggA, kAggBK);
+      const uint64_t bld = desc_mnmajor_base(sa + kAggMT * kAggA + kAggB, kAggBK);
+      for (int m = 0; m < nmt; ++m) {
+        const uint64_t ad = desc_kmajor_base(sa + m * kAggA);
 #pragma unroll
-      for (int ks = 0; ks < kAggBK / 16; ++ks) {
-        const uint64_t a = desc_advance(ad, kmajor_step_bytes(128, ks));
-        mma_ss(tmem, a, desc_advance(bhd, mnmajor_step_bytes(ks)), idesc, (kt | ks) != 0);
-        mma_ss(tmem, a, desc_advance(bld, mnmajor_step_bytes(ks)), idesc, 1);
+        for (int ks = 0; ks < kAggBK / 16; ++ks) {
+          const uint64_t a = desc_advance(ad, kmajor_step_bytes(128, ks));
+          mma_ss(tmem + m * kAggBN, a, desc_advance(bhd, mnmajor_step_bytes(ks)), idesc,
+                 (kt | ks) != 0);
+          mma_ss(tmem + m * kAggBN, a, desc_advance(bld, mnmajor_step_bytes(ks)), idesc, 1);
+        }
       }
       mma_commit(&empty[s]);
     }
@@ -234,29 +240,31 @@ __global__ void __launch_bounds__(128) agg_gemm_kernel(const __grid_constant__ C
   __syncwarp();
   const bool ok = mbar_wait(&acc_bar, 0, err, &abort_flag);
   tc_fence_after();
-  const int i = mt * 128 + warp * 32 + lane_id();
   if (ok) {
-    const size_t o = (size_t(bh) * T + i) * NN + size_t(nt) * kAggBN;
+    for (int m = 0; m < nmt; ++m) {
+      const int i = (mg * kAggMT + m) * 128 + warp * 32 + lane_id();
+      const size_t o = (size_t(bh) * T + i) * NN + size_t(nt) * kAggBN;
 #pragma unroll 1
-    for (int c0 = 0; c0 < kAggBN; c0 += 32) {
-      float vals[32];
-      tmem_ld32(tmem_addr(tmem, warp * 32, c0), vals);
-      tmem_ld_wait();
-      if (i < T && nt * kAggBN + c0 < NN) {  // NN is a multiple of 32
+      for (int c0 = 0; c0 < kAggBN; c0 += 32) {
+        float vals[32];
+        tmem_ld32(tmem_addr(tmem, warp * 32, m * kAggBN + c0), vals);
+        tmem_ld_wait();
+        if (i < T && nt * kAggBN + c0 < NN) {  // NN is a multiple of 32
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint32_t h[4], l[4];
+          for (int e = 0; e < 32; e += 8) {
+            uint32_t h[4], l[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) split2(vals[e + 2 * u], vals[e + 2 * u + 1], h[u], l[u]);
-          *reinterpret_cast<uint4*>(out_hi + o + c0 + e) = make_uint4(h[0], h[1], h[2], h[3]);
-          *reinterpret_cast<uint4*>(out_lo + o + c0 + e) = make_uint4(l[0], l[1], l[2], l[3]);
+            for (int u = 0; u < 4; ++u) split2(vals[e + 2 * u], vals[e + 2 * u + 1], h[u], l[u]);
+            *reinterpret_cast<uint4*>(out_hi + o + c0 + e) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4*>(out_lo + o + c0 + e) = make_uint4(l[0], l[1], l[2], l[3]);
+          }
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_free(tmem, 128);
+  if (warp == 0) tmem_free(tmem, 512);
 }
 
 template <typename K>
@@ -299,7 +307,7 @@ cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
   const size_t smem = 1024 + kAggStages * kAggStageBytes;
   cudaError_t e = set_smem(agg_gemm_kernel, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.Tp / 128, (NN + kAggBN - 1) / kAggBN, p.BH);
+  dim3 grid((p.Tp / 128 + kAggMT - 1) / kAggMT, (NN + kAggBN - 1) / kAggBN, p.BH);
   agg_gemm_kernel<<<grid, 128, smem, s>>>(ta, tbh, tbl, out_hi, out_lo, p.T, p.Tp, NN, err);
   return cudaGetLastError();
 }
