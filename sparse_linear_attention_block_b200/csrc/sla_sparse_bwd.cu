@@ -268,15 +268,22 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
         tmem_ld32(dp_t + c0, dpv);
         tmem_ld_wait();
         uint32_t pk[16], dk16[16];
+        // LSE and D of these 32 queries, as 16-byte broadcast loads
+        float lv[32], dv4[32];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          *reinterpret_cast<float4*>(&lv[e]) = *reinterpret_cast<const float4*>(sl + c0 + e);
+          *reinterpret_cast<float4*>(&dv4[e]) = *reinterpret_cast<const float4*>(sd + c0 + e);
+        }
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           float p0 = 0.f, p1 = 0.f;
           if (member) {
-            p0 = exp2f(fmaf(sv[e], scale_log2, -sl[c0 + e] * 1.4426950408889634f));
-            p1 = exp2f(fmaf(sv[e + 1], scale_log2, -sl[c0 + e + 1] * 1.4426950408889634f));
+            p0 = exp2f(fmaf(sv[e], scale_log2, -lv[e] * 1.4426950408889634f));
+            p1 = exp2f(fmaf(sv[e + 1], scale_log2, -lv[e + 1] * 1.4426950408889634f));
           }
           pk[e / 2] = pack_bf16(p0, p1);
-          dk16[e / 2] = pack_bf16(p0 * (dpv[e] - sd[c0 + e]), p1 * (dpv[e + 1] - sd[c0 + e + 1]));
+          dk16[e / 2] = pack_bf16(p0 * (dpv[e] - dv4[e]), p1 * (dpv[e + 1] - dv4[e + 1]));
         }
         tmem_st16(st_t + c0 / 2, pk);
         tmem_st16(dp_t + c0 / 2, dk16);
