@@ -294,7 +294,11 @@ def main():
         step()
     torch.cuda.synchronize()
     prof = slab.sla_profile_end()
-    launches_per_step = sum(n for n, _ in prof.values()) / args.steps
+    # each profiled call is one kernel launch, except the CSR build (count, scan
+    # and, when there are critical blocks, fill kernels)
+    kernels_per_call = {"crit_csr": 3 if n_crit > 0 else 2}
+    launches_per_step = sum(n * kernels_per_call.get(name, 1)
+                            for name, (n, _) in prof.items()) / args.steps
     pk, src = peaks()
     work = kernel_work(wl, n_crit)
     per_kernel = {name: {"launches": n, "ms_per_launch": tot / n,
