@@ -61,6 +61,15 @@ def executed_block_flops(wl, n_crit):
     return fwd, bwd
 
 
+# DRAM bytes (read + write) per head of one launch, from the ncu captures under
+# profiles/ of the kernels as they are now (4-head case, divided by 4; the
+# traffic grows with the number of heads).  A kernel missing here reports
+# traffic null; an entry must be dropped or re-measured when its kernel changes.
+NCU_DRAM_BYTES_PER_HEAD = {
+    "bwd_sparse": (204.957184e6 + 153.236480e6) / 4,  # bwd_sparse_wan4h_full.md
+}
+
+
 def kernel_work(wl, n_crit):
     """Algorithmic work per launch of each kernel: ('tensor', FLOP) or ('hbm', bytes)."""
     B, H, N, d, T = wl.B, wl.H, wl.N, wl.d, wl.T
@@ -306,18 +315,20 @@ def main():
                   for name, (n, tot) in prof.items()}
     dominant = max(prof, key=lambda n: prof[n][1])
     kind, amount = work.get(dominant, ("tensor", 0))
+    traffic = (NCU_DRAM_BYTES_PER_HEAD[dominant] * wl.B * wl.H
+               if dominant in NCU_DRAM_BYTES_PER_HEAD else None)
     avg_s = prof[dominant][1] / prof[dominant][0] * 1e-3
     if kind == "tensor":
         achieved = amount / avg_s / 1e12
         peak = pk["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "kernel": dominant,
+                "frac": achieved / peak, "traffic": traffic, "kernel": dominant,
                 "peak_source": f"{src} sustained bf16"}
     else:
         achieved = amount / avg_s / 1e9
         peak = pk["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None, "kernel": dominant,
+                "frac": achieved / peak, "traffic": traffic, "kernel": dominant,
                 "peak_source": f"{src} HBM copy"}
     fwd_ms = sum(prof[n][1] for n in ("summaries", "expand_marginal", "aggregate",
                                       "aggregate_z", "fwd_sparse", "fwd_linear")
@@ -330,25 +341,38 @@ def main():
     if not args.no_e2e:
         hosts = [torch.from_numpy(x).to(torch.bfloat16).pin_memory()
                  for x in (wl.q, wl.k, wl.v, wl.w_proj, wl.d_o)]
-        devs = [torch.empty_like(h, device=dev) for h in hosts]
+        # two device input sets: step i's inputs cross PCIe on a copy stream
+        # while step i-1 computes (every copy is inside the timed region)
+        sets = [[torch.empty_like(h, device=dev) for h in hosts] for _ in range(2)]
+        copy_stream = torch.cuda.Stream(dev)
+        copied = [torch.cuda.Event() for _ in range(2)]
+        used = [torch.cuda.Event() for _ in range(2)]
         dw_host = torch.empty(dw.shape, dtype=torch.float32).pin_memory()
         h2d = sum(h.numel() * h.element_size() for h in hosts)
         d2h = dw_host.numel() * dw_host.element_size()
 
-        def e2e_step():
-            for hsrc, ddst in zip(hosts, devs):
-                ddst.copy_(hsrc, non_blocking=True)
-            step(*devs)
-            dw_host.copy_(dw, non_blocking=True)
+        def e2e_run(nsteps, start=None):
+            if start is not None:
+                copy_stream.wait_event(start)
+            for i in range(nsteps):
+                b = i % 2
+                with torch.cuda.stream(copy_stream):
+                    if i >= 2:
+                        copy_stream.wait_event(used[b])
+                    for hsrc, ddst in zip(hosts, sets[b]):
+                        ddst.copy_(hsrc, non_blocking=True)
+                    copied[b].record(copy_stream)
+                stream.wait_event(copied[b])
+                step(*sets[b])
+                used[b].record(stream)
+                dw_host.copy_(dw, non_blocking=True)  # the step's result back to the host
 
-        for _ in range(3):
-            e2e_step()
+        e2e_run(3)
         torch.cuda.synchronize()
         barrier()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        e2e_run(args.steps, start=a0)
         a1.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps)
