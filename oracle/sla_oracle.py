@@ -29,6 +29,14 @@ map, the combination and the backward math; this oracle takes these readings
       sum_{u in j} phi(K_u); no epsilon; 0 when row i has no marginal block.
 * R7  O = O_s + O_l W_proj, W_proj one d x d matrix for all heads.
 * R8  gradients treat the classification as a constant.
+* R12 optional gate on the linear branch, after the page "SALAD: Achieve
+      High-Sparsity Attention via Efficient Linear Attention Tuning for Video
+      Diffusion Transformer", section "Methodologie: SALAD", items 2 (a global
+      factor in (0, 1) from a sigmoid scales the linear branch) and 3 (branches
+      with a very low factor are dropped at inference): with a caller-given
+      logit gamma and threshold tau, g = sigmoid(gamma) and
+      O = O_s + g * O_l W_proj; when g < tau the branch is dropped, O = O_s,
+      and neither the branch nor gamma gets a gradient.
 
 Arrays are [B, H, N, d]; blocks are consecutive runs of ``block`` tokens.
 """
@@ -48,6 +56,7 @@ __all__ = [
     "phi",
     "phi_prime",
     "key_block_summaries",
+    "gate_factor",
     "forward",
     "forward_bruteforce",
     "backward",
@@ -140,18 +149,33 @@ def key_block_summaries(k: np.ndarray, v: np.ndarray, block: int):
     return h, z
 
 
+def gate_factor(gate) -> tuple[float, bool]:
+    """(g, dropped) for gate = (gamma, tau) or None (reading R12).
+
+    g = 1 / (1 + exp(-gamma)); None means no gate (g = 1, never dropped).
+    """
+    if gate is None:
+        return 1.0, False
+    gamma, tau = float(gate[0]), float(gate[1])
+    g = 1.0 / (1.0 + math.exp(-gamma)) if gamma > -700 else 0.0
+    return g, g < tau
+
+
 def _tokens(blocks: np.ndarray, block: int) -> np.ndarray:
     return (blocks[:, None] * block + np.arange(block)[None, :]).reshape(-1)
 
 
 def forward(q, k, v, w_proj, cls, block: int, scale: float | None = None,
-            query_blocks=None):
+            query_blocks=None, gate=None):
     """SLA forward with a given class map ``cls`` [B,H,T,T].
 
-    Returns a dict with o, o_s, o_l [B,H,N,d], lse and den [B,H,N] (fp64).
-    ``query_blocks``, if given, restricts the work to those query-block
-    indices (other rows stay zero / -inf); used to sample large problems.
+    Returns a dict with o, o_s, o_l [B,H,N,d], lse and den [B,H,N] (fp64),
+    and the gate factor g.  ``query_blocks``, if given, restricts the work to
+    those query-block indices (other rows stay zero / -inf); used to sample
+    large problems.  ``gate`` = (gamma, tau) gates the linear branch (R12); a
+    dropped branch leaves o_l and den zero.
     """
+    g, dropped = gate_factor(gate)
     B, H, N, d = q.shape
     T = N // block
     if scale is None:
@@ -186,7 +210,7 @@ def forward(q, k, v, w_proj, cls, block: int, scale: float | None = None,
                     o_s[b, hh, t0:t1] = (e @ v64[b, hh, keys]) / l
                     lse[b, hh, t0:t1] = (m + np.log(l))[:, 0]
                 # marginal pairs: linear attention through the key-block summaries
-                if marg.size:
+                if marg.size and not dropped:
                     Hi, Zi = H_all[i], Z_all[i]
                     fq = phi(qi)
                     num = fq @ Hi
@@ -194,8 +218,8 @@ def forward(q, k, v, w_proj, cls, block: int, scale: float | None = None,
                     o_l[b, hh, t0:t1] = num / dn[:, None]
                     den[b, hh, t0:t1] = dn
                 # negligible pairs contribute nothing
-    o = o_s + np.einsum("bhta,ac->bhtc", o_l, w64)
-    return {"o": o, "o_s": o_s, "o_l": o_l, "lse": lse, "den": den}
+    o = o_s + g * np.einsum("bhta,ac->bhtc", o_l, w64)
+    return {"o": o, "o_s": o_s, "o_l": o_l, "lse": lse, "den": den, "g": g}
 
 
 def forward_bruteforce(q, k, v, w_proj, cls, block: int, scale: float | None = None):
@@ -244,7 +268,7 @@ def forward_bruteforce(q, k, v, w_proj, cls, block: int, scale: float | None = N
 
 
 def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
-             fwd=None):
+             fwd=None, gate=None):
     """Gradients of sum(O * dO) w.r.t. Q, K, V and W_proj, classes held fixed (R8).
 
     Sparse branch (standard softmax-attention backward over critical pairs):
@@ -259,21 +283,28 @@ def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
       dphi(K_u) = dh_j V_u + dz_j;  dK_u += dphi(K_u) * phi'(K_u);
       dV_u += dh_j^T phi(K_u).
     Projection: dW = sum over b, h, t of O_l,t dO_t^T.
+    Gate (R12): the linear branch sees g dO, so dO_l, dW and everything
+    downstream of them carry the factor g, and
+      d gamma = g (1 - g) sum over b, h, t of (O_l,t W) . dO_t;
+    a dropped branch contributes nothing and d gamma = 0.
     """
+    g, dropped = gate_factor(gate)
     B, H, N, d = q.shape
     T = N // block
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if fwd is None:
-        fwd = forward(q, k, v, w_proj, cls, block, scale)
+        fwd = forward(q, k, v, w_proj, cls, block, scale, gate=gate)
     q64, k64, v64, do64 = (np.asarray(a, dtype=np.float64) for a in (q, k, v, d_o))
     w64 = np.asarray(w_proj, dtype=np.float64)
     h, z = key_block_summaries(k64, v64, block)
     dq = np.zeros_like(q64)
     dk = np.zeros_like(k64)
     dv = np.zeros_like(v64)
-    dw = np.einsum("bhta,bhtc->ac", fwd["o_l"], do64)
-    do_l = np.einsum("bhtc,ac->bhta", do64, w64)
+    dw = g * np.einsum("bhta,bhtc->ac", fwd["o_l"], do64)
+    do_l = g * np.einsum("bhtc,ac->bhta", do64, w64)
+    d_gamma = 0.0 if dropped else (
+        g * (1.0 - g) * float(np.einsum("bhta,ac,bhtc->", fwd["o_l"], w64, do64)))
     for b in range(B):
         for hh in range(H):
             marg_ind = (cls[b, hh] == 0).astype(np.float64)
@@ -298,7 +329,7 @@ def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
                     ds = p * (dp - D)
                     dq[b, hh, t0:t1] += scale * (ds @ kc)
                     dk[b, hh, keys] += scale * (ds.T @ qi)
-                if marg.size:
+                if marg.size and not dropped:
                     Hi, Zi = H_all[i], Z_all[i]
                     dn = fwd["den"][b, hh, t0:t1]
                     dol = do_l[b, hh, t0:t1]
@@ -318,7 +349,7 @@ def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
                 dfk = vj @ dh[j].T + dz[j][None, :]
                 dk[b, hh, u0:u1] += dfk * phi_prime(kj)
                 dv[b, hh, u0:u1] += phi(kj) @ dh[j]
-    return {"dq": dq, "dk": dk, "dv": dv, "dw": dw}
+    return {"dq": dq, "dk": dk, "dv": dv, "dw": dw, "d_gamma": d_gamma}
 
 
 def sla(q, k, v, w_proj, block: int, k_h: float, k_l: float, scale: float | None = None):

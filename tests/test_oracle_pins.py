@@ -293,3 +293,89 @@ def test_workload_generators_shapes_and_stats():
     # zero padding past the grid
     p = sla_inputs.make_grid((1, 3, 7), H=1, name="p")
     assert p.N == 64 and p.n_valid == 21 and np.all(p.q[:, :, 21:] == 0)
+
+
+# ---------------------------------------------------------------- gated linear branch (R12)
+
+def test_gate_factor_closed_form():
+    assert oracle.gate_factor(None) == (1.0, False)
+    g, dropped = oracle.gate_factor((0.0, 0.25))
+    assert g == 0.5 and not dropped
+    g, dropped = oracle.gate_factor((math.log(3.0), 0.0))  # sigmoid(log 3) = 3/4
+    assert math.isclose(g, 0.75, rel_tol=1e-15) and not dropped
+    assert oracle.gate_factor((-math.log(9.0), 0.2)) == pytest.approx((0.1, True))
+    assert oracle.gate_factor((float("inf"), 0.5)) == (1.0, False)
+
+
+def test_gate_open_is_ungated():
+    q, k, v, w = _small(N=256, d=16, seed=40)
+    cls = _cls_from(q, k, 32, 0.25, 0.25)
+    do = np.random.default_rng(41).standard_normal(q.shape)
+    a = oracle.forward(q, k, v, w, cls, 32)
+    b = oracle.forward(q, k, v, w, cls, 32, gate=(float("inf"), 0.5))
+    assert np.array_equal(a["o"], b["o"])
+    ga = oracle.backward(q, k, v, w, cls, do, 32)
+    gb = oracle.backward(q, k, v, w, cls, do, 32, gate=(float("inf"), 0.5))
+    for n in ("dq", "dk", "dv", "dw"):
+        assert np.array_equal(ga[n], gb[n]), n
+    assert gb["d_gamma"] == 0.0  # g (1 - g) = 0
+
+
+def test_gate_scales_only_the_linear_share():
+    q, k, v, w = _small(N=256, d=16, seed=42)
+    cls = _cls_from(q, k, 32, 0.25, 0.25)
+    a = oracle.forward(q, k, v, w, cls, 32)
+    b = oracle.forward(q, k, v, w, cls, 32, gate=(-0.7, 0.05))
+    g = 1.0 / (1.0 + math.exp(0.7))
+    np.testing.assert_allclose(b["o"] - b["o_s"], g * (a["o"] - a["o_s"]), rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(a["o_s"], b["o_s"])
+
+
+def test_dropped_gate_equals_no_marginal_blocks():
+    # dropping the branch must give exactly the problem in which every
+    # marginal block is negligible instead (outputs and all gradients)
+    q, k, v, w = _small(N=256, d=16, seed=44)
+    cls = _cls_from(q, k, 32, 0.25, 0.25)
+    assert np.any(cls == 0)
+    do = np.random.default_rng(45).standard_normal(q.shape)
+    cls_nm = np.where(cls == 0, -1, cls).astype(cls.dtype)
+    gate = (-3.0, 0.1)  # g = 0.047 < 0.1
+    a = oracle.forward(q, k, v, w, cls, 32, gate=gate)
+    b = oracle.forward(q, k, v, w, cls_nm, 32)
+    np.testing.assert_array_equal(a["o"], b["o"])
+    ga = oracle.backward(q, k, v, w, cls, do, 32, gate=gate)
+    gb = oracle.backward(q, k, v, w, cls_nm, do, 32)
+    for n in ("dq", "dk", "dv", "dw"):
+        np.testing.assert_array_equal(ga[n], gb[n], err_msg=n)
+    assert ga["d_gamma"] == 0.0
+
+
+@pytest.mark.parametrize("gamma", [-1.3, 0.4, 2.0])
+def test_gate_gradient_matches_central_difference(gamma):
+    q, k, v, w = _small(B=1, H=1, N=256, d=8, seed=46)
+    cls = _cls_from(q, k, 16, 0.25, 0.25)
+    do = np.random.default_rng(47).standard_normal(q.shape)
+
+    def loss(gm):
+        return float(np.sum(oracle.forward(q, k, v, w, cls, 16, gate=(gm, 0.0))["o"] * do))
+
+    eps = 1e-5
+    fd = (loss(gamma + eps) - loss(gamma - eps)) / (2 * eps)
+    got = oracle.backward(q, k, v, w, cls, do, 16, gate=(gamma, 0.0))
+    assert math.isclose(fd, got["d_gamma"], rel_tol=1e-7, abs_tol=1e-10), (fd, got["d_gamma"])
+    # and the other gradients still match finite differences with the gate on
+    rng = np.random.default_rng(48)
+    for name in ("q", "w"):
+        arr = {"q": q, "w": w}[name]
+        grad = got["d" + name]
+        for _ in range(6):
+            idx = tuple(rng.integers(0, s) for s in arr.shape)
+            xp, xm = arr.copy(), arr.copy()
+            xp[idx] += 1e-6
+            xm[idx] -= 1e-6
+            argp = {"q": q, "w": w}
+            argm = dict(argp)
+            argp[name], argm[name] = xp, xm
+            lp = np.sum(oracle.forward(argp["q"], k, v, argp["w"], cls, 16, gate=(gamma, 0.0))["o"] * do)
+            lm = np.sum(oracle.forward(argm["q"], k, v, argm["w"], cls, 16, gate=(gamma, 0.0))["o"] * do)
+            assert math.isclose((lp - lm) / 2e-6, grad[idx], rel_tol=2e-6, abs_tol=2e-8)
