@@ -221,6 +221,10 @@ def main():
     ap.add_argument("--impl", choices=["sla", "reference"], default="sla")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gate-logit", type=float, default=None,
+                    help="run the gated entry points with this gate logit (default: ungated)")
+    ap.add_argument("--gate-skip", type=float, default=0.0,
+                    help="drop the linear branch when sigmoid(logit) is below this")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -256,11 +260,21 @@ def main():
     dw = torch.empty(w.shape, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    gate = None if args.gate_logit is None else slab.Gate(args.gate_logit, args.gate_skip)
+    d_logit = torch.empty(1, dtype=torch.float32, device=dev)
+
     def step(qq=q, kk=k, vv=v, ww=w, dd=do):
         slab.sla_classify(shape, qq, kk, buf.mask, buf.workspace, stream)
-        slab.sla_forward(shape, qq, kk, vv, ww, buf.mask, o, buf.saved, buf.workspace, stream)
-        slab.sla_backward(shape, qq, kk, vv, ww, buf.mask, buf.saved, dd, dq, dk, dv, dw,
-                          buf.workspace, stream)
+        if gate is None:
+            slab.sla_forward(shape, qq, kk, vv, ww, buf.mask, o, buf.saved, buf.workspace,
+                             stream)
+            slab.sla_backward(shape, qq, kk, vv, ww, buf.mask, buf.saved, dd, dq, dk, dv, dw,
+                              buf.workspace, stream)
+        else:
+            slab.sla_forward_gated(shape, qq, kk, vv, ww, buf.mask, gate, o, buf.saved,
+                                   buf.workspace, stream)
+            slab.sla_backward_gated(shape, qq, kk, vv, ww, buf.mask, gate, buf.saved, dd, dq, dk,
+                                    dv, dw, d_logit, buf.workspace, stream)
 
     def barrier():
         if world > 1:
@@ -331,7 +345,7 @@ def main():
                 "frac": achieved / peak, "traffic": traffic, "kernel": dominant,
                 "peak_source": f"{src} HBM copy"}
     fwd_ms = sum(prof[n][1] for n in ("summaries", "expand_marginal", "aggregate",
-                                      "aggregate_z", "fwd_sparse", "fwd_linear")
+                                      "fwd_sparse", "fwd_linear", "os_to_o")
                  if n in prof) / args.steps
     cls_ms = sum(prof[n][1] for n in ("pool", "classify", "crit_csr") if n in prof) / args.steps
     bwd_ms = sum(t for n, (_, t) in prof.items()) / args.steps - fwd_ms - cls_ms
@@ -394,11 +408,16 @@ def main():
     if rank != 0:
         return
     peak_t = pk["bf16_tflops_sustained"]
+    cfg = workload_config(wl, n_crit)
+    if gate is not None:
+        g = 1.0 / (1.0 + math.exp(-args.gate_logit))
+        cfg["gate"] = {"logit": args.gate_logit, "skip_below": args.gate_skip, "g": g,
+                       "linear_branch_dropped": g < args.gate_skip}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": workload_config(wl, n_crit),
+        "data": "synthetic", "config": cfg,
         "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "classify_ms": cls_ms,
         "fwd_tflops": fwd_flops / (fwd_ms * 1e-3) / 1e12,
         "bwd_tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12,

@@ -160,6 +160,37 @@ SLA_API sla_status sla_backward(const sla_shape* shape, const void* q, const voi
                         const void* d_o, float* dq, float* dk, float* dv, float* dw_proj,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* Gate on the linear branch, after the page "SALAD: Achieve High-Sparsity
+ * Attention via Efficient Linear Attention Tuning for Video Diffusion
+ * Transformer", section "Methodologie: SALAD", items 2 (a global factor in
+ * (0, 1) from a sigmoid scales the linear branch) and 3 (branches whose
+ * factor is very low are dropped at inference):
+ *   g = 1 / (1 + exp(-logit)),  O = O_s + g * O_l W_proj;
+ *   g < skip_below: the branch is dropped, O = O_s, its kernels are not
+ *   launched and neither the branch nor the logit gets a gradient.
+ * logit = +inf gives g = 1 (the ungated forward, bit for bit). */
+typedef struct {
+  float logit;
+  float skip_below;
+} sla_gate;
+
+/* sla_forward with a gate (gate must not be NULL; NaN fields are rejected).
+ * A dropped branch leaves saved->hz_agg unwritten and saved->den untouched. */
+SLA_API sla_status sla_forward_gated(const sla_shape* shape, const void* q, const void* k,
+                                     const void* v, const void* w_proj, const sla_mask* mask,
+                                     const sla_gate* gate, void* o, const sla_saved* saved,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* sla_backward with the same gate as the forward.  Also writes *d_logit
+ * (device fp32 scalar, overwritten): g (1 - g) times the sum over B, H, N of
+ * (O_l W_proj) . dO; 0 when the branch is dropped. */
+SLA_API sla_status sla_backward_gated(const sla_shape* shape, const void* q, const void* k,
+                                      const void* v, const void* w_proj, const sla_mask* mask,
+                                      const sla_gate* gate, const sla_saved* saved,
+                                      const void* d_o, float* dq, float* dk, float* dv,
+                                      float* dw_proj, float* d_logit, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
 /* Zero the workspace's device error word (asynchronously on `stream`).  Call
  * once on a new workspace before its first use; sla_check() clears it
  * afterwards. */

@@ -23,7 +23,7 @@ __all__ = [
     "sla_query_sizes", "sla_classify", "sla_classify_from_scores", "sla_forward",
     "sla_backward", "sla_workspace_init", "sla_check", "sla_strerror", "sla_version",
     "sla_profile_begin", "sla_profile_end", "KernelStat", "make_shape", "EXPORTED_SYMBOLS",
-    "STATUS",
+    "STATUS", "Gate", "sla_forward_gated", "sla_backward_gated",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -35,7 +35,7 @@ STATUS = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED", 3: "S
 EXPORTED_SYMBOLS = ["sla_query_sizes", "sla_classify", "sla_classify_from_scores",
                     "sla_forward", "sla_backward", "sla_workspace_init", "sla_check",
                     "sla_strerror", "sla_version", "sla_profile_begin", "sla_profile_end",
-                    "sla_classify_noalloc"]
+                    "sla_classify_noalloc", "sla_forward_gated", "sla_backward_gated"]
 
 
 class SlaError(RuntimeError):
@@ -59,6 +59,11 @@ class MaskStruct(ctypes.Structure):
 class SavedStruct(ctypes.Structure):
     _fields_ = [("lse", ctypes.c_void_p), ("o_s", ctypes.c_void_p), ("den", ctypes.c_void_p),
                 ("hz_agg", ctypes.c_void_p)]
+
+
+class Gate(ctypes.Structure):
+    """sla_gate: g = sigmoid(logit); the linear branch is dropped when g < skip_below."""
+    _fields_ = [("logit", ctypes.c_float), ("skip_below", ctypes.c_float)]
 
 
 class KernelStat(ctypes.Structure):
@@ -95,6 +100,10 @@ def lib() -> ctypes.CDLL:
                                   vp, sz, vp]
         L.sla_backward.argtypes = [P(Shape), vp, vp, vp, vp, P(MaskStruct), P(SavedStruct), vp,
                                    vp, vp, vp, vp, vp, sz, vp]
+        L.sla_forward_gated.argtypes = [P(Shape), vp, vp, vp, vp, P(MaskStruct), P(Gate), vp,
+                                        P(SavedStruct), vp, sz, vp]
+        L.sla_backward_gated.argtypes = [P(Shape), vp, vp, vp, vp, P(MaskStruct), P(Gate),
+                                         P(SavedStruct), vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_workspace_init.argtypes = [vp, sz, vp]
         L.sla_check.argtypes = [vp, vp]
         L.sla_strerror.argtypes = [st]
@@ -107,7 +116,7 @@ def lib() -> ctypes.CDLL:
         L.sla_profile_end.argtypes = [P(KernelStat), st, P(st)]
         for n in ("sla_query_sizes", "sla_classify", "sla_classify_from_scores", "sla_forward",
                   "sla_backward", "sla_workspace_init", "sla_check", "sla_profile_begin",
-                  "sla_profile_end"):
+                  "sla_profile_end", "sla_forward_gated", "sla_backward_gated"):
             getattr(L, n).restype = st
         _lib = L
     return _lib
@@ -217,6 +226,26 @@ def sla_backward(shape: Shape, q, k, v, w_proj, mask: MaskStruct, saved: SavedSt
                               _ptr(dk), _ptr(dv), _ptr(dw_proj), _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream)),
            "sla_backward")
+
+
+def sla_forward_gated(shape: Shape, q, k, v, w_proj, mask: MaskStruct, gate: Gate, o,
+                      saved: SavedStruct, workspace, stream=None):
+    _check(lib().sla_forward_gated(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(w_proj),
+                                   ctypes.byref(mask), ctypes.byref(gate), _ptr(o),
+                                   ctypes.byref(saved), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "sla_forward_gated")
+
+
+def sla_backward_gated(shape: Shape, q, k, v, w_proj, mask: MaskStruct, gate: Gate,
+                       saved: SavedStruct, d_o, dq, dk, dv, dw_proj, d_logit, workspace,
+                       stream=None):
+    _check(lib().sla_backward_gated(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(w_proj),
+                                    ctypes.byref(mask), ctypes.byref(gate), ctypes.byref(saved),
+                                    _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dw_proj),
+                                    _ptr(d_logit), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
+           "sla_backward_gated")
 
 
 @dataclasses.dataclass

@@ -282,16 +282,31 @@ static sla_status check_saved(const Problem& p, const sla_saved* sv) {
   return SLA_OK;
 }
 
-sla_status sla_forward(const sla_shape* shape, const void* q, const void* k, const void* v,
-                       const void* w_proj, const sla_mask* mask, void* o,
-                       const sla_saved* saved, void* workspace, size_t workspace_bytes,
-                       void* stream) {
+// g and whether the branch is dropped, for a gate or none (g = 1, kept)
+static bool gate_values(const sla_gate* gate, float* g, bool* dropped) {
+  *g = 1.0f;
+  *dropped = false;
+  if (!gate) return true;
+  if (std::isnan(gate->logit) || std::isnan(gate->skip_below)) return false;
+  const double gd = 1.0 / (1.0 + std::exp(-double(gate->logit)));
+  *g = float(gd);
+  *dropped = gd < double(gate->skip_below);
+  return true;
+}
+
+static sla_status forward_impl(const sla_shape* shape, const void* q, const void* k, const void* v,
+                               const void* w_proj, const sla_mask* mask, const sla_gate* gate,
+                               void* o, const sla_saved* saved, void* workspace,
+                               size_t workspace_bytes, void* stream) {
   Problem p;
   sla_status st = check_shape(shape, &p);
   if (st != SLA_OK) return st;
   if (!q || !k || !v || !w_proj || !o) return SLA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(w_proj) || !aligned16(o))
     return SLA_ERR_INVALID_ARG;
+  float g;
+  bool dropped;
+  if (!gate_values(gate, &g, &dropped)) return SLA_ERR_INVALID_ARG;
   if ((st = check_mask(p, mask, false)) != SLA_OK) return st;
   if ((st = check_saved(p, saved)) != SLA_OK) return st;
   WorkspaceLayout L;
@@ -301,23 +316,46 @@ sla_status sla_forward(const sla_shape* shape, const void* q, const void* k, con
   auto* summ_hi = at<__nv_bfloat16>(workspace, L.summ_hi);
   auto* summ_lo = at<__nv_bfloat16>(workspace, L.summ_lo);
   auto* mmat = at<__nv_bfloat16>(workspace, L.mmat);
+  auto* hz_hi = static_cast<__nv_bfloat16*>(saved->hz_agg);
+  auto* hz_lo = hz_hi + size_t(p.BH) * p.T * summary_width(p.d);
+  if (dropped) {  // sparse branch only: O = O_s
+    SLA_LAUNCH("fwd_sparse", s, launch_fwd_sparse(p, q, k, v, mask->crit_idx, saved->o_s, saved->lse, err, s));
+    SLA_LAUNCH("os_to_o", s, launch_os_to_o(p, saved->o_s, o, s));
+    return SLA_OK;
+  }
   // linear branch: (h_j | z_j) summaries, then (H_i | Z_i) by one aggregation GEMM
   SLA_LAUNCH("summaries", s, launch_summaries(p, k, v, summ_hi, summ_lo, err, s));
   SLA_LAUNCH("expand_marginal", s, launch_expand_marginal(p, mask->marg_bits, mmat, nullptr, s));
-  auto* hz_hi = static_cast<__nv_bfloat16*>(saved->hz_agg);
-  auto* hz_lo = hz_hi + size_t(p.BH) * p.T * summary_width(p.d);
   SLA_LAUNCH("aggregate", s, launch_aggregate(p, mmat, summ_hi, summ_lo, hz_hi, hz_lo, err, s));
   // sparse branch, then the combination
   SLA_LAUNCH("fwd_sparse", s, launch_fwd_sparse(p, q, k, v, mask->crit_idx, saved->o_s, saved->lse, err, s));
   SLA_LAUNCH("fwd_linear", s, launch_fwd_linear(p, q, hz_hi, hz_lo, w_proj, saved->o_s, o,
-                                                saved->den, err, s));
+                                                saved->den, g, err, s));
   return SLA_OK;
 }
 
-sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, const void* v,
-                        const void* w_proj, const sla_mask* mask, const sla_saved* saved,
-                        const void* d_o, float* dq, float* dk, float* dv, float* dw_proj,
-                        void* workspace, size_t workspace_bytes, void* stream) {
+sla_status sla_forward(const sla_shape* shape, const void* q, const void* k, const void* v,
+                       const void* w_proj, const sla_mask* mask, void* o,
+                       const sla_saved* saved, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  return forward_impl(shape, q, k, v, w_proj, mask, nullptr, o, saved, workspace,
+                      workspace_bytes, stream);
+}
+
+sla_status sla_forward_gated(const sla_shape* shape, const void* q, const void* k, const void* v,
+                             const void* w_proj, const sla_mask* mask, const sla_gate* gate,
+                             void* o, const sla_saved* saved, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (!gate) return SLA_ERR_INVALID_ARG;
+  return forward_impl(shape, q, k, v, w_proj, mask, gate, o, saved, workspace, workspace_bytes,
+                      stream);
+}
+
+static sla_status backward_impl(const sla_shape* shape, const void* q, const void* k,
+                                const void* v, const void* w_proj, const sla_mask* mask,
+                                const sla_gate* gate, const sla_saved* saved, const void* d_o,
+                                float* dq, float* dk, float* dv, float* dw_proj, float* d_logit,
+                                void* workspace, size_t workspace_bytes, void* stream) {
   Problem p;
   sla_status st = check_shape(shape, &p);
   if (st != SLA_OK) return st;
@@ -326,6 +364,9 @@ sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, co
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(w_proj) || !aligned16(d_o) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dw_proj))
     return SLA_ERR_INVALID_ARG;
+  float g;
+  bool dropped;
+  if (!gate_values(gate, &g, &dropped)) return SLA_ERR_INVALID_ARG;
   if ((st = check_mask(p, mask, true)) != SLA_OK) return st;
   if ((st = check_saved(p, saved)) != SLA_OK) return st;
   WorkspaceLayout L;
@@ -346,10 +387,19 @@ sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, co
   float* dvec = at<float>(workspace, L.dvec);
   if (cudaMemsetAsync(dw_proj, 0, size_t(p.d) * p.d * sizeof(float), s) != cudaSuccess)
     return SLA_ERR_CUDA;
+  if (d_logit && cudaMemsetAsync(d_logit, 0, sizeof(float), s) != cudaSuccess) return SLA_ERR_CUDA;
+  if (dropped) {  // sparse branch only
+    if (cudaMemsetAsync(dq, 0, size_t(p.BH) * p.N * p.d * sizeof(float), s) != cudaSuccess)
+      return SLA_ERR_CUDA;
+    SLA_LAUNCH("dvec", s, launch_dvec(p, d_o, saved->o_s, dvec, s));
+    SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
+                                 mask->crit_col_idx, dq, dk, dv, err, s));
+    return SLA_OK;
+  }
   // linear branch, query side: D, dQ's linear share (written), dW, and the
   // per-block (A_i | a_i) rows
   SLA_LAUNCH("bwd_q", s, launch_bwd_q(p, q, d_o, w_proj, saved->o_s, saved->den, hz_hi, hz_lo,
-                                      dvec, dq, summ_hi, summ_lo, dw_proj, sms, err, s));
+                                      dvec, dq, summ_hi, summ_lo, dw_proj, g, d_logit, sms, err, s));
   // (dh_j | dz_j) = sum over rows i with j marginal of (A_i | a_i): transposed aggregation
   SLA_LAUNCH("expand_marginal_t", s, launch_expand_marginal(p, mask->marg_bits, nullptr, mmat_t, s));
   SLA_LAUNCH("aggregate_t", s, launch_aggregate(p, mmat_t, summ_hi, summ_lo, dh_hi, dh_lo, err, s));
@@ -358,6 +408,25 @@ sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, co
                                mask->crit_col_idx, dq, dk, dv, err, s));
   SLA_LAUNCH("bwd_k", s, launch_bwd_k(p, k, v, dh_hi, dh_lo, dk, dv, sms, err, s));
   return SLA_OK;
+}
+
+sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, const void* v,
+                        const void* w_proj, const sla_mask* mask, const sla_saved* saved,
+                        const void* d_o, float* dq, float* dk, float* dv, float* dw_proj,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  return backward_impl(shape, q, k, v, w_proj, mask, nullptr, saved, d_o, dq, dk, dv, dw_proj,
+                       nullptr, workspace, workspace_bytes, stream);
+}
+
+sla_status sla_backward_gated(const sla_shape* shape, const void* q, const void* k,
+                              const void* v, const void* w_proj, const sla_mask* mask,
+                              const sla_gate* gate, const sla_saved* saved, const void* d_o,
+                              float* dq, float* dk, float* dv, float* dw_proj, float* d_logit,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  if (!gate || !d_logit || (reinterpret_cast<uintptr_t>(d_logit) & 3u) != 0)
+    return SLA_ERR_INVALID_ARG;
+  return backward_impl(shape, q, k, v, w_proj, mask, gate, saved, d_o, dq, dk, dv, dw_proj,
+                       d_logit, workspace, workspace_bytes, stream);
 }
 
 sla_status sla_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {

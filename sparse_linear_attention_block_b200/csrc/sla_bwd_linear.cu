@@ -67,8 +67,8 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(
     const float* __restrict__ o_s, const float* __restrict__ den,
     const __nv_bfloat16* __restrict__ hz_hi, const __nv_bfloat16* __restrict__ hz_lo,
     float* __restrict__ dvec, float* __restrict__ dq, __nv_bfloat16* __restrict__ summ_hi,
-    __nv_bfloat16* __restrict__ summ_lo, float* __restrict__ dw, int N, int T, int nblk,
-    int* err) {
+    __nv_bfloat16* __restrict__ summ_lo, float* __restrict__ dw, float gate, float gate_slope,
+    float* __restrict__ d_gate, int N, int T, int nblk, int* err) {
   constexpr int W = D * D + D;
   constexpr int kU = D / 8;
   constexpr int kRowsPerPass = 256 / kU;
@@ -180,6 +180,7 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(
   load_in(blockIdx.x);
   load_zd(blockIdx.x);
   bool ok = true;
+  float gate_acc = 0.f;  // sum over this CTA's tokens of G . O_l (threads < 64)
   int k = 0;
   for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x, ++k) {
     const size_t tok0 = tok_of(blk);
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(
         const float i0 = sInv[t0 + j], i1 = sInv[t0 + j + 1];
         const float o0 = nm[j] * i0, o1 = nm[j + 1] * i1;
         split2(o0, o1, ph[j / 2], pl[j / 2]);
-        split2(gv[j] * i0, gv[j + 1] * i1, dnh[j / 2], dnl[j / 2]);
+        split2(gv[j] * (gate * i0), gv[j + 1] * (gate * i1), dnh[j / 2], dnl[j / 2]);
         gv[j] *= o0;
         gv[j + 1] *= o1;
       }
@@ -279,8 +280,9 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(
         gs += sRed[0][w][t];
         ds += sRed[1][w][t];
       }
-      sDd[t] = -gs * sInv[t];
+      sDd[t] = -gate * gs * sInv[t];
       dvec[tok0 + t] = ds;
+      gate_acc += gs;
     }
     __syncthreads();
     tc_fence_after();
@@ -381,8 +383,15 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(
       tmem_ld32(tmem + lane_base + kDW + c0, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) atomicAdd(dw + size_t(f) * D + c0 + e, v[e]);
+      for (int e = 0; e < 32; ++e) atomicAdd(dw + size_t(f) * D + c0 + e, v[e] * gate);
     }
+  }
+  // d gamma += g (1 - g) * sum of G . O_l (the linear branch's share of
+  // sum O . dO before the gate), one reduction per warp
+  if (d_gate && ok && t < 64) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) gate_acc += __shfl_xor_sync(0xffffffffu, gate_acc, m);
+    if (lane == 0) atomicAdd(d_gate, gate_slope * gate_acc);
   }
   tc_fence_before();
   __syncthreads();
@@ -586,13 +595,45 @@ __global__ void __launch_bounds__(128, 1) bwd_k_kernel(
   if (warp == 0) tmem_free(tmem, 256);
 }
 
+// D_t = dO_t . O_s,t alone (the linear branch dropped): one warp per token.
+template <int D>
+__global__ void __launch_bounds__(256) dvec_kernel(const __nv_bfloat16* __restrict__ d_o,
+                                                   const float* __restrict__ o_s,
+                                                   float* __restrict__ dvec, size_t ntok) {
+  const size_t tk = blockIdx.x * size_t(8) + threadIdx.x / 32;
+  if (tk >= ntok) return;
+  const int lane = int(lane_id());
+  float acc = 0.f;
+#pragma unroll
+  for (int c = lane * 2; c < D; c += 64) {
+    const float2 o2 = __ldg(reinterpret_cast<const float2*>(o_s + tk * D + c));
+    const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(d_o + tk * D + c);
+    acc = fmaf(__low2float(g2), o2.x, fmaf(__high2float(g2), o2.y, acc));
+  }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if (lane == 0) dvec[tk] = acc;
+}
+
 }  // namespace
+
+cudaError_t launch_dvec(const Problem& p, const void* d_o, const float* o_s, float* dvec,
+                        cudaStream_t s) {
+  const size_t ntok = size_t(p.BH) * p.N;
+  const unsigned grid = unsigned((ntok + 7) / 8);
+  if (p.d == 128)
+    dvec_kernel<128><<<grid, 256, 0, s>>>((const __nv_bfloat16*)d_o, o_s, dvec, ntok);
+  else
+    dvec_kernel<64><<<grid, 256, 0, s>>>((const __nv_bfloat16*)d_o, o_s, dvec, ntok);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_q(const Problem& p, const void* q, const void* d_o, const void* w_proj,
                          const float* o_s, const float* den, const __nv_bfloat16* hz_hi,
                          const __nv_bfloat16* hz_lo, float* dvec, float* dq,
-                         __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* dw, int num_sms,
-                         int* err, cudaStream_t s) {
+                         __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* dw, float gate,
+                         float* d_gate, int num_sms, int* err, cudaStream_t s) {
+  const float slope = gate * (1.0f - gate);
   CUtensorMap th, tl, tdo;
   if (!make_tmap_summary(&th, hz_hi, p.BH * p.T, p.d)) return cudaErrorInvalidValue;
   if (!make_tmap_summary(&tl, hz_lo, p.BH * p.T, p.d)) return cudaErrorInvalidValue;
@@ -605,15 +646,15 @@ cudaError_t launch_bwd_q(const Problem& p, const void* q, const void* d_o, const
     if (e != cudaSuccess) return e;
     bwd_q_kernel<128><<<grid, 256, kBqSmem, s>>>(
         th, tl, tdo, (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o,
-        (const __nv_bfloat16*)w_proj, o_s, den, hz_hi, hz_lo, dvec, dq, summ_hi, summ_lo, dw, p.N,
-        p.T, nblk, err);
+        (const __nv_bfloat16*)w_proj, o_s, den, hz_hi, hz_lo, dvec, dq, summ_hi, summ_lo, dw, gate,
+        slope, d_gate, p.N, p.T, nblk, err);
   } else {
     e = cudaFuncSetAttribute(bwd_q_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBqSmem);
     if (e != cudaSuccess) return e;
     bwd_q_kernel<64><<<grid, 256, kBqSmem, s>>>(
         th, tl, tdo, (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o,
-        (const __nv_bfloat16*)w_proj, o_s, den, hz_hi, hz_lo, dvec, dq, summ_hi, summ_lo, dw, p.N,
-        p.T, nblk, err);
+        (const __nv_bfloat16*)w_proj, o_s, den, hz_hi, hz_lo, dvec, dq, summ_hi, summ_lo, dw, gate,
+        slope, d_gate, p.N, p.T, nblk, err);
   }
   return cudaGetLastError();
 }

@@ -13,7 +13,8 @@
 //   den_t = phi(Q_t) . Z_i      (fp32, from the exact phi values at load time)
 //   O_l^T = NUM^T / den         (bf16 hi + lo, an MN-major operand tile)
 //   O^T   = W^T O_l^T           (A = W^T held in TMEM; W_proj is exact in bf16)
-//   O     = O_s + O             (bf16 out; den saved for the backward)
+//   O     = O_s + g O           (bf16 out; den saved for the backward; g = 1
+//                                  unless the branch is gated)
 // Persistent: two CTAs per SM (96 KB shared memory, 256 TMEM columns each)
 // walk the blocks; W^T goes to TMEM once per CTA, and the next block's H tile
 // is requested as soon as NUM^T has consumed the current one, so the copy
@@ -38,7 +39,7 @@ __global__ void __launch_bounds__(128) fwd_linear_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ hz_hi,
     const __nv_bfloat16* __restrict__ hz_lo, const __nv_bfloat16* __restrict__ w_proj,
     const float* __restrict__ o_s, __nv_bfloat16* __restrict__ o, float* __restrict__ den_out,
-    int N, int T, int nblk, int* err) {
+    float gate, int N, int T, int nblk, int* err) {
   constexpr int W = D * D + D;
   constexpr int kU = D / 8;               // 16-byte units per token row
   constexpr int kRowsPerPass = 128 / kU;  // token rows covered by one pass of 128 threads
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(128) fwd_linear_kernel(
         if (ok) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            o[(tok0 + t0 + j) * D + t] = __float2bfloat16_rn(os[j] + v[j]);
+            o[(tok0 + t0 + j) * D + t] = __float2bfloat16_rn(fmaf(gate, v[j], os[j]));
         }
       }
     }
@@ -257,11 +258,31 @@ __global__ void __launch_bounds__(128) fwd_linear_kernel(
   __syncthreads();
   if (warp == 0) tmem_free(tmem, 256);
 }
+// O = bf16(O_s): the forward's output when the linear branch is dropped.
+__global__ void __launch_bounds__(256) os_to_o_kernel(const float4* __restrict__ o_s,
+                                                      uint2* __restrict__ o, size_t n4) {
+  for (size_t e = blockIdx.x * size_t(256) + threadIdx.x; e < n4; e += size_t(gridDim.x) * 256) {
+    const float4 x = __ldg(o_s + e);
+    o[e] = make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_os_to_o(const Problem& p, const float* o_s, void* o, cudaStream_t s) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorInvalidValue;
+  const size_t n4 = size_t(p.BH) * p.N * p.d / 4;
+  os_to_o_kernel<<<4 * sms, 256, 0, s>>>(reinterpret_cast<const float4*>(o_s),
+                                         reinterpret_cast<uint2*>(o), n4);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_fwd_linear(const Problem& p, const void* q, const __nv_bfloat16* hz_hi,
                               const __nv_bfloat16* hz_lo, const void* w_proj, const float* o_s,
-                              void* o, float* den, int* err, cudaStream_t s) {
+                              void* o, float* den, float gate, int* err, cudaStream_t s) {
   CUtensorMap th, tl;
   if (!make_tmap_summary(&th, hz_hi, p.BH * p.T, p.d)) return cudaErrorInvalidValue;
   if (!make_tmap_summary(&tl, hz_lo, p.BH * p.T, p.d)) return cudaErrorInvalidValue;
@@ -278,14 +299,14 @@ cudaError_t launch_fwd_linear(const Problem& p, const void* q, const __nv_bfloat
     if (e != cudaSuccess) return e;
     fwd_linear_kernel<128><<<grid, 128, kFlSmem, s>>>(
         th, tl, (const __nv_bfloat16*)q, hz_hi, hz_lo, (const __nv_bfloat16*)w_proj, o_s,
-        (__nv_bfloat16*)o, den, p.N, p.T, nblk, err);
+        (__nv_bfloat16*)o, den, gate, p.N, p.T, nblk, err);
   } else {
     e = cudaFuncSetAttribute(fwd_linear_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kFlSmem);
     if (e != cudaSuccess) return e;
     fwd_linear_kernel<64><<<grid, 128, kFlSmem, s>>>(
         th, tl, (const __nv_bfloat16*)q, hz_hi, hz_lo, (const __nv_bfloat16*)w_proj, o_s,
-        (__nv_bfloat16*)o, den, p.N, p.T, nblk, err);
+        (__nv_bfloat16*)o, den, gate, p.N, p.T, nblk, err);
   }
   return cudaGetLastError();
 }

@@ -70,12 +70,15 @@ cudaError_t launch_fwd_sparse(const Problem& p, const void* q, const void* k, co
                               cudaStream_t s);
 cudaError_t launch_fwd_linear(const Problem& p, const void* q, const __nv_bfloat16* hz_hi,
                               const __nv_bfloat16* hz_lo, const void* w_proj, const float* o_s,
-                              void* o, float* den, int* err, cudaStream_t s);
+                              void* o, float* den, float gate, int* err, cudaStream_t s);
+cudaError_t launch_os_to_o(const Problem& p, const float* o_s, void* o, cudaStream_t s);
+cudaError_t launch_dvec(const Problem& p, const void* d_o, const float* o_s, float* dvec,
+                        cudaStream_t s);
 cudaError_t launch_bwd_q(const Problem& p, const void* q, const void* d_o, const void* w_proj,
                          const float* o_s, const float* den, const __nv_bfloat16* hz_hi,
                          const __nv_bfloat16* hz_lo, float* dvec, float* dq,
-                         __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* dw, int num_sms,
-                         int* err, cudaStream_t s);
+                         __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* dw, float gate,
+                         float* d_gate, int num_sms, int* err, cudaStream_t s);
 cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
                               const void* d_o, const float* lse, const float* dvec,
                               const int32_t* col_ptr, const int32_t* col_idx, float* dq,

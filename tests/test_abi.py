@@ -111,3 +111,28 @@ def test_entry_points_reject_bad_arguments_without_launching(L):
     sh2 = slab.make_shape(1, 2, 1024, 96, 64, 0.25, 0.25)
     assert L.sla_classify(ctypes.byref(sh2), good, good, ctypes.byref(mg), good, 1 << 40,
                           None) == 2
+
+
+def test_gated_entry_points_reject_bad_gates_without_launching(L):
+    sh = slab.make_shape(1, 2, 1024, 64, 64, 0.25, 0.25)
+    shp = ctypes.byref(sh)
+    good = 0x7f0000000000  # aligned, never dereferenced: every check fails first
+    m = slab.MaskStruct(good, good, good, good, good, None)
+    sv = slab.SavedStruct(good, good, good, good)
+    ok_gate = slab.Gate(0.5, 0.1)
+    nan_gate = slab.Gate(float("nan"), 0.1)
+    nan_skip = slab.Gate(0.5, float("nan"))
+    fwd = lambda gate: L.sla_forward_gated(shp, good, good, good, good, ctypes.byref(m), gate,
+                                           good, ctypes.byref(sv), good, 16, None)
+    assert fwd(None) == 1
+    assert fwd(ctypes.byref(nan_gate)) == 1
+    assert fwd(ctypes.byref(nan_skip)) == 1
+    assert fwd(ctypes.byref(ok_gate)) == 3  # valid gate: the small workspace is reported
+    bwd = lambda gate, d_logit: L.sla_backward_gated(
+        shp, good, good, good, good, ctypes.byref(m), gate, ctypes.byref(sv), good, good, good,
+        good, good, d_logit, good, 16, None)
+    assert bwd(ctypes.byref(ok_gate), None) == 1
+    assert bwd(ctypes.byref(ok_gate), good + 2) == 1  # d_logit must be 4-byte aligned
+    assert bwd(None, good) == 1
+    assert bwd(ctypes.byref(nan_gate), good) == 1
+    assert bwd(ctypes.byref(ok_gate), good) == 3

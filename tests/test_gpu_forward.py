@@ -133,7 +133,7 @@ def _forward_and_compare(wl, sample_blocks=None):
     if sample_blocks is not None:
         rows = np.concatenate([np.arange(i * 64, (i + 1) * 64) for i in sample_blocks])
         o, o_s, lse, den = o[:, :, rows], o_s[:, :, rows], lse[:, :, rows], den[:, :, rows]
-        ref = {k: v[:, :, rows] for k, v in ref.items()}
+        ref = {k: v[:, :, rows] for k, v in ref.items() if isinstance(v, np.ndarray)}
     res = {"o": assert_close(o, ref["o"], "o"),
            "o_s": assert_close(o_s, ref["o_s"], "o_s", 1e-2, 2e-3)}
     fin = np.isfinite(ref["lse"])
