@@ -29,6 +29,12 @@ map, the combination and the backward math; this oracle takes these readings
       sum_{u in j} phi(K_u); no epsilon; 0 when row i has no marginal block.
 * R7  O = O_s + O_l W_proj, W_proj one d x d matrix for all heads.
 * R8  gradients treat the classification as a constant.
+* R13 optional key padding (valid length n_valid, only the last block may be
+      partial): tokens t >= n_valid do not exist for the method.  Block means,
+      softmax keys and key-block summaries use valid tokens only; padded query
+      rows output O = O_s = O_l = 0, LSE = -inf, den = 0; their dO is ignored
+      and every padded position gets zero gradient.  Without n_valid, padding
+      tokens are ordinary tokens.
 * R12 optional gate on the linear branch, after the page "SALAD: Achieve
       High-Sparsity Attention via Efficient Linear Attention Tuning for Video
       Diffusion Transformer", section "Methodologie: SALAD", items 2 (a global
@@ -73,17 +79,31 @@ def block_counts(T: int, k_h: float, k_l: float) -> tuple[int, int]:
     return n_h, n_l
 
 
-def pool(x: np.ndarray, block: int) -> np.ndarray:
-    """Mean of each block of ``block`` consecutive tokens: [B,H,N,d] -> [B,H,T,d]."""
+def _n_valid(N: int, block: int, n_valid) -> int:
+    """Checked valid length (reading R13): N when not given."""
+    if n_valid is None:
+        return N
+    n_valid = int(n_valid)
+    if not (N - block < n_valid <= N):
+        raise ValueError("n_valid must leave only the last block partially padded")
+    return n_valid
+
+
+def pool(x: np.ndarray, block: int, n_valid=None) -> np.ndarray:
+    """Mean of each block's valid tokens (R1, R13): [B,H,N,d] -> [B,H,T,d]."""
     B, H, N, d = x.shape
     if N % block:
         raise ValueError("N must be a multiple of the block size")
-    return x.astype(np.float64).reshape(B, H, N // block, block, d).mean(axis=3)
+    nv = _n_valid(N, block, n_valid)
+    w = (np.arange(N) < nv).astype(np.float64).reshape(N // block, block)
+    xb = x.astype(np.float64).reshape(B, H, N // block, block, d)
+    return np.einsum("bhtud,tu->bhtd", xb, w) / w.sum(axis=1)[:, None]
 
 
-def pooled_logits(q: np.ndarray, k: np.ndarray, block: int, scale: float) -> np.ndarray:
+def pooled_logits(q: np.ndarray, k: np.ndarray, block: int, scale: float,
+                  n_valid=None) -> np.ndarray:
     """s_ij = mean(Q_i) . mean(K_j) * scale, [B,H,T,T] (reading R1)."""
-    qb, kb = pool(q, block), pool(k, block)
+    qb, kb = pool(q, block, n_valid), pool(k, block, n_valid)
     return np.einsum("bhid,bhjd->bhij", qb, kb) * scale
 
 
@@ -134,16 +154,19 @@ def phi_prime(x: np.ndarray) -> np.ndarray:
     return np.where(x > 0, 1.0, np.exp(np.minimum(x, 0.0)))
 
 
-def key_block_summaries(k: np.ndarray, v: np.ndarray, block: int):
-    """Per key block j: h_j = phi(K_j)^T V_j [d,d] and z_j = sum_u phi(K_u) [d].
+def key_block_summaries(k: np.ndarray, v: np.ndarray, block: int, n_valid=None):
+    """Per key block j: h_j = phi(K_j)^T V_j [d,d] and z_j = sum_u phi(K_u) [d]
+    over the block's valid tokens u.
 
     These are the per-key-block summaries through which marginal pairs get
     O(N) linear attention (SLA abstract; framework step 3).
     """
     B, H, N, d = k.shape
     T = N // block
-    fk = phi(k).reshape(B, H, T, block, d)
-    vb = v.astype(np.float64).reshape(B, H, T, block, d)
+    nv = _n_valid(N, block, n_valid)
+    valid = (np.arange(N) < nv).astype(np.float64)[:, None]
+    fk = (phi(k) * valid).reshape(B, H, T, block, d)
+    vb = (v.astype(np.float64) * valid).reshape(B, H, T, block, d)
     h = np.einsum("bhtua,bhtuc->bhtac", fk, vb)
     z = fk.sum(axis=3)
     return h, z
@@ -166,14 +189,15 @@ def _tokens(blocks: np.ndarray, block: int) -> np.ndarray:
 
 
 def forward(q, k, v, w_proj, cls, block: int, scale: float | None = None,
-            query_blocks=None, gate=None):
+            query_blocks=None, gate=None, n_valid=None):
     """SLA forward with a given class map ``cls`` [B,H,T,T].
 
     Returns a dict with o, o_s, o_l [B,H,N,d], lse and den [B,H,N] (fp64),
     and the gate factor g.  ``query_blocks``, if given, restricts the work to
     those query-block indices (other rows stay zero / -inf); used to sample
     large problems.  ``gate`` = (gamma, tau) gates the linear branch (R12); a
-    dropped branch leaves o_l and den zero.
+    dropped branch leaves o_l and den zero.  ``n_valid`` masks the padding
+    tokens (R13).
     """
     g, dropped = gate_factor(gate)
     B, H, N, d = q.shape
@@ -182,7 +206,8 @@ def forward(q, k, v, w_proj, cls, block: int, scale: float | None = None,
         scale = 1.0 / math.sqrt(d)
     q64, k64, v64 = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
     w64 = np.asarray(w_proj, dtype=np.float64)
-    h, z = key_block_summaries(k64, v64, block)
+    nv = _n_valid(N, block, n_valid)
+    h, z = key_block_summaries(k64, v64, block, nv)
     o_s = np.zeros((B, H, N, d))
     o_l = np.zeros((B, H, N, d))
     lse = np.full((B, H, N), -np.inf)
@@ -196,13 +221,14 @@ def forward(q, k, v, w_proj, cls, block: int, scale: float | None = None,
             H_all = np.tensordot(marg_ind, h[b, hh], axes=(1, 0))
             Z_all = marg_ind @ z[b, hh]
             for i in rows:
-                t0, t1 = i * block, (i + 1) * block
+                t0, t1 = i * block, min((i + 1) * block, nv)  # valid query rows
                 qi = q64[b, hh, t0:t1]
                 crit = np.nonzero(cls[b, hh, i] == 1)[0]
                 marg = np.nonzero(cls[b, hh, i] == 0)[0]
-                # critical pairs: exact softmax attention over all their key tokens
+                # critical pairs: exact softmax attention over all their valid key tokens
                 if crit.size:
                     keys = _tokens(crit, block)
+                    keys = keys[keys < nv]
                     s = (qi @ k64[b, hh, keys].T) * scale
                     m = s.max(axis=1, keepdims=True)
                     e = np.exp(s - m)
@@ -222,15 +248,18 @@ def forward(q, k, v, w_proj, cls, block: int, scale: float | None = None,
     return {"o": o, "o_s": o_s, "o_l": o_l, "lse": lse, "den": den, "g": g}
 
 
-def forward_bruteforce(q, k, v, w_proj, cls, block: int, scale: float | None = None):
+def forward_bruteforce(q, k, v, w_proj, cls, block: int, scale: float | None = None,
+                       n_valid=None):
     """Per-token loops over every key with the class looked up per key.
 
     The linear branch is written per key token,
     O_l,t = sum_u (phi(Q_t).phi(K_u)) V_u / sum_u phi(Q_t).phi(K_u),
     u over marginal tokens, so agreement with ``forward`` pins the summary
-    reassociation.  Meant for N <= 256.
+    reassociation.  Meant for N <= 256.  With ``n_valid`` (R13) keys and
+    queries at t >= n_valid are skipped (padded rows stay 0).
     """
     B, H, N, d = q.shape
+    nv = N if n_valid is None else int(n_valid)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     q64, k64, v64 = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
@@ -238,13 +267,13 @@ def forward_bruteforce(q, k, v, w_proj, cls, block: int, scale: float | None = N
     o = np.zeros((B, H, N, d))
     for b in range(B):
         for hh in range(H):
-            for t in range(N):
+            for t in range(nv):
                 i = t // block
                 crit_w, crit_v = [], []
                 lin_num = np.zeros(d)
                 lin_den = 0.0
                 fq = phi(q64[b, hh, t])
-                for u in range(N):
+                for u in range(nv):
                     c = cls[b, hh, i, u // block]
                     if c == 1:
                         crit_w.append(float(q64[b, hh, t] @ k64[b, hh, u]) * scale)
@@ -268,7 +297,7 @@ def forward_bruteforce(q, k, v, w_proj, cls, block: int, scale: float | None = N
 
 
 def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
-             fwd=None, gate=None):
+             fwd=None, gate=None, n_valid=None):
     """Gradients of sum(O * dO) w.r.t. Q, K, V and W_proj, classes held fixed (R8).
 
     Sparse branch (standard softmax-attention backward over critical pairs):
@@ -287,17 +316,20 @@ def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
     downstream of them carry the factor g, and
       d gamma = g (1 - g) sum over b, h, t of (O_l,t W) . dO_t;
     a dropped branch contributes nothing and d gamma = 0.
+    Key padding (R13): dO of padded rows is ignored, padded positions get 0.
     """
     g, dropped = gate_factor(gate)
     B, H, N, d = q.shape
     T = N // block
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    nv = _n_valid(N, block, n_valid)
     if fwd is None:
-        fwd = forward(q, k, v, w_proj, cls, block, scale, gate=gate)
+        fwd = forward(q, k, v, w_proj, cls, block, scale, gate=gate, n_valid=nv)
     q64, k64, v64, do64 = (np.asarray(a, dtype=np.float64) for a in (q, k, v, d_o))
+    do64 = do64 * (np.arange(N) < nv)[:, None]  # padded rows carry no gradient
     w64 = np.asarray(w_proj, dtype=np.float64)
-    h, z = key_block_summaries(k64, v64, block)
+    h, z = key_block_summaries(k64, v64, block, nv)
     dq = np.zeros_like(q64)
     dk = np.zeros_like(k64)
     dv = np.zeros_like(v64)
@@ -313,13 +345,14 @@ def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
             dH_all = np.zeros((T, d, d))  # dL/dH_i per query block
             dZ_all = np.zeros((T, d))
             for i in range(T):
-                t0, t1 = i * block, (i + 1) * block
+                t0, t1 = i * block, min((i + 1) * block, nv)  # valid query rows
                 qi = q64[b, hh, t0:t1]
                 doi = do64[b, hh, t0:t1]
                 crit = np.nonzero(cls[b, hh, i] == 1)[0]
                 marg = np.nonzero(cls[b, hh, i] == 0)[0]
                 if crit.size:
                     keys = _tokens(crit, block)
+                    keys = keys[keys < nv]
                     kc, vc = k64[b, hh, keys], v64[b, hh, keys]
                     s = (qi @ kc.T) * scale
                     p = np.exp(s - fwd["lse"][b, hh, t0:t1, None])
@@ -344,7 +377,7 @@ def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
             dh = np.tensordot(marg_ind.T, dH_all, axes=(1, 0))
             dz = marg_ind.T @ dZ_all
             for j in range(T):
-                u0, u1 = j * block, (j + 1) * block
+                u0, u1 = j * block, min((j + 1) * block, nv)  # valid key rows
                 kj, vj = k64[b, hh, u0:u1], v64[b, hh, u0:u1]
                 dfk = vj @ dh[j].T + dz[j][None, :]
                 dk[b, hh, u0:u1] += dfk * phi_prime(kj)
@@ -352,15 +385,16 @@ def backward(q, k, v, w_proj, cls, d_o, block: int, scale: float | None = None,
     return {"dq": dq, "dk": dk, "dv": dv, "dw": dw, "d_gamma": d_gamma}
 
 
-def sla(q, k, v, w_proj, block: int, k_h: float, k_l: float, scale: float | None = None):
+def sla(q, k, v, w_proj, block: int, k_h: float, k_l: float, scale: float | None = None,
+        n_valid=None):
     """Classification from the inputs followed by the forward."""
     d = q.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     T = q.shape[2] // block
     n_h, n_l = block_counts(T, k_h, k_l)
-    logits = pooled_logits(q, k, block, scale)
+    logits = pooled_logits(q, k, block, scale, n_valid)
     cls = classify(logits, n_h, n_l)
-    out = forward(q, k, v, w_proj, cls, block, scale)
+    out = forward(q, k, v, w_proj, cls, block, scale, n_valid=n_valid)
     out.update(cls=cls, logits=logits)
     return out

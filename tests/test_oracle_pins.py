@@ -379,3 +379,93 @@ def test_gate_gradient_matches_central_difference(gamma):
             lp = np.sum(oracle.forward(argp["q"], k, v, argp["w"], cls, 16, gate=(gamma, 0.0))["o"] * do)
             lm = np.sum(oracle.forward(argm["q"], k, v, argm["w"], cls, 16, gate=(gamma, 0.0))["o"] * do)
             assert math.isclose((lp - lm) / 2e-6, grad[idx], rel_tol=2e-6, abs_tol=2e-8)
+
+
+# ---------------------------------------------------------------- key padding (R13)
+
+def test_pool_with_padding_is_mean_of_valid_tokens():
+    x = _rand((1, 2, 128, 4), 60)
+    got = oracle.pool(x, 32, n_valid=101)
+    np.testing.assert_allclose(got[:, :, :3], x.reshape(1, 2, 4, 32, 4)[:, :, :3].mean(axis=3),
+                               rtol=1e-14)
+    np.testing.assert_allclose(got[:, :, 3], x[:, :, 96:101].mean(axis=2), rtol=1e-14)
+    with pytest.raises(ValueError):
+        oracle.pool(x, 32, n_valid=96)  # a whole block of padding
+
+
+def test_padding_at_full_length_is_unpadded():
+    q, k, v, w = _small(N=256, d=16, seed=61)
+    cls = _cls_from(q, k, 32, 0.25, 0.25)
+    do = np.random.default_rng(62).standard_normal(q.shape)
+    a = oracle.forward(q, k, v, w, cls, 32)
+    b = oracle.forward(q, k, v, w, cls, 32, n_valid=256)
+    for n in ("o", "o_s", "o_l", "lse", "den"):
+        assert np.array_equal(a[n], b[n]), n
+    ga = oracle.backward(q, k, v, w, cls, do, 32)
+    gb = oracle.backward(q, k, v, w, cls, do, 32, n_valid=256)
+    for n in ("dq", "dk", "dv", "dw"):
+        assert np.array_equal(ga[n], gb[n]), n
+
+
+def test_padded_tokens_do_not_matter():
+    # two different fillings of the padding: identical outputs and gradients,
+    # zero at the padded positions
+    nv = 229
+    q, k, v, w = _small(N=256, d=16, seed=63)
+    do = np.random.default_rng(64).standard_normal(q.shape)
+    q2, k2, v2, do2 = (a.copy() for a in (q, k, v, do))
+    rng = np.random.default_rng(65)
+    for a in (q2, k2, v2, do2):
+        a[:, :, nv:] = rng.standard_normal(a[:, :, nv:].shape) * 7.0
+    n_h, n_l = oracle.block_counts(8, 0.25, 0.25)
+    cls = oracle.classify(oracle.pooled_logits(q, k, 32, 0.25, nv), n_h, n_l)
+    cls2 = oracle.classify(oracle.pooled_logits(q2, k2, 32, 0.25, nv), n_h, n_l)
+    assert np.array_equal(cls, cls2)
+    f1 = oracle.forward(q, k, v, w, cls, 32, n_valid=nv)
+    f2 = oracle.forward(q2, k2, v2, w, cls, 32, n_valid=nv)
+    for n in ("o", "o_s", "o_l", "lse", "den"):
+        assert np.array_equal(f1[n], f2[n]), n
+    assert np.all(f1["o"][:, :, nv:] == 0) and np.all(np.isneginf(f1["lse"][:, :, nv:]))
+    g1 = oracle.backward(q, k, v, w, cls, do, 32, n_valid=nv)
+    g2 = oracle.backward(q2, k2, v2, w, cls, do2, 32, n_valid=nv)
+    for n in ("dq", "dk", "dv", "dw"):
+        assert np.array_equal(g1[n], g2[n]), n
+    for n in ("dq", "dk", "dv"):
+        assert np.all(g1[n][:, :, nv:] == 0), n
+
+
+@pytest.mark.parametrize("nv", [113, 127])
+def test_padded_blockwise_equals_bruteforce(nv):
+    q, k, v, w = _small(B=1, H=2, N=128, d=8, seed=66)
+    cls = oracle.classify(oracle.pooled_logits(q, k, 16, 0.3, nv), *oracle.block_counts(8, 0.25, 0.25))
+    got = oracle.forward(q, k, v, w, cls, 16, 0.3, n_valid=nv)["o"]
+    ref = oracle.forward_bruteforce(q, k, v, w, cls, 16, 0.3, n_valid=nv)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_padded_backward_matches_central_differences():
+    nv = 247
+    q, k, v, w = _small(B=1, H=1, N=256, d=8, seed=67)
+    do = np.random.default_rng(68).standard_normal(q.shape)
+    cls = oracle.classify(oracle.pooled_logits(q, k, 16, 1 / math.sqrt(8), nv),
+                          *oracle.block_counts(16, 0.25, 0.25))
+    g = oracle.backward(q, k, v, w, cls, do, 16, n_valid=nv)
+
+    def loss(qq, kk, vv, ww):
+        o = oracle.forward(qq, kk, vv, ww, cls, 16, n_valid=nv)["o"]
+        return float(np.sum(o[:, :, :nv] * do[:, :, :nv]))
+
+    rng = np.random.default_rng(69)
+    for name in ("q", "k", "v", "w"):
+        arr = {"q": q, "k": k, "v": v, "w": w}[name]
+        grad = g["d" + name]
+        for _ in range(8):
+            idx = tuple(rng.integers(0, s) for s in arr.shape)
+            xp, xm = arr.copy(), arr.copy()
+            xp[idx] += 1e-6
+            xm[idx] -= 1e-6
+            a = {"q": q, "k": k, "v": v, "w": w}
+            bp, bm = dict(a), dict(a)
+            bp[name], bm[name] = xp, xm
+            fd = (loss(bp["q"], bp["k"], bp["v"], bp["w"]) - loss(bm["q"], bm["k"], bm["v"], bm["w"])) / 2e-6
+            assert math.isclose(fd, grad[idx], rel_tol=2e-6, abs_tol=2e-8), (name, idx, fd, grad[idx])
