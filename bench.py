@@ -223,6 +223,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gate-logit", type=float, default=None,
                     help="run the gated entry points with this gate logit (default: ungated)")
+    ap.add_argument("--key-padding", action="store_true",
+                    help="mask the grid's padding tokens (n_valid) instead of treating them as tokens")
     ap.add_argument("--gate-skip", type=float, default=0.0,
                     help="drop the linear branch when sigmoid(logit) is below this")
     args = ap.parse_args()
@@ -249,7 +251,8 @@ def main():
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     wl = sla_inputs.make("train", seed=rank)
-    shape = slab.make_shape(wl.B, wl.H, wl.N, wl.d, wl.block, wl.k_h, wl.k_l)
+    shape = slab.make_shape(wl.B, wl.H, wl.N, wl.d, wl.block, wl.k_h, wl.k_l,
+                            n_valid=wl.n_valid if args.key_padding else 0)
     buf = slab.Buffers.allocate(shape, device=dev, with_logits=False)
     n_crit = buf.sizes.n_crit
     to_dev = lambda a: torch.from_numpy(a).to(torch.bfloat16).to(dev)
@@ -409,6 +412,8 @@ def main():
         return
     peak_t = pk["bf16_tflops_sustained"]
     cfg = workload_config(wl, n_crit)
+    if args.key_padding:
+        cfg["n_valid"] = wl.n_valid
     if gate is not None:
         g = 1.0 / (1.0 + math.exp(-args.gate_logit))
         cfg["gate"] = {"logit": args.gate_logit, "skip_below": args.gate_skip, "g": g,

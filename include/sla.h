@@ -66,11 +66,20 @@ typedef enum {
   SLA_ERR_DEVICE = 6       /* a device-side invariant failed (reported by sla_check) */
 } sla_status;
 
-/* Problem shape.  softmax_scale <= 0 selects 1/sqrt(d). */
+/* Problem shape.  softmax_scale <= 0 selects 1/sqrt(d).
+ * n_valid: valid tokens per sequence (key padding); 0 means N.  Otherwise
+ * N - block < n_valid <= N (only the last block may be partial).  Tokens at
+ * t >= n_valid take no part: block means, softmax keys and key-block
+ * summaries use valid tokens only; padded rows of o, o_s, den are 0 and of lse
+ * +inf (exp(s - lse) = 0 for every key; -inf marks a real row without a
+ * critical block); d_o at padded rows is ignored; dq, dk, dv there are 0.  With
+ * n_valid = 0 padding tokens are ordinary tokens (the pages do not say how a
+ * grid is padded to whole blocks; this is the optional exact handling). */
 typedef struct {
   int B, H, N, d, block;
   double k_h, k_l;
   float softmax_scale;
+  int n_valid;
 } sla_shape;
 
 /* Classification output (written by sla_classify*, read by forward/backward;
@@ -91,7 +100,8 @@ typedef struct {
 } sla_mask;
 
 /* State saved by sla_forward for sla_backward.
- *   lse   fp32 [B,H,N]      log-sum-exp of the critical scores (-inf if none)
+ *   lse   fp32 [B,H,N]      log-sum-exp of the critical scores (-inf if none,
+ *                           +inf on a padded row, see sla_shape.n_valid)
  *   o_s   fp32 [B,H,N,d]    sparse-branch output
  *   den   fp32 [B,H,N]      phi(Q).Z_i (0 if the row has no marginal block)
  *   hz_agg bf16 [2][B,H,T,d*d+d]  per query block: H_i (d x d, row-major) then

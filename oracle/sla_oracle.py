@@ -32,8 +32,10 @@ map, the combination and the backward math; this oracle takes these readings
 * R13 optional key padding (valid length n_valid, only the last block may be
       partial): tokens t >= n_valid do not exist for the method.  Block means,
       softmax keys and key-block summaries use valid tokens only; padded query
-      rows output O = O_s = O_l = 0, LSE = -inf, den = 0; their dO is ignored
-      and every padded position gets zero gradient.  Without n_valid, padding
+      rows output O = O_s = O_l = 0 and den = 0, and LSE = +inf (no token, so
+      exp(s - LSE) = 0 for every key; -inf stays the mark of a real row with no
+      critical block); their dO is ignored and every padded position gets zero
+      gradient.  Without n_valid, padding
       tokens are ordinary tokens.
 * R12 optional gate on the linear branch, after the page "SALAD: Achieve
       High-Sparsity Attention via Efficient Linear Attention Tuning for Video
@@ -244,6 +246,7 @@ def forward(q, k, v, w_proj, cls, block: int, scale: float | None = None,
                     o_l[b, hh, t0:t1] = num / dn[:, None]
                     den[b, hh, t0:t1] = dn
                 # negligible pairs contribute nothing
+    lse[:, :, nv:] = np.inf  # padded rows (R13)
     o = o_s + g * np.einsum("bhta,ac->bhtc", o_l, w64)
     return {"o": o, "o_s": o_s, "o_l": o_l, "lse": lse, "den": den, "g": g}
 

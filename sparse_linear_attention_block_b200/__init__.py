@@ -47,7 +47,8 @@ class SlaError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
                 ("d", ctypes.c_int), ("block", ctypes.c_int), ("k_h", ctypes.c_double),
-                ("k_l", ctypes.c_double), ("softmax_scale", ctypes.c_float)]
+                ("k_l", ctypes.c_double), ("softmax_scale", ctypes.c_float),
+                ("n_valid", ctypes.c_int)]
 
 
 class MaskStruct(ctypes.Structure):
@@ -151,8 +152,9 @@ def _check(status: int, what: str):
         raise SlaError(status, what)
 
 
-def make_shape(B, H, N, d, block=64, k_h=0.05, k_l=0.10, softmax_scale=0.0) -> Shape:
-    return Shape(B, H, N, d, block, float(k_h), float(k_l), float(softmax_scale))
+def make_shape(B, H, N, d, block=64, k_h=0.05, k_l=0.10, softmax_scale=0.0,
+               n_valid=0) -> Shape:
+    return Shape(B, H, N, d, block, float(k_h), float(k_l), float(softmax_scale), int(n_valid))
 
 
 def sla_query_sizes(shape: Shape) -> Sizes:

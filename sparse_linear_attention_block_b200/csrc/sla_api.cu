@@ -119,6 +119,8 @@ sla_status check_shape(const sla_shape* s, Problem* p) {
     return SLA_ERR_INVALID_ARG;
   if (std::isnan(s->softmax_scale) || std::isinf(s->softmax_scale)) return SLA_ERR_INVALID_ARG;
   if (s->N % s->block != 0) return SLA_ERR_INVALID_ARG;
+  if (s->n_valid != 0 && (s->n_valid > s->N || s->n_valid <= s->N - s->block))
+    return SLA_ERR_INVALID_ARG;
   if (s->block != kBlock) return SLA_ERR_UNSUPPORTED;
   if (s->d != 64 && s->d != 128) return SLA_ERR_UNSUPPORTED;
   const long long bh = (long long)s->B * s->H;
@@ -133,6 +135,7 @@ sla_status check_shape(const sla_shape* s, Problem* p) {
     p->d = s->d;
     p->T = T;
     p->Tp = pad128(T);
+    p->nv = s->n_valid != 0 ? s->n_valid : s->N;
     counts(T, s->k_h, s->k_l, &p->n_crit, &p->n_negl);
     p->scale = s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / std::sqrt(float(s->d));
     p->scale_log2 = p->scale * 1.4426950408889634f;

@@ -413,7 +413,7 @@ __global__ void __launch_bounds__(128, 1) bwd_k_kernel(
     const __grid_constant__ CUtensorMap tm_dh, const __grid_constant__ CUtensorMap tm_dl,
     const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16* __restrict__ kin,
     const __nv_bfloat16* __restrict__ dh_hi, const __nv_bfloat16* __restrict__ dh_lo,
-    float* __restrict__ dk, float* __restrict__ dv, int N, int T, int nblk, int* err) {
+    float* __restrict__ dk, float* __restrict__ dv, int N, int T, int nv, int nblk, int* err) {
   constexpr int W = D * D + D;
   constexpr int kU = D / 8;
   constexpr int kRowsPerPass = 128 / kU;
@@ -506,11 +506,24 @@ __global__ void __launch_bounds__(128, 1) bwd_k_kernel(
       tmem_ld16(acc + 64 + q16, gv);
       tmem_ld_wait();
       if (write) {
+        // keys of this block that exist (key padding; all 16 except in a
+        // sequence's partial last block, where padded keys keep dK = dV = 0)
+        const int lim = nv - ((blk % T) * 64 + q16);
+        if (lim >= 16) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const size_t idx = (tk + q16 + j) * D + t;
-          dk[idx] = fmaf(gk[j] + dz, dphi_f(kk[j]), ck[j]);
-          dv[idx] = cv[j] + gv[j];
+          for (int j = 0; j < 16; ++j) {
+            const size_t idx = (tk + q16 + j) * D + t;
+            dk[idx] = fmaf(gk[j] + dz, dphi_f(kk[j]), ck[j]);
+            dv[idx] = cv[j] + gv[j];
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (j >= lim) break;
+            const size_t idx = (tk + q16 + j) * D + t;
+            dk[idx] = fmaf(gk[j] + dz, dphi_f(kk[j]), ck[j]);
+            dv[idx] = cv[j] + gv[j];
+          }
         }
       }
     }
@@ -673,12 +686,12 @@ cudaError_t launch_bwd_k(const Problem& p, const void* k, const void* v,
     e = cudaFuncSetAttribute(bwd_k_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBkSmem);
     if (e != cudaSuccess) return e;
     bwd_k_kernel<128><<<grid, 128, kBkSmem, s>>>(th, tl, tv, (const __nv_bfloat16*)k, dh_hi, dh_lo,
-                                                 dk, dv, p.N, p.T, nblk, err);
+                                                 dk, dv, p.N, p.T, p.nv, nblk, err);
   } else {
     e = cudaFuncSetAttribute(bwd_k_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBkSmem);
     if (e != cudaSuccess) return e;
     bwd_k_kernel<64><<<grid, 128, kBkSmem, s>>>(th, tl, tv, (const __nv_bfloat16*)k, dh_hi, dh_lo,
-                                                dk, dv, p.N, p.T, nblk, err);
+                                                dk, dv, p.N, p.T, p.nv, nblk, err);
   }
   return cudaGetLastError();
 }

@@ -23,7 +23,8 @@ template <int D>
 __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k,
                                                    float* __restrict__ qbar,
-                                                   float* __restrict__ kbar, int N, int T) {
+                                                   float* __restrict__ kbar, int N, int T,
+                                                   int nv) {
   constexpr int kChunks = D / 8;          // 16-byte chunks per row
   constexpr int kGroups = 128 / kChunks;  // row groups
   constexpr int kRowsPer = kBlock / kGroups;
@@ -31,6 +32,7 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
   const int j = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
   const int c8 = t % kChunks, g = t / kChunks;
   const size_t base = (size_t(bh) * N + size_t(j) * kBlock) * D;
+  const int valid = min(kBlock, nv - j * kBlock);  // tokens of this block that exist
 #pragma unroll
   for (int which = 0; which < 2; ++which) {
     const __nv_bfloat16* src = (which == 0 ? q : k) + base;
@@ -38,6 +40,7 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
 #pragma unroll
     for (int i = 0; i < kRowsPer; ++i) {
       const int row = g + i * kGroups;
+      if (row >= valid) continue;
       const uint4 u = *reinterpret_cast<const uint4*>(src + size_t(row) * D + c8 * 8);
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -56,7 +59,7 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
 #pragma unroll
     for (int gg = 0; gg < kGroups; ++gg) s += red[which][gg][col];
     float* dst = (which == 0 ? qbar : kbar) + (size_t(bh) * T + j) * D;
-    dst[col] = s * (1.0f / kBlock);
+    dst[col] = s / float(valid);
   }
 }
 
@@ -357,10 +360,10 @@ cudaError_t launch_pool(const Problem& p, const void* q, const void* k, float* q
   dim3 grid(p.T, p.BH);
   if (p.d == 128)
     pool_kernel<128><<<grid, 128, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                          qbar, kbar, p.N, p.T);
+                                          qbar, kbar, p.N, p.T, p.nv);
   else
     pool_kernel<64><<<grid, 128, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                         qbar, kbar, p.N, p.T);
+                                         qbar, kbar, p.N, p.T, p.nv);
   return cudaGetLastError();
 }
 

@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(128) fwd_linear_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ hz_hi,
     const __nv_bfloat16* __restrict__ hz_lo, const __nv_bfloat16* __restrict__ w_proj,
     const float* __restrict__ o_s, __nv_bfloat16* __restrict__ o, float* __restrict__ den_out,
-    float gate, int N, int T, int nblk, int* err) {
+    float gate, int N, int T, int nv, int nblk, int* err) {
   constexpr int W = D * D + D;
   constexpr int kU = D / 8;               // 16-byte units per token row
   constexpr int kRowsPerPass = 128 / kU;  // token rows covered by one pass of 128 threads
@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(128) fwd_linear_kernel(
   for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x, ++k) {
     const size_t tok0 = tok_of(blk);
     const int nxt = blk + int(gridDim.x);
+    const int vrows = nv - (blk % T) * 64;  // rows of this block that exist (key padding)
     // phi(Q) as hi/lo K-major tiles [64 t][a]; den_t = phi(Q_t) . Z_i in fp32,
     // each thread's 8 features summed, then over the kU threads of a row
 #pragma unroll
@@ -150,8 +151,10 @@ __global__ void __launch_bounds__(128) fwd_linear_kernel(
 #pragma unroll
       for (int m = kU / 2; m >= 1; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
       if (u == 0) {
-        sInv[rr] = part > 0.f ? 1.0f / part : 0.f;
-        den_out[tok0 + rr] = part;
+        // a padded query row (key padding) has no linear output: den = 0
+        const float dn = rr < vrows ? part : 0.f;
+        sInv[rr] = dn > 0.f ? 1.0f / dn : 0.f;
+        den_out[tok0 + rr] = dn;
       }
     }
     fence_proxy_async_smem();
@@ -299,14 +302,14 @@ cudaError_t launch_fwd_linear(const Problem& p, const void* q, const __nv_bfloat
     if (e != cudaSuccess) return e;
     fwd_linear_kernel<128><<<grid, 128, kFlSmem, s>>>(
         th, tl, (const __nv_bfloat16*)q, hz_hi, hz_lo, (const __nv_bfloat16*)w_proj, o_s,
-        (__nv_bfloat16*)o, den, gate, p.N, p.T, nblk, err);
+        (__nv_bfloat16*)o, den, gate, p.N, p.T, p.nv, nblk, err);
   } else {
     e = cudaFuncSetAttribute(fwd_linear_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kFlSmem);
     if (e != cudaSuccess) return e;
     fwd_linear_kernel<64><<<grid, 128, kFlSmem, s>>>(
         th, tl, (const __nv_bfloat16*)q, hz_hi, hz_lo, (const __nv_bfloat16*)w_proj, o_s,
-        (__nv_bfloat16*)o, den, gate, p.N, p.T, nblk, err);
+        (__nv_bfloat16*)o, den, gate, p.N, p.T, p.nv, nblk, err);
   }
   return cudaGetLastError();
 }

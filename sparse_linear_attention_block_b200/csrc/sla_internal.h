@@ -44,6 +44,7 @@ WorkspaceLayout workspace_layout(int BH, int N, int d);
 // Validated problem description handed to the launchers.
 struct Problem {
   int B, H, BH, N, d, T, Tp, n_crit, n_negl;
+  int nv;             // valid tokens per sequence (N unless key padding is on)
   float scale;        // softmax scale
   float scale_log2;   // scale * log2(e)
 };

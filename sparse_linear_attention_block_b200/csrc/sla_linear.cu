@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
                                                         const __nv_bfloat16* __restrict__ v,
                                                         __nv_bfloat16* __restrict__ summ_hi,
                                                         __nv_bfloat16* __restrict__ summ_lo,
-                                                        int N, int T, int* err) {
+                                                        int N, int T, int nv, int* err) {
   constexpr int kChunks = D / 8;
   constexpr int kGroups = 128 / kChunks;
   constexpr int kRowsPer = kBlock / kGroups;
@@ -67,6 +67,7 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
   }
   const int c8 = t % kChunks, g = t / kChunks;
   const size_t off = (size_t(bh) * N + size_t(j) * kBlock) * D;
+  const int valid = min(kBlock, nv - j * kBlock);  // keys of this block that exist
   uint4 uk[kRowsPer], uv[kRowsPer];
 #pragma unroll
   for (int i = 0; i < kRowsPer; ++i) {
@@ -75,14 +76,20 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
     uv[i] = __ldg(reinterpret_cast<const uint4*>(v + off + size_t(row) * D + c8 * 8));
   }
   float zacc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (valid < kBlock) {  // a sequence's partial last block: padded keys contribute nothing
+#pragma unroll
+    for (int i = 0; i < kRowsPer; ++i)
+      if (g + i * kGroups >= valid) uk[i] = uv[i] = make_uint4(0, 0, 0, 0);
+  }
 #pragma unroll
   for (int i = 0; i < kRowsPer; ++i) {
     const int row = g + i * kGroups;
+    const bool rv = valid == kBlock || row < valid;
     const uint32_t w[4] = {uk[i].x, uk[i].y, uk[i].z, uk[i].w};
     uint32_t ph[4], pl[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float a = phi_f(bf16_lo(w[e])), b = phi_f(bf16_hi(w[e]));
+      const float a = rv ? phi_f(bf16_lo(w[e])) : 0.f, b = rv ? phi_f(bf16_hi(w[e])) : 0.f;
       zacc[2 * e] += a;
       zacc[2 * e + 1] += b;
       split2(a, b, ph[e], pl[e]);
@@ -285,12 +292,12 @@ cudaError_t launch_summaries(const Problem& p, const void* k, const void* v,
     if ((e = set_smem(summaries_kernel<128>, smem)) != cudaSuccess) return e;
     summaries_kernel<128><<<grid, 128, smem, s>>>((const __nv_bfloat16*)k,
                                                   (const __nv_bfloat16*)v, summ_hi, summ_lo,
-                                                  p.N, p.T, err);
+                                                  p.N, p.T, p.nv, err);
   } else {
     if ((e = set_smem(summaries_kernel<64>, smem)) != cudaSuccess) return e;
     summaries_kernel<64><<<grid, 128, smem, s>>>((const __nv_bfloat16*)k,
                                                  (const __nv_bfloat16*)v, summ_hi, summ_lo, p.N,
-                                                 p.T, err);
+                                                 p.T, p.nv, err);
   }
   return cudaGetLastError();
 }

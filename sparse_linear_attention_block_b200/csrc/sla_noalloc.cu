@@ -85,6 +85,7 @@ extern "C" sla_status sla_classify_noalloc(const sla_shape* shape, const void* q
   p.d = shape->d;
   p.T = sz.T;
   p.Tp = pad128(sz.T);
+  p.nv = shape->n_valid != 0 ? shape->n_valid : shape->N;  // validated by sla_query_sizes
   p.n_crit = sz.n_crit;
   p.n_negl = sz.n_negl;
   p.scale = shape->softmax_scale > 0.f ? shape->softmax_scale : 1.0f / sqrtf(float(shape->d));

@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
     const float* __restrict__ lse, const float* __restrict__ dvec,
     const int32_t* __restrict__ col_ptr, const int32_t* __restrict__ col_idx, int N, int T,
-    int n_crit, float scale_log2, float scale, float* __restrict__ dq, float* __restrict__ dk,
+    int n_crit, int nv, float scale_log2, float scale, float* __restrict__ dq, float* __restrict__ dk,
     float* __restrict__ dv, int* err) {
   using L = SbSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -238,7 +238,9 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
     const int wg = warp >> 2, wq = warp & 3;
     const int r = wq * 32 + lane;  // key row == TMEM lane
     const int half = r >> 6;
-    const bool key_ok = (half == 0) || has1;
+    const bool key_ok = (half == 0) || has1;  // the key block exists
+    // a padded key (key padding) gets no weight; its dK, dV rows stay 0
+    const bool key_valid = key_ok && qp * 128 + r < nv;
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
     uint8_t* ds_tile = sDS + wg * L::kDS;
     bool ok = true;
@@ -259,7 +261,8 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
       const int i = ulist[n];
       if (!(ok = mbar_wait(&s_full[wg], (n >> 1) & 1, err, &abort_flag))) break;
       tc_fence_after();
-      const bool member = key_ok && ((uflag[n] >> half) & 1);
+      // (a padded query row of this block has LSE = +inf, so its P is 0)
+      const bool member = key_valid && ((uflag[n] >> half) & 1);
       const uint32_t st_t = tmem + lane_base + wg * 128, dp_t = st_t + 64;
 #pragma unroll
       for (int c0 = 0; c0 < 64; c0 += 32) {
@@ -275,6 +278,7 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
           *reinterpret_cast<float4*>(&lv[e]) = *reinterpret_cast<const float4*>(sl + c0 + e);
           *reinterpret_cast<float4*>(&dv4[e]) = *reinterpret_cast<const float4*>(sd + c0 + e);
         }
+
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           float p0 = 0.f, p1 = 0.f;
@@ -387,7 +391,7 @@ cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, co
                              int(smem));
     if (e != cudaSuccess) return e;
     bwd_sparse_kernel<128><<<grid, 320, smem, s>>>(tq, tk, tv, tdo, lse, dvec, col_ptr, col_idx,
-                                                   p.N, p.T, p.n_crit, p.scale_log2, p.scale, dq,
+                                                   p.N, p.T, p.n_crit, p.nv, p.scale_log2, p.scale, dq,
                                                    dk, dv, err);
   } else {
     const size_t smem = SbSmem<64>::total(p.T);
@@ -395,7 +399,7 @@ cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, co
                              int(smem));
     if (e != cudaSuccess) return e;
     bwd_sparse_kernel<64><<<grid, 320, smem, s>>>(tq, tk, tv, tdo, lse, dvec, col_ptr, col_idx,
-                                                  p.N, p.T, p.n_crit, p.scale_log2, p.scale, dq,
+                                                  p.N, p.T, p.n_crit, p.nv, p.scale_log2, p.scale, dq,
                                                   dk, dv, err);
   }
   return cudaGetLastError();

@@ -46,7 +46,8 @@ template <int D>
 __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ crit_idx, int N, int T,
-    int n_crit, float scale_log2, float* __restrict__ o_s, float* __restrict__ lse, int* err) {
+    int n_crit, int nv, float scale_log2, float* __restrict__ o_s, float* __restrict__ lse,
+    int* err) {
   using L = FwdSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = align_smem_1024(smem_raw);
@@ -202,6 +203,9 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
     const int half = r >> 6;
     const int blk = blk0 + half;
     const bool row_ok = blk < T;
+    // a padded query row (key padding) attends to nothing: O_s = 0, LSE = +inf
+    const bool q_valid = size_t(p) * 128 + r < size_t(nv);
+    const int last_keys = nv - (T - 1) * kBlock;  // valid keys of block T-1
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
@@ -214,9 +218,14 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
       tmem_ld32(sb, reinterpret_cast<float(&)[32]>(sv[0]));
       tmem_ld32(sb + 32, reinterpret_cast<float(&)[32]>(sv[32]));
       tmem_ld_wait();
-      const bool member = row_ok && ((uflag[n] >> half) & 1);
+      const bool member = row_ok && q_valid && ((uflag[n] >> half) & 1);
       float alpha = 1.f;
       if (member) {
+        if (int(ulist[n]) == T - 1 && last_keys < kBlock) {  // padded keys: no weight
+#pragma unroll
+          for (int e = 0; e < 64; ++e)
+            if (e >= last_keys) sv[e] = -INFINITY;
+        }
         float mx = -INFINITY;  // the scale is positive: max of the raw scores, then scaled
 #pragma unroll
         for (int e = 0; e < 64; ++e) mx = fmaxf(mx, sv[e]);
@@ -297,7 +306,8 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
     }
     if (row_ok)
       lse[size_t(bh) * N + tok] =
-          have ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+          have ? (m_run + __log2f(l_run)) * 0.69314718055994530942f
+               : (q_valid ? -INFINITY : INFINITY);  // +inf: a padded row, P = 0 everywhere
   }
   tc_fence_before();
   __syncthreads();
@@ -321,14 +331,14 @@ cudaError_t launch_fwd_sparse(const Problem& p, const void* q, const void* k, co
                              smem);
     if (e != cudaSuccess) return e;
     fwd_sparse_kernel<128><<<grid, 192, smem, s>>>(tq, tk, tv, crit_idx, p.N, p.T, p.n_crit,
-                                                   p.scale_log2, o_s, lse, err);
+                                                   p.nv, p.scale_log2, o_s, lse, err);
   } else {
     const int smem = int(FwdSmem<64>::total(p.n_crit));
     e = cudaFuncSetAttribute(fwd_sparse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem);
     if (e != cudaSuccess) return e;
     fwd_sparse_kernel<64><<<grid, 192, smem, s>>>(tq, tk, tv, crit_idx, p.N, p.T, p.n_crit,
-                                                  p.scale_log2, o_s, lse, err);
+                                                  p.nv, p.scale_log2, o_s, lse, err);
   }
   return cudaGetLastError();
 }

@@ -37,12 +37,13 @@ def assert_close(got, ref, what, max_tol=MAX_TOL, mean_tol=MEAN_TOL):
 class Run:
     """One library run (classification + forward [+ backward]) on a workload."""
 
-    def __init__(self, wl, with_logits=True):
+    def __init__(self, wl, with_logits=True, n_valid=0):
         import torch
         import sparse_linear_attention_block_b200 as slab
         self.slab = slab
         self.wl = wl
-        self.shape = slab.make_shape(wl.B, wl.H, wl.N, wl.d, wl.block, wl.k_h, wl.k_l)
+        self.shape = slab.make_shape(wl.B, wl.H, wl.N, wl.d, wl.block, wl.k_h, wl.k_l,
+                                     n_valid=n_valid)
         self.buf = slab.Buffers.allocate(self.shape, with_logits=with_logits)
         self.q = to_dev(wl.q, torch.bfloat16)
         self.k = to_dev(wl.k, torch.bfloat16)

@@ -425,7 +425,7 @@ def test_padded_tokens_do_not_matter():
     f2 = oracle.forward(q2, k2, v2, w, cls, 32, n_valid=nv)
     for n in ("o", "o_s", "o_l", "lse", "den"):
         assert np.array_equal(f1[n], f2[n]), n
-    assert np.all(f1["o"][:, :, nv:] == 0) and np.all(np.isneginf(f1["lse"][:, :, nv:]))
+    assert np.all(f1["o"][:, :, nv:] == 0) and np.all(np.isposinf(f1["lse"][:, :, nv:]))
     g1 = oracle.backward(q, k, v, w, cls, do, 32, n_valid=nv)
     g2 = oracle.backward(q2, k2, v2, w, cls, do2, 32, n_valid=nv)
     for n in ("dq", "dk", "dv", "dw"):
