@@ -45,6 +45,23 @@ map, the combination and the backward math; this oracle takes these readings
       logit gamma and threshold tau, g = sigmoid(gamma) and
       O = O_s + g * O_l W_proj; when g < tau the branch is dropped, O = O_s,
       and neither the branch nor gamma gets a gradient.
+* R14 optional hierarchical selection for long sequences, after the page
+      "Trainable Log-linear Sparse Attention for Efficient Diffusion
+      Transformers" (abstract: top-K is taken at a coarse level first and the
+      next level's top-K is restricted to the indices found there): blocks
+      are grouped into super-blocks of G consecutive blocks (the last may be
+      partial) with mean key Kc_J (equal-weight mean of its blocks' mean
+      keys); a query block's coarse scores are sc_iJ = mean(Q_i) . Kc_J *
+      scale; in the order (sc desc, J asc) its first c_hi super-blocks are the
+      critical candidates and its last c_lo the negligible candidates.  c_hi is
+      at least a caller's minimum and at least ceil(n_h / G) (+1 when T % G,
+      since the partial super-block may be chosen), so the candidates hold
+      n_h blocks; c_lo likewise for n_l; when c_hi + c_lo > TG both become
+      TG.  Critical: the first n_h candidate blocks in the order (s desc,
+      j asc) of the fine scores; negligible: the last n_l, in that order, of
+      the negligible candidates that are not critical; the rest marginal.
+      Counts are exactly n_h and n_l, and with every super-block a candidate
+      this is R1.
 
 Arrays are [B, H, N, d]; blocks are consecutive runs of ``block`` tokens.
 """
@@ -61,6 +78,11 @@ __all__ = [
     "pooled_logits",
     "classify",
     "classify_rows_bruteforce",
+    "coarse_counts",
+    "coarse_keys",
+    "coarse_logits",
+    "classify_hierarchical",
+    "classify_hierarchical_rows_bruteforce",
     "phi",
     "phi_prime",
     "key_block_summaries",
@@ -142,6 +164,107 @@ def classify_rows_bruteforce(row: list[float], n_h: int, n_l: int) -> list[int]:
         rank = sum(1 for k in range(T) if row[k] > row[j] or (row[k] == row[j] and k < j))
         out.append(1 if rank < n_h else (-1 if rank >= T - n_l else 0))
     return out
+
+
+def coarse_counts(T: int, n_h: int, n_l: int, group: int, top: int = 0, bottom: int = 0):
+    """(TG, c_hi, c_lo) of the hierarchical selection (reading R14).
+
+    TG = ceil(T / group) super-blocks.  c_hi is at least top and at least the
+    number of super-blocks that always hold n_h blocks (ceil(n_h / group),
+    plus one when the last super-block is partial, since it may be chosen);
+    c_lo likewise for n_l.  When the two candidate lists could meet
+    (c_hi + c_lo > TG) every super-block is a candidate of both, which is the
+    flat selection.
+    """
+    if group < 2:
+        raise ValueError("group must be at least 2")
+    if top < 0 or bottom < 0:
+        raise ValueError("candidate counts must be non-negative")
+    TG = -(-T // group)
+    partial = 1 if T % group else 0
+
+    def floor(n):
+        return 0 if n == 0 else -(-n // group) + partial
+
+    c_hi = min(TG, max(top, floor(n_h)))
+    c_lo = min(TG, max(bottom, floor(n_l)))
+    if c_hi + c_lo > TG:
+        c_hi = c_lo = TG
+    return TG, c_hi, c_lo
+
+
+def coarse_keys(kbar: np.ndarray, group: int) -> np.ndarray:
+    """Kc_J = equal-weight mean of the block means of super-block J: [.., T, d] -> [.., TG, d]."""
+    T = kbar.shape[-2]
+    TG = -(-T // group)
+    return np.stack([kbar[..., J * group:min((J + 1) * group, T), :].mean(axis=-2)
+                     for J in range(TG)], axis=-2)
+
+
+def coarse_logits(q: np.ndarray, k: np.ndarray, block: int, scale: float, group: int,
+                  n_valid=None) -> np.ndarray:
+    """sc_iJ = mean(Q_i) . Kc_J * scale, [B,H,T,ceil(T/group)] (reading R14)."""
+    qb = pool(q, block, n_valid)
+    kc = coarse_keys(pool(k, block, n_valid), group)
+    return np.einsum("bhid,bhjd->bhij", qb, kc) * scale
+
+
+def _order(scores: np.ndarray, among: np.ndarray) -> np.ndarray:
+    """Indices ``among`` sorted by (score desc, index asc)."""
+    among = np.asarray(among)
+    return among[np.lexsort((among, -scores[among]))]
+
+
+def classify_hierarchical(logits: np.ndarray, coarse: np.ndarray, n_h: int, n_l: int,
+                          group: int, top: int = 0, bottom: int = 0) -> np.ndarray:
+    """Three-way classes by the two-level selection of reading R14.
+
+    logits [.., T, T] fine scores s_ij and coarse [.., T, TG] scores sc_iJ;
+    only the fine scores of candidate blocks are read.  int8 in {+1, 0, -1}.
+    """
+    T = logits.shape[-1]
+    TG, c_hi, c_lo = coarse_counts(T, n_h, n_l, group, top, bottom)
+    if coarse.shape[-1] != TG or coarse.shape[:-1] != logits.shape[:-1]:
+        raise ValueError("coarse scores must be [.., T, ceil(T / group)]")
+    if np.isnan(coarse).any():
+        raise ValueError("NaN scores have no ordering")
+    lead = logits.shape[:-2]
+    L = np.asarray(logits, dtype=np.float64).reshape(-1, T, T)
+    C = np.asarray(coarse, dtype=np.float64).reshape(-1, T, TG)
+    out = np.zeros(L.shape, dtype=np.int8)
+    blocks_of = [np.arange(J * group, min((J + 1) * group, T)) for J in range(TG)]
+    for r in range(L.shape[0]):
+        for i in range(T):
+            sb = _order(C[r, i], np.arange(TG))
+            hi = np.concatenate([blocks_of[J] for J in sb[:c_hi]] + [np.zeros(0, int)])
+            lo = np.concatenate([blocks_of[J] for J in sb[TG - c_lo:]] + [np.zeros(0, int)])
+            if np.isnan(L[r, i, np.union1d(hi, lo)]).any():
+                raise ValueError("NaN scores have no ordering")
+            crit = _order(L[r, i], hi)[:n_h]
+            rest = np.setdiff1d(lo, crit)
+            neg = _order(L[r, i], rest)[len(rest) - n_l:] if n_l else rest[:0]
+            out[r, i, crit] = 1
+            out[r, i, neg] = -1
+    return out.reshape(*lead, T, T)
+
+
+def classify_hierarchical_rows_bruteforce(row, crow, n_h, n_l, group, top=0, bottom=0):
+    """Pure-Python check of ``classify_hierarchical`` for one row: membership
+    by counting, for every entry, how many entries of its set precede it."""
+    T, TG = len(row), len(crow)
+    _, c_hi, c_lo = coarse_counts(T, n_h, n_l, group, top, bottom)
+
+    def rank(vals, idxs, x):  # position of x in (value desc, index asc) among idxs
+        return sum(1 for y in idxs if vals[y] > vals[x] or (vals[y] == vals[x] and y < x))
+
+    allJ = list(range(TG))
+    hi_sb = {J for J in allJ if rank(crow, allJ, J) < c_hi}
+    lo_sb = {J for J in allJ if rank(crow, allJ, J) >= TG - c_lo}
+    hi = [j for j in range(T) if j // group in hi_sb]
+    crit = {j for j in hi if rank(row, hi, j) < n_h}
+    lo = [j for j in range(T) if j // group in lo_sb and j not in crit]
+    neg = {j for j in lo if rank(row, lo, j) >= len(lo) - n_l}
+    return [1 if j in crit else (-1 if j in neg else 0) for j in range(T)]
 
 
 def phi(x: np.ndarray) -> np.ndarray:

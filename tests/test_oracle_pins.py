@@ -469,3 +469,122 @@ def test_padded_backward_matches_central_differences():
             bp[name], bm[name] = xp, xm
             fd = (loss(bp["q"], bp["k"], bp["v"], bp["w"]) - loss(bm["q"], bm["k"], bm["v"], bm["w"])) / 2e-6
             assert math.isclose(fd, grad[idx], rel_tol=2e-6, abs_tol=2e-8), (name, idx, fd, grad[idx])
+
+
+# ---------------------------------------------------------------- hierarchical selection (R14)
+
+@pytest.mark.parametrize("args,expect", [
+    ((1182, 119, 118, 16), (74, 9, 9)),     # long sequence, partial last super-block
+    ((1182, 30, 118, 16), (74, 3, 9)),
+    ((512, 26, 51, 16), (32, 2, 4)),        # whole super-blocks only
+    ((16, 4, 4, 4), (4, 1, 1)),
+    ((16, 4, 4, 4, 3), (4, 3, 1)),          # a caller's minimum
+    ((16, 4, 4, 4, 3, 2), (4, 4, 4)),       # the lists would meet: flat
+    ((16, 0, 0, 4), (4, 0, 0)),
+    ((10, 3, 3, 4), (3, 3, 3)),             # 2 + 2 > 3: flat
+    ((10, 1, 0, 4), (3, 2, 0)),             # partial: one more than ceil(1/4)
+])
+def test_coarse_counts(args, expect):
+    assert oracle.coarse_counts(*args) == expect
+
+
+def test_coarse_counts_rejects_bad_group():
+    with pytest.raises(ValueError):
+        oracle.coarse_counts(16, 4, 4, 1)
+    with pytest.raises(ValueError):
+        oracle.coarse_counts(16, 4, 4, 4, -1)
+
+
+def test_coarse_keys_are_pooling_at_the_coarser_block():
+    # whole super-blocks: the mean of G block means is the mean of their G*b tokens
+    k = _rand((2, 3, 16 * 8, 5), 40)
+    kb = oracle.pool(k, 8)
+    np.testing.assert_allclose(oracle.coarse_keys(kb, 4), oracle.pool(k, 32), rtol=0, atol=1e-13)
+    # partial last super-block (T = 7, G = 3): blocks 6 alone
+    k7 = _rand((1, 1, 7 * 4, 3), 41)
+    kc = oracle.coarse_keys(oracle.pool(k7, 4), 3)
+    assert kc.shape == (1, 1, 3, 3)
+    np.testing.assert_allclose(kc[0, 0, 2], k7[0, 0, 24:28].mean(axis=0), atol=1e-14)
+    np.testing.assert_allclose(kc[0, 0, 1], k7[0, 0, 12:24].mean(axis=0), atol=1e-14)
+
+
+def test_coarse_logits_closed_form():
+    q, k = _rand((1, 2, 12 * 8, 6), 42), _rand((1, 2, 12 * 8, 6), 43)
+    got = oracle.coarse_logits(q, k, 8, 0.3, 3)
+    want = np.einsum("bhid,bhjd->bhij", oracle.pool(q, 8), oracle.pool(k, 24)) * 0.3
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def _hier_case(T, G, seed, ties=True):
+    rng = np.random.default_rng(seed)
+    TG = -(-T // G)
+    if ties:
+        fine = rng.integers(-3, 4, size=(2, T, T)).astype(np.float64)
+        coarse = rng.integers(-2, 3, size=(2, T, TG)).astype(np.float64)
+        fine[0, :, ::3] = -0.0
+    else:
+        fine, coarse = rng.standard_normal((2, T, T)), rng.standard_normal((2, T, TG))
+    return fine, coarse
+
+
+@pytest.mark.parametrize("T,G", [(1, 2), (5, 2), (16, 4), (21, 4), (33, 8), (40, 3)])
+@pytest.mark.parametrize("frac", [(0.0, 0.0), (0.1, 0.2), (0.25, 0.25), (0.05, 0.5)])
+@pytest.mark.parametrize("extra", [(0, 0), (1, 0), (0, 2)])
+def test_hierarchical_matches_rank_count(T, G, frac, extra):
+    n_h, n_l = oracle.block_counts(T, *frac)
+    fine, coarse = _hier_case(T, G, T * 7 + G)
+    got = oracle.classify_hierarchical(fine, coarse, n_h, n_l, G, *extra)
+    for r in range(fine.shape[0]):
+        for i in range(T):
+            want = oracle.classify_hierarchical_rows_bruteforce(
+                fine[r, i].tolist(), coarse[r, i].tolist(), n_h, n_l, G, *extra)
+            assert got[r, i].tolist() == want, (r, i)
+
+
+@pytest.mark.parametrize("T,G", [(16, 4), (21, 4), (40, 3)])
+def test_hierarchical_with_every_candidate_is_flat(T, G):
+    n_h, n_l = oracle.block_counts(T, 0.2, 0.3)
+    fine, coarse = _hier_case(T, G, 5 + T)
+    TG = coarse.shape[-1]
+    got = oracle.classify_hierarchical(fine, coarse, n_h, n_l, G, TG, TG)
+    np.testing.assert_array_equal(got, oracle.classify(fine, n_h, n_l))
+
+
+@pytest.mark.parametrize("T,G,frac", [(64, 8, (0.1, 0.2)), (61, 4, (0.05, 0.1)),
+                                      (100, 16, (0.1, 0.1))])
+def test_hierarchical_counts_and_candidate_sets(T, G, frac):
+    n_h, n_l = oracle.block_counts(T, *frac)
+    fine, coarse = _hier_case(T, G, 11 * T, ties=False)
+    TG, c_hi, c_lo = oracle.coarse_counts(T, n_h, n_l, G)
+    assert c_hi + c_lo <= TG  # a pruning case
+    got = oracle.classify_hierarchical(fine, coarse, n_h, n_l, G)
+    assert ((got == 1).sum(-1) == n_h).all() and ((got == -1).sum(-1) == n_l).all()
+    for r in range(2):
+        for i in range(T):
+            c = coarse[r, i]
+            rank = np.array([(c > c[J]).sum() for J in range(TG)])  # distinct scores
+            crit = np.flatnonzero(got[r, i] == 1)
+            neg = np.flatnonzero(got[r, i] == -1)
+            assert (rank[crit // G] < c_hi).all()
+            assert (rank[neg // G] >= TG - c_lo).all()
+            # inside its candidates the critical set is the top of the fine scores
+            cand = np.flatnonzero(rank[np.arange(T) // G] < c_hi)
+            rest = np.setdiff1d(cand, crit)
+            if len(rest) and len(crit):
+                assert fine[r, i, crit].min() >= fine[r, i, rest].max()
+
+
+@pytest.mark.parametrize("frac", [(0.1, 0.2), (0.05, 0.4), (0.3, 0.3)])
+def test_hierarchical_equals_flat_when_blocks_follow_their_super_block(frac):
+    # fine score = coarse score of the block's super-block: the coarse order
+    # agrees with the fine one (ties by index on both levels), so pruning to
+    # the candidates loses nothing
+    T, G = 48, 4
+    n_h, n_l = oracle.block_counts(T, *frac)
+    rng = np.random.default_rng(3)
+    coarse = rng.integers(-4, 5, size=(3, T, T // G)).astype(np.float64)
+    fine = np.repeat(coarse, G, axis=-1)
+    TG, c_hi, c_lo = oracle.coarse_counts(T, n_h, n_l, G)
+    assert c_hi + c_lo <= TG
+    np.testing.assert_array_equal(oracle.classify_hierarchical(fine, coarse, n_h, n_l, G),
+                                  oracle.classify(fine, n_h, n_l))
