@@ -44,12 +44,16 @@ def peaks():
 
 
 def workload_config(wl, n_crit):
+    kind = ("Wan2.1-1.3B-shaped" if wl.name == "train" else "long-sequence")
+    grid = "x".join(str(g) for g in wl.grid) if wl.grid else "none"
     return {
-        "workload": "Wan2.1-1.3B-shaped SLA training step (classify+forward+backward): "
-                    "B=1 H=12 N=32768 (21x30x52 grid padded) d=128 block=64 k_h=0.05 k_l=0.10",
+        "workload": f"{kind} SLA training step (classify+forward+backward): B={wl.B} H={wl.H} "
+                    f"N={wl.N} ({grid} grid padded) d={wl.d} block={wl.block} "
+                    f"k_h={wl.k_h:g} k_l={wl.k_l:g}",
         "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "block": wl.block, "k_h": wl.k_h,
         "k_l": wl.k_l, "n_crit": n_crit, "global_batch": wl.B, "seq_len": wl.N,
-        "l2": "inputs larger than L2 (Q/K/V/dO bf16 = 403 MB per step)",
+        "l2": f"inputs larger than L2 (Q/K/V/dO bf16 = {4 * wl.B * wl.H * wl.N * wl.d * 2 / 1e6:.0f} "
+              f"MB per step)",
         "parallelism": "independent replica per GPU",
     }
 
@@ -227,6 +231,12 @@ def main():
                     help="mask the grid's padding tokens (n_valid) instead of treating them as tokens")
     ap.add_argument("--gate-skip", type=float, default=0.0,
                     help="drop the linear branch when sigmoid(logit) is below this")
+    ap.add_argument("--workload", choices=["train", "long"], default="train",
+                    help="train: N=32768 (21x30x52 grid); long: N=75648 (21x45x80 grid)")
+    ap.add_argument("--k-h", type=float, default=None,
+                    help="critical fraction (default: the workload's 0.05)")
+    ap.add_argument("--hierarchical", type=int, default=0, metavar="G",
+                    help="classify hierarchically with super-blocks of G key blocks (0: flat)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -250,7 +260,10 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
-    wl = sla_inputs.make("train", seed=rank)
+    over = {"with_grad": True}
+    if args.k_h is not None:
+        over["k_h"] = args.k_h
+    wl = sla_inputs.make(args.workload, seed=rank, **over)
     shape = slab.make_shape(wl.B, wl.H, wl.N, wl.d, wl.block, wl.k_h, wl.k_l,
                             n_valid=wl.n_valid if args.key_padding else 0)
     buf = slab.Buffers.allocate(shape, device=dev, with_logits=False)
@@ -266,8 +279,14 @@ def main():
     gate = None if args.gate_logit is None else slab.Gate(args.gate_logit, args.gate_skip)
     d_logit = torch.empty(1, dtype=torch.float32, device=dev)
 
+    hier = slab.Hierarchy(args.hierarchical, 0, 0) if args.hierarchical else None
+
     def step(qq=q, kk=k, vv=v, ww=w, dd=do):
-        slab.sla_classify(shape, qq, kk, buf.mask, buf.workspace, stream)
+        if hier is None:
+            slab.sla_classify(shape, qq, kk, buf.mask, buf.workspace, stream)
+        else:
+            slab.sla_classify_hierarchical(shape, qq, kk, hier, buf.mask, None, buf.workspace,
+                                           stream)
         if gate is None:
             slab.sla_forward(shape, qq, kk, vv, ww, buf.mask, o, buf.saved, buf.workspace,
                              stream)
@@ -333,7 +352,7 @@ def main():
     dominant = max(prof, key=lambda n: prof[n][1])
     kind, amount = work.get(dominant, ("tensor", 0))
     traffic = (NCU_DRAM_BYTES_PER_HEAD[dominant] * wl.B * wl.H
-               if dominant in NCU_DRAM_BYTES_PER_HEAD else None)
+               if dominant in NCU_DRAM_BYTES_PER_HEAD and args.workload == "train" else None)
     avg_s = prof[dominant][1] / prof[dominant][0] * 1e-3
     if kind == "tensor":
         achieved = amount / avg_s / 1e12
@@ -350,7 +369,8 @@ def main():
     fwd_ms = sum(prof[n][1] for n in ("summaries", "expand_marginal", "aggregate",
                                       "fwd_sparse", "fwd_linear", "os_to_o")
                  if n in prof) / args.steps
-    cls_ms = sum(prof[n][1] for n in ("pool", "classify", "crit_csr") if n in prof) / args.steps
+    cls_ms = sum(prof[n][1] for n in ("pool", "classify", "coarse_keys", "hier_classify",
+                                      "crit_csr") if n in prof) / args.steps
     bwd_ms = sum(t for n, (_, t) in prof.items()) / args.steps - fwd_ms - cls_ms
 
     # ------------------------------------------------------------ end to end
@@ -399,7 +419,8 @@ def main():
 
     # ------------------------------------------------------------ CPU oracle baseline
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    default_run = args.workload == "train" and args.k_h is None and not args.hierarchical
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and default_run:
         tfl, sec = time_oracle(wl, [0], 1, 0)
         cpu = {"value": tfl, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"head 0 of 12 of this workload, one classify+forward+backward step "
@@ -414,6 +435,10 @@ def main():
     cfg = workload_config(wl, n_crit)
     if args.key_padding:
         cfg["n_valid"] = wl.n_valid
+    if hier is not None:
+        TG, c_hi, c_lo = slab.sla_hierarchy_counts(shape, hier)
+        cfg["classification"] = {"hierarchical_group": args.hierarchical, "super_blocks": TG,
+                                 "critical_candidates": c_hi, "negligible_candidates": c_lo}
     if gate is not None:
         g = 1.0 / (1.0 + math.exp(-args.gate_logit))
         cfg["gate"] = {"logit": args.gate_logit, "skip_below": args.gate_skip, "g": g,

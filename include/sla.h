@@ -156,6 +156,57 @@ SLA_API sla_status sla_classify_from_scores(const sla_shape* shape, const float*
 SLA_API sla_status sla_classify_noalloc(const sla_shape* shape, const void* q, const void* k,
                                         const sla_mask* mask, void* stream);
 
+/* Hierarchical selection for long sequences.  "Trainable Log-linear Sparse
+ * Attention for Efficient Diffusion Transformers" (abstract): top-K is taken
+ * on a coarse level first and the finer level only looks inside what the
+ * coarse level kept.  Reading (the page gives no formulas):
+ *   - super-block J = key blocks [J*group, min(T, (J+1)*group)); its key is
+ *     Kc_J = the equal-weight mean of its blocks' mean keys; TG = ceil(T/group);
+ *   - coarse scores sc_iJ = mean(Q_i) . Kc_J * scale; in the order
+ *     (sc desc, J asc) the first c_hi super-blocks of row i hold its critical
+ *     candidates, the last c_lo its negligible candidates;
+ *   - c_hi = min(TG, max(top, f(n_crit))), c_lo = min(TG, max(bottom,
+ *     f(n_negl))), f(0) = 0, f(n) = ceil(n/group) + (T % group ? 1 : 0), so
+ *     the candidates always hold enough blocks; if c_hi + c_lo > TG both are
+ *     TG and the result is exactly sla_classify's;
+ *   - critical: the n_crit candidate blocks first in the order (s desc,
+ *     j asc) of the pooled logits s_ij of sla_classify; negligible: the
+ *     n_negl negligible candidates last in that order; the rest marginal.
+ * Exactly n_crit critical and n_negl negligible blocks per row, as with
+ * sla_classify, and the mask has the same layout and meaning.
+ *   group >= 2; top, bottom >= 0 (minimum candidate counts). */
+typedef struct {
+  int group, top, bottom;
+} sla_hierarchy;
+
+/* TG, c_hi and c_lo of the reading above.  Host only; no CUDA call.  A flat
+ * case (c_hi + c_lo > TG before the clamp) reports c_hi = c_lo = TG. */
+SLA_API sla_status sla_hierarchy_counts(const sla_shape* shape, const sla_hierarchy* hier,
+                                        int* n_super, int* c_hi, int* c_lo);
+
+/* Hierarchical classification from q, k (bf16 [B,H,N,d]) into *mask, with
+ * the crit_col CSR, like sla_classify.  mask->pooled_logits, if not NULL,
+ * receives s_ij at the candidate blocks of each row (other entries are left
+ * as they were); coarse_logits (fp32 [B,H,T,TG], 16-byte aligned, or NULL)
+ * receives sc_iJ.  In a flat case the call is sla_classify: pooled_logits
+ * gets every s_ij and coarse_logits is left untouched. */
+SLA_API sla_status sla_classify_hierarchical(const sla_shape* shape, const void* q,
+                                             const void* k, const sla_hierarchy* hier,
+                                             const sla_mask* mask, float* coarse_logits,
+                                             void* workspace, size_t workspace_bytes,
+                                             void* stream);
+
+/* The same selection from caller-given scores: logits fp32 [B,H,T,T] (only
+ * the candidate entries are read) and coarse_logits fp32 [B,H,T,TG]; any
+ * values but NaN.  mask->pooled_logits is not touched.  Lets a test feed
+ * identical scores to this library and to a reference. */
+SLA_API sla_status sla_classify_hierarchical_from_scores(const sla_shape* shape,
+                                                         const float* logits,
+                                                         const float* coarse_logits,
+                                                         const sla_hierarchy* hier,
+                                                         const sla_mask* mask, void* workspace,
+                                                         size_t workspace_bytes, void* stream);
+
 /* Forward with a given mask: writes o (bf16 [B,H,N,d]) and *saved. */
 SLA_API sla_status sla_forward(const sla_shape* shape, const void* q, const void* k, const void* v,
                        const void* w_proj, const sla_mask* mask, void* o,

@@ -23,7 +23,8 @@ __all__ = [
     "sla_query_sizes", "sla_classify", "sla_classify_from_scores", "sla_forward",
     "sla_backward", "sla_workspace_init", "sla_check", "sla_strerror", "sla_version",
     "sla_profile_begin", "sla_profile_end", "KernelStat", "make_shape", "EXPORTED_SYMBOLS",
-    "STATUS", "Gate", "sla_forward_gated", "sla_backward_gated",
+    "STATUS", "Gate", "sla_forward_gated", "sla_backward_gated", "Hierarchy",
+    "sla_hierarchy_counts", "sla_classify_hierarchical", "sla_classify_hierarchical_from_scores",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -35,7 +36,9 @@ STATUS = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED", 3: "S
 EXPORTED_SYMBOLS = ["sla_query_sizes", "sla_classify", "sla_classify_from_scores",
                     "sla_forward", "sla_backward", "sla_workspace_init", "sla_check",
                     "sla_strerror", "sla_version", "sla_profile_begin", "sla_profile_end",
-                    "sla_classify_noalloc", "sla_forward_gated", "sla_backward_gated"]
+                    "sla_classify_noalloc", "sla_forward_gated", "sla_backward_gated",
+                    "sla_hierarchy_counts", "sla_classify_hierarchical",
+                    "sla_classify_hierarchical_from_scores"]
 
 
 class SlaError(RuntimeError):
@@ -65,6 +68,12 @@ class SavedStruct(ctypes.Structure):
 class Gate(ctypes.Structure):
     """sla_gate: g = sigmoid(logit); the linear branch is dropped when g < skip_below."""
     _fields_ = [("logit", ctypes.c_float), ("skip_below", ctypes.c_float)]
+
+
+class Hierarchy(ctypes.Structure):
+    """sla_hierarchy: super-blocks of `group` key blocks; `top` / `bottom` are
+    minimum numbers of critical / negligible candidate super-blocks."""
+    _fields_ = [("group", ctypes.c_int), ("top", ctypes.c_int), ("bottom", ctypes.c_int)]
 
 
 class KernelStat(ctypes.Structure):
@@ -105,6 +114,11 @@ def lib() -> ctypes.CDLL:
                                         P(SavedStruct), vp, sz, vp]
         L.sla_backward_gated.argtypes = [P(Shape), vp, vp, vp, vp, P(MaskStruct), P(Gate),
                                          P(SavedStruct), vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_hierarchy_counts.argtypes = [P(Shape), P(Hierarchy), P(st), P(st), P(st)]
+        L.sla_classify_hierarchical.argtypes = [P(Shape), vp, vp, P(Hierarchy), P(MaskStruct), vp,
+                                                vp, sz, vp]
+        L.sla_classify_hierarchical_from_scores.argtypes = [P(Shape), vp, vp, P(Hierarchy),
+                                                            P(MaskStruct), vp, sz, vp]
         L.sla_workspace_init.argtypes = [vp, sz, vp]
         L.sla_check.argtypes = [vp, vp]
         L.sla_strerror.argtypes = [st]
@@ -117,7 +131,9 @@ def lib() -> ctypes.CDLL:
         L.sla_profile_end.argtypes = [P(KernelStat), st, P(st)]
         for n in ("sla_query_sizes", "sla_classify", "sla_classify_from_scores", "sla_forward",
                   "sla_backward", "sla_workspace_init", "sla_check", "sla_profile_begin",
-                  "sla_profile_end", "sla_forward_gated", "sla_backward_gated"):
+                  "sla_profile_end", "sla_forward_gated", "sla_backward_gated",
+                  "sla_hierarchy_counts", "sla_classify_hierarchical",
+                  "sla_classify_hierarchical_from_scores"):
             getattr(L, n).restype = st
         _lib = L
     return _lib
@@ -211,6 +227,32 @@ def sla_classify_from_scores(shape: Shape, logits, mask: MaskStruct, workspace, 
                                           _ptr(workspace),
                                           workspace.numel() * workspace.element_size(),
                                           _stream(stream)), "sla_classify_from_scores")
+
+
+def sla_hierarchy_counts(shape: Shape, hier: Hierarchy) -> tuple[int, int, int]:
+    """(TG, c_hi, c_lo) of the hierarchical selection; host only."""
+    n, hi, lo = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(lib().sla_hierarchy_counts(ctypes.byref(shape), ctypes.byref(hier), ctypes.byref(n),
+                                      ctypes.byref(hi), ctypes.byref(lo)),
+           "sla_hierarchy_counts")
+    return n.value, hi.value, lo.value
+
+
+def sla_classify_hierarchical(shape: Shape, q, k, hier: Hierarchy, mask: MaskStruct,
+                              coarse_logits, workspace, stream=None):
+    _check(lib().sla_classify_hierarchical(ctypes.byref(shape), _ptr(q), _ptr(k),
+                                           ctypes.byref(hier), ctypes.byref(mask),
+                                           _ptr(coarse_logits), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(),
+                                           _stream(stream)), "sla_classify_hierarchical")
+
+
+def sla_classify_hierarchical_from_scores(shape: Shape, logits, coarse_logits, hier: Hierarchy,
+                                          mask: MaskStruct, workspace, stream=None):
+    _check(lib().sla_classify_hierarchical_from_scores(
+        ctypes.byref(shape), _ptr(logits), _ptr(coarse_logits), ctypes.byref(hier),
+        ctypes.byref(mask), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "sla_classify_hierarchical_from_scores")
 
 
 def sla_forward(shape: Shape, q, k, v, w_proj, mask: MaskStruct, o, saved: SavedStruct,

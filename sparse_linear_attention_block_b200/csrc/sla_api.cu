@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -274,6 +275,89 @@ sla_status sla_classify_from_scores(const sla_shape* shape, const float* logits,
   if (!logits || !aligned16(logits)) return SLA_ERR_INVALID_ARG;
   return classify_impl(shape, nullptr, nullptr, logits, mask, workspace, workspace_bytes,
                        stream);
+}
+
+// Super-block counts of the hierarchical selection; false on a bad argument.
+static bool hier_counts(const Problem& p, const sla_hierarchy* hz, HierCounts* h) {
+  if (!hz || hz->group < 2 || hz->top < 0 || hz->bottom < 0) return false;
+  const int G = hz->group;
+  const int TG = (p.T + G - 1) / G;
+  const int partial = p.T % G ? 1 : 0;
+  auto floor_of = [&](int n) { return n == 0 ? 0 : (n + G - 1) / G + partial; };
+  int c_hi = std::min(TG, std::max(hz->top, floor_of(p.n_crit)));
+  int c_lo = std::min(TG, std::max(hz->bottom, floor_of(p.n_negl)));
+  if (c_hi + c_lo > TG) c_hi = c_lo = TG;
+  *h = HierCounts{G, TG, c_hi, c_lo};
+  return true;
+}
+
+static bool hier_is_flat(const HierCounts& h) { return h.c_hi == h.TG && h.c_lo == h.TG; }
+
+static sla_status classify_hier_impl(const sla_shape* shape, const void* q, const void* k,
+                                     const float* logits_in, const float* coarse_in,
+                                     float* coarse_out, const sla_hierarchy* hz,
+                                     const sla_mask* mask, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  Problem p;
+  sla_status st = check_shape(shape, &p);
+  if (st != SLA_OK) return st;
+  HierCounts h;
+  if (!hier_counts(p, hz, &h)) return SLA_ERR_INVALID_ARG;
+  if ((st = check_mask(p, mask, true)) != SLA_OK) return st;
+  if (coarse_out && !aligned16(coarse_out)) return SLA_ERR_INVALID_ARG;
+  WorkspaceLayout L;
+  if ((st = check_ws(p, ws, ws_bytes, &L)) != SLA_OK) return st;
+  if (hier_is_flat(h)) return classify_impl(shape, q, k, logits_in, mask, ws, ws_bytes, stream);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* qbar = at<float>(ws, L.qbar);
+  float* kbar = at<float>(ws, L.kbar);
+  float* kc = at<float>(ws, L.summ_hi);  // forward-only region, free during classification
+  if (!logits_in) {
+    if (!q || !k || !aligned16(q) || !aligned16(k)) return SLA_ERR_INVALID_ARG;
+    SLA_LAUNCH("pool", s, launch_pool(p, q, k, qbar, kbar, s));
+    SLA_LAUNCH("coarse_keys", s, launch_coarse_keys(p, kbar, kc, h.G, s));
+  }
+  SLA_LAUNCH("hier_classify", s,
+             launch_hier_classify(p, h, qbar, kbar, kc, logits_in, coarse_in,
+                                  logits_in ? nullptr : mask->pooled_logits, coarse_out,
+                                  mask->cls, mask->crit_idx, mask->marg_bits,
+                                  at<int>(ws, L.err), s));
+  SLA_LAUNCH("crit_csr", s, launch_crit_csr(p, mask->cls, mask->crit_col_ptr, mask->crit_col_idx, s));
+  return SLA_OK;
+}
+
+sla_status sla_hierarchy_counts(const sla_shape* shape, const sla_hierarchy* hier, int* n_super,
+                                int* c_hi, int* c_lo) {
+  if (!n_super || !c_hi || !c_lo) return SLA_ERR_INVALID_ARG;
+  Problem p;
+  sla_status st = check_shape(shape, &p);
+  if (st != SLA_OK) return st;
+  HierCounts h;
+  if (!hier_counts(p, hier, &h)) return SLA_ERR_INVALID_ARG;
+  *n_super = h.TG;
+  *c_hi = h.c_hi;
+  *c_lo = h.c_lo;
+  return SLA_OK;
+}
+
+sla_status sla_classify_hierarchical(const sla_shape* shape, const void* q, const void* k,
+                                     const sla_hierarchy* hier, const sla_mask* mask,
+                                     float* coarse_logits, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (!q || !k) return SLA_ERR_INVALID_ARG;
+  return classify_hier_impl(shape, q, k, nullptr, nullptr, coarse_logits, hier, mask, workspace,
+                            workspace_bytes, stream);
+}
+
+sla_status sla_classify_hierarchical_from_scores(const sla_shape* shape, const float* logits,
+                                                 const float* coarse_logits,
+                                                 const sla_hierarchy* hier, const sla_mask* mask,
+                                                 void* workspace, size_t workspace_bytes,
+                                                 void* stream) {
+  if (!logits || !aligned16(logits) || !coarse_logits || !aligned16(coarse_logits))
+    return SLA_ERR_INVALID_ARG;
+  return classify_hier_impl(shape, nullptr, nullptr, logits, coarse_logits, nullptr, hier, mask,
+                            workspace, workspace_bytes, stream);
 }
 
 static sla_status check_saved(const Problem& p, const sla_saved* sv) {

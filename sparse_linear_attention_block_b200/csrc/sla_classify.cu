@@ -9,6 +9,8 @@
 // equivalent to ranking the row softmax of the pooled scores.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "sla_internal.h"
 #include "sla_ptx.cuh"
 
@@ -251,6 +253,256 @@ __global__ void __launch_bounds__(256) classify_kernel(
   }
 }
 
+// ------------------------------------------------------------------ hierarchical selection
+// "Trainable Log-linear Sparse Attention for Efficient Diffusion Transformers"
+// (abstract): top-K is taken on a coarse level first and the next level only
+// looks inside the indices it kept.  Here the coarse level is super-blocks of
+// G consecutive key blocks with mean key Kc_J; per query-block row its first
+// c_hi super-blocks (coarse score desc, J asc) hold the critical candidates and
+// its last c_lo the negligible ones.  The host routes the case in which the
+// two lists could meet (c_hi + c_lo > TG) to the flat kernel above, so here
+// the lists are disjoint and each holds enough blocks for its count.
+
+// Kc_J = mean of the block means of super-block J (the last may be partial).
+// One CTA per (J, head), one thread per feature.
+__global__ void coarse_keys_kernel(const float* __restrict__ kbar, float* __restrict__ kc,
+                                   int T, int TG, int G, int D) {
+  const int J = blockIdx.x, bh = blockIdx.y, a = threadIdx.x;
+  if (a >= D) return;
+  const int j0 = J * G, j1 = min(T, j0 + G);
+  const float* src = kbar + (size_t(bh) * T) * D + a;
+  float s = 0.f;
+  for (int j = j0; j < j1; ++j) s += src[size_t(j) * D];
+  kc[(size_t(bh) * TG + J) * D + a] = s / float(j1 - j0);
+}
+
+struct HierArgs {
+  const float* qbar;       // [BH,T,D]   (null with fine_in)
+  const float* kbar;       // [BH,T,D]
+  const float* kc;         // [BH,TG,D]
+  const float* fine_in;    // [BH,T,T]   caller scores, or null
+  const float* coarse_in;  // [BH,T,TG]  caller coarse scores, or null
+  float* fine_out;         // [BH,T,T]   candidate entries only, or null
+  float* coarse_out;       // [BH,T,TG]  or null
+  int8_t* cls;
+  int32_t* crit_idx;
+  uint32_t* marg_bits;
+  int* err;
+  int T, TG, G, c_hi, c_lo, cap_hi, cap_lo, n_crit, n_negl, rows;
+  float scale;
+};
+
+// Per-warp shared scratch, in floats / words.
+__host__ __device__ inline int hier_warp_words(int T, int TG, int cap_hi, int cap_lo, int c_hi,
+                                               int c_lo) {
+  const int W = (T + 31) / 32;
+  return TG + cap_hi + cap_lo + c_hi + c_lo + 256 + 2 * W;
+}
+
+// Block index of candidate position p of a list of super-blocks (ascending).
+__device__ __forceinline__ int cand_block(const int* list, int p, int G) {
+  return list[p / G] * G + p % G;
+}
+
+// Fine scores of nb candidate positions into out[]: four candidates per step,
+// eight lanes per candidate, each lane a contiguous D/8-feature slice of the
+// pooled query (registers) against the same slice of the pooled key (L2).
+template <int D>
+__device__ void fine_scores(const float* qrow, const float* kbar_h, const int* list, int nb,
+                            int G, float scale, float* out, float* fine_out_row) {
+  constexpr int kPer = D / 8;  // features per lane
+  const int lane = lane_id(), sub = lane & 7, grp = lane >> 3;
+  float qv[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; e += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(qrow + sub * kPer + e);
+    qv[e] = x.x; qv[e + 1] = x.y; qv[e + 2] = x.z; qv[e + 3] = x.w;
+  }
+  for (int p0 = 0; p0 < nb; p0 += 4) {
+    const int p = p0 + grp;
+    float acc = 0.f;
+    int j = 0;
+    if (p < nb) {
+      j = cand_block(list, p, G);
+      const float4* kr = reinterpret_cast<const float4*>(kbar_h + size_t(j) * D + sub * kPer);
+#pragma unroll
+      for (int e = 0; e < kPer / 4; ++e) {
+        const float4 y = __ldg(kr + e);
+        acc = fmaf(qv[4 * e], y.x, acc);
+        acc = fmaf(qv[4 * e + 1], y.y, acc);
+        acc = fmaf(qv[4 * e + 2], y.z, acc);
+        acc = fmaf(qv[4 * e + 3], y.w, acc);
+      }
+    }
+    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
+    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 2);
+    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 4);
+    if (p < nb && sub == 0) {
+      const float v = acc * scale;
+      out[p] = v;
+      if (fine_out_row) fine_out_row[j] = v;
+    }
+  }
+}
+
+// Candidate positions of one list whose ordered score is at or before the
+// threshold, as bits by block index.
+__device__ __forceinline__ void mark_selected(const float* cand, const int* list, int nb, int G,
+                                              Threshold t, bool flip, uint32_t* bits) {
+  for (int p = lane_id(); p < nb; p += 32) {
+    if (before_or_at(ordered_bits(cand[p]), p, t, flip)) {
+      const int j = cand_block(list, p, G);
+      atomicOr(&bits[j >> 5], 1u << (j & 31));
+    }
+  }
+}
+
+// One warp per query-block row, `rows` rows per CTA (blockDim = 32 * rows).
+template <int D>
+__global__ void __launch_bounds__(256) hier_classify_kernel(const HierArgs a) {
+  extern __shared__ __align__(16) float smem[];
+  constexpr int kStride = D + 4;
+  const int T = a.T, TG = a.TG, G = a.G, rows = a.rows;
+  const bool compute = a.fine_in == nullptr;
+  float* sq = smem;                                  // [rows][D]
+  float* sk = sq + rows * D;                         // [32][D+4]
+  float* wbase = compute ? sk + kKTile * kStride : smem;
+  const int bh = blockIdx.y, warp = threadIdx.x / 32, lane = lane_id();
+  const int i = blockIdx.x * rows + warp;
+  const bool row_ok = i < T;
+  const int W = (T + 31) / 32;
+  float* crow = wbase + size_t(warp) * hier_warp_words(T, TG, a.cap_hi, a.cap_lo, a.c_hi, a.c_lo);
+  float* cand = crow + TG;                           // [cap_hi] then [cap_lo]
+  int* list_hi = reinterpret_cast<int*>(cand + a.cap_hi + a.cap_lo);
+  int* list_lo = list_hi + a.c_hi;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(list_lo + a.c_lo);
+  uint32_t* bits_c = hist + 256;
+  uint32_t* bits_n = bits_c + W;
+
+  // ---- coarse scores sc_iJ (all warps take part in the staging)
+  if (a.coarse_in == nullptr) {
+    for (int e = threadIdx.x; e < rows * D; e += blockDim.x) {
+      const int r = e / D, f = e % D, ii = blockIdx.x * rows + r;
+      sq[e] = ii < T ? a.qbar[(size_t(bh) * T + ii) * D + f] : 0.f;
+    }
+    for (int J0 = 0; J0 < TG; J0 += kKTile) {
+      __syncthreads();
+      for (int e = threadIdx.x; e < kKTile * D; e += blockDim.x) {
+        const int r = e / D, f = e % D, JJ = J0 + r;
+        sk[r * kStride + f] = JJ < TG ? a.kc[(size_t(bh) * TG + JJ) * D + f] : 0.f;
+      }
+      __syncthreads();
+      const float4* qa = reinterpret_cast<const float4*>(sq + warp * D);
+      const float4* ka = reinterpret_cast<const float4*>(sk + lane * kStride);
+      float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+      for (int a4 = 0; a4 < D / 4; a4 += 2) {
+        const float4 x0 = qa[a4], y0 = ka[a4], x1 = qa[a4 + 1], y1 = ka[a4 + 1];
+        acc0 = fmaf(x0.x, y0.x, acc0); acc0 = fmaf(x0.y, y0.y, acc0);
+        acc0 = fmaf(x0.z, y0.z, acc0); acc0 = fmaf(x0.w, y0.w, acc0);
+        acc1 = fmaf(x1.x, y1.x, acc1); acc1 = fmaf(x1.y, y1.y, acc1);
+        acc1 = fmaf(x1.z, y1.z, acc1); acc1 = fmaf(x1.w, y1.w, acc1);
+      }
+      if (row_ok && J0 + lane < TG) crow[J0 + lane] = (acc0 + acc1) * a.scale;
+    }
+    __syncwarp();
+    if (row_ok && a.coarse_out)
+      for (int J = lane; J < TG; J += 32) a.coarse_out[(size_t(bh) * T + i) * TG + J] = crow[J];
+  } else if (row_ok) {
+    for (int J = lane; J < TG; J += 32) crow[J] = a.coarse_in[(size_t(bh) * T + i) * TG + J];
+  }
+  __syncwarp();
+  if (!row_ok) return;
+
+  // ---- candidate super-blocks, ascending
+  const Threshold thc = a.c_hi > 0 ? warp_select(crow, TG, a.c_hi, false, hist) : Threshold{0, -1};
+  const Threshold tlc = a.c_lo > 0 ? warp_select(crow, TG, a.c_lo, true, hist) : Threshold{0, -1};
+  int nh = 0, nl = 0;
+  for (int J0 = 0; J0 < TG; J0 += 32) {
+    const int J = J0 + lane;
+    bool hi = false, lo = false;
+    if (J < TG) {
+      const uint32_t o = ordered_bits(crow[J]);
+      hi = a.c_hi > 0 && before_or_at(o, J, thc, false);
+      lo = a.c_lo > 0 && before_or_at(o, J, tlc, true);
+    }
+    const uint32_t mh = __ballot_sync(0xFFFFFFFFu, hi), ml = __ballot_sync(0xFFFFFFFFu, lo);
+    const uint32_t below = (1u << lane) - 1u;
+    if (hi) {
+      const int pos = nh + __popc(mh & below);
+      if (pos < a.c_hi) list_hi[pos] = J;
+    }
+    if (lo) {
+      const int pos = nl + __popc(ml & below);
+      if (pos < a.c_lo) list_lo[pos] = J;
+    }
+    nh += __popc(mh);
+    nl += __popc(ml);
+  }
+  for (int w = lane; w < 2 * W; w += 32) bits_c[w] = 0u;
+  __syncwarp();
+  if (nh != a.c_hi || nl != a.c_lo) {  // the selection is exact: cannot happen
+    if (lane == 0) set_error(a.err, SLA_ERR_DEVICE);
+    return;
+  }
+  const int tail = TG * G - T;  // missing blocks of the last super-block
+  const int nb_hi = a.c_hi == 0 ? 0 : a.c_hi * G - (list_hi[a.c_hi - 1] == TG - 1 ? tail : 0);
+  const int nb_lo = a.c_lo == 0 ? 0 : a.c_lo * G - (list_lo[a.c_lo - 1] == TG - 1 ? tail : 0);
+  if (a.n_crit > nb_hi || a.n_negl > nb_lo) {  // the host's counts rule this out
+    if (lane == 0) set_error(a.err, SLA_ERR_DEVICE);
+    return;
+  }
+
+  // ---- fine scores of the candidate blocks only
+  float* cand_lo = cand + a.cap_hi;
+  if (compute) {
+    const float* qrow = sq + warp * D;
+    const float* kb = a.kbar + size_t(bh) * T * D;
+    float* fo = a.fine_out ? a.fine_out + (size_t(bh) * T + i) * T : nullptr;
+    fine_scores<D>(qrow, kb, list_hi, nb_hi, G, a.scale, cand, fo);
+    fine_scores<D>(qrow, kb, list_lo, nb_lo, G, a.scale, cand_lo, fo);
+  } else {
+    const float* fr = a.fine_in + (size_t(bh) * T + i) * T;
+    for (int p = lane; p < nb_hi; p += 32) cand[p] = fr[cand_block(list_hi, p, G)];
+    for (int p = lane; p < nb_lo; p += 32) cand_lo[p] = fr[cand_block(list_lo, p, G)];
+  }
+  __syncwarp();
+
+  // ---- exact selection inside the candidates (position order = block order)
+  if (a.n_crit > 0) {
+    const Threshold th = warp_select(cand, nb_hi, a.n_crit, false, hist);
+    mark_selected(cand, list_hi, nb_hi, G, th, false, bits_c);
+  }
+  if (a.n_negl > 0) {
+    const Threshold tl = warp_select(cand_lo, nb_lo, a.n_negl, true, hist);
+    mark_selected(cand_lo, list_lo, nb_lo, G, tl, true, bits_n);
+  }
+  __syncwarp();
+
+  // ---- outputs, as the flat kernel writes them
+  const size_t rbase = size_t(bh) * T + i;
+  int8_t* crw = a.cls + rbase * T;
+  int32_t* idx = a.crit_idx + rbase * a.n_crit;
+  uint32_t* mrow = a.marg_bits + rbase * W;
+  int written = 0;
+  for (int w = 0; w < W; ++w) {
+    const int j = w * 32 + lane;
+    const uint32_t bc = bits_c[w], bn = bits_n[w];
+    const bool in = j < T;
+    const bool c = (bc >> lane) & 1u, n = (bn >> lane) & 1u;
+    if (in) crw[j] = int8_t(c ? 1 : (n ? -1 : 0));
+    if (c) {
+      const int pos = written + __popc(bc & ((1u << lane) - 1u));
+      if (pos < a.n_crit) idx[pos] = j;
+    }
+    written += __popc(bc);
+    if (lane == 0) {
+      const uint32_t valid = (T - w * 32) >= 32 ? 0xFFFFFFFFu : ((1u << (T - w * 32)) - 1u);
+      mrow[w] = ~(bc | bn) & valid;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ column CSR
 // For every key block j the ascending list of query blocks i with
 // cls[i][j] == +1 (offsets relative to the head), in three launches:
@@ -389,6 +641,53 @@ cudaError_t launch_classify(const Problem& p, const float* qbar, const float* kb
     classify_kernel<64><<<grid, 256, smem, s>>>(qbar, kbar, logits_in, logits_out, cls,
                                                 crit_idx, marg_bits, p.T, p.n_crit, p.n_negl,
                                                 p.scale);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_coarse_keys(const Problem& p, const float* kbar, float* kc, int G,
+                               cudaStream_t s) {
+  const int TG = (p.T + G - 1) / G;
+  coarse_keys_kernel<<<dim3(TG, p.BH), p.d, 0, s>>>(kbar, kc, p.T, TG, G, p.d);
+  return cudaGetLastError();
+}
+
+size_t hier_smem_bytes(const Problem& p, const HierCounts& h, bool compute, int rows) {
+  const int cap_hi = std::min(h.c_hi * h.G, p.T), cap_lo = std::min(h.c_lo * h.G, p.T);
+  size_t words = size_t(rows) * hier_warp_words(p.T, h.TG, cap_hi, cap_lo, h.c_hi, h.c_lo);
+  if (compute) words += size_t(rows) * p.d + size_t(kKTile) * (p.d + 4);
+  return words * 4;
+}
+
+cudaError_t launch_hier_classify(const Problem& p, const HierCounts& h, const float* qbar,
+                                 const float* kbar, const float* kc, const float* fine_in,
+                                 const float* coarse_in, float* fine_out, float* coarse_out,
+                                 int8_t* cls, int32_t* crit_idx, uint32_t* marg_bits, int* err,
+                                 cudaStream_t s) {
+  const bool compute = fine_in == nullptr;
+  int rows = 8;
+  while (rows > 1 && hier_smem_bytes(p, h, compute, rows) > kMaxSmemPerCta) rows /= 2;
+  const size_t smem = hier_smem_bytes(p, h, compute, rows);
+  if (smem > kMaxSmemPerCta) return cudaErrorInvalidConfiguration;
+  HierArgs a;
+  a.qbar = qbar; a.kbar = kbar; a.kc = kc; a.fine_in = fine_in; a.coarse_in = coarse_in;
+  a.fine_out = fine_out; a.coarse_out = coarse_out;
+  a.cls = cls; a.crit_idx = crit_idx; a.marg_bits = marg_bits; a.err = err;
+  a.T = p.T; a.TG = h.TG; a.G = h.G; a.c_hi = h.c_hi; a.c_lo = h.c_lo;
+  a.cap_hi = std::min(h.c_hi * h.G, p.T); a.cap_lo = std::min(h.c_lo * h.G, p.T);
+  a.n_crit = p.n_crit; a.n_negl = p.n_negl; a.rows = rows; a.scale = p.scale;
+  dim3 grid((p.T + rows - 1) / rows, p.BH);
+  cudaError_t e;
+  if (p.d == 128) {
+    e = cudaFuncSetAttribute(hier_classify_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    hier_classify_kernel<128><<<grid, 32 * rows, smem, s>>>(a);
+  } else {
+    e = cudaFuncSetAttribute(hier_classify_kernel<64>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    hier_classify_kernel<64><<<grid, 32 * rows, smem, s>>>(a);
   }
   return cudaGetLastError();
 }

@@ -55,6 +55,18 @@ cudaError_t launch_pool(const Problem& p, const void* q, const void* k, float* q
 cudaError_t launch_classify(const Problem& p, const float* qbar, const float* kbar,
                             const float* logits_in, float* logits_out, int8_t* cls,
                             int32_t* crit_idx, uint32_t* marg_bits, cudaStream_t s);
+// Hierarchical selection: super-block size and candidate counts (validated).
+struct HierCounts {
+  int G, TG, c_hi, c_lo;
+};
+constexpr size_t kMaxSmemPerCta = 227 * 1024;
+cudaError_t launch_coarse_keys(const Problem& p, const float* kbar, float* kc, int G,
+                               cudaStream_t s);
+cudaError_t launch_hier_classify(const Problem& p, const HierCounts& h, const float* qbar,
+                                 const float* kbar, const float* kc, const float* fine_in,
+                                 const float* coarse_in, float* fine_out, float* coarse_out,
+                                 int8_t* cls, int32_t* crit_idx, uint32_t* marg_bits, int* err,
+                                 cudaStream_t s);
 cudaError_t launch_crit_csr(const Problem& p, const int8_t* cls, int32_t* col_ptr,
                             int32_t* col_idx, cudaStream_t s);
 cudaError_t launch_expand_marginal(const Problem& p, const uint32_t* marg_bits,

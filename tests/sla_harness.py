@@ -90,3 +90,42 @@ class Run:
         if t.dtype == torch.bfloat16:
             t = t.float()
         return t.cpu().numpy().astype(dtype)
+
+
+def expected_csr(cls):
+    B, H, T, _ = cls.shape
+    n_crit = int((cls[0, 0, 0] == 1).sum())
+    ptr = np.zeros((B, H, T + 1), np.int64)
+    idx = np.zeros((B, H, T * max(n_crit, 1)), np.int64)
+    for b in range(B):
+        for h in range(H):
+            pos = 0
+            for j in range(T):
+                ptr[b, h, j] = pos
+                rows = np.nonzero(cls[b, h, :, j] == 1)[0]
+                idx[b, h, pos:pos + rows.size] = rows
+                pos += rows.size
+            ptr[b, h, T] = pos
+    return ptr, idx
+
+
+def check_mask_outputs(run, cls_ref):
+    """crit_idx, marg_bits and the column CSR must be consistent with cls."""
+    B, H, T, _ = cls_ref.shape
+    s = run.buf.sizes
+    cls = run.cls()
+    assert np.array_equal(cls, cls_ref)
+    if s.n_crit > 0:
+        crit = run.buf.crit_idx.cpu().numpy()[..., :s.n_crit]
+        exp = np.stack([np.nonzero(r == 1)[0] for r in cls_ref.reshape(-1, T)]).reshape(
+            B, H, T, s.n_crit)
+        assert np.array_equal(crit, exp)
+    bits = run.buf.marg_bits.cpu().numpy().view(np.uint32)
+    for j in range(T):
+        got = (bits[..., j // 32] >> np.uint32(j % 32)) & 1
+        assert np.array_equal(got.astype(bool), cls_ref[..., j] == 0)
+    ptr, idx = expected_csr(cls_ref)
+    assert np.array_equal(run.buf.crit_col_ptr.cpu().numpy(), ptr)
+    n = T * s.n_crit
+    if n:
+        assert np.array_equal(run.buf.crit_col_idx.cpu().numpy()[..., :n], idx[..., :n])

@@ -136,3 +136,44 @@ def test_gated_entry_points_reject_bad_gates_without_launching(L):
     assert bwd(None, good) == 1
     assert bwd(ctypes.byref(nan_gate), good) == 1
     assert bwd(ctypes.byref(ok_gate), good) == 3
+
+
+@pytest.mark.parametrize("T,k_h,k_l", [(16, 0.25, 0.25), (128, 0.05, 0.10), (512, 0.05, 0.10),
+                                       (1182, 0.10, 0.10), (1182, 0.025, 0.10), (10, 0.3, 0.3),
+                                       (7, 0.0, 0.0)])
+@pytest.mark.parametrize("group,top,bottom", [(2, 0, 0), (4, 0, 0), (16, 0, 0), (16, 12, 3),
+                                              (8, 1, 40), (64, 0, 0)])
+def test_hierarchy_counts_match_oracle(L, T, k_h, k_l, group, top, bottom):
+    import oracle
+    sh = slab.make_shape(1, 1, 64 * T, 64, 64, k_h, k_l)
+    n_h, n_l = oracle.block_counts(T, k_h, k_l)
+    got = slab.sla_hierarchy_counts(sh, slab.Hierarchy(group, top, bottom))
+    assert got == oracle.coarse_counts(T, n_h, n_l, group, top, bottom)
+
+
+def test_hierarchical_entry_points_reject_bad_arguments_without_launching(L):
+    sh = slab.make_shape(1, 2, 1024, 64, 64, 0.25, 0.25)
+    shp = ctypes.byref(sh)
+    good = 0x7f0000000000  # aligned, never dereferenced: every check fails first
+    m = slab.MaskStruct(good, good, good, good, good, None)
+    n = ctypes.c_int()
+    for bad in (slab.Hierarchy(1, 0, 0), slab.Hierarchy(4, -1, 0), slab.Hierarchy(4, 0, -2)):
+        assert L.sla_hierarchy_counts(shp, ctypes.byref(bad), ctypes.byref(n), ctypes.byref(n),
+                                      ctypes.byref(n)) == 1
+        assert L.sla_classify_hierarchical(shp, good, good, ctypes.byref(bad), ctypes.byref(m),
+                                           None, good, 1 << 40, None) == 1
+    ok = slab.Hierarchy(4, 0, 0)
+    assert L.sla_hierarchy_counts(shp, None, ctypes.byref(n), ctypes.byref(n),
+                                  ctypes.byref(n)) == 1
+    assert L.sla_classify_hierarchical(shp, None, good, ctypes.byref(ok), ctypes.byref(m), None,
+                                       good, 1 << 40, None) == 1
+    assert L.sla_classify_hierarchical(shp, good, good, ctypes.byref(ok), ctypes.byref(m),
+                                       good + 4, good, 1 << 40, None) == 1  # coarse misaligned
+    assert L.sla_classify_hierarchical(shp, good, good, ctypes.byref(ok), ctypes.byref(m), None,
+                                       good, 16, None) == 3
+    fs = lambda lg, co: L.sla_classify_hierarchical_from_scores(
+        shp, lg, co, ctypes.byref(ok), ctypes.byref(m), good, 16, None)
+    assert fs(good, None) == 1
+    assert fs(None, good) == 1
+    assert fs(good, good + 8) == 1
+    assert fs(good, good) == 3
