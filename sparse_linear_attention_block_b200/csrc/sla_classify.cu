@@ -73,91 +73,100 @@ __device__ __forceinline__ uint32_t ordered_bits(float x) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// The n-th element (n >= 1) of one row in the order (score desc, index asc),
-// or with `flip` in the reverse order (score asc, index desc), found by one
-// warp: an exact radix select on the order-preserving 32-bit score (four
-// 8-bit digits, most significant first, histogram in shared memory) followed
-// by one pass that breaks ties by index.  Returns the element's (possibly
-// complemented) ordered score v and its index jt; an element is at or before
-// it in the order iff its value is > v, or == v with index <= jt (>= jt when
-// flipped).
+// Selection thresholds.  For the order (score desc, index asc) a threshold
+// is the n-th element's ordered score v and index jt: an element is at or
+// before it iff its ordered score is > v, or == v with index <= jt.  For the
+// reverse order (score asc, index desc) v holds the complemented score and the
+// index test is >= jt.
 struct Threshold {
   uint32_t v;
   int jt;
 };
 
-__device__ Threshold warp_select(const float* row, int T, int n, bool flip, uint32_t* hist) {
+// Row of n <= 32 * KPL scores held by one warp in registers: element j sits in
+// lane j % 32, slot j / 32, as its ordered score; slots past n hold 0, below
+// every ordered score (the smallest, of -inf, is 0x007FFFFF).
+template <int KPL>
+__device__ __forceinline__ void load_keys(const float* row, int n, uint32_t (&key)[KPL]) {
+  const int lane = lane_id();
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int j = 32 * e + lane;
+    key[e] = j < n ? ordered_bits(row[j]) : 0u;
+  }
+}
+
+// Thresholds of the n_hi-th element in the order (score desc, index asc) and
+// the n_lo-th in the reverse order, computed together by one warp (a count of
+// 0 leaves its threshold unused).  Exact bisection on the 32-bit ordered
+// score: only the bits below the common prefix of the row's smallest and
+// largest score are searched, each step counting with one warp sum per side;
+// then one pass resolves equal scores by index.  No shared memory.
+template <int KPL>
+__device__ void select2(const uint32_t (&key)[KPL], int n, int n_hi, int n_lo, Threshold* th,
+                        Threshold* tl) {
   constexpr uint32_t kAll = 0xFFFFFFFFu;
   const int lane = lane_id();
-  uint32_t prefix = 0, mask = 0;
-  int need = n;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = lane; b < 256; b += 32) hist[b] = 0;
-    __syncwarp();
-    for (int j = lane; j < T; j += 32) {
-      uint32_t o = ordered_bits(row[j]);
-      if (flip) o = ~o;
-      if ((o & mask) == prefix) atomicAdd(&hist[(o >> shift) & 255u], 1u);
-    }
-    __syncwarp();
-    // lane l owns digits 255-8l down to 248-8l; scan from the top digit
-    uint32_t c[8];
-    int s = 0;
+  const int npad = 32 * KPL - n;  // zero slots: always <= any bound, never >= one
+  uint32_t lo = ~0u, hi = 0u;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      c[e] = hist[255 - 8 * lane - e];
-      s += int(c[e]);
-    }
-    int incl = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(kAll, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const int excl = incl - s;
-    const bool mine = excl < need && need <= incl;
-    const int src = __ffs(__ballot_sync(kAll, mine)) - 1;
-    int digit = 0, above = 0;
-    if (mine) {
-      int acc = excl;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (acc + int(c[e]) >= need) {
-          digit = 255 - 8 * lane - e;
-          above = acc;
-          break;
-        }
-        acc += int(c[e]);
-      }
-    }
-    digit = __shfl_sync(kAll, digit, src);
-    above = __shfl_sync(kAll, above, src);
-    prefix |= uint32_t(digit) << shift;
-    mask |= 255u << shift;
-    need -= above;
-    __syncwarp();
+  for (int e = 0; e < KPL; ++e) {
+    lo = min(lo, 32 * e + lane < n ? key[e] : ~0u);
+    hi = max(hi, key[e]);
   }
-  // ties on the score: the need-th equal element in index order
-  int jt = -1, seen = 0;
-  const int last = ((T - 1) / 32) * 32;
-  for (int step = 0; step <= last / 32 && jt < 0; ++step) {
-    const int j0 = flip ? last - 32 * step : 32 * step;
-    const int j = j0 + lane;
-    bool eq = false;
-    if (j < T) {
-      uint32_t o = ordered_bits(row[j]);
-      if (flip) o = ~o;
-      eq = o == prefix;
+  lo = __reduce_min_sync(kAll, lo);
+  hi = __reduce_max_sync(kAll, hi);
+  const uint32_t diff = lo ^ hi;
+  const int top = diff ? 31 - __clz(diff) : -1;  // highest bit that varies in the row
+  const uint32_t vary = top < 0 ? 0u : (top == 31 ? ~0u : (2u << top) - 1u);
+  // v: the largest value with #(key >= v) >= n_hi (the n_hi-th largest key);
+  // u: the smallest value with #(key <= u) >= n_lo (the n_lo-th smallest)
+  uint32_t v = hi & ~vary, u = lo | vary;
+  for (int b = top; b >= 0; --b) {
+    const uint32_t ch = v | (1u << b), cl = u & ~(1u << b);
+    int a = 0, c = 0;
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+      a += key[e] >= ch;
+      c += key[e] <= cl;
     }
-    uint32_t m = __ballot_sync(kAll, eq);
+    a = __reduce_add_sync(kAll, a);
+    c = __reduce_add_sync(kAll, c) - npad;
+    if (a >= n_hi) v = ch;
+    if (c >= n_lo) u = cl;
+  }
+  // equal scores: the needed one among them by index
+  int gt = 0, lt = 0;
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    gt += key[e] > v;
+    lt += key[e] < u;
+  }
+  const int need_hi = n_hi - __reduce_add_sync(kAll, gt);
+  const int need_lo = n_lo - (__reduce_add_sync(kAll, lt) - npad);
+  int jh = -1, jl = -1, seen_h = 0, seen_l = 0;
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    uint32_t m = __ballot_sync(kAll, key[e] == v);  // a zero slot never equals a score
     const int cnt = __popc(m);
-    if (seen + cnt >= need) {
-      for (int k = need - seen; k > 1; --k) m &= flip ? ~(1u << (31 - __clz(m))) : (m - 1);
-      jt = j0 + (flip ? 31 - __clz(m) : __ffs(m) - 1);
+    if (jh < 0 && seen_h + cnt >= need_hi) {
+      for (int r = need_hi - seen_h; r > 1; --r) m &= m - 1u;
+      jh = 32 * e + __ffs(int(m)) - 1;
     }
-    seen += cnt;
+    seen_h += cnt;
   }
-  return {prefix, jt};
+#pragma unroll
+  for (int e = KPL - 1; e >= 0; --e) {
+    uint32_t m = __ballot_sync(kAll, key[e] == u);
+    const int cnt = __popc(m);
+    if (jl < 0 && seen_l + cnt >= need_lo) {
+      for (int r = need_lo - seen_l; r > 1; --r) m &= ~(1u << (31 - __clz(m)));
+      jl = 32 * e + 31 - __clz(m);
+    }
+    seen_l += cnt;
+  }
+  *th = Threshold{v, jh};
+  *tl = Threshold{~u, jl};
 }
 
 __device__ __forceinline__ bool before_or_at(uint32_t o, int j, Threshold t, bool flip) {
@@ -169,8 +178,9 @@ constexpr int kRowsPerCta = 8;  // one warp per query-block row
 constexpr int kKTile = 32;      // pooled keys staged per step
 
 // One CTA per 8 rows of one head.  When `logits_in` is null the pooled logits
-// are computed from qbar/kbar (fp32), otherwise read from it.
-template <int D>
+// are computed from qbar/kbar (fp32), otherwise read from it.  KPL: row
+// scores per lane in the selection (T <= 32 * KPL).
+template <int D, int KPL>
 __global__ void __launch_bounds__(256) classify_kernel(
     const float* __restrict__ qbar, const float* __restrict__ kbar,
     const float* __restrict__ logits_in, float* __restrict__ logits_out,
@@ -223,9 +233,12 @@ __global__ void __launch_bounds__(256) classify_kernel(
   }
   if (!row_ok) return;
 
-  uint32_t* hist = reinterpret_cast<uint32_t*>(sk + kKTile * kStride) + warp * 256;
-  const Threshold th = n_crit > 0 ? warp_select(row, T, n_crit, false, hist) : Threshold{0, -1};
-  const Threshold tl = n_negl > 0 ? warp_select(row, T, n_negl, true, hist) : Threshold{0, -1};
+  Threshold th{0, -1}, tl{0, -1};
+  if (n_crit > 0 || n_negl > 0) {
+    uint32_t key[KPL];
+    load_keys<KPL>(row, T, key);
+    select2<KPL>(key, T, n_crit, n_negl, &th, &tl);
+  }
   const size_t rbase = size_t(bh) * T + i;
   int8_t* crow = cls + rbase * T;
   int32_t* idx = crit_idx + rbase * n_crit;
@@ -288,15 +301,16 @@ struct HierArgs {
   int32_t* crit_idx;
   uint32_t* marg_bits;
   int* err;
-  int T, TG, G, c_hi, c_lo, cap_hi, cap_lo, n_crit, n_negl, rows;
+  int T, TG, G, c_hi, c_lo, cap_hi, cap_lo, n_crit, n_negl, rows, BH;
   float scale;
+  size_t smem;
 };
 
 // Per-warp shared scratch, in floats / words.
 __host__ __device__ inline int hier_warp_words(int T, int TG, int cap_hi, int cap_lo, int c_hi,
                                                int c_lo) {
   const int W = (T + 31) / 32;
-  return TG + cap_hi + cap_lo + c_hi + c_lo + 256 + 2 * W;
+  return TG + cap_hi + cap_lo + c_hi + c_lo + 2 * W;
 }
 
 // Block index of candidate position p of a list of super-blocks (ascending).
@@ -358,7 +372,8 @@ __device__ __forceinline__ void mark_selected(const float* cand, const int* list
 }
 
 // One warp per query-block row, `rows` rows per CTA (blockDim = 32 * rows).
-template <int D>
+// KPL: entries per lane in the selections (TG, cap_hi, cap_lo <= 32 * KPL).
+template <int D, int KPL>
 __global__ void __launch_bounds__(256) hier_classify_kernel(const HierArgs a) {
   extern __shared__ __align__(16) float smem[];
   constexpr int kStride = D + 4;
@@ -375,8 +390,7 @@ __global__ void __launch_bounds__(256) hier_classify_kernel(const HierArgs a) {
   float* cand = crow + TG;                           // [cap_hi] then [cap_lo]
   int* list_hi = reinterpret_cast<int*>(cand + a.cap_hi + a.cap_lo);
   int* list_lo = list_hi + a.c_hi;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(list_lo + a.c_lo);
-  uint32_t* bits_c = hist + 256;
+  uint32_t* bits_c = reinterpret_cast<uint32_t*>(list_lo + a.c_lo);
   uint32_t* bits_n = bits_c + W;
 
   // ---- coarse scores sc_iJ (all warps take part in the staging)
@@ -415,8 +429,12 @@ __global__ void __launch_bounds__(256) hier_classify_kernel(const HierArgs a) {
   if (!row_ok) return;
 
   // ---- candidate super-blocks, ascending
-  const Threshold thc = a.c_hi > 0 ? warp_select(crow, TG, a.c_hi, false, hist) : Threshold{0, -1};
-  const Threshold tlc = a.c_lo > 0 ? warp_select(crow, TG, a.c_lo, true, hist) : Threshold{0, -1};
+  Threshold thc, tlc;
+  {
+    uint32_t key[KPL];
+    load_keys<KPL>(crow, TG, key);
+    select2<KPL>(key, TG, a.c_hi, a.c_lo, &thc, &tlc);
+  }
   int nh = 0, nl = 0;
   for (int J0 = 0; J0 < TG; J0 += 32) {
     const int J = J0 + lane;
@@ -470,11 +488,17 @@ __global__ void __launch_bounds__(256) hier_classify_kernel(const HierArgs a) {
 
   // ---- exact selection inside the candidates (position order = block order)
   if (a.n_crit > 0) {
-    const Threshold th = warp_select(cand, nb_hi, a.n_crit, false, hist);
+    uint32_t key[KPL];
+    Threshold th, unused;
+    load_keys<KPL>(cand, nb_hi, key);
+    select2<KPL>(key, nb_hi, a.n_crit, 0, &th, &unused);
     mark_selected(cand, list_hi, nb_hi, G, th, false, bits_c);
   }
   if (a.n_negl > 0) {
-    const Threshold tl = warp_select(cand_lo, nb_lo, a.n_negl, true, hist);
+    uint32_t key[KPL];
+    Threshold tl, unused;
+    load_keys<KPL>(cand_lo, nb_lo, key);
+    select2<KPL>(key, nb_lo, 0, a.n_negl, &unused, &tl);
     mark_selected(cand_lo, list_lo, nb_lo, G, tl, true, bits_n);
   }
   __syncwarp();
@@ -506,21 +530,36 @@ __global__ void __launch_bounds__(256) hier_classify_kernel(const HierArgs a) {
 // ------------------------------------------------------------------ column CSR
 // For every key block j the ascending list of query blocks i with
 // cls[i][j] == +1 (offsets relative to the head), in three launches:
-//   csr_count_kernel  one warp per column: count -> col_ptr[j+1]
+//   csr_count_kernel  count -> col_ptr[j+1]
 //   csr_scan_kernel   one CTA per head: inclusive scan of col_ptr[1..T] in place
-//   csr_fill_kernel   one warp per column: rows in ascending order by ballots
+//   csr_fill_kernel   rows in ascending order
+// Count and fill: one CTA per 32 key blocks, lane = key block, so each row
+// step is one coalesced 32-byte read of cls; warp w scans the contiguous row
+// range [w*T/8, (w+1)*T/8), and the fill offsets each warp by the hits of the
+// warps before it, which keeps every column's list ascending.
 constexpr int kCsrWarps = 8;
+
+__device__ __forceinline__ int csr_count_rows(const int8_t* c, int T, int i0, int i1) {
+  int cnt = 0;
+#pragma unroll 8
+  for (int i = i0; i < i1; ++i) cnt += c[size_t(i) * T] == 1;
+  return cnt;
+}
 
 __global__ void __launch_bounds__(256) csr_count_kernel(const int8_t* __restrict__ cls,
                                                         int32_t* __restrict__ col_ptr, int T) {
-  const int bh = blockIdx.y, j = blockIdx.x * kCsrWarps + threadIdx.x / 32, lane = lane_id();
-  if (j >= T) return;
-  const int8_t* c = cls + size_t(bh) * T * T + j;
-  int cnt = 0;
-#pragma unroll 4
-  for (int i = lane; i < T; i += 32) cnt += c[size_t(i) * T] == 1;
-  cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-  if (lane == 0) col_ptr[size_t(bh) * (T + 1) + j + 1] = cnt;
+  __shared__ int part[kCsrWarps][32];
+  const int bh = blockIdx.y, w = threadIdx.x / 32, lane = lane_id();
+  const int j = blockIdx.x * 32 + lane;
+  const int i0 = w * T / kCsrWarps, i1 = (w + 1) * T / kCsrWarps;
+  part[w][lane] = j < T ? csr_count_rows(cls + size_t(bh) * T * T + j, T, i0, i1) : 0;
+  __syncthreads();
+  if (w == 0 && j < T) {
+    int cnt = 0;
+#pragma unroll
+    for (int x = 0; x < kCsrWarps; ++x) cnt += part[x][lane];
+    col_ptr[size_t(bh) * (T + 1) + j + 1] = cnt;
+  }
 }
 
 __global__ void __launch_bounds__(1024) csr_scan_kernel(int32_t* __restrict__ col_ptr, int T) {
@@ -565,19 +604,24 @@ __global__ void __launch_bounds__(256) csr_fill_kernel(const int8_t* __restrict_
                                                        const int32_t* __restrict__ col_ptr,
                                                        int32_t* __restrict__ col_idx, int T,
                                                        int n_crit) {
-  const int bh = blockIdx.y, j = blockIdx.x * kCsrWarps + threadIdx.x / 32, lane = lane_id();
-  if (j >= T) return;
+  __shared__ int part[kCsrWarps][32];
+  const int bh = blockIdx.y, w = threadIdx.x / 32, lane = lane_id();
+  const int j = blockIdx.x * 32 + lane;
+  const int i0 = w * T / kCsrWarps, i1 = (w + 1) * T / kCsrWarps;
   const int8_t* c = cls + size_t(bh) * T * T + j;
+  part[w][lane] = j < T ? csr_count_rows(c, T, i0, i1) : 0;
+  __syncthreads();
+  if (j >= T) return;
+  int pos = col_ptr[size_t(bh) * (T + 1) + j];
+  for (int x = 0; x < w; ++x) pos += part[x][lane];
   int32_t* out = col_idx + size_t(bh) * T * n_crit;
   const int cap = T * n_crit;
-  int pos = col_ptr[size_t(bh) * (T + 1) + j];
-  for (int i0 = 0; i0 < T; i0 += 32) {
-    const int i = i0 + lane;
-    const bool hit = i < T && c[size_t(i) * T] == 1;
-    const uint32_t m = __ballot_sync(0xFFFFFFFFu, hit);
-    const int at = pos + __popc(m & ((1u << lane) - 1u));
-    if (hit && at < cap) out[at] = i;
-    pos += __popc(m);
+#pragma unroll 8
+  for (int i = i0; i < i1; ++i) {
+    if (c[size_t(i) * T] == 1) {
+      if (pos < cap) out[pos] = i;
+      ++pos;
+    }
   }
 }
 
@@ -619,30 +663,52 @@ cudaError_t launch_pool(const Problem& p, const void* q, const void* k, float* q
   return cudaGetLastError();
 }
 
+// Scores per lane of a warp's selection (a row of up to 32 * KPL entries):
+// the smallest instantiated KPL that holds n entries.
+int kpl_for(int n) {
+  for (int k : {4, 8, 16, 24, 40, 64, 128})
+    if (32 * k >= n) return k;
+  return 0;
+}
+
+#define SLA_KPL_SWITCH(kpl, CALL)                 \
+  switch (kpl) {                                  \
+    case 4: return CALL(4);                       \
+    case 8: return CALL(8);                       \
+    case 16: return CALL(16);                     \
+    case 24: return CALL(24);                     \
+    case 40: return CALL(40);                     \
+    case 64: return CALL(64);                     \
+    case 128: return CALL(128);                   \
+    default: return cudaErrorInvalidValue;        \
+  }
+
+template <int D, int KPL>
+cudaError_t launch_classify_t(const Problem& p, size_t smem, const float* qbar, const float* kbar,
+                              const float* logits_in, float* logits_out, int8_t* cls,
+                              int32_t* crit_idx, uint32_t* marg_bits, cudaStream_t s) {
+  const cudaError_t e = cudaFuncSetAttribute(
+      classify_kernel<D, KPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.T + kRowsPerCta - 1) / kRowsPerCta, p.BH);
+  classify_kernel<D, KPL><<<grid, 256, smem, s>>>(qbar, kbar, logits_in, logits_out, cls,
+                                                  crit_idx, marg_bits, p.T, p.n_crit, p.n_negl,
+                                                  p.scale);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_classify(const Problem& p, const float* qbar, const float* kbar,
                             const float* logits_in, float* logits_out, int8_t* cls,
                             int32_t* crit_idx, uint32_t* marg_bits, cudaStream_t s) {
-  dim3 grid((p.T + kRowsPerCta - 1) / kRowsPerCta, p.BH);
   const size_t smem =
-      sizeof(float) * (size_t(kRowsPerCta) * p.T + kRowsPerCta * p.d + kKTile * (p.d + 4)) +
-      sizeof(uint32_t) * kRowsPerCta * 256;  // per-warp radix histograms
-  cudaError_t e;
-  if (p.d == 128) {
-    e = cudaFuncSetAttribute(classify_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem));
-    if (e != cudaSuccess) return e;
-    classify_kernel<128><<<grid, 256, smem, s>>>(qbar, kbar, logits_in, logits_out, cls,
-                                                 crit_idx, marg_bits, p.T, p.n_crit, p.n_negl,
-                                                 p.scale);
-  } else {
-    e = cudaFuncSetAttribute(classify_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem));
-    if (e != cudaSuccess) return e;
-    classify_kernel<64><<<grid, 256, smem, s>>>(qbar, kbar, logits_in, logits_out, cls,
-                                                crit_idx, marg_bits, p.T, p.n_crit, p.n_negl,
-                                                p.scale);
-  }
-  return cudaGetLastError();
+      sizeof(float) * (size_t(kRowsPerCta) * p.T + kRowsPerCta * p.d + kKTile * (p.d + 4));
+#define SLA_FLAT(K)                                                                         \
+  (p.d == 128 ? launch_classify_t<128, K>(p, smem, qbar, kbar, logits_in, logits_out, cls, \
+                                          crit_idx, marg_bits, s)                          \
+              : launch_classify_t<64, K>(p, smem, qbar, kbar, logits_in, logits_out, cls,  \
+                                         crit_idx, marg_bits, s))
+  SLA_KPL_SWITCH(kpl_for(p.T), SLA_FLAT)
+#undef SLA_FLAT
 }
 
 cudaError_t launch_coarse_keys(const Problem& p, const float* kbar, float* kc, int G,
@@ -657,6 +723,16 @@ size_t hier_smem_bytes(const Problem& p, const HierCounts& h, bool compute, int 
   size_t words = size_t(rows) * hier_warp_words(p.T, h.TG, cap_hi, cap_lo, h.c_hi, h.c_lo);
   if (compute) words += size_t(rows) * p.d + size_t(kKTile) * (p.d + 4);
   return words * 4;
+}
+
+template <int D, int KPL>
+cudaError_t launch_hier_t(const HierArgs& a, cudaStream_t s) {
+  const cudaError_t e = cudaFuncSetAttribute(
+      hier_classify_kernel<D, KPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(a.smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.T + a.rows - 1) / a.rows, a.BH);
+  hier_classify_kernel<D, KPL><<<grid, 32 * a.rows, a.smem, s>>>(a);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_hier_classify(const Problem& p, const HierCounts& h, const float* qbar,
@@ -675,26 +751,16 @@ cudaError_t launch_hier_classify(const Problem& p, const HierCounts& h, const fl
   a.cls = cls; a.crit_idx = crit_idx; a.marg_bits = marg_bits; a.err = err;
   a.T = p.T; a.TG = h.TG; a.G = h.G; a.c_hi = h.c_hi; a.c_lo = h.c_lo;
   a.cap_hi = std::min(h.c_hi * h.G, p.T); a.cap_lo = std::min(h.c_lo * h.G, p.T);
-  a.n_crit = p.n_crit; a.n_negl = p.n_negl; a.rows = rows; a.scale = p.scale;
-  dim3 grid((p.T + rows - 1) / rows, p.BH);
-  cudaError_t e;
-  if (p.d == 128) {
-    e = cudaFuncSetAttribute(hier_classify_kernel<128>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    hier_classify_kernel<128><<<grid, 32 * rows, smem, s>>>(a);
-  } else {
-    e = cudaFuncSetAttribute(hier_classify_kernel<64>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    hier_classify_kernel<64><<<grid, 32 * rows, smem, s>>>(a);
-  }
-  return cudaGetLastError();
+  a.n_crit = p.n_crit; a.n_negl = p.n_negl; a.rows = rows; a.scale = p.scale; a.BH = p.BH;
+  a.smem = smem;
+#define SLA_HIER(K) (p.d == 128 ? launch_hier_t<128, K>(a, s) : launch_hier_t<64, K>(a, s))
+  SLA_KPL_SWITCH(kpl_for(std::max(h.TG, std::max(a.cap_hi, a.cap_lo))), SLA_HIER)
+#undef SLA_HIER
 }
 
 cudaError_t launch_crit_csr(const Problem& p, const int8_t* cls, int32_t* col_ptr,
                             int32_t* col_idx, cudaStream_t s) {
-  dim3 grid((p.T + kCsrWarps - 1) / kCsrWarps, p.BH);
+  dim3 grid((p.T + 31) / 32, p.BH);
   csr_count_kernel<<<grid, 32 * kCsrWarps, 0, s>>>(cls, col_ptr, p.T);
   csr_scan_kernel<<<p.BH, 1024, 0, s>>>(col_ptr, p.T);
   if (p.n_crit > 0) csr_fill_kernel<<<grid, 32 * kCsrWarps, 0, s>>>(cls, col_ptr, col_idx, p.T, p.n_crit);
