@@ -21,6 +21,8 @@
 // (the combination O = O_s + (phi(Q) H_i / den) W_proj is in sla_fwd_linear.cu)
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "sla_internal.h"
 #include "sla_ptx.cuh"
 #include "sla_tile.cuh"
@@ -158,36 +160,50 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
 // marginal matrix [Tp x Tp] (K-major), B the per-block summary rows [T x W]
 // as bf16 hi/lo planes (MN-major); C (fp32 in TMEM) is written back as bf16
 // hi/lo planes [T x W] (C = hi + lo), the operand format of its consumers.
-// One CTA covers up to 512 rows (four 128 x 128 accumulators, all of TMEM)
-// of one 128-column slice, so each B slice is read once and A once per
-// slice; K in steps of 64 through a 2-stage TMA ring.  Warp 0 = TMA
-// producer, warp 1 = MMA issuer, all 4 warps = epilogue.
-constexpr int kAggBN = 128, kAggBK = 64, kAggStages = 2, kAggMT = 4;
+// Persistent and warp-specialised: a work tile is 256 rows (two 128-row
+// M tiles) x 128 columns of one head; tiles of the same column slice are
+// adjacent in the schedule, so the second M half finds its B slice in L2.
+// Warp 0 = TMA producer over a 3-stage ring (K in steps of 64), warp 1 =
+// MMA issuer into one of two TMEM accumulator buffers (256 columns each),
+// warps 2-5 = epilogue (TMEM -> hi/lo planes) of the previous tile while the
+// next one is multiplied.
+constexpr int kAggBN = 128, kAggBK = 64, kAggStages = 3, kAggMT = 2;
 constexpr int kAggA = 128 * kAggBK * 2;        // 16 KB per 128-row tile
 constexpr int kAggB = kAggBK * kAggBN * 2;     // 16 KB per plane
 constexpr int kAggStageBytes = kAggMT * kAggA + 2 * kAggB;
+constexpr int kAggThreads = 192;
 
-__global__ void __launch_bounds__(128, 1) agg_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
-                                                          const __grid_constant__ CUtensorMap tm_bh,
-                                                          const __grid_constant__ CUtensorMap tm_bl,
-                                                          __nv_bfloat16* __restrict__ out_hi,
-                                                          __nv_bfloat16* __restrict__ out_lo,
-                                                          int T, int Tp, int NN, int* err) {
+__global__ void __launch_bounds__(kAggThreads, 1) agg_gemm_kernel(
+    const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_bh,
+    const __grid_constant__ CUtensorMap tm_bl, __nv_bfloat16* __restrict__ out_hi,
+    __nv_bfloat16* __restrict__ out_lo, int T, int Tp, int NN, int BH, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = align_smem_1024(smem_raw);
-  __shared__ uint64_t full[kAggStages], empty[kAggStages], acc_bar;
+  __shared__ uint64_t full[kAggStages], empty[kAggStages], acc_full[2], acc_empty[2], fin;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
-  const int mg = blockIdx.x, nt = blockIdx.y, bh = blockIdx.z;
   const int warp = threadIdx.x / 32;
   const int nk = Tp / kAggBK;
-  const int nmt = min(kAggMT, Tp / 128 - mg * kAggMT);  // 128-row tiles of this CTA
+  const int nmg = (Tp / 128 + kAggMT - 1) / kAggMT;  // 256-row groups
+  const int nnt = (NN + kAggBN - 1) / kAggBN;         // 128-column slices
+  const int ntiles = BH * nnt * nmg;
+  const int nloc = ntiles > int(blockIdx.x) ? (ntiles - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
+  auto tile_of = [&](int n, int& mg, int& nt, int& bh) {
+    const int t = int(blockIdx.x) + n * int(gridDim.x);
+    mg = t % nmg;
+    nt = (t / nmg) % nnt;
+    bh = t / (nmg * nnt);
+  };
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAggStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(&acc_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(&fin, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -196,81 +212,117 @@ __global__ void __launch_bounds__(128, 1) agg_gemm_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
+  int it = 0;  // K steps issued (producer) or consumed (MMA issuer)
 
   if (warp == 0 && lane_id() == 0) {
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_bh);
     tma_prefetch_desc(&tm_bl);
-    int issued = 0;
-    for (int kt = 0; kt < nk; ++kt) {
-      const int s = kt % kAggStages;
-      if (kt >= kAggStages &&
-          !mbar_wait(&empty[s], ((kt / kAggStages) + 1) & 1, err, &abort_flag))
-        break;
-      uint8_t* sa = base + s * kAggStageBytes;
-      uint8_t* sb = sa + kAggMT * kAggA;
-      mbar_arrive_expect_tx(&full[s], nmt * kAggA + 2 * kAggB);
-      for (int m = 0; m < nmt; ++m)
-        tma_load_3d(sa + m * kAggA, &full[s], &tm_a, kt * kAggBK, (mg * kAggMT + m) * 128, bh);
-      for (int c = 0; c < 2; ++c) {
-        tma_load_3d(sb + c * 8192, &full[s], &tm_bh, nt * kAggBN + c * 64, kt * kAggBK, bh);
-        tma_load_3d(sb + kAggB + c * 8192, &full[s], &tm_bl, nt * kAggBN + c * 64, kt * kAggBK, bh);
-      }
-      ++issued;
-    }
-    if (abort_flag)
-      for (int kt = (issued > kAggStages ? issued - kAggStages : 0); kt < issued; ++kt)
-        mbar_wait(&full[kt % kAggStages], (kt / kAggStages) & 1, nullptr, nullptr);
-  } else if (warp == 1 && lane_id() == 0) {
-    constexpr uint32_t idesc = idesc_bf16(128, kAggBN, 0, 1);
-    for (int kt = 0; kt < nk; ++kt) {
-      const int s = kt % kAggStages;
-      if (!mbar_wait(&full[s], (kt / kAggStages) & 1, err, &abort_flag)) break;
-      tc_fence_after();
-      const uint32_t sa = smem_u32(base + s * kAggStageBytes);
-      const uint64_t bhd = desc_mnmajor_base(sa + kAggMT * kAggA, kAggBK);
-      const uint64_t bld = desc_mnmajor_base(sa + kAggMT * kAggA + kAggB, kAggBK);
-      for (int m = 0; m < nmt; ++m) {
-        const uint64_t ad = desc_kmajor_base(sa + m * kAggA);
-#pragma unroll
-        for (int ks = 0; ks < kAggBK / 16; ++ks) {
-          const uint64_t a = desc_advance(ad, kmajor_step_bytes(128, ks));
-          mma_ss(tmem + m * kAggBN, a, desc_advance(bhd, mnmajor_step_bytes(ks)), idesc,
-                 (kt | ks) != 0);
-          mma_ss(tmem + m * kAggBN, a, desc_advance(bld, mnmajor_step_bytes(ks)), idesc, 1);
+    bool ok = true;
+    for (int n = 0; n < nloc && ok; ++n) {
+      int mg, nt, bh;
+      tile_of(n, mg, nt, bh);
+      const int nmt = min(kAggMT, Tp / 128 - mg * kAggMT);
+      for (int kt = 0; kt < nk; ++kt, ++it) {
+        const int s = it % kAggStages;
+        if (it >= kAggStages &&
+            !mbar_wait(&empty[s], ((it / kAggStages) + 1) & 1, err, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sa = base + s * kAggStageBytes;
+        uint8_t* sb = sa + kAggMT * kAggA;
+        mbar_arrive_expect_tx(&full[s], nmt * kAggA + 2 * kAggB);
+        for (int m = 0; m < nmt; ++m)
+          tma_load_3d(sa + m * kAggA, &full[s], &tm_a, kt * kAggBK, (mg * kAggMT + m) * 128, bh);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(sb + c * 8192, &full[s], &tm_bh, nt * kAggBN + c * 64, kt * kAggBK, bh);
+          tma_load_3d(sb + kAggB + c * 8192, &full[s], &tm_bl, nt * kAggBN + c * 64,
+                      kt * kAggBK, bh);
         }
       }
-      mma_commit(&empty[s]);
     }
-    mma_commit(&acc_bar);
-  }
-  __syncwarp();
-  const bool ok = mbar_wait(&acc_bar, 0, err, &abort_flag);
-  tc_fence_after();
-  if (ok) {
-    for (int m = 0; m < nmt; ++m) {
-      const int i = (mg * kAggMT + m) * 128 + warp * 32 + lane_id();
-      const size_t o = (size_t(bh) * T + i) * NN + size_t(nt) * kAggBN;
+  } else if (warp == 1 && lane_id() == 0) {
+    constexpr uint32_t idesc = idesc_bf16(128, kAggBN, 0, 1);
+    bool ok = true;
+    for (int n = 0; n < nloc && ok; ++n) {
+      int mg, nt, bh;
+      tile_of(n, mg, nt, bh);
+      const int nmt = min(kAggMT, Tp / 128 - mg * kAggMT);
+      const int buf = n & 1;
+      if (n >= 2 && !mbar_wait(&acc_empty[buf], ((n >> 1) + 1) & 1, err, &abort_flag)) break;
+      tc_fence_after();
+      const uint32_t acc = tmem + uint32_t(buf) * (kAggMT * kAggBN);
+      for (int kt = 0; kt < nk; ++kt, ++it) {
+        const int s = it % kAggStages;
+        if (!mbar_wait(&full[s], (it / kAggStages) & 1, err, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(base + s * kAggStageBytes);
+        const uint64_t bhd = desc_mnmajor_base(sa + kAggMT * kAggA, kAggBK);
+        const uint64_t bld = desc_mnmajor_base(sa + kAggMT * kAggA + kAggB, kAggBK);
+        for (int m = 0; m < nmt; ++m) {
+          const uint64_t ad = desc_kmajor_base(sa + m * kAggA);
+#pragma unroll
+          for (int ks = 0; ks < kAggBK / 16; ++ks) {
+            const uint64_t av = desc_advance(ad, kmajor_step_bytes(128, ks));
+            mma_ss(acc + m * kAggBN, av, desc_advance(bhd, mnmajor_step_bytes(ks)), idesc,
+                   (kt | ks) != 0);
+            mma_ss(acc + m * kAggBN, av, desc_advance(bld, mnmajor_step_bytes(ks)), idesc, 1);
+          }
+        }
+        mma_commit(&empty[s]);
+      }
+      if (ok) mma_commit(&acc_full[buf]);
+    }
+    // every product issued has finished before TMEM is released
+    mma_commit(&fin);
+    mbar_wait(&fin, 0, nullptr, nullptr);
+  } else if (warp >= 2) {
+    const int q = warp % 4;  // the TMEM lane quadrant this warp may access
+    for (int n = 0; n < nloc; ++n) {
+      int mg, nt, bh;
+      tile_of(n, mg, nt, bh);
+      const int nmt = min(kAggMT, Tp / 128 - mg * kAggMT);
+      const int buf = n & 1;
+      if (!mbar_wait(&acc_full[buf], (n >> 1) & 1, err, &abort_flag)) break;
+      tc_fence_after();
+      for (int m = 0; m < nmt; ++m) {
+        const int i = (mg * kAggMT + m) * 128 + q * 32 + lane_id();
+        const size_t o = (size_t(bh) * T + i) * NN + size_t(nt) * kAggBN;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kAggBN; c0 += 32) {
-        float vals[32];
-        tmem_ld32(tmem_addr(tmem, warp * 32, m * kAggBN + c0), vals);
-        tmem_ld_wait();
-        if (i < T && nt * kAggBN + c0 < NN) {  // NN is a multiple of 32
+        for (int c0 = 0; c0 < kAggBN; c0 += 32) {
+          float vals[32];
+          tmem_ld32(tmem_addr(tmem, q * 32, buf * (kAggMT * kAggBN) + m * kAggBN + c0), vals);
+          tmem_ld_wait();
+          if (i < T && nt * kAggBN + c0 < NN) {  // NN is a multiple of 32
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint32_t h[4], l[4];
+            for (int e = 0; e < 32; e += 8) {
+              uint32_t h[4], l[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) split2(vals[e + 2 * u], vals[e + 2 * u + 1], h[u], l[u]);
-            *reinterpret_cast<uint4*>(out_hi + o + c0 + e) = make_uint4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<uint4*>(out_lo + o + c0 + e) = make_uint4(l[0], l[1], l[2], l[3]);
+              for (int u = 0; u < 4; ++u)
+                split2(vals[e + 2 * u], vals[e + 2 * u + 1], h[u], l[u]);
+              *reinterpret_cast<uint4*>(out_hi + o + c0 + e) = make_uint4(h[0], h[1], h[2], h[3]);
+              *reinterpret_cast<uint4*>(out_lo + o + c0 + e) = make_uint4(l[0], l[1], l[2], l[3]);
+            }
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane_id() == 0) mbar_arrive(&acc_empty[buf]);
     }
   }
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  if (abort_flag && warp == 0 && lane_id() == 0)  // copies still in flight land first
+    for (int j = (it > kAggStages ? it - kAggStages : 0); j < it; ++j)
+      mbar_wait(&full[j % kAggStages], (j / kAggStages) & 1, nullptr, nullptr);
+  __syncwarp();
   if (warp == 0) tmem_free(tmem, 512);
 }
 
@@ -314,8 +366,13 @@ cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
   const size_t smem = 1024 + kAggStages * kAggStageBytes;
   cudaError_t e = set_smem(agg_gemm_kernel, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.Tp / 128 + kAggMT - 1) / kAggMT, (NN + kAggBN - 1) / kAggBN, p.BH);
-  agg_gemm_kernel<<<grid, 128, smem, s>>>(ta, tbh, tbl, out_hi, out_lo, p.T, p.Tp, NN, err);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorUnknown;
+  const int ntiles = p.BH * ((NN + kAggBN - 1) / kAggBN) * ((p.Tp / 128 + kAggMT - 1) / kAggMT);
+  agg_gemm_kernel<<<std::min(ntiles, sms), kAggThreads, smem, s>>>(ta, tbh, tbl, out_hi, out_lo,
+                                                                  p.T, p.Tp, NN, p.BH, err);
   return cudaGetLastError();
 }
 
