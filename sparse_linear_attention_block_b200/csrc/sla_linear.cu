@@ -171,7 +171,8 @@ constexpr int kAggBN = 128, kAggBK = 64, kAggStages = 3, kAggMT = 2;
 constexpr int kAggA = 128 * kAggBK * 2;        // 16 KB per 128-row tile
 constexpr int kAggB = kAggBK * kAggBN * 2;     // 16 KB per plane
 constexpr int kAggStageBytes = kAggMT * kAggA + 2 * kAggB;
-constexpr int kAggThreads = 192;
+constexpr int kAggEpiWarps = 4;
+constexpr int kAggThreads = 64 + 32 * kAggEpiWarps;
 
 __global__ void __launch_bounds__(kAggThreads, 1) agg_gemm_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_bh,
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(kAggThreads, 1) agg_gemm_kernel(
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+      mbar_init(&acc_empty[b], kAggEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(&fin, 1);
     abort_flag = 0;
@@ -281,7 +282,7 @@ __global__ void __launch_bounds__(kAggThreads, 1) agg_gemm_kernel(
     mma_commit(&fin);
     mbar_wait(&fin, 0, nullptr, nullptr);
   } else if (warp >= 2) {
-    const int q = warp % 4;  // the TMEM lane quadrant this warp may access
+    const int q = warp % 4;                          // the TMEM lane quadrant this warp may access
     for (int n = 0; n < nloc; ++n) {
       int mg, nt, bh;
       tile_of(n, mg, nt, bh);
@@ -291,21 +292,28 @@ __global__ void __launch_bounds__(kAggThreads, 1) agg_gemm_kernel(
       tc_fence_after();
       for (int m = 0; m < nmt; ++m) {
         const int i = (mg * kAggMT + m) * 128 + q * 32 + lane_id();
-        const size_t o = (size_t(bh) * T + i) * NN + size_t(nt) * kAggBN;
 #pragma unroll 1
-        for (int c0 = 0; c0 < kAggBN; c0 += 32) {
-          float vals[32];
-          tmem_ld32(tmem_addr(tmem, q * 32, buf * (kAggMT * kAggBN) + m * kAggBN + c0), vals);
+        for (int cbase = 0; cbase < kAggBN; cbase += 64) {
+          const size_t o = (size_t(bh) * T + i) * NN + size_t(nt) * kAggBN + cbase;
+          const uint32_t col = buf * (kAggMT * kAggBN) + m * kAggBN + cbase;
+          float vals[2][32];
+          tmem_ld32(tmem_addr(tmem, q * 32, col), vals[0]);
+          tmem_ld32(tmem_addr(tmem, q * 32, col + 32), vals[1]);
           tmem_ld_wait();
-          if (i < T && nt * kAggBN + c0 < NN) {  // NN is a multiple of 32
 #pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              uint32_t h[4], l[4];
+          for (int c = 0; c < 2; ++c) {
+            if (i < T && nt * kAggBN + cbase + 32 * c < NN) {  // NN is a multiple of 32
 #pragma unroll
-              for (int u = 0; u < 4; ++u)
-                split2(vals[e + 2 * u], vals[e + 2 * u + 1], h[u], l[u]);
-              *reinterpret_cast<uint4*>(out_hi + o + c0 + e) = make_uint4(h[0], h[1], h[2], h[3]);
-              *reinterpret_cast<uint4*>(out_lo + o + c0 + e) = make_uint4(l[0], l[1], l[2], l[3]);
+              for (int e = 0; e < 32; e += 8) {
+                uint32_t h[4], l[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  split2(vals[c][e + 2 * u], vals[c][e + 2 * u + 1], h[u], l[u]);
+                *reinterpret_cast<uint4*>(out_hi + o + 32 * c + e) =
+                    make_uint4(h[0], h[1], h[2], h[3]);
+                *reinterpret_cast<uint4*>(out_lo + o + 32 * c + e) =
+                    make_uint4(l[0], l[1], l[2], l[3]);
+              }
             }
           }
         }
