@@ -177,6 +177,15 @@ __device__ __forceinline__ bool before_or_at(uint32_t o, int j, Threshold t, boo
 constexpr int kRowsPerCta = 8;  // one warp per query-block row
 constexpr int kKTile = 32;      // pooled keys staged per step
 
+// Scores of the flat classifier: a CTA's 8 rows against key tiles of 256,
+// staged 64 features at a time.  Thread (rg, kq) of the 4 x 64 grid holds the
+// 2 x 4 block rows {2rg, 2rg+1} x keys {kq + 64 j}: per 4 features it reads 2
+// query and 4 key float4s (each a conflict-free wavefront across the warp,
+// thanks to the padded rows) for 32 FMAs.
+constexpr int kSKeys = 256;      // keys per score tile
+constexpr int kSChunk = 64;      // features staged per pass
+constexpr int kSStride = kSChunk + 4;
+
 // One CTA per 8 rows of one head.  When `logits_in` is null the pooled logits
 // are computed from qbar/kbar (fp32), otherwise read from it.  KPL: row
 // scores per lane in the selection (T <= 32 * KPL).
@@ -187,42 +196,65 @@ __global__ void __launch_bounds__(256) classify_kernel(
     int8_t* __restrict__ cls, int32_t* __restrict__ crit_idx, uint32_t* __restrict__ marg_bits,
     int T, int n_crit, int n_negl, float scale) {
   extern __shared__ __align__(16) float smem[];
-  constexpr int kStride = D + 4;  // padded row of the staged pooled keys
+  constexpr int kQStride = D + 4;
   float* srow = smem;                                // [8][T]
-  float* sq = srow + kRowsPerCta * T;                // [8][D]
-  float* sk = sq + kRowsPerCta * D;                  // [32][D+4]
+  float* sq = srow + kRowsPerCta * T;                // [8][D+4]
+  float* sk = sq + kRowsPerCta * kQStride;           // [256][64+4]
   const int bh = blockIdx.y, warp = threadIdx.x / 32, lane = lane_id();
   const int i = blockIdx.x * kRowsPerCta + warp;
   const bool row_ok = i < T;
   float* row = srow + warp * T;
 
   if (logits_in == nullptr) {
-    for (int e = threadIdx.x; e < kRowsPerCta * D; e += blockDim.x) {
-      const int r = e / D, a = e % D, ii = blockIdx.x * kRowsPerCta + r;
-      sq[e] = ii < T ? qbar[(size_t(bh) * T + ii) * D + a] : 0.f;
+    for (int e = threadIdx.x; e < kRowsPerCta * D / 4; e += blockDim.x) {
+      const int r = e / (D / 4), a4 = e % (D / 4), ii = blockIdx.x * kRowsPerCta + r;
+      const float4 x = ii < T ? reinterpret_cast<const float4*>(qbar + (size_t(bh) * T + ii) * D)[a4]
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(sq + r * kQStride + 4 * a4) = x;
     }
-    for (int j0 = 0; j0 < T; j0 += kKTile) {
-      __syncthreads();
-      for (int e = threadIdx.x; e < kKTile * D; e += blockDim.x) {
-        const int r = e / D, a = e % D, jj = j0 + r;
-        sk[r * kStride + a] = jj < T ? kbar[(size_t(bh) * T + jj) * D + a] : 0.f;
+    const int rg = lane >> 3, kq = warp * 8 + (lane & 7);
+    const float* kb = kbar + size_t(bh) * T * D;
+    for (int j0 = 0; j0 < T; j0 += kSKeys) {
+      float acc[2][4];
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[r][j] = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += kSChunk) {
+        __syncthreads();  // the previous chunk has been read
+        for (int e = threadIdx.x; e < kSKeys * kSChunk / 4; e += blockDim.x) {
+          const int key = e / (kSChunk / 4), a4 = e % (kSChunk / 4), jj = j0 + key;
+          const float4 y = jj < T ? reinterpret_cast<const float4*>(kb + size_t(jj) * D + c0)[a4]
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+          *reinterpret_cast<float4*>(sk + key * kSStride + 4 * a4) = y;
+        }
+        __syncthreads();
+        const float* q0 = sq + (2 * rg) * kQStride + c0;
+        const float* q1 = q0 + kQStride;
+#pragma unroll 4
+        for (int a = 0; a < kSChunk; a += 4) {
+          const float4 x0 = *reinterpret_cast<const float4*>(q0 + a);
+          const float4 x1 = *reinterpret_cast<const float4*>(q1 + a);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float4 y = *reinterpret_cast<const float4*>(sk + (kq + 64 * j) * kSStride + a);
+            acc[0][j] = fmaf(x0.x, y.x, acc[0][j]); acc[0][j] = fmaf(x0.y, y.y, acc[0][j]);
+            acc[0][j] = fmaf(x0.z, y.z, acc[0][j]); acc[0][j] = fmaf(x0.w, y.w, acc[0][j]);
+            acc[1][j] = fmaf(x1.x, y.x, acc[1][j]); acc[1][j] = fmaf(x1.y, y.y, acc[1][j]);
+            acc[1][j] = fmaf(x1.z, y.z, acc[1][j]); acc[1][j] = fmaf(x1.w, y.w, acc[1][j]);
+          }
+        }
       }
-      __syncthreads();
-      const int j = j0 + lane;
-      const float4* qa = reinterpret_cast<const float4*>(sq + warp * D);
-      const float4* ka = reinterpret_cast<const float4*>(sk + lane * kStride);
-      float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 8
-      for (int a4 = 0; a4 < D / 4; a4 += 2) {
-        const float4 x0 = qa[a4], y0 = ka[a4], x1 = qa[a4 + 1], y1 = ka[a4 + 1];
-        acc0 = fmaf(x0.x, y0.x, acc0); acc0 = fmaf(x0.y, y0.y, acc0);
-        acc0 = fmaf(x0.z, y0.z, acc0); acc0 = fmaf(x0.w, y0.w, acc0);
-        acc1 = fmaf(x1.x, y1.x, acc1); acc1 = fmaf(x1.y, y1.y, acc1);
-        acc1 = fmaf(x1.z, y1.z, acc1); acc1 = fmaf(x1.w, y1.w, acc1);
-      }
-      if (j < T) row[j] = (acc0 + acc1) * scale;
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int jj = j0 + kq + 64 * j;
+          if (jj < T) srow[(2 * rg + r) * T + jj] = acc[r][j] * scale;
+        }
     }
-    __syncwarp();
+    __syncthreads();  // every row complete
     if (row_ok && logits_out) {
       for (int j = lane; j < T; j += 32) logits_out[(size_t(bh) * T + i) * T + j] = row[j];
     }
@@ -700,8 +732,8 @@ cudaError_t launch_classify_t(const Problem& p, size_t smem, const float* qbar, 
 cudaError_t launch_classify(const Problem& p, const float* qbar, const float* kbar,
                             const float* logits_in, float* logits_out, int8_t* cls,
                             int32_t* crit_idx, uint32_t* marg_bits, cudaStream_t s) {
-  const size_t smem =
-      sizeof(float) * (size_t(kRowsPerCta) * p.T + kRowsPerCta * p.d + kKTile * (p.d + 4));
+  const size_t smem = sizeof(float) * (size_t(kRowsPerCta) * p.T + kRowsPerCta * (p.d + 4) +
+                                       size_t(kSKeys) * kSStride);
 #define SLA_FLAT(K)                                                                         \
   (p.d == 128 ? launch_classify_t<128, K>(p, smem, qbar, kbar, logits_in, logits_out, cls, \
                                           crit_idx, marg_bits, s)                          \
