@@ -177,14 +177,31 @@ __device__ __forceinline__ bool before_or_at(uint32_t o, int j, Threshold t, boo
 constexpr int kRowsPerCta = 8;  // one warp per query-block row
 constexpr int kKTile = 32;      // pooled keys staged per step
 
-// Scores of the flat classifier: a CTA's 8 rows against key tiles of 256,
-// staged 64 features at a time.  Thread (rg, kq) of the 4 x 64 grid holds the
-// 2 x 4 block rows {2rg, 2rg+1} x keys {kq + 64 j}: per 4 features it reads 2
-// query and 4 key float4s (each a conflict-free wavefront across the warp,
-// thanks to the padded rows) for 32 FMAs.
-constexpr int kSKeys = 256;      // keys per score tile
-constexpr int kSChunk = 64;      // features staged per pass
+// Scores of the flat classifier: a CTA's 8 rows against key tiles of 128,
+// staged 32 features at a time through a cp.async double buffer (the next
+// chunk is in flight while the current one is multiplied).  Thread (rg, kq)
+// of the 4 x 64 grid holds the 2 x 2 block rows {2rg, 2rg+1} x keys
+// {kq, kq + 64}: per 4 features it reads 2 query and 2 key float4s (each a
+// conflict-free wavefront across the warp, thanks to the padded rows) for 16
+// FMAs.  The small staging buffers keep two or three CTAs on an SM.
+constexpr int kSKeys = 128;      // keys per score tile
+constexpr int kSChunk = 32;      // features staged per step
 constexpr int kSStride = kSChunk + 4;
+constexpr int kSBuf = kSKeys * kSStride;  // floats per staging buffer
+
+// 16-byte global -> shared copy; src_bytes = 0 writes zeros (out-of-range key)
+__device__ __forceinline__ void cp_async16(float* dst, const float* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // One CTA per 8 rows of one head.  When `logits_in` is null the pooled logits
 // are computed from qbar/kbar (fp32), otherwise read from it.  KPL: row
@@ -197,9 +214,10 @@ __global__ void __launch_bounds__(256) classify_kernel(
     int T, int n_crit, int n_negl, float scale) {
   extern __shared__ __align__(16) float smem[];
   constexpr int kQStride = D + 4;
+  constexpr int kChunks = D / kSChunk;
   float* srow = smem;                                // [8][T]
   float* sq = srow + kRowsPerCta * T;                // [8][D+4]
-  float* sk = sq + kRowsPerCta * kQStride;           // [256][64+4]
+  float* sk = sq + kRowsPerCta * kQStride;           // 2 x [256][32+4]
   const int bh = blockIdx.y, warp = threadIdx.x / 32, lane = lane_id();
   const int i = blockIdx.x * kRowsPerCta + warp;
   const bool row_ok = i < T;
@@ -214,45 +232,64 @@ __global__ void __launch_bounds__(256) classify_kernel(
     }
     const int rg = lane >> 3, kq = warp * 8 + (lane & 7);
     const float* kb = kbar + size_t(bh) * T * D;
-    for (int j0 = 0; j0 < T; j0 += kSKeys) {
-      float acc[2][4];
+    const int nsteps = (T + kSKeys - 1) / kSKeys * kChunks;
+    // step st = (key tile st / kChunks, feature chunk st % kChunks) into buffer st & 1
+    auto stage = [&](int st) {
+      float* dst = sk + (st & 1) * kSBuf;
+      const int j0 = (st / kChunks) * kSKeys, c0 = (st % kChunks) * kSChunk;
 #pragma unroll
-      for (int r = 0; r < 2; ++r)
+      for (int x = 0; x < kSKeys * kSChunk / 4 / 256; ++x) {
+        const int e = threadIdx.x + 256 * x;
+        const int key = e / (kSChunk / 4), a4 = e % (kSChunk / 4), jj = j0 + key;
+        const bool in = jj < T;
+        cp_async16(dst + key * kSStride + 4 * a4, in ? kb + size_t(jj) * D + c0 + 4 * a4 : kb,
+                   in ? 16 : 0);
+      }
+      cp_async_commit();
+    };
+    stage(0);
+    float acc[2][2];
+    for (int st = 0; st < nsteps; ++st) {
+      if (st + 1 < nsteps) {
+        stage(st + 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();  // step st landed for every thread's copies
+      const int chunk = st % kChunks, j0 = (st / kChunks) * kSKeys;
+      if (chunk == 0) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[r][j] = 0.f;
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += kSChunk) {
-        __syncthreads();  // the previous chunk has been read
-        for (int e = threadIdx.x; e < kSKeys * kSChunk / 4; e += blockDim.x) {
-          const int key = e / (kSChunk / 4), a4 = e % (kSChunk / 4), jj = j0 + key;
-          const float4 y = jj < T ? reinterpret_cast<const float4*>(kb + size_t(jj) * D + c0)[a4]
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-          *reinterpret_cast<float4*>(sk + key * kSStride + 4 * a4) = y;
-        }
-        __syncthreads();
-        const float* q0 = sq + (2 * rg) * kQStride + c0;
-        const float* q1 = q0 + kQStride;
-#pragma unroll 4
-        for (int a = 0; a < kSChunk; a += 4) {
-          const float4 x0 = *reinterpret_cast<const float4*>(q0 + a);
-          const float4 x1 = *reinterpret_cast<const float4*>(q1 + a);
+        for (int r = 0; r < 2; ++r)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float4 y = *reinterpret_cast<const float4*>(sk + (kq + 64 * j) * kSStride + a);
-            acc[0][j] = fmaf(x0.x, y.x, acc[0][j]); acc[0][j] = fmaf(x0.y, y.y, acc[0][j]);
-            acc[0][j] = fmaf(x0.z, y.z, acc[0][j]); acc[0][j] = fmaf(x0.w, y.w, acc[0][j]);
-            acc[1][j] = fmaf(x1.x, y.x, acc[1][j]); acc[1][j] = fmaf(x1.y, y.y, acc[1][j]);
-            acc[1][j] = fmaf(x1.z, y.z, acc[1][j]); acc[1][j] = fmaf(x1.w, y.w, acc[1][j]);
-          }
+          for (int j = 0; j < 2; ++j) acc[r][j] = 0.f;
+      }
+      const float* kbuf = sk + (st & 1) * kSBuf;
+      const float* q0 = sq + (2 * rg) * kQStride + chunk * kSChunk;
+      const float* q1 = q0 + kQStride;
+#pragma unroll
+      for (int a = 0; a < kSChunk; a += 4) {
+        const float4 x0 = *reinterpret_cast<const float4*>(q0 + a);
+        const float4 x1 = *reinterpret_cast<const float4*>(q1 + a);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float4 y = *reinterpret_cast<const float4*>(kbuf + (kq + 64 * j) * kSStride + a);
+          acc[0][j] = fmaf(x0.x, y.x, acc[0][j]); acc[0][j] = fmaf(x0.y, y.y, acc[0][j]);
+          acc[0][j] = fmaf(x0.z, y.z, acc[0][j]); acc[0][j] = fmaf(x0.w, y.w, acc[0][j]);
+          acc[1][j] = fmaf(x1.x, y.x, acc[1][j]); acc[1][j] = fmaf(x1.y, y.y, acc[1][j]);
+          acc[1][j] = fmaf(x1.z, y.z, acc[1][j]); acc[1][j] = fmaf(x1.w, y.w, acc[1][j]);
         }
       }
+      if (chunk == kChunks - 1) {
 #pragma unroll
-      for (int r = 0; r < 2; ++r)
+        for (int r = 0; r < 2; ++r)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int jj = j0 + kq + 64 * j;
-          if (jj < T) srow[(2 * rg + r) * T + jj] = acc[r][j] * scale;
-        }
+          for (int j = 0; j < 2; ++j) {
+            const int jj = j0 + kq + 64 * j;
+            if (jj < T) srow[(2 * rg + r) * T + jj] = acc[r][j] * scale;
+          }
+      }
+      __syncthreads();  // buffer st & 1 may be refilled by step st + 2
     }
     __syncthreads();  // every row complete
     if (row_ok && logits_out) {
@@ -733,7 +770,7 @@ cudaError_t launch_classify(const Problem& p, const float* qbar, const float* kb
                             const float* logits_in, float* logits_out, int8_t* cls,
                             int32_t* crit_idx, uint32_t* marg_bits, cudaStream_t s) {
   const size_t smem = sizeof(float) * (size_t(kRowsPerCta) * p.T + kRowsPerCta * (p.d + 4) +
-                                       size_t(kSKeys) * kSStride);
+                                       2 * size_t(kSBuf));
 #define SLA_FLAT(K)                                                                         \
   (p.d == 128 ? launch_classify_t<128, K>(p, smem, qbar, kbar, logits_in, logits_out, cls, \
                                           crit_idx, marg_bits, s)                          \
