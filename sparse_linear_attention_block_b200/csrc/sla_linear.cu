@@ -35,8 +35,12 @@ namespace {
 // K = token; as hi and lo bf16 tiles) and V_j (N = c) are written MN-major
 // into swizzled shared memory; h_j = phi_hi^T V + phi_lo^T V by tcgen05
 // (M=128, N=D, K=64; for D = 64 the M dimension is zero-padded to 128).
+// h_j's hi and lo planes leave through the (then free) phi tiles as swizzled
+// 64-column halves written by TMA stores, one contiguous 16 KB box each.
 template <int D>
-__global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __restrict__ k,
+__global__ void __launch_bounds__(128) summaries_kernel(const __grid_constant__ CUtensorMap tm_hi,
+                                                        const __grid_constant__ CUtensorMap tm_lo,
+                                                        const __nv_bfloat16* __restrict__ k,
                                                         const __nv_bfloat16* __restrict__ v,
                                                         __nv_bfloat16* __restrict__ summ_hi,
                                                         __nv_bfloat16* __restrict__ summ_lo,
@@ -132,24 +136,39 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
   }
   const bool ok = mbar_wait(&bar, 0, err, nullptr);
   tc_fence_after();
-  if (ok && warp * 32 < D) {
-    const int a = warp * 32 + lane_id();
-    const size_t o = rowbase + size_t(a) * D;
+  // the products have read the phi tiles: they now stage h_j's output halves
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      float vals[32];
-      tmem_ld32(tmem_addr(tmem, warp * 32, c0), vals);
+  for (int c0 = 0; c0 < D; c0 += 64) {
+    if (c0 > 0) {  // the previous half's stores have read the staging tiles
+      if (t == 0) bulk_wait_read_all();
+      __syncthreads();
+    }
+    if (ok && warp * 32 < D) {
+      const int a = warp * 32 + lane_id();
+      float vals[2][32];
+      tmem_ld32(tmem_addr(tmem, warp * 32, c0), vals[0]);
+      tmem_ld32(tmem_addr(tmem, warp * 32, c0 + 32), vals[1]);
       tmem_ld_wait();
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
+      for (int q8 = 0; q8 < 8; ++q8) {
         uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) split2(vals[q4 * 8 + 2 * e], vals[q4 * 8 + 2 * e + 1], hi[e], lo[e]);
-        *reinterpret_cast<uint4*>(summ_hi + o + c0 + q4 * 8) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(summ_lo + o + c0 + q4 * 8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        for (int e = 0; e < 4; ++e)
+          split2(vals[q8 >> 2][(q8 & 3) * 8 + 2 * e], vals[q8 >> 2][(q8 & 3) * 8 + 2 * e + 1],
+                 hi[e], lo[e]);
+        st_sw128_unit(sPhiH, D, a, q8 * 8, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+        st_sw128_unit(sPhiL, D, a, q8 * 8, make_uint4(lo[0], lo[1], lo[2], lo[3]));
       }
     }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (t == 0 && ok) {
+      tma_store_3d(&tm_hi, sPhiH, c0, 0, bh * T + j);
+      tma_store_3d(&tm_lo, sPhiL, c0, 0, bh * T + j);
+      bulk_commit();
+    }
   }
+  if (t == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_free(tmem, 128);
@@ -165,22 +184,25 @@ __global__ void __launch_bounds__(128) summaries_kernel(const __nv_bfloat16* __r
 // adjacent in the schedule, so the second M half finds its B slice in L2.
 // Warp 0 = TMA producer over a 3-stage ring (K in steps of 64), warp 1 =
 // MMA issuer into one of two TMEM accumulator buffers (256 columns each),
-// warps 2-5 = epilogue (TMEM -> hi/lo planes) of the previous tile while the
-// next one is multiplied.
+// warps 2-5 = epilogue of the previous tile while the next one is multiplied:
+// TMEM -> hi/lo bf16 -> a swizzled 128 x 64 staging tile per plane -> TMA
+// stores (whole 128-byte lines instead of one 16-byte piece per row).
 constexpr int kAggBN = 128, kAggBK = 64, kAggStages = 3, kAggMT = 2;
 constexpr int kAggA = 128 * kAggBK * 2;        // 16 KB per 128-row tile
 constexpr int kAggB = kAggBK * kAggBN * 2;     // 16 KB per plane
 constexpr int kAggStageBytes = kAggMT * kAggA + 2 * kAggB;
+constexpr int kAggOut = 128 * 64 * 2;          // staging tile: 128 rows x 64 columns
 constexpr int kAggEpiWarps = 4;
 constexpr int kAggThreads = 64 + 32 * kAggEpiWarps;
 
 __global__ void __launch_bounds__(kAggThreads, 1) agg_gemm_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_bh,
-    const __grid_constant__ CUtensorMap tm_bl, __nv_bfloat16* __restrict__ out_hi,
-    __nv_bfloat16* __restrict__ out_lo, int T, int Tp, int NN, int BH, int* err) {
+    const __grid_constant__ CUtensorMap tm_bl, const __grid_constant__ CUtensorMap tm_oh,
+    const __grid_constant__ CUtensorMap tm_ol, int T, int Tp, int NN, int BH, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = align_smem_1024(smem_raw);
-  __shared__ uint64_t full[kAggStages], empty[kAggStages], acc_full[2], acc_empty[2], fin;
+  uint8_t* sOut = base + kAggStages * kAggStageBytes;  // hi then lo staging tile
+  __shared__ uint64_t full[kAggStages], empty[kAggStages], acc_full[2], acc_empty[2], fin, esync;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   const int warp = threadIdx.x / 32;
@@ -205,6 +227,7 @@ __global__ void __launch_bounds__(kAggThreads, 1) agg_gemm_kernel(
       mbar_init(&acc_empty[b], kAggEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(&fin, 1);
+    mbar_init(&esync, 32 * kAggEpiWarps);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -282,39 +305,53 @@ __global__ void __launch_bounds__(kAggThreads, 1) agg_gemm_kernel(
     mma_commit(&fin);
     mbar_wait(&fin, 0, nullptr, nullptr);
   } else if (warp >= 2) {
-    const int q = warp % 4;                          // the TMEM lane quadrant this warp may access
-    for (int n = 0; n < nloc; ++n) {
+    const int q = warp % 4;  // the TMEM lane quadrant this warp may access
+    const int r = q * 32 + lane_id();  // row of the 128-row M tile == TMEM lane
+    const bool leader = warp == 2 && lane_id() == 0;
+    uint32_t ephase = 0;
+    // barrier of the epilogue warps with a bounded wait
+    auto epi_sync = [&]() -> bool {
+      mbar_arrive(&esync);
+      const bool okw = mbar_wait(&esync, ephase & 1, err, &abort_flag);
+      ++ephase;
+      return okw;
+    };
+    bool ok = true;
+    for (int n = 0; n < nloc && ok; ++n) {
       int mg, nt, bh;
       tile_of(n, mg, nt, bh);
       const int nmt = min(kAggMT, Tp / 128 - mg * kAggMT);
       const int buf = n & 1;
       if (!mbar_wait(&acc_full[buf], (n >> 1) & 1, err, &abort_flag)) break;
       tc_fence_after();
-      for (int m = 0; m < nmt; ++m) {
-        const int i = (mg * kAggMT + m) * 128 + q * 32 + lane_id();
+      for (int m = 0; m < nmt && ok; ++m) {
 #pragma unroll 1
         for (int cbase = 0; cbase < kAggBN; cbase += 64) {
-          const size_t o = (size_t(bh) * T + i) * NN + size_t(nt) * kAggBN + cbase;
           const uint32_t col = buf * (kAggMT * kAggBN) + m * kAggBN + cbase;
           float vals[2][32];
           tmem_ld32(tmem_addr(tmem, q * 32, col), vals[0]);
           tmem_ld32(tmem_addr(tmem, q * 32, col + 32), vals[1]);
           tmem_ld_wait();
+          // the staging tiles are free once the previous stores have read them
+          if (leader) bulk_wait_read_all();
+          if (!(ok = epi_sync())) break;
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            if (i < T && nt * kAggBN + cbase + 32 * c < NN) {  // NN is a multiple of 32
+          for (int u = 0; u < 8; ++u) {
+            uint32_t h[4], l[4];
 #pragma unroll
-              for (int e = 0; e < 32; e += 8) {
-                uint32_t h[4], l[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                  split2(vals[c][e + 2 * u], vals[c][e + 2 * u + 1], h[u], l[u]);
-                *reinterpret_cast<uint4*>(out_hi + o + 32 * c + e) =
-                    make_uint4(h[0], h[1], h[2], h[3]);
-                *reinterpret_cast<uint4*>(out_lo + o + 32 * c + e) =
-                    make_uint4(l[0], l[1], l[2], l[3]);
-              }
-            }
+            for (int e = 0; e < 4; ++e)
+              split2(vals[u >> 2][(u & 3) * 8 + 2 * e], vals[u >> 2][(u & 3) * 8 + 2 * e + 1], h[e],
+                     l[e]);
+            st_sw128_unit(sOut, 128, r, u * 8, make_uint4(h[0], h[1], h[2], h[3]));
+            st_sw128_unit(sOut + kAggOut, 128, r, u * 8, make_uint4(l[0], l[1], l[2], l[3]));
+          }
+          fence_proxy_async_smem();
+          if (!(ok = epi_sync())) break;
+          if (leader) {  // rows past T and columns past NN are clipped by the store
+            const int x = nt * kAggBN + cbase, y = (mg * kAggMT + m) * 128;
+            tma_store_3d(&tm_oh, sOut, x, y, bh);
+            tma_store_3d(&tm_ol, sOut + kAggOut, x, y, bh);
+            bulk_commit();
           }
         }
       }
@@ -322,6 +359,7 @@ __global__ void __launch_bounds__(kAggThreads, 1) agg_gemm_kernel(
       __syncwarp();
       if (lane_id() == 0) mbar_arrive(&acc_empty[buf]);
     }
+    if (leader) bulk_wait_all();
   }
   __syncwarp();
   tc_fence_before();
@@ -347,15 +385,18 @@ cudaError_t launch_summaries(const Problem& p, const void* k, const void* v,
   dim3 grid(p.T, p.BH);
   const int groups = 128 / (p.d / 8);
   const size_t smem = 1024 + 32768 + (p.d / 64) * 8192 + sizeof(float) * groups * p.d;
+  CUtensorMap th, tl;
+  if (!make_tmap_summary(&th, summ_hi, p.BH * p.T, p.d)) return cudaErrorInvalidValue;
+  if (!make_tmap_summary(&tl, summ_lo, p.BH * p.T, p.d)) return cudaErrorInvalidValue;
   cudaError_t e;
   if (p.d == 128) {
     if ((e = set_smem(summaries_kernel<128>, smem)) != cudaSuccess) return e;
-    summaries_kernel<128><<<grid, 128, smem, s>>>((const __nv_bfloat16*)k,
+    summaries_kernel<128><<<grid, 128, smem, s>>>(th, tl, (const __nv_bfloat16*)k,
                                                   (const __nv_bfloat16*)v, summ_hi, summ_lo,
                                                   p.N, p.T, p.nv, err);
   } else {
     if ((e = set_smem(summaries_kernel<64>, smem)) != cudaSuccess) return e;
-    summaries_kernel<64><<<grid, 128, smem, s>>>((const __nv_bfloat16*)k,
+    summaries_kernel<64><<<grid, 128, smem, s>>>(th, tl, (const __nv_bfloat16*)k,
                                                  (const __nv_bfloat16*)v, summ_hi, summ_lo, p.N,
                                                  p.T, p.nv, err);
   }
@@ -371,7 +412,10 @@ cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
   if (!make_tmap_3d(&ta, mmat, p.Tp, p.Tp, p.BH, 64, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_3d(&tbh, summ_hi, NN, p.T, p.BH, 64, 64)) return cudaErrorInvalidValue;
   if (!make_tmap_3d(&tbl, summ_lo, NN, p.T, p.BH, 64, 64)) return cudaErrorInvalidValue;
-  const size_t smem = 1024 + kAggStages * kAggStageBytes;
+  CUtensorMap toh, tol;
+  if (!make_tmap_3d(&toh, out_hi, NN, p.T, p.BH, 64, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_3d(&tol, out_lo, NN, p.T, p.BH, 64, 128)) return cudaErrorInvalidValue;
+  const size_t smem = 1024 + kAggStages * kAggStageBytes + 2 * kAggOut;
   cudaError_t e = set_smem(agg_gemm_kernel, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
@@ -379,8 +423,8 @@ cudaError_t launch_aggregate(const Problem& p, const __nv_bfloat16* mmat,
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return cudaErrorUnknown;
   const int ntiles = p.BH * ((NN + kAggBN - 1) / kAggBN) * ((p.Tp / 128 + kAggMT - 1) / kAggMT);
-  agg_gemm_kernel<<<std::min(ntiles, sms), kAggThreads, smem, s>>>(ta, tbh, tbl, out_hi, out_lo,
-                                                                  p.T, p.Tp, NN, p.BH, err);
+  agg_gemm_kernel<<<std::min(ntiles, sms), kAggThreads, smem, s>>>(ta, tbh, tbl, toh, tol, p.T,
+                                                                  p.Tp, NN, p.BH, err);
   return cudaGetLastError();
 }
 

@@ -156,6 +156,29 @@ __device__ __forceinline__ void tma_load_3d(void* dst, uint64_t* bar, const CUte
       : "memory");
 }
 
+// Tiled 3D store shared -> global (bulk async group; the source tile is in the
+// 128-byte swizzled layout of the map).  Issue after fence_proxy_async_smem()
+// and a barrier with the threads that wrote the tile.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* src, int x, int y,
+                                             int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// The stores committed so far have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// The stores committed so far are complete.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05: TMEM
 
 // Allocate `ncols` TMEM columns (power of two >= 32); whole warp; the base
