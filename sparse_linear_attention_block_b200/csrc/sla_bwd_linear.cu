@@ -56,13 +56,14 @@ __device__ __forceinline__ float tile_at(const uint8_t* tile, int rows, int row,
 
 constexpr int kQH = 32768;  // one H plane tile: 2 chunks x 128 rows x 128 B
 constexpr int kQT = 16384;  // a [64 t][128] or [128][64 t] bf16 tile
-// bwd_q shared memory: H hi/lo, dO, phi hi/lo, dnum^T hi/lo
-constexpr int kBqSmem = 1024 + 2 * kQH + kQT + 2 * kQT + 2 * kQT;
+// bwd_q shared memory: H hi/lo, dO, phi hi/lo, dnum^T hi/lo, A_i staging
+constexpr int kBqSmem = 1024 + 2 * kQH + kQT + 2 * kQT + 2 * kQT + 2 * kQT;
 
 template <int D>
 __global__ void __launch_bounds__(256, 1) bwd_q_kernel(
     const __grid_constant__ CUtensorMap tm_hh, const __grid_constant__ CUtensorMap tm_hl,
-    const __grid_constant__ CUtensorMap tm_do, const __nv_bfloat16* __restrict__ q,
+    const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_ah,
+    const __grid_constant__ CUtensorMap tm_al, const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* __restrict__ d_o, const __nv_bfloat16* __restrict__ w_proj,
     const float* __restrict__ o_s, const float* __restrict__ den,
     const __nv_bfloat16* __restrict__ hz_hi, const __nv_bfloat16* __restrict__ hz_lo,
@@ -85,6 +86,10 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(
   uint8_t* sPl = sPh + kQT;
   uint8_t* sNh = sPl + kQT;   // dnum^T hi [c][64 t]
   uint8_t* sNl = sNh + kQT;
+  // A_i leaves as 64-column hi/lo tiles written by TMA stores: columns [0, 64)
+  // staged in the dnum^T tiles (free once the block's products are done),
+  // columns [64, 128) in sAx
+  uint8_t* sAx = sNl + kQT;
   __shared__ float sZ[D];
   __shared__ float sInv[64], sDd[64];
   __shared__ float sRed[2][4][64];  // per-warp partial sums: G . O_l and dO . O_s
@@ -197,6 +202,7 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(
       st_sw128_unit(sPl, 64, rr, 8 * u, make_uint4(l[0], l[1], l[2], l[3]));
     }
     fence_proxy_async_smem();
+    if (t == 0) bulk_wait_read_all();  // the previous A_i stores have left the dnum tiles
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -354,8 +360,8 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(
         const float dph = fminf(tile_at(sPh, 64, t0 + j, f) + tile_at(sPl, 64, t0 + j, f), 1.0f);
         dq[(tok0 + t0 + j) * D + f] = fmaf(sDd[t0 + j], za, v[j]) * dph;
       }
-      // A_i, row a of the summary (hi/lo planes), this warpgroup's column half
-      const size_t srow = size_t(blk) * W + size_t(f) * D;
+      // A_i, row a of the summary (hi/lo planes), this warpgroup's column half,
+      // into the swizzled staging tiles
 #pragma unroll 1
       for (int c0 = g * DH; c0 < (g + 1) * DH; c0 += 32) {
         tmem_ld32(tmem + lane_base + kA + c0, v);
@@ -365,16 +371,29 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(
           uint32_t hh[4], ll[4];
 #pragma unroll
           for (int m = 0; m < 4; ++m) split2(v[e + 2 * m], v[e + 2 * m + 1], hh[m], ll[m]);
-          *reinterpret_cast<uint4*>(summ_hi + srow + c0 + e) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
-          *reinterpret_cast<uint4*>(summ_lo + srow + c0 + e) = make_uint4(ll[0], ll[1], ll[2], ll[3]);
+          const int c = c0 + e;
+          uint8_t* sth = c < 64 ? sNh : sAx;
+          uint8_t* stl = c < 64 ? sNl : sAx + kQT;
+          st_sw128_unit(sth, D, f, c & 63, make_uint4(hh[0], hh[1], hh[2], hh[3]));
+          st_sw128_unit(stl, D, f, c & 63, make_uint4(ll[0], ll[1], ll[2], ll[3]));
         }
       }
     }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();  // sZ, sDd, the phi tiles and TMEM dQ^T / A_i are free
     tc_fence_after();
+    if (t == 0) {
+#pragma unroll
+      for (int ch = 0; ch < D / 64; ++ch) {
+        tma_store_3d(&tm_ah, ch == 0 ? sNh : sAx, ch * 64, 0, blk);
+        tma_store_3d(&tm_al, ch == 0 ? sNl : sAx + kQT, ch * 64, 0, blk);
+      }
+      bulk_commit();
+    }
     if (nxt < nblk) load_zd(nxt);
   }
+  if (t == 0) bulk_wait_all();
   // this CTA's share of dW (lane = row c of dW, this warpgroup's column half)
   if (ok && k > 0 && lane_ok) {
 #pragma unroll 1
@@ -647,9 +666,11 @@ cudaError_t launch_bwd_q(const Problem& p, const void* q, const void* d_o, const
                          __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* dw, float gate,
                          float* d_gate, int num_sms, int* err, cudaStream_t s) {
   const float slope = gate * (1.0f - gate);
-  CUtensorMap th, tl, tdo;
+  CUtensorMap th, tl, tdo, tah, tal;
   if (!make_tmap_summary(&th, hz_hi, p.BH * p.T, p.d)) return cudaErrorInvalidValue;
   if (!make_tmap_summary(&tl, hz_lo, p.BH * p.T, p.d)) return cudaErrorInvalidValue;
+  if (!make_tmap_summary(&tah, summ_hi, p.BH * p.T, p.d)) return cudaErrorInvalidValue;
+  if (!make_tmap_summary(&tal, summ_lo, p.BH * p.T, p.d)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tdo, d_o, p.BH, p.N, p.d, 64)) return cudaErrorInvalidValue;
   const int nblk = p.BH * p.T;
   const int grid = nblk < num_sms ? nblk : num_sms;
@@ -658,14 +679,14 @@ cudaError_t launch_bwd_q(const Problem& p, const void* q, const void* d_o, const
     e = cudaFuncSetAttribute(bwd_q_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBqSmem);
     if (e != cudaSuccess) return e;
     bwd_q_kernel<128><<<grid, 256, kBqSmem, s>>>(
-        th, tl, tdo, (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o,
+        th, tl, tdo, tah, tal, (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o,
         (const __nv_bfloat16*)w_proj, o_s, den, hz_hi, hz_lo, dvec, dq, summ_hi, summ_lo, dw, gate,
         slope, d_gate, p.N, p.T, nblk, err);
   } else {
     e = cudaFuncSetAttribute(bwd_q_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBqSmem);
     if (e != cudaSuccess) return e;
     bwd_q_kernel<64><<<grid, 256, kBqSmem, s>>>(
-        th, tl, tdo, (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o,
+        th, tl, tdo, tah, tal, (const __nv_bfloat16*)q, (const __nv_bfloat16*)d_o,
         (const __nv_bfloat16*)w_proj, o_s, den, hz_hi, hz_lo, dvec, dq, summ_hi, summ_lo, dw, gate,
         slope, d_gate, p.N, p.T, nblk, err);
   }
