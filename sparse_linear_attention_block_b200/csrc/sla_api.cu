@@ -85,6 +85,19 @@ bool make_tmap_strided(CUtensorMap* map, const void* base, uint64_t d0, uint64_t
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_f32_bhnd(CUtensorMap* map, const float* base, int BH, int N, int d, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {uint64_t(d), uint64_t(N), uint64_t(BH)};
+  cuuint64_t strides[2] = {uint64_t(d) * 4, uint64_t(d) * uint64_t(N) * 4};
+  cuuint32_t box[3] = {32, uint32_t(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_summary(CUtensorMap* map, const void* plane, int rows, int d) {
   return make_tmap_strided(map, plane, uint64_t(d), uint64_t(d), uint64_t(rows), uint64_t(d),
                            uint64_t(summary_width(d)), 64, uint32_t(d));

@@ -114,5 +114,9 @@ bool make_tmap_strided(CUtensorMap* map, const void* base, uint64_t d0, uint64_t
 // viewed as {c, a, row} so that a box {64, d, 1} lands as a 128-byte-swizzled
 // tile of d rows (a) per 64-column chunk (c).
 bool make_tmap_summary(CUtensorMap* map, const void* plane, int rows, int d);
+// fp32 [BH][N][d] as {d, N, BH}, 32-column (128-byte) boxes of box_rows rows,
+// 128-byte swizzle (a store source: row r's 16-byte unit u at unit u ^ (r % 8)).
+bool make_tmap_f32_bhnd(CUtensorMap* map, const float* base, int BH, int N, int d, int box_rows);
+
 
 }  // namespace sla

@@ -64,6 +64,7 @@ template <int D>
 __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+    const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
     const float* __restrict__ lse, const float* __restrict__ dvec,
     const int32_t* __restrict__ col_ptr, const int32_t* __restrict__ col_idx, int N, int T,
     int n_crit, int nv, float scale_log2, float scale, float* __restrict__ dq, float* __restrict__ dk,
@@ -341,15 +342,18 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
       }
       if (!ok) break;
     }
-    // dK (warpgroup 0) and dV (warpgroup 1) of this tile's keys
+    // dK (warpgroup 0) and dV (warpgroup 1) of this tile's keys: fp32 rows
+    // staged as 128-byte swizzled 32-column tiles (in the K/V tiles for dV, the
+    // stage buffers for dK: every product has finished with them) and written
+    // by TMA stores; rows past N (a missing second key block) are clipped.
     if (nU > 0) {
       ok = mbar_wait(&fin, 0, err, &abort_flag) && ok;
       tc_fence_after();
     }
-    const size_t key = size_t(qp) * 128 + r;
-    float* dst = (wg == 0 ? dk : dv) + (size_t(bh) * N + key) * D;
+    uint8_t* stg_out = wg == 0 ? sSt : sK;
     const uint32_t acc = tmem + lane_base + (wg == 0 ? kDK : kDV);
     const float mul = wg == 0 ? scale : 1.0f;
+    const bool h = nU > 0 && ok;
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       float a[32];
@@ -357,14 +361,23 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
         tmem_ld32(acc + c0, a);
         tmem_ld_wait();
       }
-      if (key_ok) {
-        const bool h = nU > 0 && ok;
+      uint8_t* tile = stg_out + (c0 / 32) * (128 * 128);
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst + c0 + e) =
-              h ? make_float4(a[e] * mul, a[e + 1] * mul, a[e + 2] * mul, a[e + 3] * mul)
-                : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<float4*>(tile + r * 128 + ((u ^ (r & 7)) * 16)) =
+            h ? make_float4(a[4 * u] * mul, a[4 * u + 1] * mul, a[4 * u + 2] * mul,
+                            a[4 * u + 3] * mul)
+              : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    fence_proxy_async_smem();
+    const bool synced = wg_sync();
+    if (wq == 0 && lane == 0 && synced) {
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32)
+        tma_store_3d(wg == 0 ? &tm_dk : &tm_dv, stg_out + (c0 / 32) * (128 * 128), c0, qp * 128,
+                     bh);
+      bulk_commit();
+      bulk_wait_all();
     }
   }
   tc_fence_before();
@@ -378,7 +391,9 @@ cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, co
                               const void* d_o, const float* lse, const float* dvec,
                               const int32_t* col_ptr, const int32_t* col_idx, float* dq,
                               float* dk, float* dv, int* err, cudaStream_t s) {
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdk, tdv;
+  if (!make_tmap_f32_bhnd(&tdk, dk, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_f32_bhnd(&tdv, dv, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tq, q, p.BH, p.N, p.d, 64)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tk, k, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tv, v, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
@@ -390,7 +405,8 @@ cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, co
     e = cudaFuncSetAttribute(bwd_sparse_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem));
     if (e != cudaSuccess) return e;
-    bwd_sparse_kernel<128><<<grid, 320, smem, s>>>(tq, tk, tv, tdo, lse, dvec, col_ptr, col_idx,
+    bwd_sparse_kernel<128><<<grid, 320, smem, s>>>(tq, tk, tv, tdo, tdk, tdv, lse, dvec, col_ptr,
+                                                   col_idx,
                                                    p.N, p.T, p.n_crit, p.nv, p.scale_log2, p.scale, dq,
                                                    dk, dv, err);
   } else {
@@ -398,7 +414,8 @@ cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, co
     e = cudaFuncSetAttribute(bwd_sparse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem));
     if (e != cudaSuccess) return e;
-    bwd_sparse_kernel<64><<<grid, 320, smem, s>>>(tq, tk, tv, tdo, lse, dvec, col_ptr, col_idx,
+    bwd_sparse_kernel<64><<<grid, 320, smem, s>>>(tq, tk, tv, tdo, tdk, tdv, lse, dvec, col_ptr,
+                                                  col_idx,
                                                   p.N, p.T, p.n_crit, p.nv, p.scale_log2, p.scale, dq,
                                                   dk, dv, err);
   }
