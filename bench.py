@@ -108,6 +108,7 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.path = None
+        self.skip = 0
 
     def __enter__(self):
         try:
@@ -119,6 +120,18 @@ class ClockSampler:
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return self
+        # nvidia-smi takes a moment to start: wait for its first sample so that
+        # the timed region is sampled from its start; samples taken before it
+        # (the wait itself) are dropped
+        t0 = time.time()
+        while time.time() - t0 < 5.0 and self.proc.poll() is None:
+            with open(self.path) as f:
+                n = sum(1 for _ in f)
+            if n:
+                self.skip = n
+                break
+            time.sleep(0.01)
         return self
 
     def __exit__(self, *exc):
@@ -139,6 +152,9 @@ class ClockSampler:
                 if len(parts) >= 9:
                     rows.append(parts)
         os.unlink(self.path)
+        # the timed region's samples; a region shorter than the sampling
+        # interval keeps the sample closest to it
+        rows = rows[self.skip:] or rows[-1:]
         if not rows:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]

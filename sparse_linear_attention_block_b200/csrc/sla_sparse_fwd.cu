@@ -45,9 +45,9 @@ struct FwdSmem {
 template <int D>
 __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ crit_idx, int N, int T,
-    int n_crit, int nv, float scale_log2, float* __restrict__ o_s, float* __restrict__ lse,
-    int* err) {
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_os,
+    const int32_t* __restrict__ crit_idx, int N, int T, int n_crit, int nv, float scale_log2,
+    float* __restrict__ lse, int* err) {
   using L = FwdSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = align_smem_1024(smem_raw);
@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
   uint8_t* uflag = base + L::kTiles + 2 * (2 * n_crit);
 
   __shared__ uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages],
-      v_empty[kStages], s_full[2], p_full[2], o_done, mma_done;
+      v_empty[kStages], s_full[2], p_full[2], o_done, mma_done, osync;
   __shared__ uint32_t tmem_base;
   __shared__ int n_union, abort_flag;
 
@@ -81,6 +81,7 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
     }
     mbar_init(&o_done, 1);
     mbar_init(&mma_done, 1);
+    mbar_init(&osync, 128);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -283,10 +284,12 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
       ok = mbar_wait(&o_done, (nU - 1) & 1, err, &abort_flag);
       tc_fence_after();
     }
+    // O_s rows staged as 128-byte swizzled 32-column fp32 tiles in the Q and
+    // K/V buffers (every product has finished with them) and written by TMA
+    // stores; rows past N (a missing second block) are clipped by the store
     const size_t tok = size_t(p) * 128 + r;
     const bool have = ok && nU > 0 && l_run > 0.f;
     const float inv = have ? 1.0f / l_run : 0.f;
-    float* dst = o_s + (size_t(bh) * N + tok) * D;
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       float ov[32];
@@ -294,15 +297,22 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
         tmem_ld32(tm_o + lane_base + c0, ov);
         tmem_ld_wait();
       }
-      if (row_ok) {
+      uint8_t* tile = base + (c0 / 32) * (128 * 128);
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          float4 x = have ? make_float4(ov[e] * inv, ov[e + 1] * inv, ov[e + 2] * inv,
-                                        ov[e + 3] * inv)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-          *reinterpret_cast<float4*>(dst + c0 + e) = x;
-        }
-      }
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<float4*>(tile + r * 128 + ((u ^ (r & 7)) * 16)) =
+            have ? make_float4(ov[4 * u] * inv, ov[4 * u + 1] * inv, ov[4 * u + 2] * inv,
+                               ov[4 * u + 3] * inv)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&osync);
+    if (mbar_wait(&osync, 0, err, &abort_flag) && r == 0) {
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32)
+        tma_store_3d(&tm_os, base + (c0 / 32) * (128 * 128), c0, p * 128, bh);
+      bulk_commit();
+      bulk_wait_all();
     }
     if (row_ok)
       lse[size_t(bh) * N + tok] =
@@ -319,7 +329,8 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
 cudaError_t launch_fwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
                               const int32_t* crit_idx, float* o_s, float* lse, int* err,
                               cudaStream_t s) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tos;
+  if (!make_tmap_f32_bhnd(&tos, o_s, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tq, q, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tk, k, p.BH, p.N, p.d, 64)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tv, v, p.BH, p.N, p.d, 64)) return cudaErrorInvalidValue;
@@ -330,15 +341,15 @@ cudaError_t launch_fwd_sparse(const Problem& p, const void* q, const void* k, co
     e = cudaFuncSetAttribute(fwd_sparse_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem);
     if (e != cudaSuccess) return e;
-    fwd_sparse_kernel<128><<<grid, 192, smem, s>>>(tq, tk, tv, crit_idx, p.N, p.T, p.n_crit,
-                                                   p.nv, p.scale_log2, o_s, lse, err);
+    fwd_sparse_kernel<128><<<grid, 192, smem, s>>>(tq, tk, tv, tos, crit_idx, p.N, p.T, p.n_crit,
+                                                   p.nv, p.scale_log2, lse, err);
   } else {
     const int smem = int(FwdSmem<64>::total(p.n_crit));
     e = cudaFuncSetAttribute(fwd_sparse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem);
     if (e != cudaSuccess) return e;
-    fwd_sparse_kernel<64><<<grid, 192, smem, s>>>(tq, tk, tv, crit_idx, p.N, p.T, p.n_crit,
-                                                  p.nv, p.scale_log2, o_s, lse, err);
+    fwd_sparse_kernel<64><<<grid, 192, smem, s>>>(tq, tk, tv, tos, crit_idx, p.N, p.T, p.n_crit,
+                                                  p.nv, p.scale_log2, lse, err);
   }
   return cudaGetLastError();
 }
