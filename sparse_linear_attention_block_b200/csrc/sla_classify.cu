@@ -83,90 +83,106 @@ struct Threshold {
   int jt;
 };
 
-// Row of n <= 32 * KPL scores held by one warp in registers: element j sits in
-// lane j % 32, slot j / 32, as its ordered score; slots past n hold 0, below
-// every ordered score (the smallest, of -inf, is 0x007FFFFF).
+// The n-th element of a row of `len` scores (smem, len <= 32 * KPL) in the
+// order (score desc, index asc), or with `flip` in the reverse order (score
+// asc, index desc), found by one warp.  The row is held in registers as
+// order-preserving 32-bit keys (complemented when flipped; element j in lane
+// j % 32, slot j / 32; slots past len hold 0, below every key).  A bracket
+// [a, b) of key values with #(key >= a) >= n > #(key >= b) is narrowed by a
+// safeguarded interpolation search (the pivot from the two counts; a plain
+// halving whenever an interpolation step did not halve the bracket), each step
+// one count by warp sums, until it holds one key value or at most 32 elements.
+// Then either the need-th equal key in index order is taken, or the bracket's
+// elements are compacted one per lane (through 64 words of shared scratch)
+// and ranked against each other by shuffles.  Exact for any input without NaN.
 template <int KPL>
-__device__ __forceinline__ void load_keys(const float* row, int n, uint32_t (&key)[KPL]) {
+__device__ Threshold select_side(const float* row, int len, int n, bool flip,
+                                 uint32_t* scratch) {
+  constexpr uint32_t kAll = 0xFFFFFFFFu;
   const int lane = lane_id();
+  uint32_t key[KPL];
+  uint32_t kmin = ~0u, kmax = 0u;
 #pragma unroll
   for (int e = 0; e < KPL; ++e) {
     const int j = 32 * e + lane;
-    key[e] = j < n ? ordered_bits(row[j]) : 0u;
+    uint32_t k = 0u;
+    if (j < len) {
+      k = ordered_bits(row[j]);
+      if (flip) k = ~k;
+      kmin = min(kmin, k);
+    }
+    key[e] = k;
+    kmax = max(kmax, k);
   }
-}
-
-// Thresholds of the n_hi-th element in the order (score desc, index asc) and
-// the n_lo-th in the reverse order, computed together by one warp (a count of
-// 0 leaves its threshold unused).  Exact bisection on the 32-bit ordered
-// score: only the bits below the common prefix of the row's smallest and
-// largest score are searched, each step counting with one warp sum per side;
-// then one pass resolves equal scores by index.  No shared memory.
-template <int KPL>
-__device__ void select2(const uint32_t (&key)[KPL], int n, int n_hi, int n_lo, Threshold* th,
-                        Threshold* tl) {
-  constexpr uint32_t kAll = 0xFFFFFFFFu;
-  const int lane = lane_id();
-  const int npad = 32 * KPL - n;  // zero slots: always <= any bound, never >= one
-  uint32_t lo = ~0u, hi = 0u;
+  uint32_t a = __reduce_min_sync(kAll, kmin);
+  uint32_t b = __reduce_max_sync(kAll, kmax) + 1u;  // keys never reach 0xFFFFFFFF
+  int ca = len, cb = 0;
+  bool halve = false;
+  while (b - a > 1u && ca - cb > 32) {
+    const uint32_t w = b - a;
+    uint32_t p = halve ? a + w / 2u
+                       : a + 1u + uint32_t((uint64_t(w - 1u) * uint32_t(ca - n)) /
+                                           uint32_t(ca - cb));
+    p = min(max(p, a + 1u), b - 1u);
+    int c = 0;
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) c += key[e] >= p;
+    c = __reduce_add_sync(kAll, c);
+    if (c >= n) {
+      a = p;
+      ca = c;
+    } else {
+      b = p;
+      cb = c;
+    }
+    halve = !halve && uint64_t(b - a) * 2u > uint64_t(w);
+  }
+  const int need = n - cb;  // rank of the answer inside the bracket (1-based)
+  Threshold th{a, -1};
+  if (b - a == 1u) {  // one key value: the need-th equal element in index order
+    int seen = 0;
+#pragma unroll
+    for (int s = 0; s < KPL; ++s) {
+      const int e = flip ? KPL - 1 - s : s;
+      uint32_t m = __ballot_sync(kAll, key[e] == a);  // a zero slot never equals a
+      const int cnt = __popc(m);
+      if (th.jt < 0 && seen + cnt >= need) {
+        for (int r = need - seen; r > 1; --r) m &= flip ? ~(1u << (31 - __clz(m))) : m - 1u;
+        th.jt = 32 * e + (flip ? 31 - __clz(m) : __ffs(int(m)) - 1);
+      }
+      seen += cnt;
+    }
+    return th;
+  }
+  // at most 32 elements in [a, b): one per lane, then ranks by shuffles
+  int base = 0;
 #pragma unroll
   for (int e = 0; e < KPL; ++e) {
-    lo = min(lo, 32 * e + lane < n ? key[e] : ~0u);
-    hi = max(hi, key[e]);
-  }
-  lo = __reduce_min_sync(kAll, lo);
-  hi = __reduce_max_sync(kAll, hi);
-  const uint32_t diff = lo ^ hi;
-  const int top = diff ? 31 - __clz(diff) : -1;  // highest bit that varies in the row
-  const uint32_t vary = top < 0 ? 0u : (top == 31 ? ~0u : (2u << top) - 1u);
-  // v: the largest value with #(key >= v) >= n_hi (the n_hi-th largest key);
-  // u: the smallest value with #(key <= u) >= n_lo (the n_lo-th smallest)
-  uint32_t v = hi & ~vary, u = lo | vary;
-  for (int b = top; b >= 0; --b) {
-    const uint32_t ch = v | (1u << b), cl = u & ~(1u << b);
-    int a = 0, c = 0;
-#pragma unroll
-    for (int e = 0; e < KPL; ++e) {
-      a += key[e] >= ch;
-      c += key[e] <= cl;
+    const bool in = key[e] >= a && key[e] < b;
+    const uint32_t m = __ballot_sync(kAll, in);
+    if (in) {
+      const int pos = base + __popc(m & ((1u << lane) - 1u));
+      scratch[pos] = key[e];
+      scratch[32 + pos] = uint32_t(32 * e + lane);
     }
-    a = __reduce_add_sync(kAll, a);
-    c = __reduce_add_sync(kAll, c) - npad;
-    if (a >= n_hi) v = ch;
-    if (c >= n_lo) u = cl;
+    base += __popc(m);
   }
-  // equal scores: the needed one among them by index
-  int gt = 0, lt = 0;
-#pragma unroll
-  for (int e = 0; e < KPL; ++e) {
-    gt += key[e] > v;
-    lt += key[e] < u;
+  __syncwarp();
+  const int cnt = ca - cb;
+  const uint32_t mk = lane < cnt ? scratch[lane] : 0u;
+  const int mj = lane < cnt ? int(scratch[32 + lane]) : 0;
+  int rank = 0;
+  for (int l = 0; l < cnt; ++l) {
+    const uint32_t ok = __shfl_sync(kAll, mk, l);
+    const int oj = __shfl_sync(kAll, mj, l);
+    rank += ok > mk || (ok == mk && (flip ? oj > mj : oj < mj));
   }
-  const int need_hi = n_hi - __reduce_add_sync(kAll, gt);
-  const int need_lo = n_lo - (__reduce_add_sync(kAll, lt) - npad);
-  int jh = -1, jl = -1, seen_h = 0, seen_l = 0;
-#pragma unroll
-  for (int e = 0; e < KPL; ++e) {
-    uint32_t m = __ballot_sync(kAll, key[e] == v);  // a zero slot never equals a score
-    const int cnt = __popc(m);
-    if (jh < 0 && seen_h + cnt >= need_hi) {
-      for (int r = need_hi - seen_h; r > 1; --r) m &= m - 1u;
-      jh = 32 * e + __ffs(int(m)) - 1;
-    }
-    seen_h += cnt;
-  }
-#pragma unroll
-  for (int e = KPL - 1; e >= 0; --e) {
-    uint32_t m = __ballot_sync(kAll, key[e] == u);
-    const int cnt = __popc(m);
-    if (jl < 0 && seen_l + cnt >= need_lo) {
-      for (int r = need_lo - seen_l; r > 1; --r) m &= ~(1u << (31 - __clz(m)));
-      jl = 32 * e + 31 - __clz(m);
-    }
-    seen_l += cnt;
-  }
-  *th = Threshold{v, jh};
-  *tl = Threshold{~u, jl};
+  const uint32_t hit = __ballot_sync(kAll, lane < cnt && rank == need - 1);
+  const int src = __ffs(int(hit)) - 1;
+  th.v = __shfl_sync(kAll, mk, src);
+  th.jt = __shfl_sync(kAll, mj, src);
+  __syncwarp();  // scratch may be reused by the next selection
+  return th;
 }
 
 __device__ __forceinline__ bool before_or_at(uint32_t o, int j, Threshold t, bool flip) {
@@ -302,12 +318,11 @@ __global__ void __launch_bounds__(256) classify_kernel(
   }
   if (!row_ok) return;
 
-  Threshold th{0, -1}, tl{0, -1};
-  if (n_crit > 0 || n_negl > 0) {
-    uint32_t key[KPL];
-    load_keys<KPL>(row, T, key);
-    select2<KPL>(key, T, n_crit, n_negl, &th, &tl);
-  }
+  uint32_t* scratch = reinterpret_cast<uint32_t*>(sk + 2 * kSBuf) + warp * 64;
+  const Threshold th = n_crit > 0 ? select_side<KPL>(row, T, n_crit, false, scratch)
+                                  : Threshold{0, -1};
+  const Threshold tl = n_negl > 0 ? select_side<KPL>(row, T, n_negl, true, scratch)
+                                  : Threshold{0, -1};
   const size_t rbase = size_t(bh) * T + i;
   int8_t* crow = cls + rbase * T;
   int32_t* idx = crit_idx + rbase * n_crit;
@@ -379,7 +394,7 @@ struct HierArgs {
 __host__ __device__ inline int hier_warp_words(int T, int TG, int cap_hi, int cap_lo, int c_hi,
                                                int c_lo) {
   const int W = (T + 31) / 32;
-  return TG + cap_hi + cap_lo + c_hi + c_lo + 2 * W;
+  return TG + cap_hi + cap_lo + c_hi + c_lo + 2 * W + 64;
 }
 
 // Block index of candidate position p of a list of super-blocks (ascending).
@@ -461,6 +476,7 @@ __global__ void __launch_bounds__(256) hier_classify_kernel(const HierArgs a) {
   int* list_lo = list_hi + a.c_hi;
   uint32_t* bits_c = reinterpret_cast<uint32_t*>(list_lo + a.c_lo);
   uint32_t* bits_n = bits_c + W;
+  uint32_t* scratch = bits_n + W;  // 64 words for the selections
 
   // ---- coarse scores sc_iJ (all warps take part in the staging)
   if (a.coarse_in == nullptr) {
@@ -498,12 +514,10 @@ __global__ void __launch_bounds__(256) hier_classify_kernel(const HierArgs a) {
   if (!row_ok) return;
 
   // ---- candidate super-blocks, ascending
-  Threshold thc, tlc;
-  {
-    uint32_t key[KPL];
-    load_keys<KPL>(crow, TG, key);
-    select2<KPL>(key, TG, a.c_hi, a.c_lo, &thc, &tlc);
-  }
+  const Threshold thc =
+      a.c_hi > 0 ? select_side<KPL>(crow, TG, a.c_hi, false, scratch) : Threshold{0, -1};
+  const Threshold tlc =
+      a.c_lo > 0 ? select_side<KPL>(crow, TG, a.c_lo, true, scratch) : Threshold{0, -1};
   int nh = 0, nl = 0;
   for (int J0 = 0; J0 < TG; J0 += 32) {
     const int J = J0 + lane;
@@ -557,17 +571,11 @@ __global__ void __launch_bounds__(256) hier_classify_kernel(const HierArgs a) {
 
   // ---- exact selection inside the candidates (position order = block order)
   if (a.n_crit > 0) {
-    uint32_t key[KPL];
-    Threshold th, unused;
-    load_keys<KPL>(cand, nb_hi, key);
-    select2<KPL>(key, nb_hi, a.n_crit, 0, &th, &unused);
+    const Threshold th = select_side<KPL>(cand, nb_hi, a.n_crit, false, scratch);
     mark_selected(cand, list_hi, nb_hi, G, th, false, bits_c);
   }
   if (a.n_negl > 0) {
-    uint32_t key[KPL];
-    Threshold tl, unused;
-    load_keys<KPL>(cand_lo, nb_lo, key);
-    select2<KPL>(key, nb_lo, 0, a.n_negl, &unused, &tl);
+    const Threshold tl = select_side<KPL>(cand_lo, nb_lo, a.n_negl, true, scratch);
     mark_selected(cand_lo, list_lo, nb_lo, G, tl, true, bits_n);
   }
   __syncwarp();
@@ -770,7 +778,7 @@ cudaError_t launch_classify(const Problem& p, const float* qbar, const float* kb
                             const float* logits_in, float* logits_out, int8_t* cls,
                             int32_t* crit_idx, uint32_t* marg_bits, cudaStream_t s) {
   const size_t smem = sizeof(float) * (size_t(kRowsPerCta) * p.T + kRowsPerCta * (p.d + 4) +
-                                       2 * size_t(kSBuf));
+                                       2 * size_t(kSBuf) + kRowsPerCta * 64);
 #define SLA_FLAT(K)                                                                         \
   (p.d == 128 ? launch_classify_t<128, K>(p, smem, qbar, kbar, logits_in, logits_out, cls, \
                                           crit_idx, marg_bits, s)                          \
