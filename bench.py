@@ -437,10 +437,11 @@ def main():
     cpu = None
     default_run = args.workload == "train" and args.k_h is None and not args.hierarchical
     if rank == 0 and world == 1 and not args.no_cpu_baseline and default_run:
-        tfl, sec = time_oracle(wl, [0], 1, 0)
+        tfl, sec = time_oracle(wl, [0, 1, 2], 1, 0)
         cpu = {"value": tfl, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"head 0 of 12 of this workload, one classify+forward+backward step "
-                         f"of the fp64 oracle ({sec:.1f} s), same executed-block FLOP count"}
+               "sample": f"heads 0-2 of 12 of this workload, one classify+forward+backward "
+                         f"step of the fp64 oracle ({sec:.1f} s), executed-block FLOPs of "
+                         f"those heads"}
 
     if world > 1:
         dist.barrier()
