@@ -512,34 +512,35 @@ __global__ void __launch_bounds__(128, 1) bwd_k_kernel(
     const float dz = __bfloat162float(dh_hi[size_t(blk) * W + D * D + t]) +
                      __bfloat162float(dh_lo[size_t(blk) * W + D * D + t]);
 #pragma unroll 1
-    for (int q16 = 0; q16 < 64; q16 += 16) {
-      float ck[16], cv[16], kk[16], gk[16], gv[16];
+    for (int q32 = 0; q32 < 64; q32 += 32) {
+      // 32 tokens per pass: 96 independent loads per thread in flight
+      float ck[32], cv[32], kk[32], gk[32], gv[32];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const size_t idx = (tk + q16 + j) * D + t;
+      for (int j = 0; j < 32; ++j) {
+        const size_t idx = (tk + q32 + j) * D + t;
         ck[j] = dk[idx];
         cv[j] = dv[idx];
         kk[j] = __bfloat162float(kin[idx]);
       }
-      tmem_ld16(acc + q16, gk);
-      tmem_ld16(acc + 64 + q16, gv);
+      tmem_ld32(acc + q32, gk);
+      tmem_ld32(acc + 64 + q32, gv);
       tmem_ld_wait();
       if (write) {
-        // keys of this block that exist (key padding; all 16 except in a
+        // keys of this block that exist (key padding; all 32 except in a
         // sequence's partial last block, where padded keys keep dK = dV = 0)
-        const int lim = nv - ((blk % T) * 64 + q16);
-        if (lim >= 16) {
+        const int lim = nv - ((blk % T) * 64 + q32);
+        if (lim >= 32) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const size_t idx = (tk + q16 + j) * D + t;
+          for (int j = 0; j < 32; ++j) {
+            const size_t idx = (tk + q32 + j) * D + t;
             dk[idx] = fmaf(gk[j] + dz, dphi_f(kk[j]), ck[j]);
             dv[idx] = cv[j] + gv[j];
           }
         } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 32; ++j) {
             if (j >= lim) break;
-            const size_t idx = (tk + q16 + j) * D + t;
+            const size_t idx = (tk + q32 + j) * D + t;
             dk[idx] = fmaf(gk[j] + dz, dphi_f(kk[j]), ck[j]);
             dv[idx] = cv[j] + gv[j];
           }
