@@ -704,25 +704,47 @@ __global__ void __launch_bounds__(256) csr_fill_kernel(const int8_t* __restrict_
 
 // ------------------------------------------------------------------ marginal matrix
 // bf16 0/1 matrix of marginal pairs, [BH][Tp][Tp] zero-padded, and its
-// transpose; the operands of the aggregation GEMMs.
-__global__ void expand_marginal_kernel(const uint32_t* __restrict__ marg_bits,
-                                       __nv_bfloat16* __restrict__ mmat,
-                                       __nv_bfloat16* __restrict__ mmat_t, int T, int Tp) {
-  const int bh = blockIdx.z;
-  const int r = blockIdx.y;                          // row of the output
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;  // column
-  if (c >= Tp) return;
+// transpose; the operands of the aggregation GEMMs.  One thread writes 8
+// consecutive columns (16 bytes) of one row.
+__global__ void __launch_bounds__(256) expand_marginal_kernel(const uint32_t* __restrict__ marg_bits,
+                                                              __nv_bfloat16* __restrict__ mmat,
+                                                              __nv_bfloat16* __restrict__ mmat_t,
+                                                              int T, int Tp) {
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;  // 8-column group of the whole head
+  const int per_row = Tp / 8;
+  if (e >= Tp * per_row) return;
+  const int r = e / per_row, c0 = (e % per_row) * 8;
   const int words = (T + 31) / 32;
   const uint32_t* mb = marg_bits + size_t(bh) * T * words;
-  const __nv_bfloat16 one = __float2bfloat16(1.0f), zero = __float2bfloat16(0.0f);
-  const size_t o = (size_t(bh) * Tp + r) * Tp + c;
+  constexpr uint32_t kOne = 0x3F80u;  // bf16 1.0
+  const size_t o = (size_t(bh) * Tp + r) * Tp + c0;
   if (mmat) {
-    bool m = r < T && c < T && ((mb[size_t(r) * words + c / 32] >> (c % 32)) & 1u);
-    mmat[o] = m ? one : zero;
+    uint32_t bits = 0;  // bit u: column c0 + u is marginal in row r
+    if (r < T && c0 < T) {
+      bits = (mb[size_t(r) * words + c0 / 32] >> (c0 % 32)) & 0xFFu;
+      if (T - c0 < 8) bits &= (1u << (T - c0)) - 1u;
+    }
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      w[u] = ((bits >> (2 * u)) & 1u ? kOne : 0u) | ((bits >> (2 * u + 1)) & 1u ? kOne << 16 : 0u);
+    *reinterpret_cast<uint4*>(mmat + o) = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  if (mmat_t) {
-    bool m = r < T && c < T && ((mb[size_t(c) * words + r / 32] >> (r % 32)) & 1u);
-    mmat_t[o] = m ? one : zero;
+  if (mmat_t) {  // row r of the transpose = column r of the matrix
+    uint32_t bits = 0;
+    if (r < T) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + u;
+        if (c < T) bits |= ((mb[size_t(c) * words + r / 32] >> (r % 32)) & 1u) << u;
+      }
+    }
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      w[u] = ((bits >> (2 * u)) & 1u ? kOne : 0u) | ((bits >> (2 * u + 1)) & 1u ? kOne << 16 : 0u);
+    *reinterpret_cast<uint4*>(mmat_t + o) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -846,8 +868,8 @@ cudaError_t launch_crit_csr(const Problem& p, const int8_t* cls, int32_t* col_pt
 
 cudaError_t launch_expand_marginal(const Problem& p, const uint32_t* marg_bits,
                                    __nv_bfloat16* mmat, __nv_bfloat16* mmat_t, cudaStream_t s) {
-  dim3 grid((p.Tp + 127) / 128, p.Tp, p.BH);
-  expand_marginal_kernel<<<grid, 128, 0, s>>>(marg_bits, mmat, mmat_t, p.T, p.Tp);
+  dim3 grid((p.Tp * (p.Tp / 8) + 255) / 256, p.BH);
+  expand_marginal_kernel<<<grid, 256, 0, s>>>(marg_bits, mmat, mmat_t, p.T, p.Tp);
   return cudaGetLastError();
 }
 
