@@ -191,7 +191,7 @@ __device__ __forceinline__ bool before_or_at(uint32_t o, int j, Threshold t, boo
 }
 
 constexpr int kRowsPerCta = 8;  // one warp per query-block row
-constexpr int kKTile = 32;      // pooled keys staged per step
+constexpr int kKTile = 32;      // coarse keys staged per step (hierarchical selection)
 
 // Scores of the flat classifier: a CTA's 8 rows against key tiles of 128,
 // staged 32 features at a time through a cp.async double buffer (the next
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(256) classify_kernel(
   constexpr int kChunks = D / kSChunk;
   float* srow = smem;                                // [8][T]
   float* sq = srow + kRowsPerCta * T;                // [8][D+4]
-  float* sk = sq + kRowsPerCta * kQStride;           // 2 x [256][32+4]
+  float* sk = sq + kRowsPerCta * kQStride;           // 2 x [128][32+4], then 8 x 64 words
   const int bh = blockIdx.y, warp = threadIdx.x / 32, lane = lane_id();
   const int i = blockIdx.x * kRowsPerCta + warp;
   const bool row_ok = i < T;
