@@ -37,6 +37,7 @@ WorkspaceLayout workspace_layout(int BH, int N, int d) {
   L.mmat = take(bh * Tp * Tp * 2);
   L.mmat_t = take(bh * Tp * Tp * 2);
   L.dvec = take(bh * N * 4);
+  L.order = take(bh * ((T + 1) / 2) * 4);
   L.total = off;
   return L;
 }
@@ -485,6 +486,7 @@ static sla_status backward_impl(const sla_shape* shape, const void* q, const voi
   const auto* hz_hi = static_cast<const __nv_bfloat16*>(saved->hz_agg);
   const auto* hz_lo = hz_hi + size_t(p.BH) * p.T * summary_width(p.d);
   float* dvec = at<float>(workspace, L.dvec);
+  int32_t* order = at<int32_t>(workspace, L.order);
   if (cudaMemsetAsync(dw_proj, 0, size_t(p.d) * p.d * sizeof(float), s) != cudaSuccess)
     return SLA_ERR_CUDA;
   if (d_logit && cudaMemsetAsync(d_logit, 0, sizeof(float), s) != cudaSuccess) return SLA_ERR_CUDA;
@@ -492,8 +494,9 @@ static sla_status backward_impl(const sla_shape* shape, const void* q, const voi
     if (cudaMemsetAsync(dq, 0, size_t(p.BH) * p.N * p.d * sizeof(float), s) != cudaSuccess)
       return SLA_ERR_CUDA;
     SLA_LAUNCH("dvec", s, launch_dvec(p, d_o, saved->o_s, dvec, s));
+    SLA_LAUNCH("pair_order", s, launch_pair_order(p, mask->crit_col_ptr, order, s));
     SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
-                                 mask->crit_col_idx, dq, dk, dv, err, s));
+                                 mask->crit_col_idx, order, dq, dk, dv, err, s));
     return SLA_OK;
   }
   // linear branch, query side: D, dQ's linear share (written), dW, and the
@@ -503,9 +506,11 @@ static sla_status backward_impl(const sla_shape* shape, const void* q, const voi
   // (dh_j | dz_j) = sum over rows i with j marginal of (A_i | a_i): transposed aggregation
   SLA_LAUNCH("expand_marginal_t", s, launch_expand_marginal(p, mask->marg_bits, nullptr, mmat_t, s));
   SLA_LAUNCH("aggregate_t", s, launch_aggregate(p, mmat_t, summ_hi, summ_lo, dh_hi, dh_lo, err, s));
-  // sparse branch adds to dQ and writes dK, dV; the linear branch's key side adds its share
+  // sparse branch adds to dQ and writes dK, dV (its tiles longest first); the linear
+  // branch's key side adds its share
+  SLA_LAUNCH("pair_order", s, launch_pair_order(p, mask->crit_col_ptr, order, s));
   SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
-                               mask->crit_col_idx, dq, dk, dv, err, s));
+                               mask->crit_col_idx, order, dq, dk, dv, err, s));
   SLA_LAUNCH("bwd_k", s, launch_bwd_k(p, k, v, dh_hi, dh_lo, dk, dv, sms, err, s));
   return SLA_OK;
 }

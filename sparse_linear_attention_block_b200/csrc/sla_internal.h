@@ -36,6 +36,7 @@ struct WorkspaceLayout {
   size_t mmat;       // bf16 [BH,Tp,Tp] marginal 0/1 matrix, rows = query blocks
   size_t mmat_t;     // bf16 [BH,Tp,Tp] its transpose
   size_t dvec;       // fp32 [BH,N]     D_t = dO_t . O_s,t
+  size_t order;      // int32 [BH*ceil(T/2)] key-block pairs of the sparse backward, longest first
   size_t total;
 };
 
@@ -92,10 +93,15 @@ cudaError_t launch_bwd_q(const Problem& p, const void* q, const void* d_o, const
                          const __nv_bfloat16* hz_lo, float* dvec, float* dq,
                          __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* dw, float gate,
                          float* d_gate, int num_sms, int* err, cudaStream_t s);
+// Order of the sparse backward's tiles (key-block pairs, all heads): by the
+// summed length of the pair's two column lists, longest first.
+cudaError_t launch_pair_order(const Problem& p, const int32_t* col_ptr, int32_t* order,
+                              cudaStream_t s);
 cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
                               const void* d_o, const float* lse, const float* dvec,
-                              const int32_t* col_ptr, const int32_t* col_idx, float* dq,
-                              float* dk, float* dv, int* err, cudaStream_t s);
+                              const int32_t* col_ptr, const int32_t* col_idx,
+                              const int32_t* order, float* dq, float* dk, float* dv, int* err,
+                              cudaStream_t s);
 cudaError_t launch_bwd_k(const Problem& p, const void* k, const void* v,
                          const __nv_bfloat16* dh_hi, const __nv_bfloat16* dh_lo, float* dk,
                          float* dv, int num_sms, int* err, cudaStream_t s);

@@ -66,7 +66,8 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
     const float* __restrict__ lse, const float* __restrict__ dvec,
-    const int32_t* __restrict__ col_ptr, const int32_t* __restrict__ col_idx, int N, int T,
+    const int32_t* __restrict__ col_ptr, const int32_t* __restrict__ col_idx,
+    const int32_t* __restrict__ order, int N, int T,
     int n_crit, int nv, float scale_log2, float scale, float* __restrict__ dq, float* __restrict__ dk,
     float* __restrict__ dv, int* err) {
   using L = SbSmem<D>;
@@ -83,7 +84,11 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
       tfree[2], wsync[2], fin;
   __shared__ uint32_t tmem_base;
   __shared__ int n_union, abort_flag;
-  const int qp = blockIdx.x, bh = blockIdx.y;
+  // this CTA's tile: key-block pair qp of head bh, taken in the order given
+  // (longest column lists first, so the long tiles do not start last)
+  const int npairs = (T + 1) / 2;
+  const int item = order[blockIdx.x];
+  const int qp = item % npairs, bh = item / npairs;
   const int warp = threadIdx.x / 32, lane = lane_id();
   const int kb0 = 2 * qp, kb1 = 2 * qp + 1;
   const bool has1 = kb1 < T;
@@ -387,10 +392,72 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
 
 }  // namespace
 
+namespace {
+
+// ------------------------------------------------------------------ tile order
+// One CTA: a counting sort of the key-block pairs of every head by the summed
+// length of their two column lists (an upper bound of the pair's union, the
+// tile's work), longest first.  Pairs of equal length keep no particular order.
+constexpr int kOrderThreads = 1024;
+
+__global__ void __launch_bounds__(kOrderThreads) pair_order_kernel(
+    const int32_t* __restrict__ col_ptr, int32_t* __restrict__ order, int T, int BH) {
+  extern __shared__ int cnt[];  // [2T + 1] buckets, bucket b = 2T - length
+  __shared__ int part[kOrderThreads];
+  const int npairs = (T + 1) / 2, n = npairs * BH, nb = 2 * T + 1, t = threadIdx.x;
+  auto length = [&](int item) {
+    const int qp = item % npairs, bh = item / npairs;
+    const int32_t* cp = col_ptr + size_t(bh) * (T + 1);
+    const int j0 = 2 * qp, j1 = 2 * qp + 1;
+    int len = cp[j0 + 1] - cp[j0];
+    if (j1 < T) len += cp[j1 + 1] - cp[j1];
+    return min(max(len, 0), 2 * T);
+  };
+  for (int b = t; b < nb; b += kOrderThreads) cnt[b] = 0;
+  __syncthreads();
+  for (int item = t; item < n; item += kOrderThreads) atomicAdd(&cnt[2 * T - length(item)], 1);
+  __syncthreads();
+  // exclusive scan of the buckets: thread t owns a contiguous run of them
+  const int per = (nb + kOrderThreads - 1) / kOrderThreads;
+  const int b0 = min(nb, t * per), b1 = min(nb, b0 + per);
+  int sum = 0;
+  for (int b = b0; b < b1; ++b) sum += cnt[b];
+  part[t] = sum;
+  __syncthreads();
+  for (int o = 1; o < kOrderThreads; o <<= 1) {  // inclusive scan of the run sums
+    const int v = t >= o ? part[t - o] : 0;
+    __syncthreads();
+    part[t] += v;
+    __syncthreads();
+  }
+  int run = part[t] - sum;
+  for (int b = b0; b < b1; ++b) {
+    const int c = cnt[b];
+    cnt[b] = run;
+    run += c;
+  }
+  __syncthreads();
+  for (int item = t; item < n; item += kOrderThreads)
+    order[atomicAdd(&cnt[2 * T - length(item)], 1)] = item;
+}
+
+}  // namespace
+
+cudaError_t launch_pair_order(const Problem& p, const int32_t* col_ptr, int32_t* order,
+                              cudaStream_t s) {
+  const size_t smem = sizeof(int) * size_t(2 * p.T + 1);
+  cudaError_t e = cudaFuncSetAttribute(pair_order_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  pair_order_kernel<<<1, kOrderThreads, smem, s>>>(col_ptr, order, p.T, p.BH);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
                               const void* d_o, const float* lse, const float* dvec,
-                              const int32_t* col_ptr, const int32_t* col_idx, float* dq,
-                              float* dk, float* dv, int* err, cudaStream_t s) {
+                              const int32_t* col_ptr, const int32_t* col_idx,
+                              const int32_t* order, float* dq, float* dk, float* dv, int* err,
+                              cudaStream_t s) {
   CUtensorMap tq, tk, tv, tdo, tdk, tdv;
   if (!make_tmap_f32_bhnd(&tdk, dk, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_f32_bhnd(&tdv, dv, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
@@ -398,7 +465,7 @@ cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, co
   if (!make_tmap_bhnd(&tk, k, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tv, v, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tdo, d_o, p.BH, p.N, p.d, 64)) return cudaErrorInvalidValue;
-  dim3 grid((p.T + 1) / 2, p.BH);
+  dim3 grid(((p.T + 1) / 2) * p.BH);
   cudaError_t e;
   if (p.d == 128) {
     const size_t smem = SbSmem<128>::total(p.T);
@@ -406,7 +473,7 @@ cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, co
                              int(smem));
     if (e != cudaSuccess) return e;
     bwd_sparse_kernel<128><<<grid, 320, smem, s>>>(tq, tk, tv, tdo, tdk, tdv, lse, dvec, col_ptr,
-                                                   col_idx,
+                                                   col_idx, order,
                                                    p.N, p.T, p.n_crit, p.nv, p.scale_log2, p.scale, dq,
                                                    dk, dv, err);
   } else {
@@ -415,7 +482,7 @@ cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, co
                              int(smem));
     if (e != cudaSuccess) return e;
     bwd_sparse_kernel<64><<<grid, 320, smem, s>>>(tq, tk, tv, tdo, tdk, tdv, lse, dvec, col_ptr,
-                                                  col_idx,
+                                                  col_idx, order,
                                                   p.N, p.T, p.n_crit, p.nv, p.scale_log2, p.scale, dq,
                                                   dk, dv, err);
   }
