@@ -70,7 +70,7 @@ def executed_block_flops(wl, n_crit):
 # traffic grows with the number of heads).  A kernel missing here reports
 # traffic null; an entry must be dropped or re-measured when its kernel changes.
 NCU_DRAM_BYTES_PER_HEAD = {
-    "bwd_sparse": (206.550272e6 + 152.495360e6) / 4,  # bwd_sparse_wan4h_full.md
+    "bwd_sparse": (204.179968e6 + 151.736320e6) / 4,  # bwd_sparse_wan4h_full.md
 }
 
 

@@ -36,7 +36,7 @@ struct WorkspaceLayout {
   size_t mmat;       // bf16 [BH,Tp,Tp] marginal 0/1 matrix, rows = query blocks
   size_t mmat_t;     // bf16 [BH,Tp,Tp] its transpose
   size_t dvec;       // fp32 [BH,N]     D_t = dO_t . O_s,t
-  size_t order;      // int32 [BH*ceil(T/2)] key-block pairs of the sparse backward, longest first
+  size_t order;      // int32 [BH*ceil(T/2)] key-block pairs of the sparse backward, in order
   size_t total;
 };
 
@@ -93,8 +93,9 @@ cudaError_t launch_bwd_q(const Problem& p, const void* q, const void* d_o, const
                          const __nv_bfloat16* hz_lo, float* dvec, float* dq,
                          __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* dw, float gate,
                          float* d_gate, int num_sms, int* err, cudaStream_t s);
-// Order of the sparse backward's tiles (key-block pairs, all heads): by the
-// summed length of the pair's two column lists, longest first.
+// Order of the sparse backward's tiles (key-block pairs): heads in sequence,
+// within a head by the summed length of the pair's two column lists, longest
+// first.
 cudaError_t launch_pair_order(const Problem& p, const int32_t* col_ptr, int32_t* order,
                               cudaStream_t s);
 cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, const void* v,

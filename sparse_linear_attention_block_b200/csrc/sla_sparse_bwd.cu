@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
   __shared__ uint32_t tmem_base;
   __shared__ int n_union, abort_flag;
   // this CTA's tile: key-block pair qp of head bh, taken in the order given
-  // (longest column lists first, so the long tiles do not start last)
+  // (heads in sequence, each head's longest column lists first)
   const int npairs = (T + 1) / 2;
   const int item = order[blockIdx.x];
   const int qp = item % npairs, bh = item / npairs;
@@ -395,19 +395,20 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
 namespace {
 
 // ------------------------------------------------------------------ tile order
-// One CTA: a counting sort of the key-block pairs of every head by the summed
+// One CTA per head: a counting sort of the head's key-block pairs by the summed
 // length of their two column lists (an upper bound of the pair's union, the
-// tile's work), longest first.  Pairs of equal length keep no particular order.
+// tile's work), longest first.  Heads stay in sequence, so the tiles running
+// at any time share one head's Q and dO in L2, and every head's tiles end
+// with its shortest ones.  Pairs of equal length keep no particular order.
 constexpr int kOrderThreads = 1024;
 
 __global__ void __launch_bounds__(kOrderThreads) pair_order_kernel(
-    const int32_t* __restrict__ col_ptr, int32_t* __restrict__ order, int T, int BH) {
+    const int32_t* __restrict__ col_ptr, int32_t* __restrict__ order, int T) {
   extern __shared__ int cnt[];  // [2T + 1] buckets, bucket b = 2T - length
   __shared__ int part[kOrderThreads];
-  const int npairs = (T + 1) / 2, n = npairs * BH, nb = 2 * T + 1, t = threadIdx.x;
-  auto length = [&](int item) {
-    const int qp = item % npairs, bh = item / npairs;
-    const int32_t* cp = col_ptr + size_t(bh) * (T + 1);
+  const int npairs = (T + 1) / 2, nb = 2 * T + 1, t = threadIdx.x, bh = blockIdx.x;
+  const int32_t* cp = col_ptr + size_t(bh) * (T + 1);
+  auto length = [&](int qp) {
     const int j0 = 2 * qp, j1 = 2 * qp + 1;
     int len = cp[j0 + 1] - cp[j0];
     if (j1 < T) len += cp[j1 + 1] - cp[j1];
@@ -415,7 +416,7 @@ __global__ void __launch_bounds__(kOrderThreads) pair_order_kernel(
   };
   for (int b = t; b < nb; b += kOrderThreads) cnt[b] = 0;
   __syncthreads();
-  for (int item = t; item < n; item += kOrderThreads) atomicAdd(&cnt[2 * T - length(item)], 1);
+  for (int qp = t; qp < npairs; qp += kOrderThreads) atomicAdd(&cnt[2 * T - length(qp)], 1);
   __syncthreads();
   // exclusive scan of the buckets: thread t owns a contiguous run of them
   const int per = (nb + kOrderThreads - 1) / kOrderThreads;
@@ -437,8 +438,9 @@ __global__ void __launch_bounds__(kOrderThreads) pair_order_kernel(
     run += c;
   }
   __syncthreads();
-  for (int item = t; item < n; item += kOrderThreads)
-    order[atomicAdd(&cnt[2 * T - length(item)], 1)] = item;
+  int32_t* out = order + size_t(bh) * npairs;
+  for (int qp = t; qp < npairs; qp += kOrderThreads)
+    out[atomicAdd(&cnt[2 * T - length(qp)], 1)] = bh * npairs + qp;
 }
 
 }  // namespace
@@ -449,7 +451,7 @@ cudaError_t launch_pair_order(const Problem& p, const int32_t* col_ptr, int32_t*
   cudaError_t e = cudaFuncSetAttribute(pair_order_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  pair_order_kernel<<<1, kOrderThreads, smem, s>>>(col_ptr, order, p.T, p.BH);
+  pair_order_kernel<<<p.BH, kOrderThreads, smem, s>>>(col_ptr, order, p.T);
   return cudaGetLastError();
 }
 
