@@ -204,6 +204,34 @@ def time_oracle(wl, heads, steps, warmup):
     return sample / sec / 1e12, sec
 
 
+# ---------------------------------------------------------------- ranks
+# One process per GPU; every rank runs an independent replica of the step on
+# its own inputs (weak scaling, no collective on the data path).  Timing is the
+# maximum over ranks of each rank's device time; the whole-job value counts the
+# work of every rank.
+
+def rank_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks_of(x, world, dev):
+    """The maximum of a per-rank float over all ranks (a collective when world > 1)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step, ms_per_step, world):
+    """Executed-block TFLOP/s of all ranks together at the slowest rank's step time."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -314,16 +342,8 @@ def main():
             slab.sla_backward_gated(shape, qq, kk, vv, ww, buf.mask, gate, buf.saved, dd, dq, dk,
                                     dv, dw, d_logit, buf.workspace, stream)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier = lambda: rank_barrier(world)
+    max_over_ranks = lambda x: max_over_ranks_of(x, world, dev)
 
     for _ in range(args.warmup):
         step()
@@ -347,7 +367,7 @@ def main():
     clocks = clk.summary()
 
     fwd_flops, bwd_flops = executed_block_flops(wl, n_crit)
-    value = world * (fwd_flops + bwd_flops) / (ms * 1e-3) / 1e12
+    value = whole_job_tflops(fwd_flops + bwd_flops, ms, world)
 
     # ------------------------------------------------------------ per-kernel times
     slab.sla_profile_begin()
@@ -429,7 +449,7 @@ def main():
         a1.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps)
-        e2e = {"value": world * (fwd_flops + bwd_flops) / (e_ms * 1e-3) / 1e12,
+        e2e = {"value": whole_job_tflops(fwd_flops + bwd_flops, e_ms, world),
                "unit": "TFLOP/s", "ms_per_step": e_ms, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
 
