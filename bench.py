@@ -65,13 +65,12 @@ def executed_block_flops(wl, n_crit):
     return fwd, bwd
 
 
-# DRAM bytes (read + write) per head of one launch, from the ncu captures under
-# profiles/ of the kernels as they are now (4-head case, divided by 4; the
-# traffic grows with the number of heads).  A kernel missing here reports
-# traffic null; an entry must be dropped or re-measured when its kernel changes.
-NCU_DRAM_BYTES_PER_HEAD = {
-    "bwd_sparse": (204.179968e6 + 151.736320e6) / 4,  # bwd_sparse_wan4h_full.md
-}
+# DRAM bytes (read + write) per head of one launch, from an ncu capture of the
+# kernel as it is now (dram__bytes_read.sum + dram__bytes_write.sum of the
+# 4-head Wan case, divided by 4; the traffic grows with the number of heads).
+# A kernel missing here reports traffic null; an entry must be dropped or
+# re-measured whenever its kernel changes.
+NCU_DRAM_BYTES_PER_HEAD = {}
 
 
 def kernel_work(wl, n_crit):
@@ -92,6 +91,7 @@ def kernel_work(wl, n_crit):
         "bwd_q": ("hbm", tok * d * (2 + 2 + 4 + 4) + 2 * BH * T * (d * d + d) * 4 + tok * 4 * 2),
         "bwd_sparse": ("tensor", pairs * 10 * b * b * d),
         "bwd_k": ("hbm", tok * d * (2 + 2 + 8 + 8) + BH * T * (d * d + d) * 4),
+        "bias_rows": ("hbm", tok * (4 + 4) + tok * 64),
         "expand_marginal": ("hbm", BH * Tp * Tp * 2),
         "expand_marginal_t": ("hbm", BH * Tp * Tp * 2),
     }
@@ -256,6 +256,49 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def dense_sdpa_context(B, H, N, d, dev, reps=3):
+    """Dense attention at the same shape through torch SDPA (context only):
+    forward and forward+backward ms per backend, CUDA events on the current
+    stream; FLOPs 4 N^2 d (forward) and 14 N^2 d (forward + backward) per head."""
+    import torch
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    g = torch.Generator(device=dev).manual_seed(0)
+    q, k, v = (torch.randn(B, H, N, d, device=dev, dtype=torch.bfloat16, generator=g)
+               for _ in range(3))
+    fwd_flop = 4.0 * B * H * N * N * d
+    out = {}
+    for name, backend in (("flash", SDPBackend.FLASH_ATTENTION),
+                          ("cudnn", SDPBackend.CUDNN_ATTENTION)):
+        try:
+            with sdpa_kernel([backend]):
+                qq, kk, vv = (x.detach().requires_grad_(True) for x in (q, k, v))
+                def fwd():
+                    return torch.nn.functional.scaled_dot_product_attention(qq, kk, vv)
+                def fwd_bwd():
+                    o = fwd()
+                    o.backward(torch.ones_like(o))
+                for fn in (fwd, fwd_bwd):  # warm-up
+                    fn()
+                torch.cuda.synchronize()
+                res = {}
+                for label, fn in (("fwd", fwd), ("fwd_bwd", fwd_bwd)):
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    for _ in range(reps):
+                        fn()
+                    e1.record()
+                    torch.cuda.synchronize()
+                    res[label + "_ms"] = e0.elapsed_time(e1) / reps
+                res["fwd_tflops"] = fwd_flop / (res["fwd_ms"] * 1e-3) / 1e12
+                res["fwd_bwd_tflops"] = 3.5 * fwd_flop / (res["fwd_bwd_ms"] * 1e-3) / 1e12
+                out[name] = res
+        except Exception as exc:  # a backend this torch build does not offer
+            out[name] = {"unavailable": str(exc).splitlines()[0][:160]}
+    del q, k, v
+    torch.cuda.empty_cache()
+    return out
+
+
 def oracle_n_crit(wl):
     import oracle
     return oracle.block_counts(wl.T, wl.k_h, wl.k_l)[0]
@@ -269,6 +312,8 @@ def main():
     ap.add_argument("--impl", choices=["sla", "reference"], default="sla")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true",
+                    help="skip the dense torch SDPA context timing")
     ap.add_argument("--gate-logit", type=float, default=None,
                     help="run the gated entry points with this gate logit (default: ungated)")
     ap.add_argument("--key-padding", action="store_true",
@@ -385,17 +430,35 @@ def main():
     per_kernel = {name: {"launches": n, "ms_per_launch": tot / n,
                          "share": tot / sum(t for _, t in prof.values())}
                   for name, (n, tot) in prof.items()}
+    capped_k = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
+    for name, rec in per_kernel.items():
+        if name in work:
+            kk, amt = work[name]
+            sec = rec["ms_per_launch"] * 1e-3
+            if kk == "tensor":
+                rec["tflops"] = amt / sec / 1e12
+                rec["frac_of_peak"] = rec["tflops"] / (pk["bf16_tflops_sustained"] if capped_k
+                                                       else pk["bf16_tflops"])
+            else:
+                rec["gbs"] = amt / sec / 1e9
+                rec["frac_of_peak"] = rec["gbs"] / pk["hbm_gbs"]
     dominant = max(prof, key=lambda n: prof[n][1])
     kind, amount = work.get(dominant, ("tensor", 0))
     traffic = (NCU_DRAM_BYTES_PER_HEAD[dominant] * wl.B * wl.H
                if dominant in NCU_DRAM_BYTES_PER_HEAD and args.workload == "train" else None)
     avg_s = prof[dominant][1] / prof[dominant][0] * 1e-3
+    # the tensor peak: the burst figure (a kernel timed at full clock, as the
+    # clock record of the timed region shows), the sustained one (measured under
+    # the power cap) beside it
+    capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
+    tensor_peak = pk["bf16_tflops_sustained"] if capped else pk["bf16_tflops"]
+    tensor_src = f"{src} bf16 cuBLAS " + ("sustained (power cap seen)" if capped else "burst")
     if kind == "tensor":
         achieved = amount / avg_s / 1e12
-        peak = pk["bf16_tflops_sustained"]
+        peak = tensor_peak
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic, "kernel": dominant,
-                "peak_source": f"{src} sustained bf16"}
+                "frac": achieved / peak, "frac_of_sustained": achieved / pk["bf16_tflops_sustained"],
+                "traffic": traffic, "kernel": dominant, "peak_source": tensor_src}
     else:
         achieved = amount / avg_s / 1e9
         peak = pk["hbm_gbs"]
@@ -463,12 +526,17 @@ def main():
                          f"step of the fp64 oracle ({sec:.1f} s), executed-block FLOPs of "
                          f"those heads"}
 
+    dense = None
+    if rank == 0 and world == 1 and not args.no_dense and args.workload == "train":
+        dense = dense_sdpa_context(wl.B, wl.H, wl.N, wl.d, dev)
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
-    peak_t = pk["bf16_tflops_sustained"]
+    peak_t = pk["bf16_tflops_sustained"] if (clocks and "sw_power_cap" in clocks.get("reasons", [])) \
+        else pk["bf16_tflops"]
     cfg = workload_config(wl, n_crit)
     if args.key_padding:
         cfg["n_valid"] = wl.n_valid
@@ -489,6 +557,7 @@ def main():
         "fwd_tflops": fwd_flops / (fwd_ms * 1e-3) / 1e12,
         "bwd_tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12,
         "frac_of_bf16_peak": value / world / peak_t,
+        "dense_attention_context": dense,
         "kernels": per_kernel, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
         "clocks": clocks, "gpu_launches": int(round(launches_per_step * args.steps)),
     }

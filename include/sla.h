@@ -127,7 +127,10 @@ typedef struct {
 SLA_API sla_status sla_query_sizes(const sla_shape* shape, sla_sizes* out);
 
 /* Pool Q and K per block, score the pooled rows and classify every
- * (query block, key block) pair into *mask.  q, k: bf16 [B,H,N,d]. */
+ * (query block, key block) pair into *mask.  q, k: bf16 [B,H,N,d].
+ * Defined by: SLA paper card, "technical framework" step 1 and core point 2
+ * (the weights split into critical, marginal and negligible), English
+ * abstract; the pooled-score ranking is the reading above. */
 SLA_API sla_status sla_classify(const sla_shape* shape, const void* q, const void* k,
                         const sla_mask* mask, void* workspace, size_t workspace_bytes,
                         void* stream);
@@ -152,7 +155,10 @@ SLA_API sla_status sla_classify_from_scores(const sla_shape* shape, const float*
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
  *   - Every call shares the one array: calls that overlap on the GPU (other
- *     streams, other threads) race on it and must be serialized by the caller. */
+ *     streams, other threads) race on it and must be serialized by the caller.
+ *   - The looked-up address is kept per device for the life of the process;
+ *     after cudaDeviceReset() on a device it is stale, so do not call this
+ *     entry point on that device again in the same process. */
 SLA_API sla_status sla_classify_noalloc(const sla_shape* shape, const void* q, const void* k,
                                         const sla_mask* mask, void* stream);
 
@@ -207,7 +213,11 @@ SLA_API sla_status sla_classify_hierarchical_from_scores(const sla_shape* shape,
                                                          const sla_mask* mask, void* workspace,
                                                          size_t workspace_bytes, void* stream);
 
-/* Forward with a given mask: writes o (bf16 [B,H,N,d]) and *saved. */
+/* Forward with a given mask: writes o (bf16 [B,H,N,d]) and *saved.
+ * Defined by: SLA English abstract and paper card "technical framework" steps
+ * 2-4 (critical pairs: exact attention; marginal: linear attention; negligible:
+ * skipped) and step 5 (one fused computation); the combination is the reading
+ * above. */
 SLA_API sla_status sla_forward(const sla_shape* shape, const void* q, const void* k, const void* v,
                        const void* w_proj, const sla_mask* mask, void* o,
                        const sla_saved* saved, void* workspace, size_t workspace_bytes,
@@ -215,7 +225,9 @@ SLA_API sla_status sla_forward(const sla_shape* shape, const void* q, const void
 
 /* Backward of sum(O * dO) with the mask held fixed.  Needs the *saved state
  * of the forward on the same inputs and mask.  Writes dq, dk, dv (fp32
- * [B,H,N,d]) and dw_proj (fp32 [d,d], summed over B, H, N; overwritten). */
+ * [B,H,N,d]) and dw_proj (fp32 [d,d], summed over B, H, N; overwritten).
+ * Defined by: SLA English abstract (the kernel supports the backward pass)
+ * and paper card step 5; the gradients are those of the forward above. */
 SLA_API sla_status sla_backward(const sla_shape* shape, const void* q, const void* k, const void* v,
                         const void* w_proj, const sla_mask* mask, const sla_saved* saved,
                         const void* d_o, float* dq, float* dk, float* dv, float* dw_proj,
@@ -260,6 +272,18 @@ SLA_API sla_status sla_workspace_init(void* workspace, size_t workspace_bytes, v
 /* Synchronize `stream`, then return and clear the workspace's device error
  * word (SLA_OK if no device-side error was recorded). */
 SLA_API sla_status sla_check(void* workspace, void* stream);
+
+/* Test hook for the device-side failure paths.  Writes `what` into a word of
+ * the workspace header that the kernels read at launch (asynchronously on
+ * `stream`; sla_workspace_init() and what = 0 clear it):
+ *   SLA_INJECT_WITHHOLD_LOADS  the sparse forward's copy warp issues none of
+ *     its copies, so every wait on them runs out after its time limit
+ *     (about 2 s); the kernel winds down with nothing in flight and
+ *     sla_check() reports SLA_ERR_TIMEOUT.
+ * No fault, trap or hang is involved; the CUDA context stays usable.  The
+ * paper has no counterpart. */
+#define SLA_INJECT_WITHHOLD_LOADS 1
+SLA_API sla_status sla_debug_inject(void* workspace, int what, void* stream);
 
 /* Static description of a status code. */
 SLA_API const char* sla_strerror(sla_status status);

@@ -25,6 +25,7 @@ __all__ = [
     "sla_profile_begin", "sla_profile_end", "KernelStat", "make_shape", "EXPORTED_SYMBOLS",
     "STATUS", "Gate", "sla_forward_gated", "sla_backward_gated", "Hierarchy",
     "sla_hierarchy_counts", "sla_classify_hierarchical", "sla_classify_hierarchical_from_scores",
+    "sla_debug_inject", "INJECT_WITHHOLD_LOADS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -38,7 +39,9 @@ EXPORTED_SYMBOLS = ["sla_query_sizes", "sla_classify", "sla_classify_from_scores
                     "sla_strerror", "sla_version", "sla_profile_begin", "sla_profile_end",
                     "sla_classify_noalloc", "sla_forward_gated", "sla_backward_gated",
                     "sla_hierarchy_counts", "sla_classify_hierarchical",
-                    "sla_classify_hierarchical_from_scores"]
+                    "sla_classify_hierarchical_from_scores", "sla_debug_inject"]
+
+INJECT_WITHHOLD_LOADS = 1  # SLA_INJECT_WITHHOLD_LOADS of sla.h
 
 
 class SlaError(RuntimeError):
@@ -121,6 +124,7 @@ def lib() -> ctypes.CDLL:
                                                             P(MaskStruct), vp, sz, vp]
         L.sla_workspace_init.argtypes = [vp, sz, vp]
         L.sla_check.argtypes = [vp, vp]
+        L.sla_debug_inject.argtypes = [vp, st, vp]
         L.sla_strerror.argtypes = [st]
         L.sla_strerror.restype = ctypes.c_char_p
         L.sla_version.argtypes = []
@@ -133,7 +137,7 @@ def lib() -> ctypes.CDLL:
                   "sla_backward", "sla_workspace_init", "sla_check", "sla_profile_begin",
                   "sla_profile_end", "sla_forward_gated", "sla_backward_gated",
                   "sla_hierarchy_counts", "sla_classify_hierarchical",
-                  "sla_classify_hierarchical_from_scores"):
+                  "sla_classify_hierarchical_from_scores", "sla_debug_inject"):
             getattr(L, n).restype = st
         _lib = L
     return _lib
@@ -206,6 +210,13 @@ def sla_workspace_init(workspace, stream=None):
 
 def sla_check(workspace, stream=None):
     _check(lib().sla_check(_ptr(workspace), _stream(stream)), "sla_check")
+
+
+def sla_debug_inject(workspace, what: int, stream=None):
+    """Set (what = INJECT_WITHHOLD_LOADS) or clear (what = 0) the workspace's
+    fault-injection word; a test hook for the device-side timeout path."""
+    _check(lib().sla_debug_inject(_ptr(workspace), int(what), _stream(stream)),
+           "sla_debug_inject")
 
 
 def sla_classify(shape: Shape, q, k, mask: MaskStruct, workspace, stream=None):

@@ -17,7 +17,7 @@
 
 namespace sla {
 
-WorkspaceLayout workspace_layout(int BH, int N, int d) {
+WorkspaceLayout workspace_layout(int BH, int N, int d, int n_crit) {
   const int T = N / kBlock, Tp = pad128(T);
   WorkspaceLayout L{};
   size_t off = 0;
@@ -38,6 +38,10 @@ WorkspaceLayout workspace_layout(int BH, int N, int d) {
   L.mmat_t = take(bh * Tp * Tp * 2);
   L.dvec = take(bh * N * 4);
   L.order = take(bh * ((T + 1) / 2) * 4);
+  L.ulen = take(bh * ((T + 1) / 2) * 4);
+  L.ulist = take(bh * T * size_t(n_crit) * 2);
+  L.uflag = take(bh * T * size_t(n_crit));
+  L.bias = take(2 * bh * size_t(N) * 16 * 2);
   L.total = off;
   return L;
 }
@@ -95,6 +99,19 @@ bool make_tmap_f32_bhnd(CUtensorMap* map, const float* base, int BH, int N, int 
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_rows16(CUtensorMap* map, const void* base, int BH, int N) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {16, uint64_t(N), uint64_t(BH)};
+  cuuint64_t strides[2] = {32, uint64_t(N) * 32};
+  cuuint32_t box[3] = {16, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -175,7 +192,7 @@ sla_status fill_sizes(const Problem& p, sla_sizes* o) {
   o->o_s_bytes = bh * N * d * 4;
   o->den_bytes = bh * N * 4;
   o->hz_agg_bytes = bh * T * size_t(summary_width(p.d)) * 4;
-  o->workspace_bytes = workspace_layout(p.BH, p.N, p.d).total;
+  o->workspace_bytes = workspace_layout(p.BH, p.N, p.d, p.n_crit).total;
   return SLA_OK;
 }
 
@@ -192,7 +209,7 @@ sla_status check_mask(const Problem& p, const sla_mask* m, bool need_csr) {
 
 sla_status check_ws(const Problem& p, void* ws, size_t ws_bytes, WorkspaceLayout* L) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return SLA_ERR_INVALID_ARG;
-  *L = workspace_layout(p.BH, p.N, p.d);
+  *L = workspace_layout(p.BH, p.N, p.d, p.n_crit);
   if (ws_bytes < L->total) return SLA_ERR_WORKSPACE;
   return SLA_OK;
 }
@@ -214,27 +231,28 @@ std::mutex g_prof_mu;
 bool g_prof_on = false;
 std::vector<ProfRec> g_prof;
 
-bool prof_mark(cudaStream_t s, cudaEvent_t* ev) {
-  if (cudaEventCreate(ev) != cudaSuccess) return false;
-  return cudaEventRecord(*ev, s) == cudaSuccess;
+}  // namespace
+
+namespace sla {
+
+bool profiler_on() {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  return g_prof_on;
 }
 
-template <typename F>
-cudaError_t launch_named(const char* name, cudaStream_t s, F&& launch) {
-  bool on;
-  {
-    std::lock_guard<std::mutex> g(g_prof_mu);
-    on = g_prof_on;
-  }
-  if (!on) return launch();
-  ProfRec r{name, nullptr, nullptr};
-  if (!prof_mark(s, &r.a)) return cudaErrorUnknown;
-  const cudaError_t e = launch();
-  if (!prof_mark(s, &r.b)) return cudaErrorUnknown;
-  std::lock_guard<std::mutex> g(g_prof_mu);
-  g_prof.push_back(r);
-  return e;
+cudaError_t profiler_mark(cudaStream_t s, cudaEvent_t* ev) {
+  const cudaError_t e = cudaEventCreate(ev);
+  return e != cudaSuccess ? e : cudaEventRecord(*ev, s);
 }
+
+void profiler_record(const char* name, cudaEvent_t a, cudaEvent_t b) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  g_prof.push_back(ProfRec{name, a, b});
+}
+
+}  // namespace sla
+
+namespace {
 
 #define SLA_LAUNCH(name, stream, expr)                                            \
   do {                                                                            \
@@ -487,6 +505,11 @@ static sla_status backward_impl(const sla_shape* shape, const void* q, const voi
   const auto* hz_lo = hz_hi + size_t(p.BH) * p.T * summary_width(p.d);
   float* dvec = at<float>(workspace, L.dvec);
   int32_t* order = at<int32_t>(workspace, L.order);
+  int32_t* ulen = at<int32_t>(workspace, L.ulen);
+  uint16_t* ulist = at<uint16_t>(workspace, L.ulist);
+  uint8_t* uflag = at<uint8_t>(workspace, L.uflag);
+  int* sched = at<int>(workspace, L.err + 128);
+  auto* bias = at<__nv_bfloat16>(workspace, L.bias);
   if (cudaMemsetAsync(dw_proj, 0, size_t(p.d) * p.d * sizeof(float), s) != cudaSuccess)
     return SLA_ERR_CUDA;
   if (d_logit && cudaMemsetAsync(d_logit, 0, sizeof(float), s) != cudaSuccess) return SLA_ERR_CUDA;
@@ -494,9 +517,12 @@ static sla_status backward_impl(const sla_shape* shape, const void* q, const voi
     if (cudaMemsetAsync(dq, 0, size_t(p.BH) * p.N * p.d * sizeof(float), s) != cudaSuccess)
       return SLA_ERR_CUDA;
     SLA_LAUNCH("dvec", s, launch_dvec(p, d_o, saved->o_s, dvec, s));
-    SLA_LAUNCH("pair_order", s, launch_pair_order(p, mask->crit_col_ptr, order, s));
-    SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
-                                 mask->crit_col_idx, order, dq, dk, dv, err, s));
+    SLA_LAUNCH("pair_order", s, launch_pair_order(p, mask->crit_col_ptr, mask->crit_col_idx,
+                                                  ulist, uflag, ulen, order, sched, err, s));
+    SLA_LAUNCH("bias_rows", s, launch_bias_rows(p, saved->lse, dvec, bias, s));
+    SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, bias, mask->crit_col_ptr,
+                                                  ulist, uflag, ulen, order, sched, dq, dk, dv,
+                                                  sms, err, s));
     return SLA_OK;
   }
   // linear branch, query side: D, dQ's linear share (written), dW, and the
@@ -508,9 +534,12 @@ static sla_status backward_impl(const sla_shape* shape, const void* q, const voi
   SLA_LAUNCH("aggregate_t", s, launch_aggregate(p, mmat_t, summ_hi, summ_lo, dh_hi, dh_lo, err, s));
   // sparse branch adds to dQ and writes dK, dV (its tiles longest first); the linear
   // branch's key side adds its share
-  SLA_LAUNCH("pair_order", s, launch_pair_order(p, mask->crit_col_ptr, order, s));
-  SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
-                               mask->crit_col_idx, order, dq, dk, dv, err, s));
+  SLA_LAUNCH("pair_order", s, launch_pair_order(p, mask->crit_col_ptr, mask->crit_col_idx,
+                                                ulist, uflag, ulen, order, sched, err, s));
+  SLA_LAUNCH("bias_rows", s, launch_bias_rows(p, saved->lse, dvec, bias, s));
+  SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, bias, mask->crit_col_ptr, ulist,
+                                                uflag, ulen, order, sched, dq, dk, dv, sms, err,
+                                                s));
   SLA_LAUNCH("bwd_k", s, launch_bwd_k(p, k, v, dh_hi, dh_lo, dk, dv, sms, err, s));
   return SLA_OK;
 }
@@ -537,6 +566,21 @@ sla_status sla_backward_gated(const sla_shape* shape, const void* q, const void*
 sla_status sla_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
   if (!workspace || workspace_bytes < 256) return SLA_ERR_INVALID_ARG;
   if (cudaMemsetAsync(workspace, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SLA_ERR_CUDA;
+  return SLA_OK;
+}
+
+sla_status sla_debug_inject(void* workspace, int what, void* stream) {
+  if (!workspace || what < 0) return SLA_ERR_INVALID_ARG;
+  static int values[2] = {0, SLA_INJECT_WITHHOLD_LOADS};
+  const int* src = what == 0 ? &values[0] : what == SLA_INJECT_WITHHOLD_LOADS ? &values[1] : nullptr;
+  if (!src) return SLA_ERR_INVALID_ARG;
+  // a synchronous copy from a static host value: the word is set (or cleared)
+  // before any later launch on `stream`
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SLA_ERR_CUDA;
+  if (cudaMemcpy(static_cast<uint8_t*>(workspace) + kInjectWordOffset, src, sizeof(int),
+                 cudaMemcpyHostToDevice) != cudaSuccess)
     return SLA_ERR_CUDA;
   return SLA_OK;
 }

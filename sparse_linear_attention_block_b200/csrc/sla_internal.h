@@ -15,6 +15,10 @@ namespace sla {
 constexpr int kBlock = 64;       // tokens per block (the only supported block size)
 constexpr int kMaxT = 4096;      // blocks per sequence
 constexpr size_t kAlign = 1024;  // alignment of every workspace region
+// Workspace header (256 bytes): the device error word at 0, the fault
+// injection word of sla_debug_inject at 64, the sparse backward's tile counter
+// at 128.
+constexpr size_t kInjectWordOffset = 64;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -27,7 +31,7 @@ inline int summary_width(int d) { return d * d + d; }
 
 // Byte offsets of the regions inside the caller's workspace.
 struct WorkspaceLayout {
-  size_t err;        // int32 device error word (+ padding)
+  size_t err;        // the 256-byte header: error word, injection word, tile counter
   size_t qbar;       // fp32 [BH,T,d]   pooled Q
   size_t kbar;       // fp32 [BH,T,d]   pooled K
   size_t summ_hi;    // bf16 [BH,T,d*d+d] (h_j|z_j) forward, (A_i|a_i) backward: high part
@@ -37,10 +41,14 @@ struct WorkspaceLayout {
   size_t mmat_t;     // bf16 [BH,Tp,Tp] its transpose
   size_t dvec;       // fp32 [BH,N]     D_t = dO_t . O_s,t
   size_t order;      // int32 [BH*ceil(T/2)] key-block pairs of the sparse backward, in order
+  size_t ulen;       // int32 [BH*ceil(T/2)] union length of each key-block pair
+  size_t ulist;      // uint16 [BH*T*n_crit] each pair's union, in the pair's column-CSR slot
+  size_t uflag;      // uint8 [BH*T*n_crit] membership bits of the union entries
+  size_t bias;       // bf16 [2][BH,N,16] rows (hi, lo, 0...) of -LSE/scale, then of -D
   size_t total;
 };
 
-WorkspaceLayout workspace_layout(int BH, int N, int d);
+WorkspaceLayout workspace_layout(int BH, int N, int d, int n_crit);
 
 // Validated problem description handed to the launchers.
 struct Problem {
@@ -93,23 +101,53 @@ cudaError_t launch_bwd_q(const Problem& p, const void* q, const void* d_o, const
                          const __nv_bfloat16* hz_lo, float* dvec, float* dq,
                          __nv_bfloat16* summ_hi, __nv_bfloat16* summ_lo, float* dw, float gate,
                          float* d_gate, int num_sms, int* err, cudaStream_t s);
-// Order of the sparse backward's tiles (key-block pairs): heads in sequence,
-// within a head by the summed length of the pair's two column lists, longest
-// first.
-cudaError_t launch_pair_order(const Problem& p, const int32_t* col_ptr, int32_t* order,
-                              cudaStream_t s);
+// The sparse backward's tiles (key-block pairs): the sorted union of each
+// pair's two column lists with membership bits (written into the pair's slot
+// of the column CSR), its length, and the tile order: heads in sequence, the
+// longest unions of a window of a few heads first.
+// `sched` (one int) is reset here for the sparse backward's tile counter.
+cudaError_t launch_pair_order(const Problem& p, const int32_t* col_ptr, const int32_t* col_idx,
+                              uint16_t* ulist, uint8_t* uflag, int32_t* ulen, int32_t* order,
+                              int* sched, int* err, cudaStream_t s);
+// The sparse backward's bias rows: for every token t, (hi, lo) bf16 pairs of
+// -LSE_t/scale and of -D_t, each padded to 16 values.
+cudaError_t launch_bias_rows(const Problem& p, const float* lse, const float* dvec,
+                             __nv_bfloat16* bias, cudaStream_t s);
+// Persistent: min(tiles, num_sms) CTAs take the tiles in order from the
+// counter `sched` (zero at launch).
 cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
-                              const void* d_o, const float* lse, const float* dvec,
-                              const int32_t* col_ptr, const int32_t* col_idx,
-                              const int32_t* order, float* dq, float* dk, float* dv, int* err,
-                              cudaStream_t s);
+                              const void* d_o, const __nv_bfloat16* bias, const int32_t* col_ptr,
+                              const uint16_t* ulist, const uint8_t* uflag, const int32_t* ulen,
+                              const int32_t* order, int* sched, float* dq, float* dk, float* dv,
+                              int num_sms, int* err, cudaStream_t s);
 cudaError_t launch_bwd_k(const Problem& p, const void* k, const void* v,
                          const __nv_bfloat16* dh_hi, const __nv_bfloat16* dh_lo, float* dk,
                          float* dv, int num_sms, int* err, cudaStream_t s);
 
+// Opt-in per-kernel profiler (sla_profile_begin / sla_profile_end): while it
+// is on, every launch made through launch_named() is bracketed by two CUDA
+// events on its stream and recorded under `name`.
+bool profiler_on();
+cudaError_t profiler_mark(cudaStream_t s, cudaEvent_t* ev);
+void profiler_record(const char* name, cudaEvent_t a, cudaEvent_t b);
+
+template <typename F>
+cudaError_t launch_named(const char* name, cudaStream_t s, F&& launch) {
+  if (!profiler_on()) return launch();
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (profiler_mark(s, &a) != cudaSuccess) return cudaErrorUnknown;
+  const cudaError_t e = launch();
+  if (profiler_mark(s, &b) != cudaSuccess) return cudaErrorUnknown;
+  profiler_record(name, a, b);
+  return e;
+}
+
 // TMA descriptor for a bf16 [BH, N, d] tensor viewed as 3D {d, N, BH} with a
 // box of {64, rows, 1} and 128-byte swizzle.  Returns false on failure.
 bool make_tmap_bhnd(CUtensorMap* map, const void* base, int BH, int N, int d, int box_rows);
+// TMA descriptor for a bf16 [BH, N, 16] tensor with a box {16, 64, 1} and
+// 32-byte swizzle (one MMA K-step of 64 rows).
+bool make_tmap_rows16(CUtensorMap* map, const void* base, int BH, int N);
 // TMA descriptor for a bf16 3D tensor {inner, rows, batch} (row pitch = inner).
 bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
                   uint64_t batch, uint32_t box_inner, uint32_t box_rows);

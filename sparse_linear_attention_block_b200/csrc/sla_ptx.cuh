@@ -156,6 +156,16 @@ __device__ __forceinline__ void tma_load_3d(void* dst, uint64_t* bar, const CUte
       : "memory");
 }
 
+// Prefetch a tile of a 3D tensor map into L2 (no shared-memory destination,
+// no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // Tiled 3D store shared -> global (bulk async group; the source tile is in the
 // 128-byte swizzled layout of the map).  Issue after fence_proxy_async_smem()
 // and a barrier with the threads that wrote the tile.
@@ -271,6 +281,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          (uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46)  // descriptor version
          | (2ull << 61);                                               // SWIZZLE_128B
+}
+
+// K-major operand tile of 16 bf16 per row (32-byte rows, 32-byte swizzle, as
+// a TMA box {16, rows} with CU_TENSOR_MAP_SWIZZLE_32B writes it): one MMA
+// K-step; 8-row groups 256 bytes apart.
+__device__ __forceinline__ uint64_t sdesc_sw32_kmajor(uint32_t saddr) {
+  return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t(1) << 16) | (uint64_t(256 >> 4) << 32) |
+         (1ull << 46)    // descriptor version
+         | (6ull << 61);  // SWIZZLE_32B
 }
 
 // K-major operand tile stored as column chunks of 64 bf16 (128 B per row),

@@ -8,21 +8,43 @@
 //   dV_u += P_tu dO_t,  dS_tu = P_tu (dO_t.V_u - D_t)
 //   dQ_t += scale dS_tu K_u,  dK_u += scale dS_tu Q_t
 //
-// Design (sm_100a).  One CTA owns 128 keys = key blocks 2q, 2q+1 and walks the
-// sorted union of their critical query blocks (column CSR).  Per query block
-// i (64 queries): S^T = K Q_i^T and dP^T = V dO_i^T (tcgen05, M = 128 keys),
-// P^T and dS^T back to TMEM (bf16) for dV += P^T dO_i and dK += dS^T Q_i (A
-// from TMEM), and dQ_i^T = K^T dS^T (dS^T via shared memory).  Warp roles:
-//   warps 0-3 / 4-7  two compute warpgroups taking alternate query blocks, so
-//                    one computes P, dS while the other drains its dQ;
-//   warp 8           TMA producer: K, V once; Q_i, dO_i, LSE_i, D_i per stage;
-//   warp 9           single-thread tcgen05 issuer.
-// The warpgroup returns the stage to the producer as soon as the MMAs of its
-// query block are done, reads dQ_i^T from TMEM into registers (freeing the
-// buffer for the next S^T) and adds it into fp32 dQ with coalesced
-// fire-and-forget reductions.
-// TMEM (512 columns): per buffer b in {0,1}: S^T at 128b (later dQ^T), dP^T at
-// 128b + 64; dV at 256, dK at 256 + d.
+// Design (sm_100a).  A tile is 128 keys = key blocks 2q, 2q+1; its work is the
+// sorted union of their critical query blocks (column CSR), one query block
+// (64 queries) per iteration.  The kernel is persistent: one CTA per SM walks
+// tiles in the order given (heads in sequence, longest unions first), with one
+// iteration counter g that runs on across tiles, so that the stage ring, the
+// TMEM chunks and the two compute warpgroups keep their rhythm at a tile
+// boundary.  Per iteration g (query block i):
+//   S'^T = K Q_i^T - LSE_i/scale, dP'^T = V dO_i^T - D_i
+//                                        (tcgen05, M = 128 keys, N = 64; the
+//                                        shifts are one more K-step each: an
+//                                        all-ones tile times the (hi, lo) bf16
+//                                        rows of -LSE/scale and -D)
+//   P^T = exp2(scale log2(e) S'^T) -> TMEM over S'^T, dS^T = P^T dP'^T -> shared
+//                                        memory (compute warpgroup g & 1; no
+//                                        per-query operand besides the TMEM tiles)
+//   dV += P^T dO_i, dK += dS^T Q_i       (A = P^T from TMEM, dS^T from smem)
+//   dQ_i^T = K^T dS^T                    (M = d, N = 64)
+//   dQ_i += scale dQ_i^T^T               (fp32 bulk reductions, TMA engine)
+// TMEM: dV at column 256, dK at 256 + d; four 64-column chunks at 0..255
+// rotate through S^T(g) -> dQ^T(g) in chunk g % 4 and dP^T(g) in chunk
+// (g + 1) % 4, so a chunk's life is S^T(g), dQ^T(g), dP^T(g + 3), S^T(g + 4).
+// The tensor pipe runs S(g + 1), G(g), S(g + 2), G(g + 1), ... (G = dV, dK,
+// dQ^T) and no product waits for the one issued just before it: S(g + 1)
+// needs only the warpgroup's loads of S^T(g), dP^T(g) and the drain of
+// dQ^T(g - 2); G(g) needs P^T(g), dS^T(g), computed while S(g + 1) runs.
+// Warp roles (512 threads; registers rebalanced with setmaxnreg):
+//   warps 0-3 / 4-7  compute warpgroups (even / odd g): P^T, dS^T, and the
+//                    tile's dK (warpgroup 0) / dV (1) epilogue  [168 registers]
+//   warps 8-11       dQ warpgroup: dQ^T out of TMEM, transposed into a shared
+//                    fp32 tile of 32 query rows, added into dQ by one bulk
+//                    reduction of the TMA engine per half (the rows of a query
+//                    block are contiguous in dQ), so that neither the compute
+//                    warps nor the mbarrier traffic queue behind 8192 scalar
+//                    reductions per iteration  [96]
+//   warp 12          TMA producer: K, V per tile; Q_i, dO_i and the bias rows
+//                    of query block i per iteration into a 3-stage ring  [80]
+//   warp 13          single-thread tcgen05 issuer (warps 14-15 idle)  [80]
 #include <cuda_bf16.h>
 
 #include "sla_internal.h"
@@ -38,351 +60,480 @@ template <int D>
 struct SbSmem {
   static constexpr int kKV = 128 * D * 2;       // K or V tile (128 keys)
   static constexpr int kQ = 64 * D * 2;         // Q_i or dO_i tile (64 queries)
-  static constexpr int kStage = 2 * kQ + 1024;  // Q, dO, LSE[64], D[64] (1024-aligned)
-  static constexpr int kDS = 128 * 64 * 2;      // dS^T bf16 [128 keys][64 q], per warpgroup
-  static constexpr int kTiles = 2 * kKV + kNSt * kStage + 2 * kDS;
-  static size_t total(int T) { return 1024 + kTiles + size_t(2 * T) * 3 + 16; }
+  static constexpr int kBias = 64 * 32;         // 64 bias rows of 16 bf16
+  static constexpr int kStage = 2 * kQ + 2 * kBias;  // Q, dO, -LSE/scale rows, -D rows
+  static constexpr int kDS = 128 * 64 * 2;      // dS^T bf16 [128 keys][64 queries]
+  static constexpr int kOnes = 128 * 32;        // all-ones A tile of the bias K-step
+  static constexpr int kStg = 32 * D * 4;       // fp32 dQ rows of 32 queries
+  static constexpr int kTotal = 1024 + 2 * kKV + kNSt * kStage + 2 * kDS + kOnes + kStg;
 };
 
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
+// The waits of this kernel poll with test_wait instead of a suspending
+// try_wait (measured faster here: the waiting warps resume without a
+// wake-up delay); the same time limit and abort flag as mbar_wait.
+__device__ __forceinline__ bool wait_spin(uint64_t* bar, uint32_t phase, int* err,
+                                          volatile int* abort_flag) {
+  if (mbar_test(bar, phase)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_test(bar, phase)) return true;
+    if (abort_flag && *abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      set_error(err, SLA_ERR_TIMEOUT);
+      if (abort_flag) *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// dst[0 .. bytes/4) += src[...] (fp32), by the TMA engine, in the bulk async
+// group of the issuing thread; both addresses 16-byte aligned, bytes a multiple
+// of 16
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const float* src, uint32_t bytes) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      "cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+      "r"(smem_u32(src)), "r"(bytes)
       : "memory");
 }
 
-// 16-byte fire-and-forget fp32 reduction into global memory
-__device__ __forceinline__ void red_add_v4(float* dst, float4 v) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y),
-               "f"(v.z), "f"(v.w)
-               : "memory");
+// A tile: key-block pair qp of head bh, its union length, where its union list
+// starts (the pair's slot in the column CSR); valid = false ends the walk.
+struct Tile {
+  int bh, qp, n, valid;
+  long long slot;
+};
+
+__device__ __forceinline__ Tile tile_at(const int32_t* order, const int32_t* ulen,
+                                        const int32_t* col_ptr, int idx, int n_tiles, int T,
+                                        int n_crit) {
+  Tile t{0, 0, 0, 0, 0};
+  if (idx >= n_tiles) return t;
+  const int npairs = (T + 1) / 2;
+  const int item = order[idx];
+  t.qp = item % npairs;
+  t.bh = item / npairs;
+  t.n = ulen[item];
+  t.slot = (long long)t.bh * T * n_crit + col_ptr[size_t(t.bh) * (T + 1) + 2 * t.qp];
+  t.valid = 1;
+  return t;
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
+__global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-    const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-    const float* __restrict__ lse, const float* __restrict__ dvec,
-    const int32_t* __restrict__ col_ptr, const int32_t* __restrict__ col_idx,
-    const int32_t* __restrict__ order, int N, int T,
-    int n_crit, int nv, float scale_log2, float scale, float* __restrict__ dq, float* __restrict__ dk,
-    float* __restrict__ dv, int* err) {
+    const __grid_constant__ CUtensorMap tm_bias, int BH, const int32_t* __restrict__ col_ptr,
+    const uint16_t* __restrict__ ulist,
+    const uint8_t* __restrict__ uflag, const int32_t* __restrict__ ulen,
+    const int32_t* __restrict__ order, int* __restrict__ sched, int n_tiles, int N, int T,
+    int n_crit, int nv, float scale_log2, float scale, float* __restrict__ dq,
+    float* __restrict__ dk, float* __restrict__ dv, int* err) {
   using L = SbSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = align_smem_1024(smem_raw);
   uint8_t* sK = base;
   uint8_t* sV = sK + L::kKV;
   uint8_t* sSt = sV + L::kKV;
-  uint8_t* sDS = sSt + kNSt * L::kStage;
-  uint16_t* ulist = reinterpret_cast<uint16_t*>(sDS + 2 * L::kDS);
-  uint8_t* uflag = reinterpret_cast<uint8_t*>(ulist + 2 * T);
+  uint8_t* sDS = sSt + kNSt * L::kStage;  // two buffers, for even and odd iterations
+  uint8_t* sOnes = sDS + 2 * L::kDS;
+  float* sStg = reinterpret_cast<float*>(sOnes + L::kOnes);  // dQ staging for bulk reductions
 
-  __shared__ uint64_t kv_full, st_full[kNSt], st_empty[kNSt], s_full[2], p_full[2], m_done[2],
-      tfree[2], wsync[2], fin;
+  __shared__ uint64_t kv_full, tile_done, acc_free, st_full[kNSt], st_empty[kNSt], s_full[2],
+      ld_done[2], p_full[2], m_done[2], dq_free[2], tq_full[2], tq_empty[2], dsync, fin;
+  __shared__ Tile tq[2];  // the tile walk, published by the producer
   __shared__ uint32_t tmem_base;
-  __shared__ int n_union, abort_flag;
-  // this CTA's tile: key-block pair qp of head bh, taken in the order given
-  // (heads in sequence, each head's longest column lists first)
-  const int npairs = (T + 1) / 2;
-  const int item = order[blockIdx.x];
-  const int qp = item % npairs, bh = item / npairs;
+  __shared__ int abort_flag;
   const int warp = threadIdx.x / 32, lane = lane_id();
-  const int kb0 = 2 * qp, kb1 = 2 * qp + 1;
-  const bool has1 = kb1 < T;
   constexpr uint32_t kDV = 256, kDK = 256 + D;
 
   if (warp == 0) tmem_alloc(&tmem_base, 512);
   if (threadIdx.x == 32) {
     mbar_init(&kv_full, 1);
+    mbar_init(&tile_done, 1);
+    mbar_init(&acc_free, 256);
     for (int s = 0; s < kNSt; ++s) {
       mbar_init(&st_full[s], 1);
       mbar_init(&st_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
+      mbar_init(&ld_done[b], 128);
       mbar_init(&p_full[b], 128);
       mbar_init(&m_done[b], 1);
-      mbar_init(&tfree[b], 128);
-      mbar_init(&wsync[b], 128);
+      mbar_init(&dq_free[b], 128);
+      mbar_init(&tq_full[b], 1);
+      mbar_init(&tq_empty[b], 1 + 3 * 128);  // the issuer and three warpgroups
     }
+    mbar_init(&dsync, 128);
     mbar_init(&fin, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 8) {
-    // union of the critical query blocks of key blocks 2q and 2q+1; flag bit h
-    // = query block critical for key block 2q+h (bitmap scratch in the still
-    // idle stage buffers)
-    const int32_t* cp = col_ptr + size_t(bh) * (T + 1);
-    const int32_t* ci = col_idx + size_t(bh) * T * n_crit;
-    int a = cp[kb0], ae = cp[kb0 + 1];
-    int b = has1 ? cp[kb1] : 0, be = has1 ? cp[kb1 + 1] : 0;
-    const int cap = T * n_crit;
-    if (a < 0 || ae > cap || a > ae || b < 0 || be > cap || b > be || ae - a > T || be - b > T) {
-      if (lane == 0) set_error(err, SLA_ERR_DEVICE);
-      a = ae = b = be = 0;
-    }
-    const int n = warp_union(ci + a, ae - a, ci + b, be - b, T, reinterpret_cast<uint32_t*>(sSt),
-                             ulist, uflag, err);
-    if (lane == 0) n_union = n;
-  }
+  for (int x = threadIdx.x; x < L::kOnes / 16; x += blockDim.x)  // bf16 1.0 everywhere
+    reinterpret_cast<uint4*>(sOnes)[x] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u,
+                                                    0x3F803F80u);
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
-  const int nU = n_union;
 
-  if (warp == 8) {
+  // The m-th tile of this CTA, as published by the producer (consumers only).
+  auto next_tile = [&](long m, Tile* t) -> bool {
+    if (!wait_spin(&tq_full[m & 1], uint32_t(m >> 1) & 1, err, &abort_flag)) return false;
+    *t = tq[m & 1];
+    mbar_arrive(&tq_empty[m & 1]);
+    return t->valid != 0;
+  };
+
+  // registers: launched with 128 per thread (65536 in all); the compute
+  // warpgroups take 168, the dQ warpgroup 96 and the last warpgroup 80
+  // (2 x 168 + 96 + 80 = 512 per thread slot of a warpgroup = 65536 / 128)
+  // (each warpgroup executes its one setmaxnreg at the top of its branch)
+  if (warp >= 12) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 80;" ::: "memory");
+   if (warp == 12 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && nU > 0) {
-      fence_proxy_async_smem();  // the union's scratch used these buffers generically
+    {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(&kv_full, 2 * L::kKV);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_bias);
+      long g = 0;       // iterations issued before the current tile
+      int tw = 0;       // tiles with work so far
+      long issued = 0;  // stage loads issued
+      bool kv_pending = false, ok = true;
+      // tiles are taken from a counter shared by all CTAs, in the order given
+      auto fetch = [&]() -> Tile {
+        return tile_at(order, ulen, col_ptr, atomicAdd(sched, 1), n_tiles, T, n_crit);
+      };
+      auto publish = [&](long m, const Tile& t) -> bool {
+        if (m >= 2 && !wait_spin(&tq_empty[m & 1], uint32_t((m >> 1) - 1) & 1, err, &abort_flag))
+          return false;
+        tq[m & 1] = t;
+        mbar_arrive(&tq_full[m & 1]);
+        return true;
+      };
+      // two tiles of look-ahead: the next tile is published while the
+      // current one starts, the one after it is fetched once the current
+      // tile's loads are out (the counter and the tile's lookups take a few
+      // round trips to global memory)
+      Tile cur = fetch();
+      Tile after = cur.valid ? fetch() : cur;
+      ok = publish(0, cur);
+      for (long m = 0; ok && cur.valid; ++m) {
+        const Tile t = cur;
+        cur = after;
+        if (!(ok = publish(m + 1, cur))) break;
+        if (t.n <= 0) {
+          after = cur.valid ? fetch() : cur;
+          continue;
+        }
+        if (cur.valid && cur.n > 0) {  // the next tile's K/V into L2 meanwhile
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(sK + c * 128 * 128, &kv_full, &tm_k, c * 64, qp * 128, bh);
-        tma_load_3d(sV + c * 128 * 128, &kv_full, &tm_v, c * 64, qp * 128, bh);
-      }
-      int issued = 0;
-      for (int n = 0; n < nU; ++n) {
-        const int s = n % kNSt;
-        if (n >= kNSt && !mbar_wait(&st_empty[s], ((n / kNSt) + 1) & 1, err, &abort_flag)) break;
-        uint8_t* st = sSt + s * L::kStage;
-        const int i = ulist[n];
-        mbar_arrive_expect_tx(&st_full[s], 2 * L::kQ + 512);
+          for (int c = 0; c < D / 64; ++c) {
+            tma_prefetch_l2_3d(&tm_k, c * 64, cur.qp * 128, cur.bh);
+            tma_prefetch_l2_3d(&tm_v, c * 64, cur.qp * 128, cur.bh);
+          }
+        }
+        auto load_stage = [&](int k) -> bool {
+          const long gg = g + k;
+          const int s = int(gg % kNSt);
+          if (gg >= kNSt &&
+              !wait_spin(&st_empty[s], uint32_t((gg / kNSt) + 1) & 1, err, &abort_flag))
+            return false;
+          uint8_t* st = sSt + s * L::kStage;
+          const int i = ulist[t.slot + k];
+          mbar_arrive_expect_tx(&st_full[s], L::kStage);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_3d(st + c * 64 * 128, &st_full[s], &tm_q, c * 64, i * 64, t.bh);
+            tma_load_3d(st + L::kQ + c * 64 * 128, &st_full[s], &tm_do, c * 64, i * 64, t.bh);
+          }
+          tma_load_3d(st + 2 * L::kQ, &st_full[s], &tm_bias, 0, i * 64, t.bh);
+          tma_load_3d(st + 2 * L::kQ + L::kBias, &st_full[s], &tm_bias, 0, i * 64, BH + t.bh);
+          ++issued;
+          return true;
+        };
+        // stages of the first iterations need only earlier iterations' stages
+        // back, not the end of the previous tile: issue them before its K/V wait
+        const int early = t.n < kNSt - 1 ? t.n : kNSt - 1;
+        for (int k = 0; ok && k < early; ++k) ok = load_stage(k);
+        if (ok && tw > 0) ok = wait_spin(&tile_done, uint32_t(tw - 1) & 1, err, &abort_flag);
+        if (!ok) break;
+        // every product of the previous tile is done: K, V may be replaced
+        mbar_arrive_expect_tx(&kv_full, 2 * L::kKV);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(st + c * 64 * 128, &st_full[s], &tm_q, c * 64, i * 64, bh);
-          tma_load_3d(st + L::kQ + c * 64 * 128, &st_full[s], &tm_do, c * 64, i * 64, bh);
+          tma_load_3d(sK + c * 128 * 128, &kv_full, &tm_k, c * 64, t.qp * 128, t.bh);
+          tma_load_3d(sV + c * 128 * 128, &kv_full, &tm_v, c * 64, t.qp * 128, t.bh);
         }
-        bulk_load(st + 2 * L::kQ, lse + size_t(bh) * N + size_t(i) * 64, 256, &st_full[s]);
-        bulk_load(st + 2 * L::kQ + 256, dvec + size_t(bh) * N + size_t(i) * 64, 256, &st_full[s]);
-        ++issued;
+        kv_pending = true;
+        for (int k = early; ok && k < t.n; ++k) ok = load_stage(k);
+        after = cur.valid ? fetch() : cur;
+        g += t.n;
+        ++tw;
       }
       if (abort_flag) {
-        mbar_wait(&kv_full, 0, nullptr, nullptr);
-        for (int n = (issued > kNSt ? issued - kNSt : 0); n < issued; ++n)
-          mbar_wait(&st_full[n % kNSt], (n / kNSt) & 1, nullptr, nullptr);
+        // let copies already in flight land before the CTA exits
+        if (kv_pending) wait_spin(&kv_full, uint32_t(tw - 1) & 1, nullptr, nullptr);
+        for (long n = (issued > kNSt ? issued - kNSt : 0); n < issued; ++n)
+          wait_spin(&st_full[n % kNSt], uint32_t(n / kNSt) & 1, nullptr, nullptr);
       }
     }
-  } else if (warp == 9) {
+   } else if (warp == 13 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nU > 0) {
+    {
       constexpr uint32_t id_s = idesc_bf16(128, 64, 0, 0);  // S^T, dP^T
-      constexpr uint32_t id_g = idesc_bf16(128, D, 0, 1);   // dV, dK (A from TMEM)
+      constexpr uint32_t id_g = idesc_bf16(128, D, 0, 1);   // dV (A from TMEM), dK
       constexpr uint32_t id_q = idesc_bf16(128, 64, 1, 1);  // dQ^T = K^T dS^T
-      bool ok = mbar_wait(&kv_full, 0, err, &abort_flag);
       const uint64_t kd_k = desc_kmajor_base(smem_u32(sK)), vd_k = desc_kmajor_base(smem_u32(sV));
       const uint64_t kd_mn = desc_mnmajor_base(smem_u32(sK), 128);
-      // Two in-order streams, issued whichever is ready first:
-      //   S(n):  S^T_n, dP^T_n into buffer n&1 (needs stage n loaded and, for
-      //          n >= 2, dQ^T_{n-2} drained from that buffer; at most one
-      //          S ahead of the G stream, so every barrier stays within a phase)
-      //   G(n):  dV, dK += ...; dQ^T_n (needs P_n, dS_n from the warpgroup)
-      int ns = 0, ng = 0;
-      uint64_t t_last = globaltimer_ns();
-      while (ok && ng < nU) {
-        bool progressed = false;
-        if (ns < nU && ns <= ng + 1 && mbar_test(&st_full[ns % kNSt], (ns / kNSt) & 1) &&
-            (ns < 2 || mbar_test(&tfree[ns & 1], ((ns >> 1) - 1) & 1))) {
-          tc_fence_after();
-          const uint32_t q0 = smem_u32(sSt + (ns % kNSt) * L::kStage), do0 = q0 + L::kQ;
-          const uint32_t st_t = tmem + (ns & 1) * 128, dp_t = st_t + 64;
-          const uint64_t qd = desc_kmajor_base(q0), dod = desc_kmajor_base(do0);
+      const uint64_t ones_d = sdesc_sw32_kmajor(smem_u32(sOnes));
+      long g = 0;
+      int tw = 0;
+      bool ok = true;
+      // dQ^T(x) drained from its chunk, waited for at most once and in
+      // increasing x: the first S of a tile needs the drain of dQ^T(L - 2),
+      // L the previous tile's last iteration, but G(L) is issued before it and
+      // the drain of dQ^T(L) completes the same barrier's next phase, so that
+      // wait is taken before G(L) is issued
+      long dq_waited = -1;
+      auto need_dq = [&](long x) -> bool {
+        if (x <= dq_waited) return true;
+        dq_waited = x;
+        return wait_spin(&dq_free[x & 1], uint32_t(x >> 1) & 1, err, &abort_flag);
+      };
+      // S(gg): S^T into chunk gg % 4, dP^T into chunk (gg + 1) % 4
+      auto issue_s = [&](long gg) -> bool {
+        const int s = int(gg % kNSt);
+        if (!wait_spin(&st_full[s], uint32_t(gg / kNSt) & 1, err, &abort_flag)) return false;
+        if (gg >= 1 &&
+            !wait_spin(&ld_done[(gg - 1) & 1], uint32_t((gg - 1) >> 1) & 1, err, &abort_flag))
+          return false;
+        if (gg >= 3 && !need_dq(gg - 3)) return false;
+        tc_fence_after();
+        const uint32_t q0 = smem_u32(sSt + s * L::kStage), do0 = q0 + L::kQ;
+        const uint32_t cs = tmem + uint32_t(gg & 3) * 64, cp = tmem + uint32_t((gg + 1) & 3) * 64;
+        const uint64_t qd = desc_kmajor_base(q0), dod = desc_kmajor_base(do0);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            mma_ss(st_t, desc_advance(kd_k, kmajor_step_bytes(128, ks)),
-                   desc_advance(qd, kmajor_step_bytes(64, ks)), id_s, ks > 0);
-            mma_ss(dp_t, desc_advance(vd_k, kmajor_step_bytes(128, ks)),
-                   desc_advance(dod, kmajor_step_bytes(64, ks)), id_s, ks > 0);
-          }
-          mma_commit(&s_full[ns & 1]);
-          ++ns;
-          progressed = true;
+        for (int ks = 0; ks < D / 16; ++ks) {
+          mma_ss(cs, desc_advance(kd_k, kmajor_step_bytes(128, ks)),
+                 desc_advance(qd, kmajor_step_bytes(64, ks)), id_s, ks > 0);
+          mma_ss(cp, desc_advance(vd_k, kmajor_step_bytes(128, ks)),
+                 desc_advance(dod, kmajor_step_bytes(64, ks)), id_s, ks > 0);
         }
-        if (ng < ns && mbar_test(&p_full[ng & 1], (ng >> 1) & 1)) {
-          tc_fence_after();
-          const int b = ng & 1;
-          const uint32_t q0 = smem_u32(sSt + (ng % kNSt) * L::kStage), do0 = q0 + L::kQ;
-          const uint32_t st_t = tmem + b * 128, dp_t = st_t + 64;
-          const uint64_t qd = desc_mnmajor_base(q0, 64), dod = desc_mnmajor_base(do0, 64);
+        // the shifts: ones x (hi, lo) rows of -LSE/scale and of -D
+        mma_ss(cs, ones_d, sdesc_sw32_kmajor(q0 + 2 * L::kQ), id_s, 1);
+        mma_ss(cp, ones_d, sdesc_sw32_kmajor(q0 + 2 * L::kQ + L::kBias), id_s, 1);
+        mma_commit(&s_full[gg & 1]);
+        return true;
+      };
+      // G(gg): dV += P^T dO_i (P^T in chunk gg % 4), dK += dS^T Q_i, then dQ^T
+      // over the same chunk (the pipe runs in order: dV has read P^T by then)
+      auto issue_g = [&](long gg, bool first, bool last) -> bool {
+        if (!wait_spin(&p_full[gg & 1], uint32_t(gg >> 1) & 1, err, &abort_flag)) return false;
+        if (first && tw > 0 &&
+            !wait_spin(&acc_free, uint32_t(tw - 1) & 1, err, &abort_flag))
+          return false;
+        if (last && gg >= 2 && !need_dq(gg - 2)) return false;
+        tc_fence_after();
+        const int s = int(gg % kNSt);
+        const uint32_t q0 = smem_u32(sSt + s * L::kStage), do0 = q0 + L::kQ;
+        const uint64_t qmn = desc_mnmajor_base(q0, 64), domn = desc_mnmajor_base(do0, 64);
+        const uint32_t cs = tmem + uint32_t(gg & 3) * 64;
+        const uint32_t ds0 = smem_u32(sDS + (gg & 1) * L::kDS);
+        const uint64_t dsd_k = desc_kmajor_base(ds0), dsd_mn = desc_mnmajor_base(ds0, 128);
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            mma_ts(tmem + kDV, st_t + ks * 8, desc_advance(dod, mnmajor_step_bytes(ks)), id_g,
-                   (ng | ks) != 0);
-            mma_ts(tmem + kDK, dp_t + ks * 8, desc_advance(qd, mnmajor_step_bytes(ks)), id_g,
-                   (ng | ks) != 0);
-          }
-          const uint64_t dsd = desc_mnmajor_base(smem_u32(sDS + b * L::kDS), 128);
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint32_t acc = (!first || ks > 0) ? 1u : 0u;
+          mma_ts(tmem + kDV, cs + ks * 8, desc_advance(domn, mnmajor_step_bytes(ks)), id_g, acc);
+          mma_ss(tmem + kDK, desc_advance(dsd_k, kmajor_step_bytes(128, ks)),
+                 desc_advance(qmn, mnmajor_step_bytes(ks)), id_g, acc);
+        }
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks)  // dQ^T overwrites S^T (its P was consumed by dV above)
-            mma_ss(st_t, desc_advance(kd_mn, mnmajor_step_bytes(ks)),
-                   desc_advance(dsd, mnmajor_step_bytes(ks)), id_q, ks > 0);
-          mma_commit(&m_done[b]);
-          ++ng;
-          progressed = true;
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss(cs, desc_advance(kd_mn, mnmajor_step_bytes(ks)),
+                 desc_advance(dsd_mn, mnmajor_step_bytes(ks)), id_q, ks > 0);
+        mma_commit(&m_done[gg & 1]);
+        mma_commit(&st_empty[s]);
+        if (last) mma_commit(&tile_done);
+        return true;
+      };
+      Tile t;
+      for (long m = 0; ok && (ok = next_tile(m, &t)); ++m) {
+        if (t.n <= 0) continue;
+        if (!(ok = wait_spin(&kv_full, uint32_t(tw) & 1, err, &abort_flag))) break;
+        for (int k = 0; ok && k <= t.n; ++k) {
+          if (k < t.n) ok = issue_s(g + k);
+          if (ok && k >= 1) ok = issue_g(g + k - 1, k == 1, k == t.n);
         }
-        if (progressed) {
-          t_last = globaltimer_ns();
-        } else if (abort_flag) {
-          ok = false;
-        } else if (globaltimer_ns() - t_last > kWaitLimitNs) {
-          set_error(err, SLA_ERR_TIMEOUT);
-          abort_flag = 1;
-          ok = false;
-        }
+        g += t.n;
+        ++tw;
       }
       mma_commit(&fin);
-      mbar_wait(&fin, 0, nullptr, nullptr);
+      wait_spin(&fin, 0, nullptr, nullptr);
     }
-  } else {
-    // ------------------------------------------------------------ compute warpgroups
-    const int wg = warp >> 2, wq = warp & 3;
-    const int r = wq * 32 + lane;  // key row == TMEM lane
-    const int half = r >> 6;
-    const bool key_ok = (half == 0) || has1;  // the key block exists
-    // a padded key (key padding) gets no weight; its dK, dV rows stay 0
-    const bool key_valid = key_ok && qp * 128 + r < nv;
+   }
+  } else if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
+    // ------------------------------------------------------------ dQ warpgroup
+    // dQ_i^T (lane = feature, 64 query columns) of every iteration: each half
+    // (32 queries) is written transposed into the staging tile [32][d] (a
+    // warp's stores for one query cover 32 consecutive features) and added into
+    // the 32 contiguous dQ rows by one bulk reduction, issued by thread 256
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
-    uint8_t* ds_tile = sDS + wg * L::kDS;
-    bool ok = true;
-    uint32_t wphase = 0;
+    const bool leader = threadIdx.x == 256;
+    uint32_t dph = 0;
     // warpgroup barrier with a bounded wait (a thread that gave up cannot
     // leave the other 127 stuck, as a named barrier would)
-    auto wg_sync = [&]() -> bool {
-      mbar_arrive(&wsync[wg]);
-      const bool r = mbar_wait(&wsync[wg], wphase & 1, err, &abort_flag);
-      ++wphase;
-      return r;
+    auto dq_sync = [&]() -> bool {
+      mbar_arrive(&dsync);
+      const bool r2 = wait_spin(&dsync, dph & 1, err, &abort_flag);
+      ++dph;
+      return r2;
     };
-    for (int n = wg; n < nU; n += 2) {
-      const int s = n % kNSt;
-      uint8_t* st = sSt + s * L::kStage;
-      const float* sl = reinterpret_cast<const float*>(st + 2 * L::kQ);
-      const float* sd = sl + 64;
-      const int i = ulist[n];
-      if (!(ok = mbar_wait(&s_full[wg], (n >> 1) & 1, err, &abort_flag))) break;
-      tc_fence_after();
-      // (a padded query row of this block has LSE = +inf, so its P is 0)
-      const bool member = key_valid && ((uflag[n] >> half) & 1);
-      const uint32_t st_t = tmem + lane_base + wg * 128, dp_t = st_t + 64;
-#pragma unroll
-      for (int c0 = 0; c0 < 64; c0 += 32) {
-        float sv[32], dpv[32];
-        tmem_ld32(st_t + c0, sv);
-        tmem_ld32(dp_t + c0, dpv);
-        tmem_ld_wait();
-        uint32_t pk[16], dk16[16];
-        // LSE and D of these 32 queries, as 16-byte broadcast loads
-        float lv[32], dv4[32];
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          *reinterpret_cast<float4*>(&lv[e]) = *reinterpret_cast<const float4*>(sl + c0 + e);
-          *reinterpret_cast<float4*>(&dv4[e]) = *reinterpret_cast<const float4*>(sd + c0 + e);
+    long g = 0;
+    bool ok = true;
+    Tile t;
+    for (long m = 0; ok && (ok = next_tile(m, &t)); ++m) {
+      for (int k = 0; ok && k < t.n; ++k) {
+        const long gg = g + k;
+        const int i = ulist[t.slot + k];
+        float* gdq = dq + (size_t(t.bh) * N + size_t(i) * 64) * D;
+        const uint32_t cs = tmem + lane_base + uint32_t(gg & 3) * 64;
+        if (!(ok = wait_spin(&m_done[gg & 1], uint32_t(gg >> 1) & 1, err, &abort_flag))) break;
+        tc_fence_after();
+        float v[64];
+        if (wq * 32 < D) {
+          tmem_ld32(cs, reinterpret_cast<float(&)[32]>(v[0]));
+          tmem_ld32(cs + 32, reinterpret_cast<float(&)[32]>(v[32]));
+          tmem_ld_wait();
         }
-
+        tc_fence_before();
+        mbar_arrive(&dq_free[gg & 1]);
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float p0 = 0.f, p1 = 0.f;
-          if (member) {
-            p0 = exp2f(fmaf(sv[e], scale_log2, -lv[e] * 1.4426950408889634f));
-            p1 = exp2f(fmaf(sv[e + 1], scale_log2, -lv[e + 1] * 1.4426950408889634f));
+        for (int h = 0; h < 2; ++h) {
+          if (leader) bulk_wait_read_all();  // the previous reduction has read the tile
+          if (!(ok = dq_sync())) break;
+          if (r < D) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) sStg[c * D + r] = v[32 * h + c] * scale;
           }
-          pk[e / 2] = pack_bf16(p0, p1);
-          dk16[e / 2] = pack_bf16(p0 * (dpv[e] - dv4[e]), p1 * (dpv[e + 1] - dv4[e + 1]));
+          fence_proxy_async_smem();
+          if (!(ok = dq_sync())) break;
+          if (leader) {
+            bulk_reduce_add_f32(gdq + size_t(32 * h) * D, sStg, 32 * D * 4);
+            bulk_commit();
+          }
         }
-        tmem_st16(st_t + c0 / 2, pk);
-        tmem_st16(dp_t + c0 / 2, dk16);
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          st_sw128_unit(ds_tile, 128, r, c0 + 8 * u,
-                        make_uint4(dk16[4 * u], dk16[4 * u + 1], dk16[4 * u + 2], dk16[4 * u + 3]));
       }
-      fence_proxy_async_smem();
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[wg]);
-      if (!(ok = mbar_wait(&m_done[wg], (n >> 1) & 1, err, &abort_flag))) break;
-      tc_fence_after();
-      // The MMAs are done with Q_i, dO_i and this warpgroup read LSE_i, D_i:
-      // hand the stage back to the producer before draining dQ.
-      if (wq == 0 && lane == 0) mbar_arrive(&st_empty[s]);
-      // dQ_i^T (lane = feature a, 64 query columns) added into dQ with
-      // fire-and-forget fp32 reductions.
-      float v[64];
-      if (wq * 32 < D) {
-        tmem_ld32(st_t, reinterpret_cast<float(&)[32]>(v[0]));
-        tmem_ld32(st_t + 32, reinterpret_cast<float(&)[32]>(v[32]));
-        tmem_ld_wait();
+      g += t.n > 0 ? t.n : 0;
+    }
+    if (leader) bulk_wait_all();
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 168;" ::: "memory");
+    // ------------------------------------------------------------ compute warpgroups
+    const int wg = warp >> 2, wq = warp & 3;
+    const int r = wq * 32 + lane;  // key row == TMEM lane (dQ^T: feature row)
+    const int half = r >> 6;
+    const uint32_t lane_base = uint32_t(wq * 32) << 16;
+    long g = 0;
+    int tw = 0;
+    bool ok = true;
+    Tile t;
+    for (long m = 0; ok && (ok = next_tile(m, &t)); ++m) {
+      const bool key_ok = (half == 0) || (2 * t.qp + 1 < T);  // the key block exists
+      const int key = t.qp * 128 + r;
+      // a padded key (key padding) gets no weight; its dK, dV rows stay 0
+      const bool key_valid = key_ok && key < nv;
+      float* out_row = (wg == 0 ? dk : dv) + (size_t(t.bh) * N + key) * D;
+      if (t.n <= 0) {
+        if (key_ok) {
+#pragma unroll 4
+          for (int c = 0; c < D; c += 4)
+            *reinterpret_cast<float4*>(out_row + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        continue;
       }
-      tc_fence_before();
-      mbar_arrive(&tfree[wg]);  // the buffer is free once dQ^T is in registers
-      // Transpose through this warpgroup's dS^T tile (its MMA is done and the
-      // tile is not written again before this warpgroup's next query block),
-      // 32 queries at a time, then add 16-byte vectors into dQ.
-      float* stg = reinterpret_cast<float*>(ds_tile);
-      float* gdq = dq + (size_t(bh) * N + size_t(i) * 64) * D;
+      for (int k = int((wg - g) & 1); k < t.n; k += 2) {
+        const long gg = g + k;
+        const uint32_t j = uint32_t(gg >> 1);
+        const int fl = uflag[t.slot + k];
+        const uint32_t cs = tmem + lane_base + uint32_t(gg & 3) * 64;
+        const uint32_t cp = tmem + lane_base + uint32_t((gg + 1) & 3) * 64;
+        if (!(ok = wait_spin(&s_full[wg], j & 1, err, &abort_flag))) break;
+        tc_fence_after();
+        // (a padded query row of this block has LSE = +inf, so its P is 0)
+        const bool member = key_valid && ((fl >> half) & 1);
+        uint32_t pk[32], dsk[32];
+        // dP'^T first: its chunk is the next S^T's, so it is handed back as soon
+        // as it is in registers; then S'^T in two halves of 32 query columns
+        // (P^T goes back over S'^T)
+        float dpa[64];
+        tmem_ld32(cp, reinterpret_cast<float(&)[32]>(dpa[0]));
+        tmem_ld32(cp + 32, reinterpret_cast<float(&)[32]>(dpa[32]));
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&ld_done[wg]);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (ok) {
-          if (wq * 32 < D) {
+        for (int h = 0; h < 2; ++h) {
+          float sv[32];
+          tmem_ld32(cs + 32 * h, sv);
+          tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) stg[e * D + r] = v[32 * h + e] * scale;
+          for (int e = 0; e < 32; e += 2) {
+            float p0 = 0.f, p1 = 0.f;
+            if (member) {
+              p0 = exp2f(sv[e] * scale_log2);
+              p1 = exp2f(sv[e + 1] * scale_log2);
+            }
+            pk[16 * h + e / 2] = pack_bf16(p0, p1);
+            dsk[16 * h + e / 2] = pack_bf16(p0 * dpa[32 * h + e], p1 * dpa[32 * h + e + 1]);
           }
-          ok = wg_sync();
         }
-        if (ok) {
-          const float4* s4 = reinterpret_cast<const float4*>(stg);
+        // P^T (bf16) over the first 32 columns of the S^T chunk; dS^T into this
+        // iteration's buffer once its last reader, G(gg - 2), is done
+        tmem_st16(cs, reinterpret_cast<const uint32_t(&)[16]>(pk[0]));
+        tmem_st16(cs + 16, reinterpret_cast<const uint32_t(&)[16]>(pk[16]));
+        if (gg >= 2 &&
+            !(ok = wait_spin(&m_done[gg & 1], uint32_t((gg - 2) >> 1) & 1, err, &abort_flag)))
+          break;
+        uint8_t* ds_tile = sDS + (gg & 1) * L::kDS;
 #pragma unroll
-          for (int idx = r; idx < 32 * D / 4; idx += 128) {
-            const int qq = idx / (D / 4), a4 = idx % (D / 4);
-            red_add_v4(gdq + size_t(32 * h + qq) * D + a4 * 4, s4[idx]);
-          }
-          ok = wg_sync();
-        }
+        for (int u = 0; u < 8; ++u)
+          st_sw128_unit(ds_tile, 128, r, 8 * u,
+                        make_uint4(dsk[4 * u], dsk[4 * u + 1], dsk[4 * u + 2], dsk[4 * u + 3]));
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[wg]);
       }
       if (!ok) break;
-    }
-    // dK (warpgroup 0) and dV (warpgroup 1) of this tile's keys: fp32 rows
-    // staged as 128-byte swizzled 32-column tiles (in the K/V tiles for dV, the
-    // stage buffers for dK: every product has finished with them) and written
-    // by TMA stores; rows past N (a missing second key block) are clipped.
-    if (nU > 0) {
-      ok = mbar_wait(&fin, 0, err, &abort_flag) && ok;
+      // the tile's dK (warpgroup 0) / dV (warpgroup 1) rows, straight from TMEM
+      if (!(ok = wait_spin(&tile_done, uint32_t(tw) & 1, err, &abort_flag))) break;
       tc_fence_after();
-    }
-    uint8_t* stg_out = wg == 0 ? sSt : sK;
-    const uint32_t acc = tmem + lane_base + (wg == 0 ? kDK : kDV);
-    const float mul = wg == 0 ? scale : 1.0f;
-    const bool h = nU > 0 && ok;
+      const uint32_t acc = tmem + lane_base + (wg == 0 ? kDK : kDV);
+      const float mul = wg == 0 ? scale : 1.0f;
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      float a[32];
-      if (nU > 0) {
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float a[32];
         tmem_ld32(acc + c0, a);
         tmem_ld_wait();
+        if (key_ok) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(out_row + c0 + c) =
+                make_float4(a[c] * mul, a[c + 1] * mul, a[c + 2] * mul, a[c + 3] * mul);
+        }
       }
-      uint8_t* tile = stg_out + (c0 / 32) * (128 * 128);
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        *reinterpret_cast<float4*>(tile + r * 128 + ((u ^ (r & 7)) * 16)) =
-            h ? make_float4(a[4 * u] * mul, a[4 * u + 1] * mul, a[4 * u + 2] * mul,
-                            a[4 * u + 3] * mul)
-              : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    fence_proxy_async_smem();
-    const bool synced = wg_sync();
-    if (wq == 0 && lane == 0 && synced) {
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32)
-        tma_store_3d(wg == 0 ? &tm_dk : &tm_dv, stg_out + (c0 / 32) * (128 * 128), c0, qp * 128,
-                     bh);
-      bulk_commit();
-      bulk_wait_all();
+      tc_fence_before();
+      mbar_arrive(&acc_free);  // the accumulators may be overwritten by the next tile
+      g += t.n;
+      ++tw;
     }
   }
   tc_fence_before();
@@ -390,39 +541,106 @@ __global__ void __launch_bounds__(320, 1) bwd_sparse_kernel(
   if (warp == 0) tmem_free(tmem, 512);
 }
 
-}  // namespace
+// ------------------------------------------------------------------ bias rows
+// For every token: row 0 = (hi, lo) of -LSE/scale, row 1 = (hi, lo) of -D,
+// padded with zeros to 16 bf16 (one MMA K-step), hi = bf16(x), lo = bf16(x -
+// hi).  A padded query row (LSE = +inf) and a row without critical blocks
+// (LSE = -inf, never in a union) both get -inf, so that P = 0.
+__global__ void __launch_bounds__(256) bias_rows_kernel(const float* __restrict__ lse,
+                                                        const float* __restrict__ dvec,
+                                                        uint4* __restrict__ bias, long long ntok,
+                                                        float inv_scale) {
+  const long long t = blockIdx.x * 256ll + threadIdx.x;
+  if (t >= ntok) return;
+  auto row = [&](float x, uint4* out) {
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    const __nv_bfloat16 lo = isfinite(x) ? __float2bfloat16_rn(x - __bfloat162float(hi))
+                                         : __float2bfloat16_rn(0.f);
+    const uint32_t w = uint32_t(__bfloat16_as_ushort(hi)) | (uint32_t(__bfloat16_as_ushort(lo)) << 16);
+    out[0] = make_uint4(w, 0u, 0u, 0u);
+    out[1] = make_uint4(0u, 0u, 0u, 0u);
+  };
+  const float l = lse[t];
+  row(isfinite(l) ? -l * inv_scale : -INFINITY, bias + 2 * t);
+  row(-dvec[t], bias + 2 * (ntok + t));
+}
 
-namespace {
+// ------------------------------------------------------------------ tile unions
+// One warp per key-block pair: the sorted union of the critical query blocks of
+// key blocks 2q and 2q+1 (column CSR), written into the pair's slot of the CSR
+// (its two lists' entries, which the union never outnumbers), with flag bit h
+// = query block critical for key block 2q+h, and the union's length.
+constexpr int kUnionWarps = 8;
+
+__global__ void __launch_bounds__(kUnionWarps * 32) pair_union_kernel(
+    const int32_t* __restrict__ col_ptr, const int32_t* __restrict__ col_idx, int BH, int T,
+    int n_crit, uint16_t* __restrict__ ulist, uint8_t* __restrict__ uflag,
+    int32_t* __restrict__ ulen, int* err) {
+  extern __shared__ uint32_t ubits[];  // [kUnionWarps][2 * ceil(T/32)]
+  const int npairs = (T + 1) / 2;
+  const int w = threadIdx.x / 32, lane = lane_id();
+  const int item = blockIdx.x * kUnionWarps + w;
+  if (item >= BH * npairs) return;
+  const int bh = item / npairs, qp = item % npairs;
+  const int kb0 = 2 * qp, kb1 = 2 * qp + 1;
+  const bool has1 = kb1 < T;
+  const int32_t* cp = col_ptr + size_t(bh) * (T + 1);
+  const int32_t* ci = col_idx + size_t(bh) * T * n_crit;
+  int a = cp[kb0], ae = cp[kb0 + 1];
+  int b = has1 ? cp[kb1] : ae, be = has1 ? cp[kb1 + 1] : ae;
+  const int cap = T * n_crit;
+  if (a < 0 || ae > cap || a > ae || b != ae || be > cap || b > be || ae - a > T || be - b > T) {
+    if (lane == 0) set_error(err, SLA_ERR_DEVICE);
+    if (lane == 0) ulen[item] = 0;
+    return;
+  }
+  const size_t slot = size_t(bh) * T * n_crit + a;
+  const int n = warp_union(ci + a, ae - a, ci + b, be - b, T,
+                           ubits + w * 2 * ((T + 31) / 32), ulist + slot, uflag + slot, err);
+  if (lane == 0) ulen[item] = n;
+}
 
 // ------------------------------------------------------------------ tile order
-// One CTA per head: a counting sort of the head's key-block pairs by the summed
-// length of their two column lists (an upper bound of the pair's union, the
-// tile's work), longest first.  Heads stay in sequence, so the tiles running
-// at any time share one head's Q and dO in L2, and every head's tiles end
-// with its shortest ones.  Pairs of equal length keep no particular order.
+// One CTA: a counting sort of all key-block pairs by the key
+//   head + kStagger * (1 - length / longest length),
+// ascending.  Heads come in sequence, so the tiles running at any time share
+// the Q and dO of a few heads in L2, and within the window of kStagger heads
+// the longest unions (the tiles' work) start first, so that no long tile of
+// the last heads starts near the end of the walk.  Pairs in one bucket keep no
+// particular order.
 constexpr int kOrderThreads = 1024;
+constexpr int kOrderBuckets = 8192;
+constexpr float kStagger = 4.0f;
 
 __global__ void __launch_bounds__(kOrderThreads) pair_order_kernel(
-    const int32_t* __restrict__ col_ptr, int32_t* __restrict__ order, int T) {
-  extern __shared__ int cnt[];  // [2T + 1] buckets, bucket b = 2T - length
+    const int32_t* __restrict__ ulen, int32_t* __restrict__ order, int* __restrict__ sched,
+    int n_items, int npairs, int BH) {
+  __shared__ int cnt[kOrderBuckets];
   __shared__ int part[kOrderThreads];
-  const int npairs = (T + 1) / 2, nb = 2 * T + 1, t = threadIdx.x, bh = blockIdx.x;
-  const int32_t* cp = col_ptr + size_t(bh) * (T + 1);
-  auto length = [&](int qp) {
-    const int j0 = 2 * qp, j1 = 2 * qp + 1;
-    int len = cp[j0 + 1] - cp[j0];
-    if (j1 < T) len += cp[j1 + 1] - cp[j1];
-    return min(max(len, 0), 2 * T);
-  };
-  for (int b = t; b < nb; b += kOrderThreads) cnt[b] = 0;
+  __shared__ int longest;
+  const int t = threadIdx.x;
+  if (t == 0) longest = 1;
+  for (int b = t; b < kOrderBuckets; b += kOrderThreads) cnt[b] = 0;
   __syncthreads();
-  for (int qp = t; qp < npairs; qp += kOrderThreads) atomicAdd(&cnt[2 * T - length(qp)], 1);
+  int mx = 1;
+  for (int i = t; i < n_items; i += kOrderThreads) mx = max(mx, ulen[i]);
+  atomicMax(&longest, mx);
+  __syncthreads();
+  const float inv_len = 1.0f / float(longest);
+  const float per = float(kOrderBuckets) / (float(BH) + kStagger);
+  auto bucket = [&](int i) {
+    const float len = float(min(max(ulen[i], 0), longest));
+    const int b = int((float(i / npairs) + kStagger * (1.0f - len * inv_len)) * per);
+    return min(max(b, 0), kOrderBuckets - 1);
+  };
+  for (int i = t; i < n_items; i += kOrderThreads) atomicAdd(&cnt[bucket(i)], 1);
   __syncthreads();
   // exclusive scan of the buckets: thread t owns a contiguous run of them
-  const int per = (nb + kOrderThreads - 1) / kOrderThreads;
-  const int b0 = min(nb, t * per), b1 = min(nb, b0 + per);
+  constexpr int kPer = kOrderBuckets / kOrderThreads;
+  const int b0 = t * kPer;
   int sum = 0;
-  for (int b = b0; b < b1; ++b) sum += cnt[b];
+#pragma unroll
+  for (int b = 0; b < kPer; ++b) sum += cnt[b0 + b];
   part[t] = sum;
   __syncthreads();
   for (int o = 1; o < kOrderThreads; o <<= 1) {  // inclusive scan of the run sums
@@ -432,61 +650,72 @@ __global__ void __launch_bounds__(kOrderThreads) pair_order_kernel(
     __syncthreads();
   }
   int run = part[t] - sum;
-  for (int b = b0; b < b1; ++b) {
-    const int c = cnt[b];
-    cnt[b] = run;
+#pragma unroll
+  for (int b = 0; b < kPer; ++b) {
+    const int c = cnt[b0 + b];
+    cnt[b0 + b] = run;
     run += c;
   }
   __syncthreads();
-  int32_t* out = order + size_t(bh) * npairs;
-  for (int qp = t; qp < npairs; qp += kOrderThreads)
-    out[atomicAdd(&cnt[2 * T - length(qp)], 1)] = bh * npairs + qp;
+  for (int i = t; i < n_items; i += kOrderThreads) order[atomicAdd(&cnt[bucket(i)], 1)] = i;
+  if (t == 0) *sched = 0;  // the sparse backward's tile counter
 }
 
 }  // namespace
 
-cudaError_t launch_pair_order(const Problem& p, const int32_t* col_ptr, int32_t* order,
-                              cudaStream_t s) {
-  const size_t smem = sizeof(int) * size_t(2 * p.T + 1);
-  cudaError_t e = cudaFuncSetAttribute(pair_order_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+cudaError_t launch_pair_order(const Problem& p, const int32_t* col_ptr, const int32_t* col_idx,
+                              uint16_t* ulist, uint8_t* uflag, int32_t* ulen, int32_t* order,
+                              int* sched, int* err, cudaStream_t s) {
+  const int npairs = (p.T + 1) / 2;
+  const size_t ubytes = sizeof(uint32_t) * kUnionWarps * 2 * size_t((p.T + 31) / 32);
+  const int ublocks = (p.BH * npairs + kUnionWarps - 1) / kUnionWarps;
+  pair_union_kernel<<<ublocks, kUnionWarps * 32, ubytes, s>>>(col_ptr, col_idx, p.BH, p.T,
+                                                              p.n_crit, ulist, uflag, ulen, err);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  pair_order_kernel<<<p.BH, kOrderThreads, smem, s>>>(col_ptr, order, p.T);
+  pair_order_kernel<<<1, kOrderThreads, 0, s>>>(ulen, order, sched, p.BH * npairs, npairs, p.BH);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bias_rows(const Problem& p, const float* lse, const float* dvec,
+                             __nv_bfloat16* bias, cudaStream_t s) {
+  const long long ntok = (long long)p.BH * p.N;
+  bias_rows_kernel<<<unsigned((ntok + 255) / 256), 256, 0, s>>>(
+      lse, dvec, reinterpret_cast<uint4*>(bias), ntok, 1.0f / p.scale);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
-                              const void* d_o, const float* lse, const float* dvec,
-                              const int32_t* col_ptr, const int32_t* col_idx,
-                              const int32_t* order, float* dq, float* dk, float* dv, int* err,
-                              cudaStream_t s) {
-  CUtensorMap tq, tk, tv, tdo, tdk, tdv;
-  if (!make_tmap_f32_bhnd(&tdk, dk, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
-  if (!make_tmap_f32_bhnd(&tdv, dv, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
+                              const void* d_o, const __nv_bfloat16* bias, const int32_t* col_ptr,
+                              const uint16_t* ulist, const uint8_t* uflag, const int32_t* ulen,
+                              const int32_t* order, int* sched, float* dq, float* dk, float* dv,
+                              int num_sms, int* err, cudaStream_t s) {
+  CUtensorMap tq, tk, tv, tdo, tb;
+  if (!make_tmap_rows16(&tb, bias, 2 * p.BH, p.N)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tq, q, p.BH, p.N, p.d, 64)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tk, k, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tv, v, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tdo, d_o, p.BH, p.N, p.d, 64)) return cudaErrorInvalidValue;
-  dim3 grid(((p.T + 1) / 2) * p.BH);
+  const int n_tiles = ((p.T + 1) / 2) * p.BH;
+  dim3 grid(std::min(n_tiles, std::max(num_sms, 1)));
   cudaError_t e;
   if (p.d == 128) {
-    const size_t smem = SbSmem<128>::total(p.T);
+    constexpr size_t smem = SbSmem<128>::kTotal;
     e = cudaFuncSetAttribute(bwd_sparse_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem));
     if (e != cudaSuccess) return e;
-    bwd_sparse_kernel<128><<<grid, 320, smem, s>>>(tq, tk, tv, tdo, tdk, tdv, lse, dvec, col_ptr,
-                                                   col_idx, order,
-                                                   p.N, p.T, p.n_crit, p.nv, p.scale_log2, p.scale, dq,
-                                                   dk, dv, err);
+    bwd_sparse_kernel<128><<<grid, 512, smem, s>>>(tq, tk, tv, tdo, tb, p.BH, col_ptr, ulist,
+                                                   uflag, ulen, order, sched, n_tiles, p.N, p.T,
+                                                   p.n_crit, p.nv, p.scale_log2, p.scale, dq, dk,
+                                                   dv, err);
   } else {
-    const size_t smem = SbSmem<64>::total(p.T);
+    constexpr size_t smem = SbSmem<64>::kTotal;
     e = cudaFuncSetAttribute(bwd_sparse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem));
     if (e != cudaSuccess) return e;
-    bwd_sparse_kernel<64><<<grid, 320, smem, s>>>(tq, tk, tv, tdo, tdk, tdv, lse, dvec, col_ptr,
-                                                  col_idx, order,
-                                                  p.N, p.T, p.n_crit, p.nv, p.scale_log2, p.scale, dq,
-                                                  dk, dv, err);
+    bwd_sparse_kernel<64><<<grid, 512, smem, s>>>(tq, tk, tv, tdo, tb, p.BH, col_ptr, ulist,
+                                                  uflag, ulen, order, sched, n_tiles, p.N, p.T, p.n_crit,
+                                                  p.nv, p.scale_log2, p.scale, dq, dk, dv, err);
   }
   return cudaGetLastError();
 }

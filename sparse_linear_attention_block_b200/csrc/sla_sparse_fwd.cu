@@ -102,7 +102,10 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
 
   if (warp == 4) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0 && nU > 0) {
+    // (sla_debug_inject's SLA_INJECT_WITHHOLD_LOADS: issue none of the copies,
+    // so that every wait on them runs out with nothing in flight)
+    const bool withhold = (err[kInjectWordOffset / 4] & SLA_INJECT_WITHHOLD_LOADS) != 0;
+    if (lane == 0 && nU > 0 && !withhold) {
       fence_proxy_async_smem();  // the union's scratch used these buffers generically
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
