@@ -29,10 +29,10 @@
 // TMEM: dV at column 256, dK at 256 + d; four 64-column chunks at 0..255
 // rotate through S^T(g) -> dQ^T(g) in chunk g % 4 and dP^T(g) in chunk
 // (g + 1) % 4, so a chunk's life is S^T(g), dQ^T(g), dP^T(g + 3), S^T(g + 4).
-// The tensor pipe runs S(g + 1), G(g), S(g + 2), G(g + 1), ... (G = dV, dK,
-// dQ^T) and no product waits for the one issued just before it: S(g + 1)
-// needs only the warpgroup's loads of S^T(g), dP^T(g) and the drain of
-// dQ^T(g - 2); G(g) needs P^T(g), dS^T(g), computed while S(g + 1) runs.
+// The S groups (S'^T, dP'^T) and the G groups (dV, dK, dQ^T) come from two
+// issuing threads and interleave in the tensor pipe: S(g + 1) needs only the
+// warpgroup's load of dP^T(g) and the drain of dQ^T(g - 2); G(g) needs P^T(g),
+// dS^T(g), computed while S(g + 1) runs.
 // Warp roles (512 threads; registers rebalanced with setmaxnreg):
 //   warps 0-3 / 4-7  compute warpgroups (even / odd g): P^T, dS^T, and the
 //                    tile's dK (warpgroup 0) / dV (1) epilogue  [168 registers]
@@ -44,7 +44,8 @@
 //                    reductions per iteration  [96]
 //   warp 12          TMA producer: K, V per tile; Q_i, dO_i and the bias rows
 //                    of query block i per iteration into a 3-stage ring  [80]
-//   warp 13          single-thread tcgen05 issuer (warps 14-15 idle)  [80]
+//   warps 13 / 14    single-thread tcgen05 issuers of the S and the G groups
+//                    (warp 15 idle)  [80]
 #include <cuda_bf16.h>
 
 #include "sla_internal.h"
@@ -84,6 +85,11 @@ __device__ __forceinline__ bool wait_spin(uint64_t* bar, uint32_t phase, int* er
       return false;
     }
   }
+}
+
+// At most one committed bulk group of this thread is still reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_le1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
 // dst[0 .. bytes/4) += src[...] (fp32), by the TMA engine, in the bulk async
@@ -139,7 +145,7 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
   float* sStg = reinterpret_cast<float*>(sOnes + L::kOnes);  // dQ staging for bulk reductions
 
   __shared__ uint64_t kv_full, tile_done, acc_free, st_full[kNSt], st_empty[kNSt], s_full[2],
-      ld_done[2], p_full[2], m_done[2], dq_free[2], tq_full[2], tq_empty[2], dsync, fin;
+      ld_done[2], p_full[2], m_done[4], dq_free[4], tq_full[2], tq_empty[2], fin;
   __shared__ Tile tq[2];  // the tile walk, published by the producer
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
@@ -160,12 +166,13 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
       mbar_init(&ld_done[b], 128);
       mbar_init(&p_full[b], 128);
       mbar_init(&m_done[b], 1);
+      mbar_init(&m_done[b + 2], 1);
       mbar_init(&dq_free[b], 128);
+      mbar_init(&dq_free[b + 2], 128);
       mbar_init(&tq_full[b], 1);
-      mbar_init(&tq_empty[b], 1 + 3 * 128);  // the issuer and three warpgroups
+      mbar_init(&tq_empty[b], 2 + 3 * 128);  // the two issuers and three warpgroups
     }
-    mbar_init(&dsync, 128);
-    mbar_init(&fin, 1);
+    mbar_init(&fin, 2);  // one commit from each issuer
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -282,8 +289,15 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
           wait_spin(&st_full[n % kNSt], uint32_t(n / kNSt) & 1, nullptr, nullptr);
       }
     }
-   } else if (warp == 13 && lane == 0) {
-    // ------------------------------------------------------------ MMA issuer
+   } else if ((warp == 13 || warp == 14) && lane == 0) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two threads feed the tensor pipe: warp 13 the S groups, warp 14 the G
+    // groups.  The pipe takes only a few instructions ahead of execution, so a
+    // single issuer that checks barriers between groups leaves it idle for
+    // every check; with two, one stream's checks overlap the other's
+    // products.  The two streams touch different TMEM chunks (the chunk
+    // rotation above), so only the barriers order them; each commit tracks its
+    // own thread's products.
     {
       constexpr uint32_t id_s = idesc_bf16(128, 64, 0, 0);  // S^T, dP^T
       constexpr uint32_t id_g = idesc_bf16(128, D, 0, 1);   // dV (A from TMEM), dK
@@ -291,28 +305,22 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
       const uint64_t kd_k = desc_kmajor_base(smem_u32(sK)), vd_k = desc_kmajor_base(smem_u32(sV));
       const uint64_t kd_mn = desc_mnmajor_base(smem_u32(sK), 128);
       const uint64_t ones_d = sdesc_sw32_kmajor(smem_u32(sOnes));
+      const bool s_stream = warp == 13;
       long g = 0;
       int tw = 0;
       bool ok = true;
-      // dQ^T(x) drained from its chunk, waited for at most once and in
-      // increasing x: the first S of a tile needs the drain of dQ^T(L - 2),
-      // L the previous tile's last iteration, but G(L) is issued before it and
-      // the drain of dQ^T(L) completes the same barrier's next phase, so that
-      // wait is taken before G(L) is issued
-      long dq_waited = -1;
-      auto need_dq = [&](long x) -> bool {
-        if (x <= dq_waited) return true;
-        dq_waited = x;
-        return wait_spin(&dq_free[x & 1], uint32_t(x >> 1) & 1, err, &abort_flag);
-      };
-      // S(gg): S^T into chunk gg % 4, dP^T into chunk (gg + 1) % 4
+      // S(gg): S^T into chunk gg % 4, dP^T into chunk (gg + 1) % 4, once the
+      // stage is loaded, dP^T(gg - 1) is out of its chunk and dQ^T(gg - 3) is
+      // drained
       auto issue_s = [&](long gg) -> bool {
         const int s = int(gg % kNSt);
         if (!wait_spin(&st_full[s], uint32_t(gg / kNSt) & 1, err, &abort_flag)) return false;
         if (gg >= 1 &&
             !wait_spin(&ld_done[(gg - 1) & 1], uint32_t((gg - 1) >> 1) & 1, err, &abort_flag))
           return false;
-        if (gg >= 3 && !need_dq(gg - 3)) return false;
+        if (gg >= 3 &&
+            !wait_spin(&dq_free[(gg - 3) & 3], uint32_t((gg - 3) >> 2) & 1, err, &abort_flag))
+          return false;
         tc_fence_after();
         const uint32_t q0 = smem_u32(sSt + s * L::kStage), do0 = q0 + L::kQ;
         const uint32_t cs = tmem + uint32_t(gg & 3) * 64, cp = tmem + uint32_t((gg + 1) & 3) * 64;
@@ -331,13 +339,14 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
         return true;
       };
       // G(gg): dV += P^T dO_i (P^T in chunk gg % 4), dK += dS^T Q_i, then dQ^T
-      // over the same chunk (the pipe runs in order: dV has read P^T by then)
+      // over the same chunk (one thread's products run in order: dV has read
+      // P^T by then).  G(gg) follows S(gg) through p_full, so its commit also
+      // frees the stage for the producer.
       auto issue_g = [&](long gg, bool first, bool last) -> bool {
         if (!wait_spin(&p_full[gg & 1], uint32_t(gg >> 1) & 1, err, &abort_flag)) return false;
         if (first && tw > 0 &&
             !wait_spin(&acc_free, uint32_t(tw - 1) & 1, err, &abort_flag))
           return false;
-        if (last && gg >= 2 && !need_dq(gg - 2)) return false;
         tc_fence_after();
         const int s = int(gg % kNSt);
         const uint32_t q0 = smem_u32(sSt + s * L::kStage), do0 = q0 + L::kQ;
@@ -356,7 +365,7 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
         for (int ks = 0; ks < 8; ++ks)
           mma_ss(cs, desc_advance(kd_mn, mnmajor_step_bytes(ks)),
                  desc_advance(dsd_mn, mnmajor_step_bytes(ks)), id_q, ks > 0);
-        mma_commit(&m_done[gg & 1]);
+        mma_commit(&m_done[gg & 3]);
         mma_commit(&st_empty[s]);
         if (last) mma_commit(&tile_done);
         return true;
@@ -364,48 +373,64 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
       Tile t;
       for (long m = 0; ok && (ok = next_tile(m, &t)); ++m) {
         if (t.n <= 0) continue;
-        if (!(ok = wait_spin(&kv_full, uint32_t(tw) & 1, err, &abort_flag))) break;
-        for (int k = 0; ok && k <= t.n; ++k) {
-          if (k < t.n) ok = issue_s(g + k);
-          if (ok && k >= 1) ok = issue_g(g + k - 1, k == 1, k == t.n);
+        if (s_stream) {
+          if (!(ok = wait_spin(&kv_full, uint32_t(tw) & 1, err, &abort_flag))) break;
+          for (int k = 0; ok && k < t.n; ++k) ok = issue_s(g + k);
+        } else {
+          for (int k = 0; ok && k < t.n; ++k) ok = issue_g(g + k, k == 0, k == t.n - 1);
         }
         g += t.n;
         ++tw;
       }
       mma_commit(&fin);
-      wait_spin(&fin, 0, nullptr, nullptr);
+      mbar_wait(&fin, 0, nullptr, nullptr);
     }
    }
   } else if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
     // ------------------------------------------------------------ dQ warpgroup
-    // dQ_i^T (lane = feature, 64 query columns) of every iteration: each half
-    // (32 queries) is written transposed into the staging tile [32][d] (a
-    // warp's stores for one query cover 32 consecutive features) and added into
-    // the 32 contiguous dQ rows by one bulk reduction, issued by thread 256
+    // dQ_i^T (lane = feature, 64 query columns) of every iteration, in four
+    // quarters of 16 queries: each is written transposed into one of two
+    // staging buffers [16][d] (a warp's stores for one query cover 32
+    // consecutive features) and added into the 16 contiguous dQ rows by one
+    // bulk reduction issued by thread 256; the reduction of one quarter reads
+    // its buffer while the next quarter is written into the other.
+    // The warpgroup synchronizes with hardware named barrier 1.  Every thread
+    // runs the same sequence of them: the trip counts come from the shared
+    // tile queue, and each wait's outcome is made common to the warpgroup with
+    // bar.red.and before anything depends on it, so no thread can be left at
+    // a barrier that another has skipped.
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
     const bool leader = threadIdx.x == 256;
-    uint32_t dph = 0;
-    // warpgroup barrier with a bounded wait (a thread that gave up cannot
-    // leave the other 127 stuck, as a named barrier would)
-    auto dq_sync = [&]() -> bool {
-      mbar_arrive(&dsync);
-      const bool r2 = wait_spin(&dsync, dph & 1, err, &abort_flag);
-      ++dph;
-      return r2;
+    auto wg_bar = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
+    auto wg_all = [](bool p) -> bool {
+      uint32_t res;
+      asm volatile(
+          "{\n\t.reg .pred a, b;\n\t"
+          "setp.ne.b32 a, %1, 0;\n\t"
+          "bar.red.and.pred b, 1, 128, a;\n\t"
+          "selp.b32 %0, 1, 0, b;\n\t}"
+          : "=r"(res)
+          : "r"(uint32_t(p))
+          : "memory");
+      return res != 0;
     };
+    float* stg[2] = {sStg, sStg + 16 * D};
     long g = 0;
     bool ok = true;
     Tile t;
-    for (long m = 0; ok && (ok = next_tile(m, &t)); ++m) {
-      for (int k = 0; ok && k < t.n; ++k) {
+    for (long m = 0; ok; ++m) {
+      const bool got = next_tile(m, &t);
+      if (!wg_all(got)) break;
+      for (int k = 0; k < t.n; ++k) {
         const long gg = g + k;
         const int i = ulist[t.slot + k];
         float* gdq = dq + (size_t(t.bh) * N + size_t(i) * 64) * D;
         const uint32_t cs = tmem + lane_base + uint32_t(gg & 3) * 64;
-        if (!(ok = wait_spin(&m_done[gg & 1], uint32_t(gg >> 1) & 1, err, &abort_flag))) break;
+        const bool w = wait_spin(&m_done[gg & 3], uint32_t(gg >> 2) & 1, err, &abort_flag);
+        if (!(ok = wg_all(w))) break;
         tc_fence_after();
         float v[64];
         if (wq * 32 < D) {
@@ -414,19 +439,20 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
           tmem_ld_wait();
         }
         tc_fence_before();
-        mbar_arrive(&dq_free[gg & 1]);
+        mbar_arrive(&dq_free[gg & 3]);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (leader) bulk_wait_read_all();  // the previous reduction has read the tile
-          if (!(ok = dq_sync())) break;
+        for (int qt = 0; qt < 4; ++qt) {
+          float* buf = stg[qt & 1];
+          if (leader) bulk_wait_read_le1();  // the reduction that read this buffer is done with it
+          wg_bar();
           if (r < D) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) sStg[c * D + r] = v[32 * h + c] * scale;
+            for (int c = 0; c < 16; ++c) buf[c * D + r] = v[16 * qt + c] * scale;
           }
           fence_proxy_async_smem();
-          if (!(ok = dq_sync())) break;
+          wg_bar();
           if (leader) {
-            bulk_reduce_add_f32(gdq + size_t(32 * h) * D, sStg, 32 * D * 4);
+            bulk_reduce_add_f32(gdq + size_t(16 * qt) * D, buf, 16 * D * 4);
             bulk_commit();
           }
         }
@@ -500,7 +526,7 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
         tmem_st16(cs, reinterpret_cast<const uint32_t(&)[16]>(pk[0]));
         tmem_st16(cs + 16, reinterpret_cast<const uint32_t(&)[16]>(pk[16]));
         if (gg >= 2 &&
-            !(ok = wait_spin(&m_done[gg & 1], uint32_t((gg - 2) >> 1) & 1, err, &abort_flag)))
+            !(ok = wait_spin(&m_done[(gg - 2) & 3], uint32_t((gg - 2) >> 2) & 1, err, &abort_flag)))
           break;
         uint8_t* ds_tile = sDS + (gg & 1) * L::kDS;
 #pragma unroll
