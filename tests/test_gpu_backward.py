@@ -83,19 +83,50 @@ def test_backward_all_critical_matches_torch_autograd():
 
 
 def test_backward_sparse_key_gradient_sums_to_zero():
-    # no marginal pairs: only the softmax branch, whose K-shift invariance
-    # makes the key gradients of each head sum to zero
+    """No marginal pairs: only the softmax branch, whose invariance to a shift
+    of all keys makes the key gradients of each head sum to zero:
+    sum_u dK_u = scale sum_t Q_t r_t with r_t = sum_u dS_tu = sum_u P_tu dP_tu
+    - D_t sum_u P_tu = 0 in exact arithmetic.  The library rounds P to bf16 in
+    the forward's P V product (which D_t = dO_t . O_s,t carries) and dS to
+    bf16 before the dK product.  Each rounding is an independent relative error
+    uniform in +-2^-9 (standard deviation 2^-9 / sqrt(3)), so r_t has variance
+    s^2 sum_u ((P_tu dP_tu)^2 + dS_tu^2) and component c of sum_u dK_u has
+    variance sum_t (scale Q_tc)^2 var(r_t); the residual's l1 norm must stay
+    within 6 standard deviations summed over the components.  The variances
+    are evaluated with the oracle's P, dP and dS on the same inputs and
+    classes.  (fp32 accumulation errors are orders of magnitude smaller.)"""
     wl = sla_inputs.make("tiny", k_h=0.5, k_l=0.5, with_grad=True)
     run = Run(wl)
     run.classify()
     run.forward()
     run.backward(wl.d_o)
+    cls = run.cls()
     dk = run.np(run.dk)
-    # exact only in exact arithmetic: bf16 P in the forward's P V product makes
-    # D = dO . O_s differ slightly from sum_u P dP, a per-row common mode
-    resid = np.abs(dk.sum(axis=2)).sum(axis=-1)
+    resid = np.abs(dk.sum(axis=2)).sum(axis=-1)  # [B, H]
+    fwd = oracle.forward(wl.q, wl.k, wl.v, wl.w_proj, cls, wl.block, wl.scale)
+    q, k, v, do = (np.asarray(x, np.float64) for x in (wl.q, wl.k, wl.v, wl.d_o))
+    B, H, N, d = q.shape
+    s2 = (2.0 ** -9) ** 2 / 3.0
+    bound = np.zeros((B, H))
+    for b in range(B):
+        for h in range(H):
+            var = np.zeros(d)
+            for i in range(wl.T):
+                crit = np.nonzero(cls[b, h, i] == 1)[0]
+                if crit.size == 0:
+                    continue
+                keys = np.concatenate([np.arange(j * 64, (j + 1) * 64) for j in crit])
+                rows = slice(i * 64, (i + 1) * 64)
+                p = np.exp(q[b, h, rows] @ k[b, h, keys].T * wl.scale
+                           - fwd["lse"][b, h, rows, None])
+                dp = do[b, h, rows] @ v[b, h, keys].T
+                ds = p * (dp - np.sum(do[b, h, rows] * fwd["o_s"][b, h, rows], 1, keepdims=True))
+                var_r = s2 * ((p * dp) ** 2 + ds ** 2).sum(axis=1)
+                var += ((wl.scale * q[b, h, rows]) ** 2 * var_r[:, None]).sum(axis=0)
+            bound[b, h] = 6.0 * np.sqrt(var).sum()
     total = np.abs(dk).sum(axis=(2, 3))
-    assert np.all(resid <= 3e-3 * total), (resid / total)
+    print("key-gradient sums / sum|dK|:", resid / total, "bound:", bound / total)
+    assert np.all(resid <= bound), (resid, bound)
 
 
 def test_backward_wan_full_size_sampled():
