@@ -132,6 +132,22 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// named barrier over a subset of warps that also ANDs a predicate over them:
+// every participant gets the same result (callers decide on it together, so
+// that none is left waiting at a barrier another has skipped)
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bool p) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t.reg .pred a, b;\n\t"
+      "setp.ne.b32 a, %1, 0;\n\t"
+      "bar.red.and.pred b, %2, %3, a;\n\t"
+      "selp.b32 %0, 1, 0, b;\n\t}"
+      : "=r"(res)
+      : "r"(uint32_t(p)), "r"(id), "r"(nthreads)
+      : "memory");
+  return res != 0;
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {

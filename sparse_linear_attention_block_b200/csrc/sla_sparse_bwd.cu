@@ -21,21 +21,27 @@
 //                                        all-ones tile times the (hi, lo) bf16
 //                                        rows of -LSE/scale and -D)
 //   P^T = exp2(scale log2(e) S'^T) -> TMEM over S'^T, dS^T = P^T dP'^T -> shared
-//                                        memory (compute warpgroup g & 1; no
-//                                        per-query operand besides the TMEM tiles)
+//                                        memory (both compute warpgroups, 32
+//                                        query columns each; no per-query
+//                                        operand besides the TMEM tiles)
 //   dV += P^T dO_i, dK += dS^T Q_i       (A = P^T from TMEM, dS^T from smem)
 //   dQ_i^T = K^T dS^T                    (M = d, N = 64)
 //   dQ_i += scale dQ_i^T^T               (fp32 bulk reductions, TMA engine)
 // TMEM: dV at column 256, dK at 256 + d; four 64-column chunks at 0..255
 // rotate through S^T(g) -> dQ^T(g) in chunk g % 4 and dP^T(g) in chunk
 // (g + 1) % 4, so a chunk's life is S^T(g), dQ^T(g), dP^T(g + 3), S^T(g + 4).
+// P^T(g) (bf16, two per column) of queries 32w..32w+31 lies over the first 16
+// of those queries' own S^T columns, 32w..32w+15 of the chunk.
 // The S groups (S'^T, dP'^T) and the G groups (dV, dK, dQ^T) come from two
 // issuing threads and interleave in the tensor pipe: S(g + 1) needs only the
-// warpgroup's load of dP^T(g) and the drain of dQ^T(g - 2); G(g) needs P^T(g),
-// dS^T(g), computed while S(g + 1) runs.
+// warpgroups' load of dP^T(g) and the drain of dQ^T(g - 2); G(g) needs P^T(g),
+// dS^T(g), computed while S(g + 1) runs.  Both warpgroups work on every
+// iteration, each on half of its query columns, so that the chain from S(g)
+// to G(g) is as short as the compute allows.
 // Warp roles (512 threads; registers rebalanced with setmaxnreg):
-//   warps 0-3 / 4-7  compute warpgroups (even / odd g): P^T, dS^T, and the
-//                    tile's dK (warpgroup 0) / dV (1) epilogue  [168 registers]
+//   warps 0-3 / 4-7  compute warpgroups (query columns 0-31 / 32-63 of every
+//                    g): P^T, dS^T, and the tile's dK (warpgroup 0) / dV (1)
+//                    epilogue  [168 registers]
 //   warps 8-11       dQ warpgroup: dQ^T out of TMEM, transposed into a shared
 //                    fp32 tile of 32 query rows, added into dQ by one bulk
 //                    reduction of the TMA engine per half (the rows of a query
@@ -163,8 +169,8 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&ld_done[b], 128);
-      mbar_init(&p_full[b], 128);
+      mbar_init(&ld_done[b], 256);
+      mbar_init(&p_full[b], 256);
       mbar_init(&m_done[b], 1);
       mbar_init(&m_done[b + 2], 1);
       mbar_init(&dq_free[b], 128);
@@ -252,6 +258,14 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
             return false;
           uint8_t* st = sSt + s * L::kStage;
           const int i = ulist[t.slot + k];
+          if (k + kNSt < t.n) {  // this tile's Q, dO three iterations ahead into L2
+            const int ia = ulist[t.slot + k + kNSt];
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+              tma_prefetch_l2_3d(&tm_q, c * 64, ia * 64, t.bh);
+              tma_prefetch_l2_3d(&tm_do, c * 64, ia * 64, t.bh);
+            }
+          }
           mbar_arrive_expect_tx(&st_full[s], L::kStage);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
@@ -338,10 +352,11 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
         mma_commit(&s_full[gg & 1]);
         return true;
       };
-      // G(gg): dV += P^T dO_i (P^T in chunk gg % 4), dK += dS^T Q_i, then dQ^T
+      // G(gg): dV += P^T dO_i (P^T in chunk gg % 4, queries 16k..16k+15 at
+      // column 8 (k & 1) + 32 (k >> 1)), dK += dS^T Q_i, then dQ^T
       // over the same chunk (one thread's products run in order: dV has read
-      // P^T by then).  G(gg) follows S(gg) through p_full, so its commit also
-      // frees the stage for the producer.
+      // P^T by then).  G(gg) follows S(gg) through p_full, so the commit after
+      // dV and dK frees the stage for the producer.
       auto issue_g = [&](long gg, bool first, bool last) -> bool {
         if (!wait_spin(&p_full[gg & 1], uint32_t(gg >> 1) & 1, err, &abort_flag)) return false;
         if (first && tw > 0 &&
@@ -357,16 +372,17 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t acc = (!first || ks > 0) ? 1u : 0u;
-          mma_ts(tmem + kDV, cs + ks * 8, desc_advance(domn, mnmajor_step_bytes(ks)), id_g, acc);
+          mma_ts(tmem + kDV, cs + (ks & 1) * 8 + (ks >> 1) * 32,
+                 desc_advance(domn, mnmajor_step_bytes(ks)), id_g, acc);
           mma_ss(tmem + kDK, desc_advance(dsd_k, kmajor_step_bytes(128, ks)),
                  desc_advance(qmn, mnmajor_step_bytes(ks)), id_g, acc);
         }
+        mma_commit(&st_empty[s]);  // the last products that read the stage
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_ss(cs, desc_advance(kd_mn, mnmajor_step_bytes(ks)),
                  desc_advance(dsd_mn, mnmajor_step_bytes(ks)), id_q, ks > 0);
         mma_commit(&m_done[gg & 3]);
-        mma_commit(&st_empty[s]);
         if (last) mma_commit(&tile_done);
         return true;
       };
@@ -485,62 +501,60 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
         }
         continue;
       }
-      for (int k = int((wg - g) & 1); k < t.n; k += 2) {
+      for (int k = 0; k < t.n; ++k) {
         const long gg = g + k;
-        const uint32_t j = uint32_t(gg >> 1);
         const int fl = uflag[t.slot + k];
-        const uint32_t cs = tmem + lane_base + uint32_t(gg & 3) * 64;
-        const uint32_t cp = tmem + lane_base + uint32_t((gg + 1) & 3) * 64;
-        if (!(ok = wait_spin(&s_full[wg], j & 1, err, &abort_flag))) break;
+        // this warpgroup's 32 query columns of the S^T and dP^T chunks
+        const uint32_t cs = tmem + lane_base + uint32_t(gg & 3) * 64 + 32 * wg;
+        const uint32_t cp = tmem + lane_base + uint32_t((gg + 1) & 3) * 64 + 32 * wg;
+        // (each wait's outcome is made common to the warp: the TMEM loads and
+        // stores that follow are warp-collective)
+        ok = __all_sync(0xFFFFFFFFu, wait_spin(&s_full[gg & 1], uint32_t(gg >> 1) & 1, err, &abort_flag));
+        if (!ok) break;
         tc_fence_after();
         // (a padded query row of this block has LSE = +inf, so its P is 0)
         const bool member = key_valid && ((fl >> half) & 1);
-        uint32_t pk[32], dsk[32];
+        uint32_t pk[16], dsk[16];
         // dP'^T first: its chunk is the next S^T's, so it is handed back as soon
-        // as it is in registers; then S'^T in two halves of 32 query columns
-        // (P^T goes back over S'^T)
-        float dpa[64];
-        tmem_ld32(cp, reinterpret_cast<float(&)[32]>(dpa[0]));
-        tmem_ld32(cp + 32, reinterpret_cast<float(&)[32]>(dpa[32]));
+        // as it is in registers; then S'^T (P^T goes back over S'^T)
+        float dpa[32], sv[32];
+        tmem_ld32(cp, dpa);
         tmem_ld_wait();
         tc_fence_before();
-        mbar_arrive(&ld_done[wg]);
+        mbar_arrive(&ld_done[gg & 1]);
+        tmem_ld32(cs, sv);
+        tmem_ld_wait();
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float sv[32];
-          tmem_ld32(cs + 32 * h, sv);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float p0 = 0.f, p1 = 0.f;
-            if (member) {
-              p0 = exp2f(sv[e] * scale_log2);
-              p1 = exp2f(sv[e + 1] * scale_log2);
-            }
-            pk[16 * h + e / 2] = pack_bf16(p0, p1);
-            dsk[16 * h + e / 2] = pack_bf16(p0 * dpa[32 * h + e], p1 * dpa[32 * h + e + 1]);
+        for (int e = 0; e < 32; e += 2) {
+          float p0 = 0.f, p1 = 0.f;
+          if (member) {
+            p0 = exp2f(sv[e] * scale_log2);
+            p1 = exp2f(sv[e + 1] * scale_log2);
           }
+          pk[e / 2] = pack_bf16(p0, p1);
+          dsk[e / 2] = pack_bf16(p0 * dpa[e], p1 * dpa[e + 1]);
         }
-        // P^T (bf16) over the first 32 columns of the S^T chunk; dS^T into this
-        // iteration's buffer once its last reader, G(gg - 2), is done
-        tmem_st16(cs, reinterpret_cast<const uint32_t(&)[16]>(pk[0]));
-        tmem_st16(cs + 16, reinterpret_cast<const uint32_t(&)[16]>(pk[16]));
-        if (gg >= 2 &&
-            !(ok = wait_spin(&m_done[(gg - 2) & 3], uint32_t((gg - 2) >> 2) & 1, err, &abort_flag)))
-          break;
+        tmem_st16(cs, pk);
+        // dS^T into this iteration's buffer once its last reader, G(gg - 2), is done
+        if (gg >= 2) {
+          ok = __all_sync(0xFFFFFFFFu, wait_spin(&m_done[(gg - 2) & 3], uint32_t((gg - 2) >> 2) & 1,
+                                                 err, &abort_flag));
+          if (!ok) break;
+        }
         uint8_t* ds_tile = sDS + (gg & 1) * L::kDS;
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          st_sw128_unit(ds_tile, 128, r, 8 * u,
+        for (int u = 0; u < 4; ++u)
+          st_sw128_unit(ds_tile, 128, r, 32 * wg + 8 * u,
                         make_uint4(dsk[4 * u], dsk[4 * u + 1], dsk[4 * u + 2], dsk[4 * u + 3]));
         fence_proxy_async_smem();
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&p_full[wg]);
+        mbar_arrive(&p_full[gg & 1]);
       }
       if (!ok) break;
       // the tile's dK (warpgroup 0) / dV (warpgroup 1) rows, straight from TMEM
-      if (!(ok = wait_spin(&tile_done, uint32_t(tw) & 1, err, &abort_flag))) break;
+      ok = __all_sync(0xFFFFFFFFu, wait_spin(&tile_done, uint32_t(tw) & 1, err, &abort_flag));
+      if (!ok) break;
       tc_fence_after();
       const uint32_t acc = tmem + lane_base + (wg == 0 ? kDK : kDV);
       const float mul = wg == 0 ? scale : 1.0f;
