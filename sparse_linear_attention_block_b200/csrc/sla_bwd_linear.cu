@@ -22,7 +22,9 @@
 //                 dQ's linear share (written; the sparse branch adds to it),
 //                 dW accumulated in TMEM across the CTA's blocks
 //   bwd_k_kernel  persistent, per key block: dK, dV linear shares added to
-//                 the sparse branch's values, inputs double-buffered
+//                 the sparse branch's values, inputs double-buffered; two
+//                 warpgroups, one per half of the block's tokens, in the
+//                 read-modify-write of dK, dV
 #include <cuda_bf16.h>
 
 #include "sla_internal.h"
@@ -423,19 +425,20 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(
 //   dV^T = dh^T phi(K)^T (split products)  (M = c, N = 64 keys, K = a)
 //   dk[t][a] += (dK^T[a][t] + dz_a) * phi'(k[t][a]);  dv[t][c] += dV^T[c][t]
 // Stage n % 2 holds block n's dh tiles and V; TMEM buffer n % 2 its products,
-// so block n's products run while block n-1's sums are added to dk, dv.
+// so block n's products run while block n-1's sums are added to dk, dv
+// (warpgroup h: tokens 32h..32h+31, its thread f: feature f).
 constexpr int kBkStage = 2 * kQH + kQT;                 // dh hi, dh lo, V
 constexpr int kBkSmem = 1024 + 2 * kBkStage + 2 * kQT;  // + phi(K) hi/lo
 
 template <int D>
-__global__ void __launch_bounds__(128, 1) bwd_k_kernel(
+__global__ void __launch_bounds__(256, 1) bwd_k_kernel(
     const __grid_constant__ CUtensorMap tm_dh, const __grid_constant__ CUtensorMap tm_dl,
     const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16* __restrict__ kin,
     const __nv_bfloat16* __restrict__ dh_hi, const __nv_bfloat16* __restrict__ dh_lo,
     float* __restrict__ dk, float* __restrict__ dv, int N, int T, int nv, int nblk, int* err) {
   constexpr int W = D * D + D;
   constexpr int kU = D / 8;
-  constexpr int kRowsPerPass = 128 / kU;
+  constexpr int kRowsPerPass = 256 / kU;
   constexpr int kPass = 64 / kRowsPerPass;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = align_smem_1024(smem_raw);
@@ -444,8 +447,9 @@ __global__ void __launch_bounds__(128, 1) bwd_k_kernel(
   __shared__ uint64_t full[2], done[2];
   __shared__ uint32_t tmem_base;
   const int t = threadIdx.x, warp = t / 32;
-  const bool lane_ok = warp * 32 < D;
-  const uint32_t lane_base = uint32_t(warp * 32) << 16;
+  const int f = t & 127, th = t >> 7;  // feature (TMEM lane), token half
+  const bool lane_ok = (warp & 3) * 32 < D;
+  const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
   auto tok_of = [&](int blk) { return size_t(blk / T) * N + size_t(blk % T) * 64; };
   auto blk_of = [&](int n) { return int(blockIdx.x) + n * int(gridDim.x); };
   const int nloc = nblk > int(blockIdx.x) ? (nblk - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
@@ -461,12 +465,12 @@ __global__ void __launch_bounds__(128, 1) bwd_k_kernel(
   if (D == 64) {  // zero the feature padding of the dh and phi tiles
     for (int st = 0; st < 2; ++st) {
       uint8_t* sg = base + st * kBkStage;
-      for (int e = t; e < (kQH - 8192) / 16; e += 128) {
+      for (int e = t; e < (kQH - 8192) / 16; e += 256) {
         reinterpret_cast<uint4*>(sg + 8192)[e] = make_uint4(0, 0, 0, 0);
         reinterpret_cast<uint4*>(sg + kQH + 8192)[e] = make_uint4(0, 0, 0, 0);
       }
     }
-    for (int e = t; e < 8192 / 16; e += 128) {
+    for (int e = t; e < 8192 / 16; e += 256) {
       reinterpret_cast<uint4*>(sPh + 8192)[e] = make_uint4(0, 0, 0, 0);
       reinterpret_cast<uint4*>(sPl + 8192)[e] = make_uint4(0, 0, 0, 0);
     }
@@ -503,21 +507,22 @@ __global__ void __launch_bounds__(128, 1) bwd_k_kernel(
     for (int b = 0; b < kPass; ++b)
       kv[b] = __ldg(reinterpret_cast<const uint4*>(kin + (tk + r0 + b * kRowsPerPass) * D) + u);
   };
-  // block n's sums (TMEM buffer n % 2) added into dk, dv; lane = feature
+  // block n's sums (TMEM buffer n % 2) added into dk, dv; lane = feature,
+  // this warpgroup's 32 tokens
   auto epilogue = [&](int n, bool write) {
     if (!lane_ok) return;
     const int blk = blk_of(n);
     const size_t tk = tok_of(blk);
     const uint32_t acc = tmem + lane_base + uint32_t(n & 1) * 128;
-    const float dz = __bfloat162float(dh_hi[size_t(blk) * W + D * D + t]) +
-                     __bfloat162float(dh_lo[size_t(blk) * W + D * D + t]);
-#pragma unroll 1
-    for (int q32 = 0; q32 < 64; q32 += 32) {
-      // 32 tokens per pass: 96 independent loads per thread in flight
+    const float dz = __bfloat162float(dh_hi[size_t(blk) * W + D * D + f]) +
+                     __bfloat162float(dh_lo[size_t(blk) * W + D * D + f]);
+    {
+      const int q32 = 32 * th;
+      // 96 independent loads per thread in flight
       float ck[32], cv[32], kk[32], gk[32], gv[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const size_t idx = (tk + q32 + j) * D + t;
+        const size_t idx = (tk + q32 + j) * D + f;
         ck[j] = dk[idx];
         cv[j] = dv[idx];
         kk[j] = __bfloat162float(kin[idx]);
@@ -532,7 +537,7 @@ __global__ void __launch_bounds__(128, 1) bwd_k_kernel(
         if (lim >= 32) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const size_t idx = (tk + q32 + j) * D + t;
+            const size_t idx = (tk + q32 + j) * D + f;
             dk[idx] = fmaf(gk[j] + dz, dphi_f(kk[j]), ck[j]);
             dv[idx] = cv[j] + gv[j];
           }
@@ -540,7 +545,7 @@ __global__ void __launch_bounds__(128, 1) bwd_k_kernel(
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (j >= lim) break;
-            const size_t idx = (tk + q32 + j) * D + t;
+            const size_t idx = (tk + q32 + j) * D + f;
             dk[idx] = fmaf(gk[j] + dz, dphi_f(kk[j]), ck[j]);
             dv[idx] = cv[j] + gv[j];
           }
@@ -707,12 +712,12 @@ cudaError_t launch_bwd_k(const Problem& p, const void* k, const void* v,
   if (p.d == 128) {
     e = cudaFuncSetAttribute(bwd_k_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBkSmem);
     if (e != cudaSuccess) return e;
-    bwd_k_kernel<128><<<grid, 128, kBkSmem, s>>>(th, tl, tv, (const __nv_bfloat16*)k, dh_hi, dh_lo,
+    bwd_k_kernel<128><<<grid, 256, kBkSmem, s>>>(th, tl, tv, (const __nv_bfloat16*)k, dh_hi, dh_lo,
                                                  dk, dv, p.N, p.T, p.nv, nblk, err);
   } else {
     e = cudaFuncSetAttribute(bwd_k_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBkSmem);
     if (e != cudaSuccess) return e;
-    bwd_k_kernel<64><<<grid, 128, kBkSmem, s>>>(th, tl, tv, (const __nv_bfloat16*)k, dh_hi, dh_lo,
+    bwd_k_kernel<64><<<grid, 256, kBkSmem, s>>>(th, tl, tv, (const __nv_bfloat16*)k, dh_hi, dh_lo,
                                                 dk, dv, p.N, p.T, p.nv, nblk, err);
   }
   return cudaGetLastError();

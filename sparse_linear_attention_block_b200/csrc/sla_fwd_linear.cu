@@ -225,28 +225,24 @@ __global__ void __launch_bounds__(128) fwd_linear_kernel(
       load_q(nxt);
       load_z(nxt);  // sZ was last read by this block's den
     }
-    float os[32];
+    float os[64];  // all 64 tokens' loads in flight at once
     if (lane_ok) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) os[j] = __ldg(o_s + (tok0 + j) * D + t);
+      for (int j = 0; j < 64; ++j) os[j] = __ldg(o_s + (tok0 + j) * D + t);
     }
     ok = mbar_wait(&bar_o, k & 1, err, nullptr);
     tc_fence_after();
     // O = O_s + O^T (lane = output feature c', 64 tokens), bf16
     if (lane_ok) {
-#pragma unroll 1
-      for (int t0 = 0; t0 < 64; t0 += 32) {
-        if (t0 > 0) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) os[j] = __ldg(o_s + (tok0 + t0 + j) * D + t);
-        }
+      for (int t0 = 0; t0 < 64; t0 += 32) {
         float v[32];
         tmem_ld32(tmem + lane_base + kOut + t0, v);
         tmem_ld_wait();
         if (ok) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            o[(tok0 + t0 + j) * D + t] = __float2bfloat16_rn(fmaf(gate, v[j], os[j]));
+            o[(tok0 + t0 + j) * D + t] = __float2bfloat16_rn(fmaf(gate, v[j], os[t0 + j]));
         }
       }
     }
