@@ -91,7 +91,6 @@ def kernel_work(wl, n_crit):
         "bwd_q": ("hbm", tok * d * (2 + 2 + 4 + 4) + 2 * BH * T * (d * d + d) * 4 + tok * 4 * 2),
         "bwd_sparse": ("tensor", pairs * 10 * b * b * d),
         "bwd_k": ("hbm", tok * d * (2 + 2 + 8 + 8) + BH * T * (d * d + d) * 4),
-        "bias_rows": ("hbm", tok * (4 + 4) + tok * 64),
         "expand_marginal": ("hbm", BH * Tp * Tp * 2),
         "expand_marginal_t": ("hbm", BH * Tp * Tp * 2),
     }

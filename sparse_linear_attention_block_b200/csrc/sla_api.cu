@@ -41,7 +41,6 @@ WorkspaceLayout workspace_layout(int BH, int N, int d, int n_crit) {
   L.ulen = take(bh * ((T + 1) / 2) * 4);
   L.ulist = take(bh * T * size_t(n_crit) * 2);
   L.uflag = take(bh * T * size_t(n_crit));
-  L.bias = take(2 * bh * size_t(N) * 16 * 2);
   L.total = off;
   return L;
 }
@@ -99,19 +98,6 @@ bool make_tmap_f32_bhnd(CUtensorMap* map, const float* base, int BH, int N, int 
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-bool make_tmap_rows16(CUtensorMap* map, const void* base, int BH, int N) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {16, uint64_t(N), uint64_t(BH)};
-  cuuint64_t strides[2] = {32, uint64_t(N) * 32};
-  cuuint32_t box[3] = {16, 64, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
-                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -509,7 +495,6 @@ static sla_status backward_impl(const sla_shape* shape, const void* q, const voi
   uint16_t* ulist = at<uint16_t>(workspace, L.ulist);
   uint8_t* uflag = at<uint8_t>(workspace, L.uflag);
   int* sched = at<int>(workspace, L.err + 128);
-  auto* bias = at<__nv_bfloat16>(workspace, L.bias);
   if (cudaMemsetAsync(dw_proj, 0, size_t(p.d) * p.d * sizeof(float), s) != cudaSuccess)
     return SLA_ERR_CUDA;
   if (d_logit && cudaMemsetAsync(d_logit, 0, sizeof(float), s) != cudaSuccess) return SLA_ERR_CUDA;
@@ -519,8 +504,7 @@ static sla_status backward_impl(const sla_shape* shape, const void* q, const voi
     SLA_LAUNCH("dvec", s, launch_dvec(p, d_o, saved->o_s, dvec, s));
     SLA_LAUNCH("pair_order", s, launch_pair_order(p, mask->crit_col_ptr, mask->crit_col_idx,
                                                   ulist, uflag, ulen, order, sched, err, s));
-    SLA_LAUNCH("bias_rows", s, launch_bias_rows(p, saved->lse, dvec, bias, s));
-    SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, bias, mask->crit_col_ptr,
+    SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr,
                                                   ulist, uflag, ulen, order, sched, dq, dk, dv,
                                                   sms, err, s));
     return SLA_OK;
@@ -536,8 +520,7 @@ static sla_status backward_impl(const sla_shape* shape, const void* q, const voi
   // branch's key side adds its share
   SLA_LAUNCH("pair_order", s, launch_pair_order(p, mask->crit_col_ptr, mask->crit_col_idx,
                                                 ulist, uflag, ulen, order, sched, err, s));
-  SLA_LAUNCH("bias_rows", s, launch_bias_rows(p, saved->lse, dvec, bias, s));
-  SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, bias, mask->crit_col_ptr, ulist,
+  SLA_LAUNCH("bwd_sparse", s, launch_bwd_sparse(p, q, k, v, d_o, saved->lse, dvec, mask->crit_col_ptr, ulist,
                                                 uflag, ulen, order, sched, dq, dk, dv, sms, err,
                                                 s));
   SLA_LAUNCH("bwd_k", s, launch_bwd_k(p, k, v, dh_hi, dh_lo, dk, dv, sms, err, s));

@@ -44,7 +44,6 @@ struct WorkspaceLayout {
   size_t ulen;       // int32 [BH*ceil(T/2)] union length of each key-block pair
   size_t ulist;      // uint16 [BH*T*n_crit] each pair's union, in the pair's column-CSR slot
   size_t uflag;      // uint8 [BH*T*n_crit] membership bits of the union entries
-  size_t bias;       // bf16 [2][BH,N,16] rows (hi, lo, 0...) of -LSE/scale, then of -D
   size_t total;
 };
 
@@ -109,17 +108,13 @@ cudaError_t launch_bwd_q(const Problem& p, const void* q, const void* d_o, const
 cudaError_t launch_pair_order(const Problem& p, const int32_t* col_ptr, const int32_t* col_idx,
                               uint16_t* ulist, uint8_t* uflag, int32_t* ulen, int32_t* order,
                               int* sched, int* err, cudaStream_t s);
-// The sparse backward's bias rows: for every token t, (hi, lo) bf16 pairs of
-// -LSE_t/scale and of -D_t, each padded to 16 values.
-cudaError_t launch_bias_rows(const Problem& p, const float* lse, const float* dvec,
-                             __nv_bfloat16* bias, cudaStream_t s);
 // Persistent: min(tiles, num_sms) CTAs take the tiles in order from the
 // counter `sched` (zero at launch).
 cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
-                              const void* d_o, const __nv_bfloat16* bias, const int32_t* col_ptr,
-                              const uint16_t* ulist, const uint8_t* uflag, const int32_t* ulen,
-                              const int32_t* order, int* sched, float* dq, float* dk, float* dv,
-                              int num_sms, int* err, cudaStream_t s);
+                              const void* d_o, const float* lse, const float* dvec,
+                              const int32_t* col_ptr, const uint16_t* ulist, const uint8_t* uflag,
+                              const int32_t* ulen, const int32_t* order, int* sched, float* dq,
+                              float* dk, float* dv, int num_sms, int* err, cudaStream_t s);
 cudaError_t launch_bwd_k(const Problem& p, const void* k, const void* v,
                          const __nv_bfloat16* dh_hi, const __nv_bfloat16* dh_lo, float* dk,
                          float* dv, int num_sms, int* err, cudaStream_t s);
@@ -145,9 +140,6 @@ cudaError_t launch_named(const char* name, cudaStream_t s, F&& launch) {
 // TMA descriptor for a bf16 [BH, N, d] tensor viewed as 3D {d, N, BH} with a
 // box of {64, rows, 1} and 128-byte swizzle.  Returns false on failure.
 bool make_tmap_bhnd(CUtensorMap* map, const void* base, int BH, int N, int d, int box_rows);
-// TMA descriptor for a bf16 [BH, N, 16] tensor with a box {16, 64, 1} and
-// 32-byte swizzle (one MMA K-step of 64 rows).
-bool make_tmap_rows16(CUtensorMap* map, const void* base, int BH, int N);
 // TMA descriptor for a bf16 3D tensor {inner, rows, batch} (row pitch = inner).
 bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
                   uint64_t batch, uint32_t box_inner, uint32_t box_rows);

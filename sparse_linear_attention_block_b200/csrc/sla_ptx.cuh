@@ -150,6 +150,17 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bo
 
 // ------------------------------------------------------------------ TMA
 
+// Plain bulk copy global -> shared, completing on `bar` (complete_tx): both
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
@@ -297,15 +308,6 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          (uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46)  // descriptor version
          | (2ull << 61);                                               // SWIZZLE_128B
-}
-
-// K-major operand tile of 16 bf16 per row (32-byte rows, 32-byte swizzle, as
-// a TMA box {16, rows} with CU_TENSOR_MAP_SWIZZLE_32B writes it): one MMA
-// K-step; 8-row groups 256 bytes apart.
-__device__ __forceinline__ uint64_t sdesc_sw32_kmajor(uint32_t saddr) {
-  return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t(1) << 16) | (uint64_t(256 >> 4) << 32) |
-         (1ull << 46)    // descriptor version
-         | (6ull << 61);  // SWIZZLE_32B
 }
 
 // K-major operand tile stored as column chunks of 64 bf16 (128 B per row),

@@ -15,24 +15,22 @@
 // iteration counter g that runs on across tiles, so that the stage ring, the
 // TMEM chunks and the two compute warpgroups keep their rhythm at a tile
 // boundary.  Per iteration g (query block i):
-//   S'^T = K Q_i^T - LSE_i/scale, dP'^T = V dO_i^T - D_i
-//                                        (tcgen05, M = 128 keys, N = 64; the
-//                                        shifts are one more K-step each: an
-//                                        all-ones tile times the (hi, lo) bf16
-//                                        rows of -LSE/scale and -D)
-//   P^T = exp2(scale log2(e) S'^T) -> TMEM over S'^T, dS^T = P^T dP'^T -> shared
-//                                        memory (both compute warpgroups, 32
-//                                        query columns each; no per-query
-//                                        operand besides the TMEM tiles)
-//   dV += P^T dO_i, dK += dS^T Q_i       (A = P^T from TMEM, dS^T from smem)
+//   S^T = K Q_i^T, dP^T = V dO_i^T       (tcgen05, M = 128 keys, N = 64)
+//   P^T = exp2(log2(e) (scale S^T - LSE_i)) -> TMEM over S^T,
+//   dS^T = P^T (dP^T - D_i) -> TMEM over S^T and shared memory
+//                                        (both compute warpgroups, 32 query
+//                                        columns each; LSE_i, D_i come with
+//                                        the stage)
+//   dV += P^T dO_i, dK += dS^T Q_i       (A = P^T, dS^T from TMEM)
 //   dQ_i^T = K^T dS^T                    (M = d, N = 64)
 //   dQ_i += scale dQ_i^T^T               (fp32 bulk reductions, TMA engine)
 // TMEM: dV at column 256, dK at 256 + d; four 64-column chunks at 0..255
 // rotate through S^T(g) -> dQ^T(g) in chunk g % 4 and dP^T(g) in chunk
 // (g + 1) % 4, so a chunk's life is S^T(g), dQ^T(g), dP^T(g + 3), S^T(g + 4).
 // P^T(g) (bf16, two per column) of queries 32w..32w+31 lies over the first 16
-// of those queries' own S^T columns, 32w..32w+15 of the chunk.
-// The S groups (S'^T, dP'^T) and the G groups (dV, dK, dQ^T) come from two
+// of those queries' own S^T columns, 32w..32w+15 of the chunk, and dS^T(g)
+// over the next 16, 32w+16..32w+31.
+// The S groups (S^T, dP^T) and the G groups (dV, dK, dQ^T) come from two
 // issuing threads and interleave in the tensor pipe: S(g + 1) needs only the
 // warpgroups' load of dP^T(g) and the drain of dQ^T(g - 2); G(g) needs P^T(g),
 // dS^T(g), computed while S(g + 1) runs.  Both warpgroups work on every
@@ -48,8 +46,8 @@
 //                    block are contiguous in dQ), so that neither the compute
 //                    warps nor the mbarrier traffic queue behind 8192 scalar
 //                    reductions per iteration  [96]
-//   warp 12          TMA producer: K, V per tile; Q_i, dO_i and the bias rows
-//                    of query block i per iteration into a 3-stage ring  [80]
+//   warp 12          TMA producer: K, V per tile; Q_i, dO_i, LSE_i and D_i of
+//                    query block i per iteration into a 3-stage ring  [80]
 //   warps 13 / 14    single-thread tcgen05 issuers of the S and the G groups
 //                    (warp 15 idle)  [80]
 #include <cuda_bf16.h>
@@ -62,17 +60,18 @@ namespace sla {
 namespace {
 
 constexpr int kNSt = 3;  // Q/dO stages
+constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct SbSmem {
   static constexpr int kKV = 128 * D * 2;       // K or V tile (128 keys)
   static constexpr int kQ = 64 * D * 2;         // Q_i or dO_i tile (64 queries)
-  static constexpr int kBias = 64 * 32;         // 64 bias rows of 16 bf16
-  static constexpr int kStage = 2 * kQ + 2 * kBias;  // Q, dO, -LSE/scale rows, -D rows
+  static constexpr int kLD = 1024;              // LSE_i, D_i (64 fp32 each; 1024-byte pitch)
+  static constexpr int kStage = 2 * kQ + kLD;   // Q, dO, LSE_i, D_i
+  static constexpr int kStageBytes = 2 * kQ + 512;  // what a stage's copies bring
   static constexpr int kDS = 128 * 64 * 2;      // dS^T bf16 [128 keys][64 queries]
-  static constexpr int kOnes = 128 * 32;        // all-ones A tile of the bias K-step
   static constexpr int kStg = 32 * D * 4;       // fp32 dQ rows of 32 queries
-  static constexpr int kTotal = 1024 + 2 * kKV + kNSt * kStage + 2 * kDS + kOnes + kStg;
+  static constexpr int kTotal = 1024 + 2 * kKV + kNSt * kStage + 2 * kDS + kStg;
 };
 
 // The waits of this kernel poll with test_wait instead of a suspending
@@ -134,11 +133,11 @@ template <int D>
 __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-    const __grid_constant__ CUtensorMap tm_bias, int BH, const int32_t* __restrict__ col_ptr,
+    const float* __restrict__ lse, const float* __restrict__ dvec, const int32_t* __restrict__ col_ptr,
     const uint16_t* __restrict__ ulist,
     const uint8_t* __restrict__ uflag, const int32_t* __restrict__ ulen,
     const int32_t* __restrict__ order, int* __restrict__ sched, int n_tiles, int N, int T,
-    int n_crit, int nv, float scale_log2, float scale, float* __restrict__ dq,
+    int n_crit, int nv, float scale, float* __restrict__ dq,
     float* __restrict__ dk, float* __restrict__ dv, int* err) {
   using L = SbSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -147,8 +146,7 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
   uint8_t* sV = sK + L::kKV;
   uint8_t* sSt = sV + L::kKV;
   uint8_t* sDS = sSt + kNSt * L::kStage;  // two buffers, for even and odd iterations
-  uint8_t* sOnes = sDS + 2 * L::kDS;
-  float* sStg = reinterpret_cast<float*>(sOnes + L::kOnes);  // dQ staging for bulk reductions
+  float* sStg = reinterpret_cast<float*>(sDS + 2 * L::kDS);  // dQ staging for bulk reductions
 
   __shared__ uint64_t kv_full, tile_done, acc_free, st_full[kNSt], st_empty[kNSt], s_full[2],
       ld_done[2], p_full[2], m_done[4], dq_free[4], tq_full[2], tq_empty[2], fin;
@@ -182,10 +180,6 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
     abort_flag = 0;
     fence_barrier_init();
   }
-  for (int x = threadIdx.x; x < L::kOnes / 16; x += blockDim.x)  // bf16 1.0 everywhere
-    reinterpret_cast<uint4*>(sOnes)[x] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u,
-                                                    0x3F803F80u);
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -212,7 +206,6 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
       tma_prefetch_desc(&tm_do);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_bias);
       long g = 0;       // iterations issued before the current tile
       int tw = 0;       // tiles with work so far
       long issued = 0;  // stage loads issued
@@ -266,14 +259,15 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
               tma_prefetch_l2_3d(&tm_do, c * 64, ia * 64, t.bh);
             }
           }
-          mbar_arrive_expect_tx(&st_full[s], L::kStage);
+          mbar_arrive_expect_tx(&st_full[s], L::kStageBytes);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
             tma_load_3d(st + c * 64 * 128, &st_full[s], &tm_q, c * 64, i * 64, t.bh);
             tma_load_3d(st + L::kQ + c * 64 * 128, &st_full[s], &tm_do, c * 64, i * 64, t.bh);
           }
-          tma_load_3d(st + 2 * L::kQ, &st_full[s], &tm_bias, 0, i * 64, t.bh);
-          tma_load_3d(st + 2 * L::kQ + L::kBias, &st_full[s], &tm_bias, 0, i * 64, BH + t.bh);
+          const size_t row0 = size_t(t.bh) * N + size_t(i) * 64;
+          bulk_load(st + 2 * L::kQ, lse + row0, 256, &st_full[s]);
+          bulk_load(st + 2 * L::kQ + 256, dvec + row0, 256, &st_full[s]);
           ++issued;
           return true;
         };
@@ -318,7 +312,6 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
       constexpr uint32_t id_q = idesc_bf16(128, 64, 1, 1);  // dQ^T = K^T dS^T
       const uint64_t kd_k = desc_kmajor_base(smem_u32(sK)), vd_k = desc_kmajor_base(smem_u32(sV));
       const uint64_t kd_mn = desc_mnmajor_base(smem_u32(sK), 128);
-      const uint64_t ones_d = sdesc_sw32_kmajor(smem_u32(sOnes));
       const bool s_stream = warp == 13;
       long g = 0;
       int tw = 0;
@@ -346,14 +339,12 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
           mma_ss(cp, desc_advance(vd_k, kmajor_step_bytes(128, ks)),
                  desc_advance(dod, kmajor_step_bytes(64, ks)), id_s, ks > 0);
         }
-        // the shifts: ones x (hi, lo) rows of -LSE/scale and of -D
-        mma_ss(cs, ones_d, sdesc_sw32_kmajor(q0 + 2 * L::kQ), id_s, 1);
-        mma_ss(cp, ones_d, sdesc_sw32_kmajor(q0 + 2 * L::kQ + L::kBias), id_s, 1);
         mma_commit(&s_full[gg & 1]);
         return true;
       };
-      // G(gg): dV += P^T dO_i (P^T in chunk gg % 4, queries 16k..16k+15 at
-      // column 8 (k & 1) + 32 (k >> 1)), dK += dS^T Q_i, then dQ^T
+      // G(gg): dV += P^T dO_i, dK += dS^T Q_i (both A operands in chunk gg % 4:
+      // queries 16k..16k+15 of P^T at column 8 (k & 1) + 32 (k >> 1), of dS^T 16
+      // columns further), then dQ^T
       // over the same chunk (one thread's products run in order: dV has read
       // P^T by then).  G(gg) follows S(gg) through p_full, so the commit after
       // dV and dK frees the stage for the producer.
@@ -368,14 +359,13 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
         const uint64_t qmn = desc_mnmajor_base(q0, 64), domn = desc_mnmajor_base(do0, 64);
         const uint32_t cs = tmem + uint32_t(gg & 3) * 64;
         const uint32_t ds0 = smem_u32(sDS + (gg & 1) * L::kDS);
-        const uint64_t dsd_k = desc_kmajor_base(ds0), dsd_mn = desc_mnmajor_base(ds0, 128);
+        const uint64_t dsd_mn = desc_mnmajor_base(ds0, 128);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t acc = (!first || ks > 0) ? 1u : 0u;
-          mma_ts(tmem + kDV, cs + (ks & 1) * 8 + (ks >> 1) * 32,
-                 desc_advance(domn, mnmajor_step_bytes(ks)), id_g, acc);
-          mma_ss(tmem + kDK, desc_advance(dsd_k, kmajor_step_bytes(128, ks)),
-                 desc_advance(qmn, mnmajor_step_bytes(ks)), id_g, acc);
+          const uint32_t pa = cs + (ks & 1) * 8 + (ks >> 1) * 32;
+          mma_ts(tmem + kDV, pa, desc_advance(domn, mnmajor_step_bytes(ks)), id_g, acc);
+          mma_ts(tmem + kDK, pa + 16, desc_advance(qmn, mnmajor_step_bytes(ks)), id_g, acc);
         }
         mma_commit(&st_empty[s]);  // the last products that read the stage
 #pragma unroll
@@ -509,14 +499,17 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
         const uint32_t cp = tmem + lane_base + uint32_t((gg + 1) & 3) * 64 + 32 * wg;
         // (each wait's outcome is made common to the warp: the TMEM loads and
         // stores that follow are warp-collective)
+        // (the stage's LSE_i, D_i, read below, landed before S(gg) was issued:
+        // its issuer waited for the stage's copies, and this wait is ordered
+        // before the reads)
         ok = __all_sync(0xFFFFFFFFu, wait_spin(&s_full[gg & 1], uint32_t(gg >> 1) & 1, err, &abort_flag));
         if (!ok) break;
         tc_fence_after();
         // (a padded query row of this block has LSE = +inf, so its P is 0)
         const bool member = key_valid && ((fl >> half) & 1);
         uint32_t pk[16], dsk[16];
-        // dP'^T first: its chunk is the next S^T's, so it is handed back as soon
-        // as it is in registers; then S'^T (P^T goes back over S'^T)
+        // dP^T first: its chunk is the next S^T's, so it is handed back as soon
+        // as it is in registers; then S^T (P^T and dS^T go back over S^T)
         float dpa[32], sv[32];
         tmem_ld32(cp, dpa);
         tmem_ld_wait();
@@ -524,17 +517,28 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
         mbar_arrive(&ld_done[gg & 1]);
         tmem_ld32(cs, sv);
         tmem_ld_wait();
+        // LSE, D of this warpgroup's 32 queries, from the iteration's stage (the
+        // stage is released only after G(gg), which waits for this thread's p_full)
+        const float* ld = reinterpret_cast<const float*>(sSt + (gg % kNSt) * L::kStage + 2 * L::kQ) +
+                          32 * wg;
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float p0 = 0.f, p1 = 0.f;
-          if (member) {
-            p0 = exp2f(sv[e] * scale_log2);
-            p1 = exp2f(sv[e + 1] * scale_log2);
+        for (int e = 0; e < 32; e += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(ld + e);
+          const float4 d4 = *reinterpret_cast<const float4*>(ld + 64 + e);
+          const float lq[4] = {l4.x, l4.y, l4.z, l4.w}, dq4[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int m = 0; m < 4; m += 2) {
+            float p0 = 0.f, p1 = 0.f;
+            if (member) {
+              p0 = exp2f(kLog2e * fmaf(sv[e + m], scale, -lq[m]));
+              p1 = exp2f(kLog2e * fmaf(sv[e + m + 1], scale, -lq[m + 1]));
+            }
+            pk[(e + m) / 2] = pack_bf16(p0, p1);
+            dsk[(e + m) / 2] = pack_bf16(p0 * (dpa[e + m] - dq4[m]), p1 * (dpa[e + m + 1] - dq4[m + 1]));
           }
-          pk[e / 2] = pack_bf16(p0, p1);
-          dsk[e / 2] = pack_bf16(p0 * dpa[e], p1 * dpa[e + 1]);
         }
         tmem_st16(cs, pk);
+        tmem_st16(cs + 16, dsk);
         // dS^T into this iteration's buffer once its last reader, G(gg - 2), is done
         if (gg >= 2) {
           ok = __all_sync(0xFFFFFFFFu, wait_spin(&m_done[(gg - 2) & 3], uint32_t((gg - 2) >> 2) & 1,
@@ -579,30 +583,6 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_free(tmem, 512);
-}
-
-// ------------------------------------------------------------------ bias rows
-// For every token: row 0 = (hi, lo) of -LSE/scale, row 1 = (hi, lo) of -D,
-// padded with zeros to 16 bf16 (one MMA K-step), hi = bf16(x), lo = bf16(x -
-// hi).  A padded query row (LSE = +inf) and a row without critical blocks
-// (LSE = -inf, never in a union) both get -inf, so that P = 0.
-__global__ void __launch_bounds__(256) bias_rows_kernel(const float* __restrict__ lse,
-                                                        const float* __restrict__ dvec,
-                                                        uint4* __restrict__ bias, long long ntok,
-                                                        float inv_scale) {
-  const long long t = blockIdx.x * 256ll + threadIdx.x;
-  if (t >= ntok) return;
-  auto row = [&](float x, uint4* out) {
-    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-    const __nv_bfloat16 lo = isfinite(x) ? __float2bfloat16_rn(x - __bfloat162float(hi))
-                                         : __float2bfloat16_rn(0.f);
-    const uint32_t w = uint32_t(__bfloat16_as_ushort(hi)) | (uint32_t(__bfloat16_as_ushort(lo)) << 16);
-    out[0] = make_uint4(w, 0u, 0u, 0u);
-    out[1] = make_uint4(0u, 0u, 0u, 0u);
-  };
-  const float l = lse[t];
-  row(isfinite(l) ? -l * inv_scale : -INFINITY, bias + 2 * t);
-  row(-dvec[t], bias + 2 * (ntok + t));
 }
 
 // ------------------------------------------------------------------ tile unions
@@ -717,21 +697,15 @@ cudaError_t launch_pair_order(const Problem& p, const int32_t* col_ptr, const in
   return cudaGetLastError();
 }
 
-cudaError_t launch_bias_rows(const Problem& p, const float* lse, const float* dvec,
-                             __nv_bfloat16* bias, cudaStream_t s) {
-  const long long ntok = (long long)p.BH * p.N;
-  bias_rows_kernel<<<unsigned((ntok + 255) / 256), 256, 0, s>>>(
-      lse, dvec, reinterpret_cast<uint4*>(bias), ntok, 1.0f / p.scale);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, const void* v,
-                              const void* d_o, const __nv_bfloat16* bias, const int32_t* col_ptr,
-                              const uint16_t* ulist, const uint8_t* uflag, const int32_t* ulen,
-                              const int32_t* order, int* sched, float* dq, float* dk, float* dv,
-                              int num_sms, int* err, cudaStream_t s) {
-  CUtensorMap tq, tk, tv, tdo, tb;
-  if (!make_tmap_rows16(&tb, bias, 2 * p.BH, p.N)) return cudaErrorInvalidValue;
+                              const void* d_o, const float* lse, const float* dvec,
+                              const int32_t* col_ptr, const uint16_t* ulist, const uint8_t* uflag,
+                              const int32_t* ulen, const int32_t* order, int* sched, float* dq,
+                              float* dk, float* dv, int num_sms, int* err, cudaStream_t s) {
+  // LSE_i and D_i go to shared memory by bulk copies: 16-byte aligned rows
+  if ((reinterpret_cast<uintptr_t>(lse) | reinterpret_cast<uintptr_t>(dvec)) % 16 != 0)
+    return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv, tdo;
   if (!make_tmap_bhnd(&tq, q, p.BH, p.N, p.d, 64)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tk, k, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_bhnd(&tv, v, p.BH, p.N, p.d, 128)) return cudaErrorInvalidValue;
@@ -744,18 +718,18 @@ cudaError_t launch_bwd_sparse(const Problem& p, const void* q, const void* k, co
     e = cudaFuncSetAttribute(bwd_sparse_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem));
     if (e != cudaSuccess) return e;
-    bwd_sparse_kernel<128><<<grid, 512, smem, s>>>(tq, tk, tv, tdo, tb, p.BH, col_ptr, ulist,
+    bwd_sparse_kernel<128><<<grid, 512, smem, s>>>(tq, tk, tv, tdo, lse, dvec, col_ptr, ulist,
                                                    uflag, ulen, order, sched, n_tiles, p.N, p.T,
-                                                   p.n_crit, p.nv, p.scale_log2, p.scale, dq, dk,
+                                                   p.n_crit, p.nv, p.scale, dq, dk,
                                                    dv, err);
   } else {
     constexpr size_t smem = SbSmem<64>::kTotal;
     e = cudaFuncSetAttribute(bwd_sparse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem));
     if (e != cudaSuccess) return e;
-    bwd_sparse_kernel<64><<<grid, 512, smem, s>>>(tq, tk, tv, tdo, tb, p.BH, col_ptr, ulist,
+    bwd_sparse_kernel<64><<<grid, 512, smem, s>>>(tq, tk, tv, tdo, lse, dvec, col_ptr, ulist,
                                                   uflag, ulen, order, sched, n_tiles, p.N, p.T, p.n_crit,
-                                                  p.nv, p.scale_log2, p.scale, dq, dk, dv, err);
+                                                  p.nv, p.scale, dq, dk, dv, err);
   }
   return cudaGetLastError();
 }
