@@ -456,7 +456,8 @@ def main():
         achieved = amount / avg_s / 1e12
         peak = tensor_peak
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "frac_of_sustained": achieved / pk["bf16_tflops_sustained"],
+                "frac": achieved / peak, "frac_of_burst": achieved / pk["bf16_tflops"],
+                "frac_of_sustained": achieved / pk["bf16_tflops_sustained"],
                 "traffic": traffic, "kernel": dominant, "peak_source": tensor_src}
     else:
         achieved = amount / avg_s / 1e9
