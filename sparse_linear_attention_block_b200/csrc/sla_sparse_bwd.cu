@@ -410,19 +410,8 @@ __global__ void __launch_bounds__(512, 1) bwd_sparse_kernel(
     const int r = wq * 32 + lane;
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
     const bool leader = threadIdx.x == 256;
-    auto wg_bar = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
-    auto wg_all = [](bool p) -> bool {
-      uint32_t res;
-      asm volatile(
-          "{\n\t.reg .pred a, b;\n\t"
-          "setp.ne.b32 a, %1, 0;\n\t"
-          "bar.red.and.pred b, 1, 128, a;\n\t"
-          "selp.b32 %0, 1, 0, b;\n\t}"
-          : "=r"(res)
-          : "r"(uint32_t(p))
-          : "memory");
-      return res != 0;
-    };
+    auto wg_bar = [] { named_bar_sync(1, 128); };
+    auto wg_all = [](bool p) -> bool { return named_bar_and(1, 128, p); };
     float* stg[2] = {sStg, sStg + 16 * D};
     long g = 0;
     bool ok = true;
