@@ -16,11 +16,16 @@
 //              TMEM (bf16, aliasing S), lazy rescaling of O in TMEM
 //   warp 4     TMA producer: Q tile once; K_j tiles into a 2-slot ring whose
 //              slot is freed as soon as S_n = Q K_n^T has been computed, V_j
-//              into a 2-slot ring freed by P_n V_n (separate rings keep the K
-//              copies off the softmax -> P V -> S chain)
+//              into a 3-slot ring freed by P_n V_n (separate rings keep the K
+//              copies off the softmax -> P V -> S chain; the third V slot
+//              gives a V copy two iterations to land)
 //   warp 5     MMA issuer (one thread): S_n into one of two TMEM buffers,
 //              O += P_n V_n with P read from TMEM
 // TMEM: S buffers at columns [0,64) and [64,128), O at [128, 128+D).
+// Shared memory: Q, the K and V slots, the union list and the barriers, all in
+// the dynamic region (no static shared memory, so that two CTAs fit on an SM
+// with the third V slot; the region starts 1024-byte aligned, which is
+// checked).
 #include <cuda_bf16.h>
 
 #include "sla_internal.h"
@@ -30,16 +35,28 @@
 namespace sla {
 namespace {
 
-constexpr int kStages = 2;
+constexpr int kStages = 2;   // K slots
+constexpr int kVStages = 3;  // V slots
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct FwdBars {
+  uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kVStages], v_empty[kVStages],
+      s_full[2], p_full[2], o_done, mma_done, osync;
+  uint32_t tmem_base;
+  int n_union, abort_flag;
+};
 
 template <int D>
 struct FwdSmem {
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVBytes = 64 * D * 2;  // one K or V tile
-  static constexpr int kTiles = kQBytes + 2 * kStages * kKVBytes;  // K slots, then V slots
-  // + the union list: 2*n_crit uint16 block indices, then 2*n_crit flag bytes
-  static size_t total(int n_crit) { return 1024 + kTiles + size_t(2 * n_crit) * 3 + 16; }
+  static constexpr int kTiles = kQBytes + (kStages + kVStages) * kKVBytes;  // K slots, then V slots
+  // then the union list (2*n_crit uint16 block indices, then 2*n_crit flag
+  // bytes) and the barriers
+  __host__ __device__ static size_t bars(int n_crit) {
+    return kTiles + (size_t(2 * n_crit) * 3 + 15) / 16 * 16;
+  }
+  static size_t total(int n_crit) { return bars(n_crit) + sizeof(FwdBars); }
 };
 
 template <int D>
@@ -49,17 +66,25 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
     const int32_t* __restrict__ crit_idx, int N, int T, int n_crit, int nv, float scale_log2,
     float* __restrict__ lse, int* err) {
   using L = FwdSmem<D>;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = align_smem_1024(smem_raw);
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  // the swizzled tiles need 1024-byte alignment: the kernel has no static
+  // shared memory, so the dynamic region starts at the CTA's window; if it
+  // does not, nothing is done and the launch reports an error
+  if ((smem_u32(smem_raw) & 1023u) != 0u) {
+    if (threadIdx.x == 0) set_error(err, SLA_ERR_DEVICE);
+    return;
+  }
+  uint8_t* base = smem_raw;
   uint8_t* sQ = base;
   uint8_t* sKV = base + L::kQBytes;
   uint16_t* ulist = reinterpret_cast<uint16_t*>(base + L::kTiles);
   uint8_t* uflag = base + L::kTiles + 2 * (2 * n_crit);
-
-  __shared__ uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages],
-      v_empty[kStages], s_full[2], p_full[2], o_done, mma_done, osync;
-  __shared__ uint32_t tmem_base;
-  __shared__ int n_union, abort_flag;
+  FwdBars& bb = *reinterpret_cast<FwdBars*>(base + L::bars(n_crit));
+  uint64_t &q_full = bb.q_full, &o_done = bb.o_done, &mma_done = bb.mma_done, &osync = bb.osync;
+  uint64_t *k_full = bb.k_full, *k_empty = bb.k_empty, *v_full = bb.v_full,
+           *v_empty = bb.v_empty, *s_full = bb.s_full, *p_full = bb.p_full;
+  uint32_t& tmem_base = bb.tmem_base;
+  int &n_union = bb.n_union, &abort_flag = bb.abort_flag;
 
   const int p = blockIdx.x, bh = blockIdx.y;
   const int warp = threadIdx.x / 32, lane = lane_id();
@@ -72,6 +97,8 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
@@ -113,9 +140,9 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
       mbar_arrive_expect_tx(&q_full, L::kQBytes);
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * 128 * 128, &q_full, &tm_q, c * 64, p * 128, bh);
-      // K_n needs S_{n-2} done, V_n needs P_{n-2} V_{n-2} done; the pipe
+      // K_n needs S_{n-2} done, V_n needs P_{n-3} V_{n-3} done; the pipe
       // completes S_0, S_1, PV_0, S_2, PV_1, S_3, ... so requests go out in
-      // that order: K_0 V_0 K_1 V_1 K_2 K_3, then V_m K_{m+2} for m >= 2.
+      // that order: K_0 V_0 K_1 V_1 V_2 K_2 K_3, then V_m K_{m+1} for m >= 3.
       int nk = 0, nv = 0;  // K and V copies issued
       auto load_k = [&](int n) -> bool {
         const int s = n % kStages;
@@ -130,8 +157,8 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
         return true;
       };
       auto load_v = [&](int n) -> bool {
-        const int s = n % kStages;
-        if (n >= kStages && !mbar_wait(&v_empty[s], ((n / kStages) + 1) & 1, err, &abort_flag))
+        const int s = n % kVStages;
+        if (n >= kVStages && !mbar_wait(&v_empty[s], ((n / kVStages) + 1) & 1, err, &abort_flag))
           return false;
         uint8_t* sv = sKV + (kStages + s) * L::kKVBytes;
         mbar_arrive_expect_tx(&v_full[s], L::kKVBytes);
@@ -142,19 +169,20 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
         return true;
       };
       bool go = true;
-      for (int n = 0; go && n < kStages && n < nU; ++n) go = load_k(n) && load_v(n);
-      for (int n = kStages; go && n < 2 * kStages && n < nU; ++n) go = load_k(n);
-      for (int m = kStages; go && m < nU; ++m) {
+      for (int n = 0; go && n < 2 && n < nU; ++n) go = load_k(n) && load_v(n);
+      if (go && 2 < nU) go = load_v(2);
+      for (int n = 2; go && n < 4 && n < nU; ++n) go = load_k(n);
+      for (int m = 3; go && m < nU; ++m) {
         go = load_v(m);
-        if (go && m + kStages < nU) go = load_k(m + kStages);
+        if (go && m + 1 >= 4 && m + 1 < nU) go = load_k(m + 1);
       }
       if (abort_flag) {
         // let copies already in flight land before the CTA exits
         mbar_wait(&q_full, 0, nullptr, nullptr);
         for (int n = (nk > kStages ? nk - kStages : 0); n < nk; ++n)
           mbar_wait(&k_full[n % kStages], (n / kStages) & 1, nullptr, nullptr);
-        for (int n = (nv > kStages ? nv - kStages : 0); n < nv; ++n)
-          mbar_wait(&v_full[n % kStages], (n / kStages) & 1, nullptr, nullptr);
+        for (int n = (nv > kVStages ? nv - kVStages : 0); n < nv; ++n)
+          mbar_wait(&v_full[n % kVStages], (n / kVStages) & 1, nullptr, nullptr);
       }
     }
   } else if (warp == 5) {
@@ -178,9 +206,9 @@ __global__ void __launch_bounds__(192, 2) fwd_sparse_kernel(
         return true;
       };
       auto issue_pv = [&](int n) -> bool {
-        const int s = n % kStages;
+        const int s = n % kVStages;
         if (!mbar_wait(&p_full[n & 1], (n >> 1) & 1, err, &abort_flag) ||
-            !mbar_wait(&v_full[s], (n / kStages) & 1, err, &abort_flag))
+            !mbar_wait(&v_full[s], (n / kVStages) & 1, err, &abort_flag))
           return false;
         tc_fence_after();
         const uint64_t vd = desc_mnmajor_base(smem_u32(sKV + (kStages + s) * L::kKVBytes), 64);
