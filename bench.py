@@ -73,9 +73,6 @@ def executed_block_flops(wl, n_crit):
 NCU_DRAM_BYTES_PER_HEAD = {
     "bwd_sparse": (395.572224e6 + 233.325056e6) / 4,
     "fwd_sparse": (100.750592e6 + 35.872512e6) / 4,
-    "bwd_k": (337.421568e6 + 90.642432e6) / 4,
-    "fwd_linear": (236.025088e6 + 20.761856e6) / 4,
-    "bwd_q": (270.171904e6 + 155.145472e6) / 4,
     "pool": (67.117824e6 + 0.468992e6) / 4,
     "summaries": (67.146496e6 + 79.487232e6) / 4,
 }

@@ -192,6 +192,13 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(
   for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x, ++k) {
     const size_t tok0 = tok_of(blk);
     const int nxt = blk + int(gridDim.x);
+    if (t == 0 && nxt < nblk) {  // the next block's Q, dO, O_s rows and H, Z into L2 meanwhile
+      bulk_prefetch_l2(q + tok_of(nxt) * D, 64 * D * 2);
+      bulk_prefetch_l2(d_o + tok_of(nxt) * D, 64 * D * 2);
+      bulk_prefetch_l2(o_s + tok_of(nxt) * D, 64 * D * 4);
+      bulk_prefetch_l2(hz_hi + size_t(nxt) * W, W * 2);
+      bulk_prefetch_l2(hz_lo + size_t(nxt) * W, W * 2);
+    }
     // ---- phi(Q) as hi/lo K-major tiles [64 t][a]
 #pragma unroll
     for (int b = 0; b < kPass; ++b) {
@@ -558,6 +565,14 @@ __global__ void __launch_bounds__(256, 1) bwd_k_kernel(
   if (nloc > 0) load_k(0);
   for (int n = 0; n < nloc; ++n) {
     const int b = n & 1;
+    if (t == 0) {  // into L2 meanwhile: the dK, dV rows of block n (added to in the next
+                   // iteration) and the K rows of block n+1 (prefetching dh two blocks
+                   // ahead as well measured slower)
+      const size_t tk = tok_of(blk_of(n));
+      bulk_prefetch_l2(dk + tk * D, 64 * D * 4);
+      bulk_prefetch_l2(dv + tk * D, 64 * D * 4);
+      if (n + 1 < nloc) bulk_prefetch_l2(kin + tok_of(blk_of(n + 1)) * D, 64 * D * 2);
+    }
     if (n > 0) {  // block n-1's products done: the phi tiles and stage (n-1) % 2 are free
       ok = mbar_wait(&done[(n - 1) & 1], ((n - 1) >> 1) & 1, err, nullptr);
       tc_fence_after();

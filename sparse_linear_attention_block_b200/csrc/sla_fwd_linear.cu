@@ -132,6 +132,10 @@ __global__ void __launch_bounds__(128) fwd_linear_kernel(
     const size_t tok0 = tok_of(blk);
     const int nxt = blk + int(gridDim.x);
     const int vrows = nv - (blk % T) * 64;  // rows of this block that exist (key padding)
+    if (t == 0 && nxt < nblk) {  // the next block's Q and O_s rows into L2 meanwhile
+      bulk_prefetch_l2(q + tok_of(nxt) * D, 64 * D * 2);
+      bulk_prefetch_l2(o_s + tok_of(nxt) * D, 64 * D * 4);
+    }
     // phi(Q) as hi/lo K-major tiles [64 t][a]; den_t = phi(Q_t) . Z_i in fp32,
     // each thread's 8 features summed, then over the kU threads of a row
 #pragma unroll

@@ -193,6 +193,12 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int x, 
       : "memory");
 }
 
+// Plain bulk prefetch of global memory into L2 (address 16-byte aligned, bytes
+// a multiple of 16); no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Tiled 3D store shared -> global (bulk async group; the source tile is in the
 // 128-byte swizzled layout of the map).  Issue after fence_proxy_async_smem()
 // and a barrier with the threads that wrote the tile.
